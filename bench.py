@@ -1,0 +1,409 @@
+#!/usr/bin/env python3
+"""Decode-step benchmark: sparse mixed-precision paged decode attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c1] [--impl kvq|reference]
+
+One step = one decode step of one attention layer for the whole batch, all of it in
+libkvq kernels: append the new token (quantise + pack + summary), score every page,
+select top-k + sink + recent pages, sparse split-K attention + log-sum-exp combine.
+
+Timing: W untimed steps, then K steps timed on the device with CUDA events on the
+launching stream (one event between kernels, so per-kernel durations come from the
+same run); L2 is flushed by writing a 512 MiB buffer before every timed step, outside
+the events.  The whole-step time is bracketed by a barrier + synchronize; with N > 1
+(torchrun, one process per GPU, NCCL) every rank runs its own independent batch (weak
+scaling: sequences are independent problems, no collective on the data path) and the
+max time over ranks is used.  Rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle (the plain fp64 restatement of the method)
+on the host cores on a bounded sample of the same workload and prints the same line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-step attn tokens/s and achieved HBM GB/s (% of roofline), 1×B200"
+FLUSH_BYTES = 512 << 20
+
+DESCR = {
+    "c0": "tiny: 1 seq, 8 q / 2 kv heads, D 64, 1024 tokens, fp16, all 16-bit pages, top-8 + page 0 + last page",
+    "c1": "Llama-3-8B-shaped layer: batch 8, 32 q / 8 kv heads, D 128, context 32768 (+1 appended token), "
+          "bf16 pages, 5% of pages + sink + 4 recent selected per kv head",
+    "c2": "c1 shape, tiers 16-bit/int8/int4/int2 = 10/20/30/40%, 10% selected, +1 appended token",
+    "c3": "batch 1, 32 q / 8 kv heads, D 128, context 131072 (+1), int4 cold / 16-bit hot pages, "
+          "permuted block table, 5% + sink + 16 recent",
+    "c4": "ragged Qwen2.5-3B-shaped layer: batch 64, 16 q / 2 kv heads, D 128, contexts log-uniform 2k-64k, "
+          "tiers 16-bit/int4/int2/1-bit = 10/30/40/20%, 8% + sink + 4 recent",
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock / throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "50", "-i", str(self.index)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        rows = [l.split(", ") for (t, l) in self.lines if t0 <= t <= t1 + 0.06]
+        rows = [r for r in rows if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- bytes
+def algorithmic_bytes(w, sel: np.ndarray, cnt: np.ndarray, tier_tbl: np.ndarray):
+    """Bytes the step must move: (attention, scores, select, append) per launch."""
+    from sparse_mixed_precision_kvq_b200.kvq import kvq_chunk_bytes
+    cb = np.array([2 * kvq_chunk_bytes(t, w.D) for t in range(5)], dtype=np.int64)
+    attn = 0
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            pages = sel[b, g, :cnt[b, g]]
+            attn += int(cb[tier_tbl[b, pages]].sum())
+    q_bytes = w.B * w.Hq * w.D * 2
+    attn += q_bytes + w.B * w.Hq * w.D * 2 + int(cnt.sum()) * 4          # q, out, page list
+    P = np.array([w.pages_after(b) for b in range(w.B)])
+    score = int(P.sum()) * w.Hkv * w.D * 2 + q_bytes + w.B * w.Hkv * w.max_pages * 4
+    select = w.B * w.Hkv * w.max_pages * 4 + int(cnt.sum()) * 4
+    append = w.B * w.Hkv * w.D * 2 * 2 if w.append else 0
+    return dict(attn=attn, score=score, select=select, append=append)
+
+
+def kernel_traffic(kernel_file: str):
+    """ncu DRAM bytes per launch recorded for the current source of a kernel, else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "sparse_mixed_precision_kvq_b200", "csrc", kernel_file)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    e = d.get(kernel_file)
+    if not e or e.get("source_sha256_16") != h:
+        return None
+    return e
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_kvq(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    from sparse_mixed_precision_kvq_b200 import kvq
+    from sparse_mixed_precision_kvq_b200 import workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = W.make(args.config, seed=W.make(args.config).seed + 1000 * rank)
+    cache = kvq.cache_from_workload(w, device=dev)
+    step = kvq.DecodeStep(w, cache, device=dev)
+    tier_tbl, _, _ = w.slot_map()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step.run()
+    torch.cuda.synchronize(dev)
+    assert cache.err_bits() == 0, f"device error bits {cache.err_bits():#x}"
+    sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
+    nbytes = algorithmic_bytes(w, sel, cnt, tier_tbl)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[0])
+                          if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local_rank)
+    if rank == 0:
+        clocks.start()
+        time.sleep(1.0)  # let nvidia-smi start sampling
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    for k in range(K):
+        flush.fill_(k & 0xFF)
+        e = ev[k]
+        e[0].record(stream)
+        step.append()
+        e[1].record(stream)
+        step.scores_()
+        e[2].record(stream)
+        step.select()
+        e[3].record(stream)
+        step.attend()
+        e[4].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t1 = time.time()
+    clocks.stop()
+    per = np.array([[ev[k][i].elapsed_time(ev[k][i + 1]) for i in range(4)] for k in range(K)])  # ms
+    step_ms = per.sum(1)
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    tokens = world * w.B * K
+    value = tokens / (total_ms / 1e3)
+
+    # end to end through the public API: host q / new token in, host out / lse back
+    pin = dict(q=step.q.cpu().pin_memory())
+    if w.append:
+        pin["k"], pin["v"] = step.k_new.cpu().pin_memory(), step.v_new.cpu().pin_memory()
+    out_h = torch.empty_like(step.out, device="cpu").pin_memory()
+    lse_h = torch.empty_like(step.lse, device="cpu").pin_memory()
+    KE = max(1, min(K, 500))
+    e_start = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
+    e_end = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
+    for k in range(KE):
+        flush.fill_(k & 0xFF)
+        e_start[k].record(stream)
+        step.q.copy_(pin["q"], non_blocking=True)
+        if w.append:
+            step.k_new.copy_(pin["k"], non_blocking=True)
+            step.v_new.copy_(pin["v"], non_blocking=True)
+        step.run()
+        out_h.copy_(step.out, non_blocking=True)
+        lse_h.copy_(step.lse, non_blocking=True)
+        e_end[k].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = float(np.mean([e_start[k].elapsed_time(e_end[k]) for k in range(KE)]))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = pin["q"].numel() * 2 + (pin["k"].numel() * 2 * 2 if w.append else 0)
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+
+    # optional dense reference point: every page selected (c1's dense run)
+    dense_ms = None
+    if args.dense and rank == 0:
+        dense_ms = time_dense(w, cache, step, flush, stream, dev)
+
+    if rank != 0:
+        return None
+    peak, peak_kind = load_peaks()
+    names = ["append", "page_scores", "select_topk", "sparse_decode_attn"]
+    avg = per.mean(0)
+    dom = int(np.argmax(avg))
+    dom_bytes = [nbytes["append"], nbytes["score"], nbytes["select"], nbytes["attn"]][dom]
+    achieved = dom_bytes / (avg[dom] * 1e-3) / 1e9
+    files = ["append.cu", "score.cu", "select.cu", "attn.cu"]
+    tr = kernel_traffic(files[dom])
+    step_bytes = nbytes["attn"] + nbytes["score"] + nbytes["select"] + nbytes["append"]
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f16",
+        "data": "synthetic (seeded; shapes and value laws of the workload; no model weights)",
+        "config": {"workload": f"{args.config}: {DESCR[args.config]}", "batch_per_gpu": w.B,
+                   "context": int(w.lens.max()), "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
+                   "selected_pages": int(cnt.sum()), "l2": "flushed (512 MiB write) before every timed step",
+                   "parallelism": f"replicas x{world} (independent batches)"},
+        "step_hbm": {"bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3) / 1e9,
+                     "peak_gbs": peak, "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak,
+                     "peak_kind": peak_kind},
+        "kernels_ms": {n: float(a) for n, a in zip(names, avg)},
+        "roofline": {"bound": "hbm", "kernel": names[dom], "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
+                     "algorithmic_bytes_per_launch": dom_bytes,
+                     "traffic": None if tr is None else tr["dram_bytes_per_launch"]},
+        "e2e": {"value": world * w.B / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
+        "gpu_launches": 5 * K,
+        "clocks": clocks.summary(t0, t1),
+    }
+    if dense_ms is not None:
+        line["dense_all_pages_ms"] = dense_ms
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
+    return line
+
+
+def time_dense(w, cache, step, flush, stream, dev, reps=20):
+    import torch
+    from sparse_mixed_precision_kvq_b200 import kvq
+    P = np.array([w.pages_after(b) for b in range(w.B)])
+    kmax = int(P.max())
+    sel = np.zeros((w.B, w.Hkv, kmax), dtype=np.int32)
+    for b in range(w.B):
+        sel[b, :, :P[b]] = np.arange(P[b])
+    sel_t = torch.from_numpy(sel).to(dev)
+    cnt_t = torch.from_numpy(np.repeat(P[:, None], w.Hkv, 1).astype(np.int32)).to(dev)
+    ws = torch.empty(kvq.kvq_workspace_size(cache, kmax) // 4 + 4, dtype=torch.float32, device=dev)
+    out = torch.empty_like(step.out)
+    ts = []
+    for r in range(reps + 3):
+        flush.fill_(r & 0xFF)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        kvq.kvq_sparse_decode_attn(cache, step.q, sel_t, cnt_t, kmax, w.sm_scale, out, None, ws)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        if r >= 3:
+            ts.append(a.elapsed_time(b_))
+    return float(np.mean(ts))
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def cpu_baseline(w, budget_s: float = 15.0):
+    """The oracle's decode step timed on the host cores on a bounded sample of (b, g) pairs.
+
+    Cache construction (the oracle's quantise/pack of the prefilled context) is excluded;
+    each timed unit is the oracle step of one (sequence, kv head): append, score,
+    select, attention of its G query heads.  tokens/s = B / (mean unit time * B * Hkv).
+    """
+    import copy
+    from threadpoolctl import threadpool_limits
+    from oracle.fp import bits16_to_f64
+    from oracle.step import prepare, step_pair
+
+    q = bits16_to_f64(w.query_bits(), w.dtype)
+    kn, vn = w.new_kv_bits() if w.append else (None, None)
+    pairs = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+    rng = np.random.default_rng(0)
+    order = [pairs[i] for i in rng.permutation(len(pairs))][:4]
+    prepared = [(b, g, prepare(w, b, g)) for b, g in order]
+    times = []
+    spent = 0.0
+    with threadpool_limits(limits=1):
+        while spent < budget_s:
+            for b, g, sh in prepared:
+                sh2 = copy.deepcopy(sh)
+                t0 = time.perf_counter()
+                step_pair(w, sh2, b, g, q[b], None if kn is None else kn[b, g], None if vn is None else vn[b, g])
+                dt = time.perf_counter() - t0
+                times.append(dt)
+                spent += dt
+            if len(times) >= 400:
+                break
+    unit = float(np.mean(times))
+    t_step = unit * w.B * w.Hkv
+    return {"value": w.B / t_step, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{len(times)} timed oracle steps of single (sequence, kv head) units drawn from "
+                      f"{len(prepared)} units of the same workload; step time = mean unit time x {w.B * w.Hkv} "
+                      f"units; cache construction excluded; numpy/BLAS limited to 1 thread"}
+
+
+def run_reference(args, rank: int, world: int):
+    from sparse_mixed_precision_kvq_b200 import workloads as W
+    if rank != 0:
+        return None
+    w = W.make(args.config)
+    K = args.steps
+    budget = max(5.0, min(60.0, 150.0 / max(1, K + args.warmup)))
+    base = cpu_baseline(w, budget_s=budget)
+    line = {
+        "metric": METRIC, "value": base["value"], "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": 1e3 * w.B / base["value"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.config}: {DESCR[args.config]}", "batch_per_gpu": w.B},
+        "impl": "reference", "cpu_baseline": base,
+        "e2e": {"value": base["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="c1", choices=sorted(DESCR))
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--dense", action="store_true", help="also time attention over every page")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import datetime
+            import torch
+            import torch.distributed as dist
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        line = run_kvq(args, rank, world, local_rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if line is not None and rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,213 @@
+/*
+ * kvq.h -- C ABI of libkvq: sparse mixed-precision paged decode attention on B200.
+ *
+ * One decode step of one attention layer over a paged KV cache:
+ *
+ *   kvq_append             write the step's new K/V token into its page (quantised to the
+ *                          page's tier) and refresh the page's mean-key summary;
+ *   kvq_page_scores        score every page from its summary;
+ *   kvq_select_topk        pick the top pages plus forced sink/recent pages;
+ *   kvq_sparse_decode_attn attend only the selected pages (split-K + log-sum-exp combine),
+ *                          unpacking and dequantising cold pages in registers.
+ *
+ * Sources: AMASS "decode-time sparse KV-cache attention for vLLM" (amass-kv 0.1.1),
+ * section "What is in the box" (per-page summary -> page score -> small selected working
+ * set -> sparse paged kernel reading only those pages) and "Quickstart" (budget: fixed
+ * selected fraction); ARGUS "Virtual Memory for Transformers" (argus_cache 0.1.7.1),
+ * sections "The One-Minute Explanation" / "Visual Architecture" (fp16 hot pages, INT8,
+ * INT4 2-way, INT2 4-way, 1-bit 8-way packed cold pages, reconstruction only when a query
+ * touches a page), "Why It Works" (dequantise, then attend) and "Quickstart"
+ * (sink_tokens).
+ *
+ * Conventions (every call):
+ *  - Pointers named "device" are device memory owned by the caller; the library never
+ *    allocates, frees or synchronises.  All work is enqueued on the given stream; a call
+ *    returns after enqueueing.  Host structs (kvq_cache, kvq_select_params) are read
+ *    during the call only.
+ *  - Return: KVQ_OK, or an argument error found on the host before anything is enqueued
+ *    (KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED / KVQ_ERR_WORKSPACE), or KVQ_ERR_CUDA when
+ *    the launch itself failed (cudaGetLastError).
+ *  - Data errors found on the device (bad block-table entry, page or position out of
+ *    range, non-finite input, fp16 metadata overflow, NaN score, too many selected pages,
+ *    a pipeline wait that ran out) set bits in *err_word (sticky; the caller clears it).
+ *    The offending unit is skipped or clamped.  Kernels never trap.
+ *  - Calls on different streams that write the same cache memory must not overlap.
+ *
+ * Cache layout (all device memory, T = 16 tokens per page, D in {64, 128}):
+ *  - block_table [B][max_pages] int32: entry = (tier << 29) | slot, tier in kvq_tier.
+ *    A logical page's tier is shared by all kv heads.
+ *  - pool[tier]: pool_slots[tier] physical slots; slot s holds, for kv head g and kind
+ *    k (0 = K, 1 = V), one chunk of kvq_chunk_bytes(tier, D) bytes at byte offset
+ *    ((s * Hkv + g) * 2 + k) * kvq_chunk_bytes(tier, D).  Base must be 16-byte aligned.
+ *    Chunk = codes then meta.  Codes order: each element (t, d) belongs to lane
+ *    lam, register pair R = 4*(d/16) + r and half h, with c = d % 16:
+ *      K:  lam = 4*(t%8) + (c%8)/2,  r = 2*(c/8) + t/8,  h = c%2
+ *      V:  lam = 4*(c%8) + (t%8)/2,  r = 2*(t/8) + c/8,  h = t%2
+ *    16-bit tier: half h of uint32 word (d/16*32 + lam)*4 + r.
+ *    b-bit tiers: lane word w = R/(16/b), slot j = R%(16/b); low code at bits b*j,
+ *    high code at bits 16 + b*j; NW = D*b/64 words per lane, PW = min(4, NW); lane word
+ *    w is uint32 ((w/PW)*32 + lam)*PW + w%PW of the codes area.  1-bit code 1 = +.
+ *    Meta: b = 8/4/2: uint32 [T][D/32] = scale_fp16 | zero_fp16 << 16;
+ *          1-bit:     uint16 [T][D/32] = magnitude fp16.  Empty slots are zero.
+ *    Value read back: 16-bit: as stored; b-bit: fp32(c * scale + zero) (one rounding);
+ *    1-bit: +m or -m.
+ *  - summary [B][Hkv][max_pages][D] fp16: fp16(mean of the page's keys as they arrived).
+ *  - open_ksum [B][Hkv][D] double: running fp64 sum of the keys of the page that holds
+ *    position seq_len-1 when that page is not full.
+ *  - seq_len [B] int32: tokens in each sequence (read by scores/select/attention; the
+ *    caller advances it after kvq_append).
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* kvq_stream_t; /* identical to cudaStream_t; NULL = legacy stream */
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1,
+  KVQ_ERR_UNSUPPORTED = 2,
+  KVQ_ERR_WORKSPACE = 3,
+  KVQ_ERR_CUDA = 4
+} kvq_status;
+
+typedef enum { KVQ_DT_F16 = 0, KVQ_DT_BF16 = 1 } kvq_dtype;
+
+typedef enum {
+  KVQ_TIER_16 = 0, /* cache dtype, unchanged */
+  KVQ_TIER_I8 = 1, /* 8-bit codes, per-32-channel fp16 scale/zero */
+  KVQ_TIER_I4 = 2, /* 4-bit codes, two per byte */
+  KVQ_TIER_I2 = 3, /* 2-bit codes, four per byte */
+  KVQ_TIER_I1 = 4  /* sign bits, eight per byte, per-32-channel fp16 magnitude */
+} kvq_tier;
+
+/* device error-word bits */
+#define KVQ_DERR_BAD_PAGE 0x1u      /* block-table entry with bad tier/slot, or page out of range */
+#define KVQ_DERR_FP16_RANGE 0x2u    /* fp16 scale/zero/magnitude/summary saturated at +-65504 */
+#define KVQ_DERR_NAN_SCORE 0x4u     /* NaN page score (ranked lowest) */
+#define KVQ_DERR_KMAX 0x8u          /* more selected pages than kmax (list truncated) */
+#define KVQ_DERR_NONFINITE 0x10u    /* non-finite key/value quantised */
+#define KVQ_DERR_TIMEOUT 0x20u      /* a bounded pipeline wait ran out (work skipped) */
+#define KVQ_DERR_BAD_POS 0x40u      /* append position outside the block table */
+
+typedef struct {
+  int32_t B, Hq, Hkv, D;   /* batch, query heads, kv heads (Hq % Hkv == 0, Hq/Hkv <= 8), head dim */
+  int32_t page_size;       /* must be 16 */
+  int32_t max_pages;       /* block-table row length (logical pages per sequence) */
+  int32_t dtype;           /* kvq_dtype of keys, values, queries and outputs */
+  int32_t reserved;
+  int32_t* block_table;    /* device [B][max_pages] */
+  int32_t* seq_len;        /* device [B] */
+  void* pool[5];           /* device, per tier (NULL if unused) */
+  int64_t pool_slots[5];   /* slots in each pool */
+  uint16_t* summary;       /* device [B][Hkv][max_pages][D] fp16 bits */
+  double* open_ksum;       /* device [B][Hkv][D] */
+  uint32_t* err_word;      /* device, 1 word */
+} kvq_cache;
+
+typedef struct {
+  int32_t k_abs;      /* >= 0: select this many pages; < 0: use k_frac_bp */
+  int32_t k_frac_bp;  /* fraction in basis points: k = ceil(P * k_frac_bp / 10000) per sequence */
+  int32_t n_sink;     /* first n_sink pages always attended (in addition to k) */
+  int32_t n_recent;   /* last n_recent pages always attended (in addition to k) */
+} kvq_select_params;
+
+/* Bytes of one chunk (one page, one kv head, K or V) of a tier; 0 for a bad tier/D. */
+size_t kvq_chunk_bytes(int32_t tier, int32_t D);
+
+/* Human-readable status. */
+const char* kvq_status_string(kvq_status s);
+
+/*
+ * kvq_append -- write one new token per sequence into the cache.
+ * (ARGUS "The One-Minute Explanation": new tokens are hot; cold tiers per "Visual
+ *  Architecture".  AMASS "What is in the box": the per-page summary the score reads.)
+ *  pos    device [B] int32: logical position written for each sequence (normally
+ *         seq_len[b]); pos < 0 skips the sequence.  The page pos/16 must already have a
+ *         block-table entry; when pos % 16 == 0 the page's chunks are cleared first.
+ *  k_new, v_new  device [B][Hkv][D] in the cache dtype.
+ *  Quantises the token into its page's tier (per 32-channel group: zero = fp16(min),
+ *  scale = fp16((max-min)/(2^b-1)), code = clamp(rint((x-zero)/scale)); 1-bit: sign and
+ *  fp16(mean|x|)), sets open_ksum = (pos%16 ? open_ksum : 0) + k (fp64) and
+ *  summary[b][g][pos/16] = fp16(open_ksum / (pos%16 + 1)).  Does not change seq_len.
+ *  A page written by append must not be shared with another sequence.
+ */
+kvq_status kvq_append(const kvq_cache* cache, const int32_t* pos, const void* k_new,
+                      const void* v_new, kvq_stream_t stream);
+
+/*
+ * kvq_build_pages -- store a prefilled context (bulk form of kvq_append).
+ *  k_src, v_src  device [Hkv][src_tokens][D] in the cache dtype; sequence b's token i is
+ *                row cu_seqlens[b] + i.
+ *  cu_seqlens    device [B+1] int64.
+ *  Stores tokens [0, seq_len[b]) of every sequence into the pages named by the block
+ *  table (same quantiser as kvq_append), writes every page's summary and the open page's
+ *  open_ksum.  Token slots past seq_len are zero.
+ */
+kvq_status kvq_build_pages(const kvq_cache* cache, const void* k_src, const void* v_src,
+                           const int64_t* cu_seqlens, int64_t src_tokens, kvq_stream_t stream);
+
+/*
+ * kvq_page_scores -- page score (AMASS "What is in the box": compact per-page score;
+ * its "quad" form is not given, the mean-key form is used).
+ *  q       device [B][Hq][D] in the cache dtype.
+ *  scores  device [B][Hkv][max_pages] fp32 out:
+ *          scores[b][g][p] = max over h in [g*G, g*G+G) of sum_d q[b][h][d] * summary[b][g][p][d]
+ *          for p < ceil(seq_len[b]/16), and -inf for the remaining pages.
+ */
+kvq_status kvq_page_scores(const kvq_cache* cache, const void* q, float* scores,
+                           kvq_stream_t stream);
+
+/*
+ * kvq_select_topk -- per (sequence, kv head) page selection (AMASS "Quickstart" budget;
+ * ARGUS "Quickstart" sink_tokens).
+ *  scores  device [B][Hkv][max_pages] fp32 (as written by kvq_page_scores).
+ *  params  host: budget k and forced sink/recent page counts.
+ *  sel     device [B][Hkv][kmax] int32 out: forced pages plus the k best other pages
+ *          (score descending, lower page index first on ties, NaN lowest), ascending.
+ *  cnt     device [B][Hkv] int32 out: entries written to sel (<= kmax).
+ *  kmax    row length of sel; a longer selection is truncated and flagged.
+ */
+kvq_status kvq_select_topk(const kvq_cache* cache, const float* scores,
+                           const kvq_select_params* params, int32_t* sel, int32_t* cnt,
+                           int32_t kmax, kvq_stream_t stream);
+
+/* Workspace bytes kvq_sparse_decode_attn needs on the current device for this cache. */
+kvq_status kvq_workspace_size(const kvq_cache* cache, int32_t kmax, size_t* bytes);
+
+/*
+ * kvq_sparse_decode_attn -- attention of each query head over the tokens of its kv
+ * head's selected pages (AMASS "What is in the box"; ARGUS "Why It Works": low-bit
+ * values are turned back into high precision before attention).
+ *  q         device [B][Hq][D], cache dtype.
+ *  sel, cnt  as written by kvq_select_topk (pages must be < ceil(seq_len/16)).
+ *  sm_scale  softmax scale (1/sqrt(D) for standard attention).
+ *  out       device [B][Hq][D] cache dtype out: softmax(sm_scale * q.k) v over the tokens
+ *            of the selected pages; zeros when a kv head has no selected page.
+ *  lse       device [B][Hq] fp32 out (may be NULL): natural-log log-sum-exp of the
+ *            scaled logits (-inf when nothing is selected).
+ *  workspace device scratch of at least kvq_workspace_size() bytes (split-K partials).
+ */
+kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const int32_t* sel,
+                                  const int32_t* cnt, int32_t kmax, float sm_scale, void* out,
+                                  float* lse, void* workspace, size_t ws_bytes,
+                                  kvq_stream_t stream);
+
+/*
+ * kvq_dequant_page -- values read back from storage for one logical page (testing aid).
+ *  out device [Hkv][2][16][D] fp32: for each kv head, K then V, every token slot: the
+ *  16-bit value, fp32(c * scale + zero), or +-m, per the page's tier.
+ */
+kvq_status kvq_dequant_page(const kvq_cache* cache, int32_t b, int32_t page, float* out,
+                            kvq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVQ_H_ */

@@ -1,0 +1,188 @@
+// extern "C" entry points of libkvq (see include/kvq.h): host-side argument checks, then
+// one or two kernel launches on the caller's stream.  No allocation, no synchronisation.
+#include <stdint.h>
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+// kvq_dequant_page: the value read back from storage for every element of one page.
+__global__ void dequant_kernel(DevCache c, int b, int page, float* __restrict__ out) {
+  const int g = blockIdx.x >> 1, kind = blockIdx.x & 1;
+  const int D = c.D;
+  int tier;
+  const unsigned char* ck;
+  if (!page_chunk(c, b, page, g, tier, ck)) return;
+  const unsigned char* chunk = ck + (size_t)kind * c.chunk[tier];
+  const int ng = D / kGroup;
+  for (int e = threadIdx.x; e < kPage * D; e += blockDim.x) {
+    const int t = e / D, d = e % D;
+    int w, bit;
+    elem_pos(kind, tier, D, t, d, w, bit);
+    const uint32_t word = reinterpret_cast<const uint32_t*>(chunk)[w];
+    float v;
+    if (tier == KVQ_TIER_16) {
+      const uint16_t x = static_cast<uint16_t>(word >> bit);
+      v = c.dtype == KVQ_DT_BF16 ? bits_to_float<true>(x) : bits_to_float<false>(x);
+    } else {
+      const int bits = tier_bits(tier);
+      const uint32_t code = (word >> bit) & ((1u << bits) - 1u);
+      const unsigned char* meta = chunk + codes_bytes(tier, D);
+      if (tier == KVQ_TIER_I1) {
+        const float m = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(meta)[t * ng + d / kGroup]));
+        v = code ? m : -m;
+      } else {
+        const uint32_t mw = reinterpret_cast<const uint32_t*>(meta)[t * ng + d / kGroup];
+        const float scale = __half2float(__ushort_as_half(static_cast<uint16_t>(mw & 0xFFFFu)));
+        const float zero = __half2float(__ushort_as_half(static_cast<uint16_t>(mw >> 16)));
+        v = fmaf(static_cast<float>(code), scale, zero);
+      }
+    }
+    out[(((size_t)g * 2 + kind) * kPage + t) * D + d] = v;
+  }
+}
+
+bool g_supported_g(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
+
+kvq_status to_dev(const kvq_cache* k, DevCache& c) {
+  if (k == nullptr) return KVQ_ERR_INVALID_ARG;
+  if (k->B < 1 || k->Hq < 1 || k->Hkv < 1 || k->max_pages < 1 || k->Hq % k->Hkv != 0)
+    return KVQ_ERR_INVALID_ARG;
+  if (k->page_size != kPage || (k->D != 64 && k->D != 128)) return KVQ_ERR_UNSUPPORTED;
+  if (k->dtype != KVQ_DT_F16 && k->dtype != KVQ_DT_BF16) return KVQ_ERR_UNSUPPORTED;
+  if (!g_supported_g(k->Hq / k->Hkv)) return KVQ_ERR_UNSUPPORTED;
+  if ((long long)k->B * k->Hkv > 65535) return KVQ_ERR_UNSUPPORTED;
+  if (k->block_table == nullptr || k->seq_len == nullptr || k->summary == nullptr ||
+      k->open_ksum == nullptr || k->err_word == nullptr)
+    return KVQ_ERR_INVALID_ARG;
+  c.B = k->B;
+  c.Hq = k->Hq;
+  c.Hkv = k->Hkv;
+  c.G = k->Hq / k->Hkv;
+  c.D = k->D;
+  c.max_pages = k->max_pages;
+  c.dtype = k->dtype;
+  c.block_table = k->block_table;
+  c.seq_len = k->seq_len;
+  bool any = false;
+  for (int t = 0; t < kNumTiers; ++t) {
+    c.pool[t] = static_cast<unsigned char*>(k->pool[t]);
+    c.pool_slots[t] = k->pool[t] ? k->pool_slots[t] : 0;
+    c.chunk[t] = chunk_bytes(t, k->D);
+    if (k->pool[t] && (reinterpret_cast<uintptr_t>(k->pool[t]) % 16 != 0 || k->pool_slots[t] < 0))
+      return KVQ_ERR_INVALID_ARG;
+    any |= k->pool[t] != nullptr;
+  }
+  if (!any) return KVQ_ERR_INVALID_ARG;
+  c.summary = k->summary;
+  c.open_ksum = k->open_ksum;
+  c.err = k->err_word;
+  return KVQ_OK;
+}
+
+kvq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) d = 0;
+  return d;
+}
+
+}  // namespace
+}  // namespace kvq
+
+using namespace kvq;
+
+extern "C" {
+
+size_t kvq_chunk_bytes(int32_t tier, int32_t D) {
+  if (tier < 0 || tier >= kNumTiers || (D != 64 && D != 128)) return 0;
+  return static_cast<size_t>(chunk_bytes(tier, D));
+}
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case KVQ_ERR_WORKSPACE: return "workspace too small";
+    case KVQ_ERR_CUDA: return "CUDA launch error";
+  }
+  return "unknown status";
+}
+
+kvq_status kvq_append(const kvq_cache* cache, const int32_t* pos, const void* k_new, const void* v_new,
+                      kvq_stream_t stream) {
+  DevCache c;
+  kvq_status st = to_dev(cache, c);
+  if (st != KVQ_OK) return st;
+  if (pos == nullptr || k_new == nullptr || v_new == nullptr) return KVQ_ERR_INVALID_ARG;
+  return cuda_status(launch_append(c, pos, k_new, v_new, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_build_pages(const kvq_cache* cache, const void* k_src, const void* v_src,
+                           const int64_t* cu_seqlens, int64_t src_tokens, kvq_stream_t stream) {
+  DevCache c;
+  kvq_status st = to_dev(cache, c);
+  if (st != KVQ_OK) return st;
+  if (k_src == nullptr || v_src == nullptr || cu_seqlens == nullptr || src_tokens < 0) return KVQ_ERR_INVALID_ARG;
+  return cuda_status(launch_build(c, k_src, v_src, cu_seqlens, src_tokens, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_page_scores(const kvq_cache* cache, const void* q, float* scores, kvq_stream_t stream) {
+  DevCache c;
+  kvq_status st = to_dev(cache, c);
+  if (st != KVQ_OK) return st;
+  if (q == nullptr || scores == nullptr || !aligned16(q)) return KVQ_ERR_INVALID_ARG;
+  return cuda_status(launch_scores(c, q, scores, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_select_topk(const kvq_cache* cache, const float* scores, const kvq_select_params* params,
+                           int32_t* sel, int32_t* cnt, int32_t kmax, kvq_stream_t stream) {
+  DevCache c;
+  kvq_status st = to_dev(cache, c);
+  if (st != KVQ_OK) return st;
+  if (scores == nullptr || params == nullptr || sel == nullptr || cnt == nullptr || kmax < 1)
+    return KVQ_ERR_INVALID_ARG;
+  if ((size_t)c.max_pages * 4 > 200 * 1024) return KVQ_ERR_UNSUPPORTED;
+  return cuda_status(launch_select(c, scores, *params, sel, cnt, kmax, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_workspace_size(const kvq_cache* cache, int32_t kmax, size_t* bytes) {
+  DevCache c;
+  kvq_status st = to_dev(cache, c);
+  if (st != KVQ_OK) return st;
+  if (bytes == nullptr || kmax < 1) return KVQ_ERR_INVALID_ARG;
+  *bytes = attn_workspace_bytes(c, attn_num_ctas(current_device()));
+  return KVQ_OK;
+}
+
+kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const int32_t* sel, const int32_t* cnt,
+                                  int32_t kmax, float sm_scale, void* out, float* lse, void* workspace,
+                                  size_t ws_bytes, kvq_stream_t stream) {
+  DevCache c;
+  kvq_status st = to_dev(cache, c);
+  if (st != KVQ_OK) return st;
+  if (q == nullptr || sel == nullptr || cnt == nullptr || out == nullptr || workspace == nullptr || kmax < 1)
+    return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(workspace) || !(sm_scale > 0.f)) return KVQ_ERR_INVALID_ARG;
+  if ((long long)c.B * c.Hkv + 1 > 8192) return KVQ_ERR_UNSUPPORTED;  // segment offsets live in shared memory
+  const int n = attn_num_ctas(current_device());
+  if (ws_bytes < attn_workspace_bytes(c, n)) return KVQ_ERR_WORKSPACE;
+  return cuda_status(launch_attn(c, q, sel, cnt, kmax, sm_scale, out, lse, workspace, n,
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_dequant_page(const kvq_cache* cache, int32_t b, int32_t page, float* out, kvq_stream_t stream) {
+  DevCache c;
+  kvq_status st = to_dev(cache, c);
+  if (st != KVQ_OK) return st;
+  if (out == nullptr || b < 0 || b >= c.B || page < 0 || page >= c.max_pages) return KVQ_ERR_INVALID_ARG;
+  dequant_kernel<<<c.Hkv * 2, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(c, b, page, out);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

@@ -1,0 +1,273 @@
+"""Python binding of libkvq (ctypes): the C ABI of ``include/kvq.h`` with the same names.
+
+Every function here only marshals arguments (``torch.Tensor.data_ptr()``, the current
+CUDA stream) and raises on a non-OK status; all work runs in the CUDA kernels of
+``libkvq.so``.  There is no CPU fallback: importing this module fails when the library
+has not been built, and calls fail when no CUDA device is present.
+
+``PagedCache`` allocates the cache's device tensors with PyTorch (plumbing only) and
+fills a ``kvq_cache`` struct that points at them.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_float, c_int32, c_int64, c_size_t, c_void_p
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libkvq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libkvq.so not found at {LIB_PATH}: build it with "
+        "`python -m sparse_mixed_precision_kvq_b200.build` (there is no CPU fallback)")
+_lib = ctypes.CDLL(LIB_PATH)
+
+TIER_16, TIER_I8, TIER_I4, TIER_I2, TIER_I1 = 0, 1, 2, 3, 4
+DT_F16, DT_BF16 = 0, 1
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "workspace too small", 4: "CUDA error"}
+
+DERR_BAD_PAGE, DERR_FP16_RANGE, DERR_NAN_SCORE, DERR_KMAX = 0x1, 0x2, 0x4, 0x8
+DERR_NONFINITE, DERR_TIMEOUT, DERR_BAD_POS = 0x10, 0x20, 0x40
+
+EXPORTS = ["kvq_chunk_bytes", "kvq_status_string", "kvq_append", "kvq_build_pages", "kvq_page_scores",
+           "kvq_select_topk", "kvq_workspace_size", "kvq_sparse_decode_attn", "kvq_dequant_page"]
+
+
+class KvqCache(ctypes.Structure):
+    _fields_ = [("B", c_int32), ("Hq", c_int32), ("Hkv", c_int32), ("D", c_int32),
+                ("page_size", c_int32), ("max_pages", c_int32), ("dtype", c_int32), ("reserved", c_int32),
+                ("block_table", c_void_p), ("seq_len", c_void_p), ("pool", c_void_p * 5),
+                ("pool_slots", c_int64 * 5), ("summary", c_void_p), ("open_ksum", c_void_p),
+                ("err_word", c_void_p)]
+
+
+class SelectParams(ctypes.Structure):
+    _fields_ = [("k_abs", c_int32), ("k_frac_bp", c_int32), ("n_sink", c_int32), ("n_recent", c_int32)]
+
+
+_P = POINTER(KvqCache)
+_lib.kvq_chunk_bytes.argtypes, _lib.kvq_chunk_bytes.restype = [c_int32, c_int32], c_size_t
+_lib.kvq_status_string.argtypes, _lib.kvq_status_string.restype = [c_int32], c_char_p
+_lib.kvq_append.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p]
+_lib.kvq_build_pages.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_int64, c_void_p]
+_lib.kvq_page_scores.argtypes = [_P, c_void_p, c_void_p, c_void_p]
+_lib.kvq_select_topk.argtypes = [_P, c_void_p, POINTER(SelectParams), c_void_p, c_void_p, c_int32, c_void_p]
+_lib.kvq_workspace_size.argtypes = [_P, c_int32, POINTER(c_size_t)]
+_lib.kvq_sparse_decode_attn.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_int32, c_float, c_void_p,
+                                        c_void_p, c_void_p, c_size_t, c_void_p]
+_lib.kvq_dequant_page.argtypes = [_P, c_int32, c_int32, c_void_p, c_void_p]
+for _f in EXPORTS[2:]:
+    getattr(_lib, _f).restype = c_int32
+
+
+class KvqError(RuntimeError):
+    pass
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise KvqError(f"{what}: {_lib.kvq_status_string(st).decode()} ({st})")
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    return int(getattr(stream, "cuda_stream", stream))
+
+
+def kvq_chunk_bytes(tier: int, D: int) -> int:
+    return int(_lib.kvq_chunk_bytes(tier, D))
+
+
+def kvq_status_string(st: int) -> str:
+    return _lib.kvq_status_string(st).decode()
+
+
+def kvq_append(cache, pos, k_new, v_new, stream=None):
+    _check(_lib.kvq_append(cache.ref(), _ptr(pos), _ptr(k_new), _ptr(v_new), _stream(stream)), "kvq_append")
+
+
+def kvq_build_pages(cache, k_src, v_src, cu_seqlens, stream=None):
+    _check(_lib.kvq_build_pages(cache.ref(), _ptr(k_src), _ptr(v_src), _ptr(cu_seqlens), int(k_src.shape[1]),
+                                _stream(stream)), "kvq_build_pages")
+
+
+def kvq_page_scores(cache, q, scores, stream=None):
+    _check(_lib.kvq_page_scores(cache.ref(), _ptr(q), _ptr(scores), _stream(stream)), "kvq_page_scores")
+
+
+def kvq_select_topk(cache, scores, params: SelectParams, sel, cnt, kmax: int, stream=None):
+    _check(_lib.kvq_select_topk(cache.ref(), _ptr(scores), ctypes.byref(params), _ptr(sel), _ptr(cnt), kmax,
+                                _stream(stream)), "kvq_select_topk")
+
+
+def kvq_workspace_size(cache, kmax: int) -> int:
+    n = c_size_t(0)
+    _check(_lib.kvq_workspace_size(cache.ref(), kmax, ctypes.byref(n)), "kvq_workspace_size")
+    return int(n.value)
+
+
+def kvq_sparse_decode_attn(cache, q, sel, cnt, kmax: int, sm_scale: float, out, lse, workspace, stream=None):
+    _check(_lib.kvq_sparse_decode_attn(cache.ref(), _ptr(q), _ptr(sel), _ptr(cnt), kmax, sm_scale, _ptr(out),
+                                       _ptr(lse), _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                                       _stream(stream)), "kvq_sparse_decode_attn")
+
+
+def kvq_dequant_page(cache, b: int, page: int, out, stream=None):
+    _check(_lib.kvq_dequant_page(cache.ref(), b, page, _ptr(out), _stream(stream)), "kvq_dequant_page")
+
+
+# ------------------------------------------------------------------------- allocation
+def encode_block_table(tier_tbl: np.ndarray, slot_tbl: np.ndarray) -> np.ndarray:
+    """(tier << 29) | slot as int32; unused entries (tier < 0) get an invalid tier (7)."""
+    t = np.where(tier_tbl < 0, 7, tier_tbl).astype(np.int64)
+    s = np.where(slot_tbl < 0, 0, slot_tbl).astype(np.int64)
+    return ((t << 29) | s).astype(np.uint32).view(np.int32)
+
+
+class PagedCache:
+    """Device tensors of a paged cache plus the ``kvq_cache`` struct pointing at them."""
+
+    def __init__(self, B, Hq, Hkv, D, max_pages, dtype: str, pool_slots, device="cuda"):
+        import torch
+        self.B, self.Hq, self.Hkv, self.D, self.max_pages = B, Hq, Hkv, D, max_pages
+        self.dtype = dtype
+        self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float16
+        dev = torch.device(device)
+        self.device = dev
+        self.block_table = torch.full((B, max_pages), -1, dtype=torch.int32, device=dev)
+        self.seq_len = torch.zeros(B, dtype=torch.int32, device=dev)
+        self.pool_slots = [int(x) for x in pool_slots]
+        self.pools = []
+        for tier, n in enumerate(self.pool_slots):
+            if n > 0:
+                nbytes = n * Hkv * 2 * kvq_chunk_bytes(tier, D)
+                self.pools.append(torch.zeros(nbytes, dtype=torch.uint8, device=dev))
+            else:
+                self.pools.append(None)
+        self.summary = torch.zeros((B, Hkv, max_pages, D), dtype=torch.float16, device=dev)
+        self.open_ksum = torch.zeros((B, Hkv, D), dtype=torch.float64, device=dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self._s = KvqCache()
+        s = self._s
+        s.B, s.Hq, s.Hkv, s.D, s.page_size, s.max_pages = B, Hq, Hkv, D, 16, max_pages
+        s.dtype = DT_BF16 if dtype == "bf16" else DT_F16
+        s.block_table, s.seq_len = _ptr(self.block_table), _ptr(self.seq_len)
+        for i in range(5):
+            s.pool[i] = _ptr(self.pools[i]) if self.pools[i] is not None else None
+            s.pool_slots[i] = self.pool_slots[i]
+        s.summary, s.open_ksum, s.err_word = _ptr(self.summary), _ptr(self.open_ksum), _ptr(self.err)
+
+    def ref(self):
+        return ctypes.byref(self._s)
+
+    def err_bits(self) -> int:
+        return int(self.err.item()) & 0xFFFFFFFF
+
+    def pool_bytes(self) -> int:
+        return sum(p.numel() for p in self.pools if p is not None)
+
+    def chunk_view(self, b: int, page: int, g: int, kind: int):
+        """Bytes (uint8 tensor view) of one chunk of logical page ``page`` (host-side lookup)."""
+        e = int(self.block_table[b, page].item()) & 0xFFFFFFFF
+        tier, slot = e >> 29, e & 0x1FFFFFFF
+        cb = kvq_chunk_bytes(tier, self.D)
+        o = ((slot * self.Hkv + g) * 2 + kind) * cb
+        return tier, self.pools[tier][o:o + cb]
+
+
+def cache_from_workload(w, device="cuda", threads: int = 8):
+    """Allocate a cache for workload ``w`` and store its prefilled context with kvq_build_pages.
+
+    After the call ``seq_len`` holds the prefilled lengths (before the step's append).
+    """
+    import torch
+    from concurrent.futures import ThreadPoolExecutor
+    tier_tbl, slot_tbl, counts = w.slot_map()
+    cache = PagedCache(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.dtype, counts, device)
+    cache.block_table.copy_(torch.from_numpy(encode_block_table(tier_tbl, slot_tbl)))
+    lens = np.asarray(w.lens, dtype=np.int64)
+    cache.seq_len.copy_(torch.from_numpy(lens.astype(np.int32)))
+    cu = np.zeros(w.B + 1, dtype=np.int64)
+    cu[1:] = np.cumsum(lens)
+    total = int(cu[-1])
+    ksrc = torch.empty((w.Hkv, max(total, 1), w.D), dtype=torch.int16, device=device)
+    vsrc = torch.empty_like(ksrc)
+    pairs = [(b, g) for b in range(w.B) for g in range(w.Hkv) if lens[b] > 0]
+
+    def draw(bg):
+        b, g = bg
+        return bg, w.keys_bits(b, g), w.values_bits(b, g)
+
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        for (b, g), kb, vb in ex.map(draw, pairs):
+            s, e = int(cu[b]), int(cu[b + 1])
+            ksrc[g, s:e].copy_(torch.from_numpy(kb.view(np.int16)))
+            vsrc[g, s:e].copy_(torch.from_numpy(vb.view(np.int16)))
+    cu_t = torch.from_numpy(cu).to(device)
+    kvq_build_pages(cache, ksrc, vsrc, cu_t)
+    torch.cuda.synchronize(device)
+    del ksrc, vsrc
+    return cache
+
+
+def select_params(w) -> SelectParams:
+    return SelectParams(w.k_abs, w.k_frac_bp, w.n_sink, w.n_recent)
+
+
+class DecodeStep:
+    """The buffers and calls of one decode step of workload ``w`` on ``cache``.
+
+    ``run()`` enqueues: kvq_append (if the workload appends) -> kvq_page_scores ->
+    kvq_select_topk -> kvq_sparse_decode_attn, all on the current stream.
+    """
+
+    def __init__(self, w, cache: PagedCache, device="cuda"):
+        import torch
+        self.w, self.cache = w, cache
+        dt = cache.tdtype
+        bits = w.query_bits()
+        self.q = torch.from_numpy(bits.view(np.int16)).to(device).view(dt)
+        if w.append:
+            kn, vn = w.new_kv_bits()
+            self.k_new = torch.from_numpy(kn.view(np.int16)).to(device).view(dt)
+            self.v_new = torch.from_numpy(vn.view(np.int16)).to(device).view(dt)
+            self.pos = torch.from_numpy(np.asarray(w.lens, dtype=np.int32)).to(device)
+        self.kmax = w.kmax()
+        self.params = select_params(w)
+        self.scores = torch.empty((w.B, w.Hkv, w.max_pages), dtype=torch.float32, device=device)
+        self.sel = torch.zeros((w.B, w.Hkv, self.kmax), dtype=torch.int32, device=device)
+        self.cnt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device=device)
+        self.out = torch.empty((w.B, w.Hq, w.D), dtype=dt, device=device)
+        self.lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
+        nws = kvq_workspace_size(cache, self.kmax)
+        self.ws = torch.empty((nws + 15) // 16 * 4, dtype=torch.float32, device=device)
+        cache.seq_len.copy_(torch.from_numpy(w.final_lens().astype(np.int32)))
+
+    def append(self):
+        if self.w.append:
+            kvq_append(self.cache, self.pos, self.k_new, self.v_new)
+
+    def scores_(self):
+        kvq_page_scores(self.cache, self.q, self.scores)
+
+    def select(self):
+        kvq_select_topk(self.cache, self.scores, self.params, self.sel, self.cnt, self.kmax)
+
+    def attend(self):
+        kvq_sparse_decode_attn(self.cache, self.q, self.sel, self.cnt, self.kmax, self.w.sm_scale, self.out,
+                               self.lse, self.ws)
+
+    def run(self):
+        self.append()
+        self.scores_()
+        self.select()
+        self.attend()

@@ -1,0 +1,108 @@
+"""Shared helpers for the GPU-vs-oracle parity tests (imported by tests, not collected)."""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import cache as ocache
+from oracle.fp import bits16_to_f64
+from oracle.layout import chunk_bytes
+from oracle.select import kth_margin
+from oracle.step import prepare, step_pair
+
+# Output tolerance for bf16/fp16 attention outputs: max |gpu - oracle| <= 1e-2 and
+# ||gpu - oracle||_2 / ||oracle||_2 <= 5e-3 (checked per (sequence, kv head) group).
+ATOL_MAX = 1e-2
+REL_L2 = 5e-3
+# Selected sets must match wherever the k-th score margin exceeds this (relative).
+MARGIN = 1e-5
+
+
+def pools_to_cpu(cache):
+    return [None if p is None else p.cpu().numpy() for p in cache.pools]
+
+
+def gpu_chunk(pools, bt: np.ndarray, Hkv: int, D: int, b: int, p: int, g: int, kind: int):
+    e = int(bt[b, p]) & 0xFFFFFFFF
+    tier, slot = e >> 29, e & 0x1FFFFFFF
+    cb = chunk_bytes(tier, D)
+    o = ((slot * Hkv + g) * 2 + kind) * cb
+    return tier, pools[tier][o:o + cb]
+
+
+def snapshot(cache):
+    return dict(pools=pools_to_cpu(cache), bt=cache.block_table.cpu().numpy(),
+                summary=cache.summary.cpu().numpy().view(np.uint16),
+                ksum=cache.open_ksum.cpu().numpy())
+
+
+def check_pages(snap, sh, w, b, g, pages):
+    """Chunk bytes of the listed pages, bit for bit."""
+    for p in pages:
+        for kind, kk in ((0, "k"), (1, "v")):
+            tier, got = gpu_chunk(snap["pools"], snap["bt"], w.Hkv, w.D, b, p, g, kind)
+            want = ocache.page_bytes(sh, p, kk)
+            assert tier == int(sh.tiers[p])
+            if not np.array_equal(got, want):
+                bad = np.nonzero(got != want)[0]
+                raise AssertionError(f"b={b} g={g} page={p} kind={kk} tier={tier}: {bad.size} bytes differ, "
+                                     f"first at {bad[:8]}")
+
+
+def check_summary(snap, sh, b, g, P):
+    got = snap["summary"][b, g, :P]
+    want = sh.summary_bits[:P]
+    assert np.array_equal(got, want), f"summary differs at pages {np.nonzero((got != want).any(1))[0][:8]}"
+
+
+def check_scores(gpu_scores: np.ndarray, ref: np.ndarray, q_group: np.ndarray, summary: np.ndarray, P: int):
+    """fp32 scores within the fp32 accumulation bound of the fp64 oracle's."""
+    assert np.all(np.isneginf(gpu_scores[P:]))
+    if P == 0:
+        return
+    mag = (np.abs(summary[:P]) @ np.abs(q_group).T).max(1)
+    err = np.abs(gpu_scores[:P].astype(np.float64) - ref[:P])
+    assert np.all(err <= 2e-6 * mag + 1e-30), f"max score error {err.max()}"
+
+
+def check_selection(gpu_sel: np.ndarray, ref_sel: np.ndarray, scores: np.ndarray, w, P: int) -> bool:
+    """Sets must be equal when the k-th margin is > MARGIN; returns whether they are equal."""
+    same = np.array_equal(np.sort(gpu_sel), ref_sel)
+    if not same:
+        m = kth_margin(scores, P, w.k_abs, w.k_frac_bp, w.n_sink, w.n_recent)
+        assert m <= MARGIN, f"selection differs with margin {m}"
+    assert np.all(np.diff(gpu_sel) > 0), "selection not ascending"
+    return same
+
+
+def out_ulp(ref: np.ndarray, dtype: str) -> np.ndarray:
+    """One unit in the last place of the output dtype at |ref| (normal range)."""
+    mant = 7 if dtype == "bf16" else 10
+    e = np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -14)))
+    return 2.0 ** (e - mant)
+
+
+def check_output(gpu: np.ndarray, ref: np.ndarray, what="", dtype="bf16"):
+    """max |gpu - ref| <= 1e-2 (or one output-dtype ulp where that is larger: a bf16 value
+    of magnitude >= 4 cannot be rounded to within 1e-2), and rel L2 <= 5e-3."""
+    err = np.abs(gpu - ref)
+    rel = np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-30)
+    bound = np.maximum(ATOL_MAX, out_ulp(ref, dtype))
+    assert np.all(err <= bound), f"{what}: max abs err {err.max()} (bound {bound[np.argmax(err - bound)]})"
+    assert rel <= REL_L2, f"{what}: rel L2 {rel}"
+    return float(err.max()), float(rel)
+
+
+def out_to_f64(t, dtype: str) -> np.ndarray:
+    return bits16_to_f64(t.cpu().contiguous().view(__import__("torch").int16).numpy().view(np.uint16), dtype)
+
+
+def query_and_new(w):
+    q = bits16_to_f64(w.query_bits(), w.dtype)
+    kn, vn = w.new_kv_bits() if w.append else (None, None)
+    return q, kn, vn
+
+
+def oracle_step(w, sh, b: int, g: int, q, kn, vn, sel=None):
+    """Run the oracle step on a prepared (b, g) cache (mutates it by the append)."""
+    return step_pair(w, sh, b, g, q[b], None if kn is None else kn[b, g], None if vn is None else vn[b, g],
+                     sel=sel)

@@ -1,0 +1,253 @@
+"""GPU path vs the CPU oracle on reduced workloads (every element compared).
+
+Covers, per workload: stored page bytes after the bulk build (bit-exact), the page
+summaries and open-page key sums (bit-exact), the appended token's page bytes and
+summary (bit-exact), the page scores (fp32 accumulation bound), the selected pages
+(bit-exact where the k-th margin exceeds 1e-5), and the attention outputs (max abs
+<= 1e-2, rel L2 <= 5e-3) and log-sum-exp.  All calls go through the C ABI.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import cache as ocache
+from oracle.step import prepare
+from sparse_mixed_precision_kvq_b200 import workloads as W
+from tests.parity_helpers import (check_output, check_pages, check_scores, check_selection, check_summary,
+                                  oracle_step, out_to_f64, query_and_new, snapshot)
+
+pytestmark = pytest.mark.gpu
+
+ALL_TIERS = {W.TIER_F16: 0.2, W.TIER_I8: 0.2, W.TIER_I4: 0.2, W.TIER_I2: 0.2, W.TIER_I1: 0.2}
+VARIANTS = {
+    "c0": lambda: W.small("c0"),
+    "c0_alltiers_fp16_d64": lambda: W.make("c0", lens=np.array([1000]), append=True, tier_fracs=ALL_TIERS),
+    "c1": lambda: W.small("c1"),
+    "c2": lambda: W.small("c2"),
+    "c3": lambda: W.small("c3"),
+    "c4": lambda: W.small("c4"),
+    "g1_alltiers": lambda: W.make("c1", B=2, Hq=8, Hkv=8, lens=np.array([700, 333]), tier_fracs=ALL_TIERS,
+                                  k_frac_bp=2000),
+    "g2_alltiers": lambda: W.make("c4", B=3, Hq=16, Hkv=8, lens=np.array([513, 64, 2047]), tier_fracs=ALL_TIERS),
+}
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    from sparse_mixed_precision_kvq_b200 import kvq as k
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return k
+
+
+def _run(kvq, w):
+    cache = kvq.cache_from_workload(w)
+    pre = snapshot(cache)
+    step = kvq.DecodeStep(w, cache)
+    step.run()
+    torch.cuda.synchronize()
+    post = snapshot(cache)
+    return cache, step, pre, post
+
+
+@pytest.mark.parametrize("name", list(VARIANTS))
+def test_step_matches_oracle(kvq, name):
+    w = VARIANTS[name]()
+    cache, step, pre, post = _run(kvq, w)
+    assert cache.err_bits() == 0, hex(cache.err_bits())
+    q, kn, vn = query_and_new(w)
+    scores = step.scores.cpu().numpy()
+    sel = step.sel.cpu().numpy()
+    cnt = step.cnt.cpu().numpy()
+    out = out_to_f64(step.out, w.dtype)
+    lse = step.lse.cpu().numpy()
+    n_same = 0
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            sh = prepare(w, b, g)
+            P0 = sh.P
+            check_pages(pre, sh, w, b, g, range(P0))
+            check_summary(pre, sh, b, g, P0)
+            if int(w.lens[b]) % 16:
+                assert np.array_equal(pre["ksum"][b, g], sh.ksum)
+            r = oracle_step(w, sh, b, g, q, kn, vn)
+            P = r["P"]
+            if w.append:
+                pa = int(w.lens[b]) // 16
+                check_pages(post, sh, w, b, g, [pa])
+                check_summary(post, sh, b, g, P)
+                assert np.array_equal(post["ksum"][b, g], sh.ksum)
+            G = w.G
+            check_scores(scores[b, g], r["scores"], q[b, g * G:(g + 1) * G], sh.summary, P)
+            got_sel = sel[b, g, :cnt[b, g]]
+            if check_selection(got_sel, r["sel"], r["scores"], w, P):
+                n_same += 1
+                for i in range(G):
+                    h = g * G + i
+                    check_output(out[b, h], r["out"][i], f"{name} b={b} h={h}", w.dtype)
+                    assert abs(lse[b, h] - r["lse"][i]) <= 1e-3 * max(1.0, abs(r["lse"][i]))
+    assert n_same >= (w.B * w.Hkv + 1) // 2
+
+
+@pytest.mark.parametrize("name", ["c0_alltiers_fp16_d64", "g1_alltiers", "c4"])
+def test_dequant_values_bit_exact(kvq, name):
+    """The values read back from every tier equal the oracle's fp32(c*scale+zero) / +-m / 16-bit."""
+    w = VARIANTS[name]()
+    cache = kvq.cache_from_workload(w)
+    out = torch.empty((w.Hkv, 2, 16, w.D), dtype=torch.float32, device="cuda")
+    for b in range(min(w.B, 2)):
+        shs = [prepare(w, b, g) for g in range(w.Hkv)]
+        P = shs[0].P
+        for p in range(P):
+            kvq.kvq_dequant_page(cache, b, p, out)
+            got = out.cpu().numpy().astype(np.float64)
+            n = min(16, int(w.lens[b]) - 16 * p)
+            for g in range(w.Hkv):
+                s = slice(16 * p, 16 * p + n)
+                assert np.array_equal(got[g, 0, :n], shs[g].khat[s]), (b, p, g)
+                assert np.array_equal(got[g, 1, :n], shs[g].vhat[s]), (b, p, g)
+    assert cache.err_bits() == 0
+
+
+def test_select_isolated_ties_and_nans(kvq):
+    """Given identical fp32 scores (many ties, NaNs), the GPU selection is the oracle's exactly."""
+    from oracle.select import select
+    rng = np.random.default_rng(5)
+    w = W.make("c4", B=16, Hq=8, Hkv=2, lens=rng.integers(0, 1200, 16), append=False)
+    cache = kvq.cache_from_workload(w)
+    P_cap = w.max_pages
+    sc = rng.integers(-4, 5, (w.B, w.Hkv, P_cap)).astype(np.float32)
+    sc[rng.random(sc.shape) < 0.02] = np.nan
+    sc[rng.random(sc.shape) < 0.02] = -0.0
+    for params in [(-1, 800, 1, 4), (5, 0, 0, 0), (-1, 10000, 2, 2), (0, 0, 3, 0), (1000, 0, 1, 1)]:
+        prm = kvq.SelectParams(*params)
+        kmax = P_cap
+        scores = torch.from_numpy(sc).cuda()
+        selt = torch.full((w.B, w.Hkv, kmax), -7, dtype=torch.int32, device="cuda")
+        cntt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+        cache.err.zero_()
+        kvq.kvq_select_topk(cache, scores, prm, selt, cntt, kmax)
+        got_s, got_c = selt.cpu().numpy(), cntt.cpu().numpy()
+        for b in range(w.B):
+            P = (int(w.lens[b]) + 15) // 16
+            for g in range(w.Hkv):
+                want = select(sc[b, g].astype(np.float64), P, *params)
+                assert list(got_s[b, g, :got_c[b, g]]) == list(want), (params, b, g)
+        nan_any = any(np.isnan(sc[b, g, :(int(w.lens[b]) + 15) // 16]).any() for b in range(w.B) for g in range(w.Hkv))
+        assert bool(cache.err_bits() & kvq.DERR_NAN_SCORE) == nan_any
+
+
+def test_select_kmax_truncation_flag(kvq):
+    w = W.small("c1", append=False)
+    cache = kvq.cache_from_workload(w)
+    step = kvq.DecodeStep(w, cache)
+    step.scores_()
+    small = 7
+    sel = torch.zeros((w.B, w.Hkv, small), dtype=torch.int32, device="cuda")
+    cnt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+    kvq.kvq_select_topk(cache, step.scores, step.params, sel, cnt, small)
+    assert int(cnt.max()) == small
+    assert cache.err_bits() & kvq.DERR_KMAX
+
+
+@pytest.mark.parametrize("name", ["c2", "c4", "c0_alltiers_fp16_d64"])
+def test_attention_isolated_random_selection(kvq, name):
+    """Attention over a given (random) page list equals the oracle's over the same list."""
+    w = VARIANTS[name]()
+    cache = kvq.cache_from_workload(w)
+    step = kvq.DecodeStep(w, cache)
+    step.append()
+    rng = np.random.default_rng(11)
+    q, kn, vn = query_and_new(w)
+    lists = {}
+    selh = np.zeros((w.B, w.Hkv, step.kmax), dtype=np.int32)
+    cnth = np.zeros((w.B, w.Hkv), dtype=np.int32)
+    for b in range(w.B):
+        P = w.pages_after(b)
+        for g in range(w.Hkv):
+            n = int(rng.integers(0, min(P, step.kmax) + 1)) if P else 0
+            s = np.sort(rng.choice(P, size=n, replace=False)) if n else np.zeros(0, np.int64)
+            lists[(b, g)] = s
+            selh[b, g, :n] = s
+            cnth[b, g] = n
+    step.sel.copy_(torch.from_numpy(selh))
+    step.cnt.copy_(torch.from_numpy(cnth))
+    step.attend()
+    torch.cuda.synchronize()
+    assert cache.err_bits() == 0
+    out = out_to_f64(step.out, w.dtype)
+    lse = step.lse.cpu().numpy()
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            sh = prepare(w, b, g)
+            r = oracle_step(w, sh, b, g, q, kn, vn, sel=lists[(b, g)])
+            for i in range(w.G):
+                h = g * w.G + i
+                if lists[(b, g)].size == 0:
+                    assert np.all(out[b, h] == 0) and np.isneginf(lse[b, h])
+                else:
+                    check_output(out[b, h], r["out"][i], f"{name} b={b} h={h}", w.dtype)
+
+
+def test_edge_cases_empty_short_and_overlapping(kvq):
+    """Empty sequences, P < k (everything selected), sink/recent overlap, a page-aligned
+    append that opens a page, and a ragged last page."""
+    w = W.make("c4", B=6, Hq=8, Hkv=2, lens=np.array([0, 1, 15, 16, 40, 200]), append=True,
+               n_sink=3, n_recent=3, k_abs=2, tier_fracs=ALL_TIERS)
+    cache, step, pre, post = _run(kvq, w)
+    assert cache.err_bits() == 0
+    q, kn, vn = query_and_new(w)
+    out = out_to_f64(step.out, w.dtype)
+    sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            sh = prepare(w, b, g)
+            r = oracle_step(w, sh, b, g, q, kn, vn)
+            assert list(sel[b, g, :cnt[b, g]]) == list(r["sel"])
+            check_pages(post, sh, w, b, g, range(sh.P))
+            for i in range(w.G):
+                check_output(out[b, g * w.G + i], r["out"][i], f"edge b={b}", w.dtype)
+
+
+def test_empty_selection_gives_zero_output(kvq):
+    w = W.make("c4", B=3, Hq=8, Hkv=2, lens=np.array([0, 35, 0]), append=False)
+    cache, step, pre, post = _run(kvq, w)
+    out = step.out.float().cpu().numpy()
+    lse = step.lse.cpu().numpy()
+    assert np.all(out[0] == 0) and np.all(out[2] == 0)
+    assert np.all(np.isneginf(lse[0])) and np.all(np.isneginf(lse[2]))
+    assert np.all(np.isfinite(lse[1]))
+
+
+def test_bad_block_table_entry_is_flagged_not_fatal(kvq):
+    """A selected page whose block-table entry names a bad tier is skipped and flagged."""
+    w = W.small("c1", append=False)
+    cache, step, pre, post = _run(kvq, w)
+    bt = cache.block_table.clone()
+    p = int(step.sel[0, 0, 3].item())
+    cache.block_table[0, p] = -1          # tier 7: invalid
+    cache.err.zero_()
+    step.attend()
+    torch.cuda.synchronize()
+    assert cache.err_bits() & kvq.DERR_BAD_PAGE
+    assert torch.isfinite(step.out.float()).all()
+    cache.block_table.copy_(bt)
+
+
+def test_fp16_metadata_saturation_flag(kvq):
+    """A token whose group range exceeds fp16 saturates scale/zero like the oracle and is flagged."""
+    w = W.make("c4", B=1, Hq=8, Hkv=2, lens=np.array([20]), append=True,
+               tier_fracs={W.TIER_I4: 1.0})
+    cache = kvq.cache_from_workload(w)
+    step = kvq.DecodeStep(w, cache)
+    big = np.zeros((1, 2, 128), dtype=np.float32)
+    big[0, :, 0], big[0, :, 1] = -3e5, 3e5
+    bits = W.f32_to_bf16_bits(big)
+    step.k_new.copy_(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16))
+    step.append()
+    torch.cuda.synchronize()
+    assert cache.err_bits() & kvq.DERR_FP16_RANGE
+    sh = prepare(w, 0, 0)
+    ocache.append(sh, 20, bits[0, 0], w.new_kv_bits()[1][0, 0])
+    check_pages(snapshot(cache), sh, w, 0, 0, [1])

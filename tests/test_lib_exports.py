@@ -1,0 +1,57 @@
+"""The C-ABI library loads and exports every symbol include/kvq.h declares (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvq.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_mixed_precision_kvq_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_binding_mirrors_the_header():
+    from sparse_mixed_precision_kvq_b200 import kvq
+    assert sorted(kvq.EXPORTS) == _declared()
+    for n in kvq.EXPORTS:
+        assert callable(getattr(kvq, n))
+
+
+def test_host_helpers_without_gpu():
+    from sparse_mixed_precision_kvq_b200 import kvq
+    assert [2 * kvq.kvq_chunk_bytes(t, 128) for t in range(5)] == [8192, 4608, 2560, 1536, 768]
+    assert kvq.kvq_chunk_bytes(5, 128) == 0 and kvq.kvq_chunk_bytes(0, 96) == 0
+    assert kvq.kvq_status_string(0) == "ok" and "workspace" in kvq.kvq_status_string(3)
+
+
+def test_invalid_arguments_rejected_on_host():
+    """Argument checks run before any CUDA call, so they work without a device."""
+    from sparse_mixed_precision_kvq_b200 import kvq
+    c = kvq.KvqCache()
+    c.B, c.Hq, c.Hkv, c.D, c.page_size, c.max_pages, c.dtype = 1, 8, 2, 96, 16, 4, 0
+    st = kvq._lib.kvq_page_scores(ctypes.byref(c), None, None, None)
+    assert st == 2          # D = 96 unsupported
+    c.D = 64
+    st = kvq._lib.kvq_page_scores(ctypes.byref(c), None, None, None)
+    assert st == 1          # null pointers
+    c.Hq = 24               # G = 12 > 8
+    assert kvq._lib.kvq_append(ctypes.byref(c), None, None, None, None) == 2
