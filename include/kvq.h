@@ -200,6 +200,26 @@ kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const i
                                   kvq_stream_t stream);
 
 /*
+ * kvq_sparse_decode_attn_noalloc -- kvq_sparse_decode_attn without a caller workspace.
+ * (The source pages have no counterpart: this is an interface for callers that cannot
+ *  allocate device memory at decode time, e.g. an engine that gave all device memory to
+ *  its own KV page pool, or a plugin with no allocation hook.)
+ *  Same arguments and results as kvq_sparse_decode_attn minus the workspace.  The split-K
+ *  scratch is a static device array of kvq_noalloc_scratch_bytes() (4 MiB) inside the
+ *  library, held by every GPU that loads it until the process exits.  Allocates nothing
+ *  (no cudaMalloc/cudaFree).  Returns KVQ_ERR_WORKSPACE when kvq_workspace_size() for
+ *  this cache exceeds the static size.  The first call on a device looks up the array's
+ *  device address (cudaGetSymbolAddress); make it before any stream capture.  All calls
+ *  share the array: calls whose work overlaps on the GPU race.
+ */
+kvq_status kvq_sparse_decode_attn_noalloc(const kvq_cache* cache, const void* q, const int32_t* sel,
+                                          const int32_t* cnt, int32_t kmax, float sm_scale, void* out,
+                                          float* lse, kvq_stream_t stream);
+
+/* Size in bytes of the static scratch used by kvq_sparse_decode_attn_noalloc. */
+size_t kvq_noalloc_scratch_bytes(void);
+
+/*
  * kvq_dequant_page -- values read back from storage for one logical page (testing aid).
  *  out device [Hkv][2][16][D] fp32: for each kv head, K then V, every token slot: the
  *  16-bit value, fp32(c * scale + zero), or +-m, per the page's tier.

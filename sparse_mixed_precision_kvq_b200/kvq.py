@@ -33,7 +33,8 @@ DERR_BAD_PAGE, DERR_FP16_RANGE, DERR_NAN_SCORE, DERR_KMAX = 0x1, 0x2, 0x4, 0x8
 DERR_NONFINITE, DERR_TIMEOUT, DERR_BAD_POS = 0x10, 0x20, 0x40
 
 EXPORTS = ["kvq_chunk_bytes", "kvq_status_string", "kvq_append", "kvq_build_pages", "kvq_page_scores",
-           "kvq_select_topk", "kvq_workspace_size", "kvq_sparse_decode_attn", "kvq_dequant_page"]
+           "kvq_select_topk", "kvq_workspace_size", "kvq_sparse_decode_attn", "kvq_dequant_page",
+           "kvq_sparse_decode_attn_noalloc", "kvq_noalloc_scratch_bytes"]
 
 
 class KvqCache(ctypes.Structure):
@@ -59,7 +60,10 @@ _lib.kvq_workspace_size.argtypes = [_P, c_int32, POINTER(c_size_t)]
 _lib.kvq_sparse_decode_attn.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_int32, c_float, c_void_p,
                                         c_void_p, c_void_p, c_size_t, c_void_p]
 _lib.kvq_dequant_page.argtypes = [_P, c_int32, c_int32, c_void_p, c_void_p]
-for _f in EXPORTS[2:]:
+_lib.kvq_sparse_decode_attn_noalloc.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_int32, c_float, c_void_p,
+                                                c_void_p, c_void_p]
+_lib.kvq_noalloc_scratch_bytes.argtypes, _lib.kvq_noalloc_scratch_bytes.restype = [], c_size_t
+for _f in EXPORTS[2:9] + ["kvq_sparse_decode_attn_noalloc"]:
     getattr(_lib, _f).restype = c_int32
 
 
@@ -119,6 +123,17 @@ def kvq_sparse_decode_attn(cache, q, sel, cnt, kmax: int, sm_scale: float, out, 
     _check(_lib.kvq_sparse_decode_attn(cache.ref(), _ptr(q), _ptr(sel), _ptr(cnt), kmax, sm_scale, _ptr(out),
                                        _ptr(lse), _ptr(workspace), int(workspace.numel() * workspace.element_size()),
                                        _stream(stream)), "kvq_sparse_decode_attn")
+
+
+def kvq_sparse_decode_attn_noalloc(cache, q, sel, cnt, kmax: int, sm_scale: float, out, lse, stream=None):
+    """kvq_sparse_decode_attn with the library's static device scratch: allocates nothing."""
+    _check(_lib.kvq_sparse_decode_attn_noalloc(cache.ref(), _ptr(q), _ptr(sel), _ptr(cnt), kmax, sm_scale,
+                                               _ptr(out), _ptr(lse), _stream(stream)),
+           "kvq_sparse_decode_attn_noalloc")
+
+
+def kvq_noalloc_scratch_bytes() -> int:
+    return int(_lib.kvq_noalloc_scratch_bytes())
 
 
 def kvq_dequant_page(cache, b: int, page: int, out, stream=None):

@@ -1,0 +1,61 @@
+"""kvq_sparse_decode_attn_noalloc: the attention entry point that allocates nothing.
+
+Callers that cannot allocate device memory at decode time (an engine that gave its device
+memory to its own KV page pool, a plugin without an allocation hook) use this variant; its
+split-K scratch is a static device array inside the library.  This file is collected last
+so that a run stopping at the first failure has run every other test first.
+
+The check: through the C ABI, on two calls in a row (two different workloads, so stale
+scratch from the first call cannot hide a bug in the second), the output and
+log-sum-exp equal those of kvq_sparse_decode_attn with a caller workspace, within the
+output tolerance the parity tests use.
+"""
+import numpy as np
+import pytest
+import torch
+
+from sparse_mixed_precision_kvq_b200 import workloads as W
+from tests.parity_helpers import check_output, out_to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(kvq, w):
+    cache = kvq.cache_from_workload(w)
+    step = kvq.DecodeStep(w, cache)
+    step.run()                                   # reference: caller-provided workspace
+    torch.cuda.synchronize()
+    ref_out, ref_lse = out_to_f64(step.out, w.dtype), step.lse.cpu().numpy()
+    out = torch.full_like(step.out, float("nan"))
+    lse = torch.full_like(step.lse, float("nan"))
+    kvq.kvq_sparse_decode_attn_noalloc(cache, step.q, step.sel, step.cnt, step.kmax, w.sm_scale, out, lse)
+    torch.cuda.synchronize()
+    assert cache.err_bits() == 0
+    got_out, got_lse = out_to_f64(out, w.dtype), lse.cpu().numpy()
+    for b in range(w.B):
+        for h in range(w.Hq):
+            check_output(got_out[b, h], ref_out[b, h], f"noalloc b={b} h={h}", w.dtype)
+    fin = np.isfinite(ref_lse)
+    assert np.array_equal(fin, np.isfinite(got_lse))
+    assert np.allclose(got_lse[fin], ref_lse[fin], rtol=1e-6, atol=1e-6)
+
+
+def test_noalloc_matches_workspace_entry_point_twice():
+    from sparse_mixed_precision_kvq_b200 import kvq
+    assert torch.cuda.is_available()
+    assert kvq.kvq_noalloc_scratch_bytes() == 4 << 20
+    _case(kvq, W.small("c4"))                   # first call: ragged batch, all four tiers, G = 8
+    _case(kvq, W.small("c1"))                   # second call: other shapes, 16-bit pages, G = 4
+
+
+def test_noalloc_rejects_a_batch_beyond_the_static_scratch():
+    from sparse_mixed_precision_kvq_b200 import kvq
+    w = W.make("c4", B=1200, Hq=16, Hkv=2, lens=np.full(1200, 16), append=False)
+    cache = kvq.PagedCache(w.B, w.Hq, w.Hkv, w.D, 2, w.dtype, [w.B * 2, 0, 0, 0, 0])
+    assert kvq.kvq_workspace_size(cache, 2) > kvq.kvq_noalloc_scratch_bytes()
+    q = torch.zeros((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    sel = torch.zeros((w.B, w.Hkv, 2), dtype=torch.int32, device="cuda")
+    cnt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+    out = torch.empty_like(q)
+    with pytest.raises(kvq.KvqError, match="workspace"):
+        kvq.kvq_sparse_decode_attn_noalloc(cache, q, sel, cnt, 2, w.sm_scale, out, None)
