@@ -7,10 +7,11 @@ One step = one decode step of one attention layer for the whole batch, all of it
 libkvq kernels: append the new token (quantise + pack + summary), score every page,
 select top-k + sink + recent pages, sparse split-K attention + log-sum-exp combine.
 
-Timing: W untimed steps, then K steps timed on the device with CUDA events on the
-launching stream (one event between kernels, so per-kernel durations come from the
-same run); L2 is flushed by writing a 512 MiB buffer before every timed step, outside
-the events.  The whole-step time is bracketed by a barrier + synchronize; with N > 1
+Timing: W untimed steps, then K steps replayed from a CUDA graph of the four calls and
+timed on the device with CUDA events on the launching stream around each replay (L2 is
+flushed by writing a 512 MiB buffer before every timed step, outside the events).
+Per-kernel durations come from a second graph of the same step with events between the
+calls, replayed right after the timed loop.  The whole-step time is bracketed by a barrier + synchronize; with N > 1
 (torchrun, one process per GPU, NCCL) every rank runs its own independent batch (weak
 scaling: sequences are independent problems, no collective on the data path) and the
 max time over ranks is used.  Rank 0 prints one JSON line.
@@ -37,7 +38,6 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decode-step attn tokens/s and achieved HBM GB/s (% of roofline), 1×B200"
-FLUSH_BYTES = 512 << 20
 
 DESCR = {
     "c0": "tiny: 1 seq, 8 q / 2 kv heads, D 64, 1024 tokens, fp16, all 16-bit pages, top-8 + page 0 + last page",
@@ -151,11 +151,14 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = W.make(args.config, seed=W.make(args.config).seed + 1000 * rank)
+    over = {} if args.batch is None else dict(B=args.batch)
+    if args.batch is not None and args.config != "c4":
+        over["lens"] = np.resize(W.make(args.config).lens, args.batch)
+    w = W.make(args.config, seed=W.make(args.config).seed + 1000 * rank, **over)
     cache = kvq.cache_from_workload(w, device=dev)
     step = kvq.DecodeStep(w, cache, device=dev)
     tier_tbl, _, _ = w.slot_map()
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
@@ -167,7 +170,40 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     nbytes = algorithmic_bytes(w, sel, cnt, tier_tbl)
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    # The step is replayed from CUDA graphs so the CPU never starves the GPU:
+    #  g_step: the four calls, nothing between them (programmatic launch overlap intact);
+    #  g_prof: the same calls with timing events between them (per-kernel durations).
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        step.run()
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        step.run()
+    pev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
+    g_prof = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_prof):
+        cs = torch.cuda.current_stream()
+        pev[0].record(cs)
+        step.append()
+        pev[1].record(cs)
+        step.scores_()
+        pev[2].record(cs)
+        step.select()
+        pev[3].record(cs)
+        step.attend()
+        pev[4].record(cs)
+    for _ in range(3):
+        flush.fill_(1)
+        g_step.replay()
+        g_prof.replay()
+    torch.cuda.synchronize(dev)
+    assert cache.err_bits() == 0, f"device error bits {cache.err_bits():#x}"
+
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[0])
                           if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local_rank)
     if rank == 0:
@@ -179,23 +215,23 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     t0 = time.time()
     for k in range(K):
         flush.fill_(k & 0xFF)
-        e = ev[k]
-        e[0].record(stream)
-        step.append()
-        e[1].record(stream)
-        step.scores_()
-        e[2].record(stream)
-        step.select()
-        e[3].record(stream)
-        step.attend()
-        e[4].record(stream)
+        e0[k].record(stream)
+        g_step.replay()
+        e1[k].record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     t1 = time.time()
+    # per-kernel durations: the same step with events between the kernels (one step at a time)
+    KP = min(K, 300)
+    per = np.zeros((KP, 4))
+    for k in range(KP):
+        flush.fill_(k & 0xFF)
+        g_prof.replay()
+        torch.cuda.synchronize(dev)
+        per[k] = [pev[i].elapsed_time(pev[i + 1]) for i in range(4)]
     clocks.stop()
-    per = np.array([[ev[k][i].elapsed_time(ev[k][i + 1]) for i in range(4)] for k in range(K)])  # ms
-    step_ms = per.sum(1)
+    step_ms = np.array([e0[k].elapsed_time(e1[k]) for k in range(K)])
     total_ms = float(step_ms.sum())
     if world > 1:
         t = torch.tensor([total_ms], device=dev)
@@ -221,7 +257,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
         if w.append:
             step.k_new.copy_(pin["k"], non_blocking=True)
             step.v_new.copy_(pin["v"], non_blocking=True)
-        step.run()
+        g_step.replay()
         out_h.copy_(step.out, non_blocking=True)
         lse_h.copy_(step.lse, non_blocking=True)
         e_end[k].record(stream)
@@ -233,6 +269,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
         e2e_ms = float(t.item())
     h2d = pin["q"].numel() * 2 + (pin["k"].numel() * 2 * 2 if w.append else 0)
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    del g_prof, g_step
 
     # optional dense reference point: every page selected (c1's dense run)
     dense_ms = None
@@ -265,7 +302,8 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
         "data": "synthetic (seeded; shapes and value laws of the workload; no model weights)",
         "config": {"workload": f"{args.config}: {DESCR[args.config]}", "batch_per_gpu": w.B,
                    "context": int(w.lens.max()), "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
-                   "selected_pages": int(cnt.sum()), "l2": "flushed (512 MiB write) before every timed step",
+                   "selected_pages": int(cnt.sum()),
+                   "l2": f"flushed ({args.flush_mib} MiB write) before every timed step",
                    "parallelism": f"replicas x{world} (independent batches)"},
         "step_hbm": {"bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3) / 1e9,
                      "peak_gbs": peak, "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak,
@@ -277,7 +315,9 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
                      "traffic": None if tr is None else tr["dram_bytes_per_launch"]},
         "e2e": {"value": world * w.B / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
-        "gpu_launches": 5 * K,
+        "gpu_launches": 4 * K,
+        "timing": "step: CUDA-graph replay of the 4 calls timed with events around each replay; "
+                  "kernels_ms: a second graph with events between the calls (no launch overlap)",
         "clocks": clocks.summary(t0, t1),
     }
     if dense_ms is not None:
@@ -298,6 +338,7 @@ def time_dense(w, cache, step, flush, stream, dev, reps=20):
     sel_t = torch.from_numpy(sel).to(dev)
     cnt_t = torch.from_numpy(np.repeat(P[:, None], w.Hkv, 1).astype(np.int32)).to(dev)
     ws = torch.empty(kvq.kvq_workspace_size(cache, kmax) // 4 + 4, dtype=torch.float32, device=dev)
+    kvq.kvq_workspace_init(ws)
     out = torch.empty_like(step.out)
     ts = []
     for r in range(reps + 3):
@@ -379,6 +420,8 @@ def main():
     ap.add_argument("--dense", action="store_true", help="also time attention over every page")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling runs)")
+    ap.add_argument("--flush-mib", type=int, default=512, help="L2 flush buffer (must exceed the 126 MB L2)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

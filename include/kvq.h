@@ -182,6 +182,14 @@ kvq_status kvq_select_topk(const kvq_cache* cache, const float* scores,
 kvq_status kvq_workspace_size(const kvq_cache* cache, int32_t kmax, size_t* bytes);
 
 /*
+ * kvq_workspace_init -- make a newly allocated workspace ready (zeroes its first 24 KiB,
+ * the per-segment arrival counters of the split-K combine; a workspace that is all zero
+ * is ready too).  Enqueued on stream.  Every kvq_sparse_decode_attn call leaves the
+ * counters zero again, so this is needed once per workspace, not per call.
+ */
+kvq_status kvq_workspace_init(void* workspace, size_t ws_bytes, kvq_stream_t stream);
+
+/*
  * kvq_sparse_decode_attn -- attention of each query head over the tokens of its kv
  * head's selected pages (AMASS "What is in the box"; ARGUS "Why It Works": low-bit
  * values are turned back into high precision before attention).
@@ -192,7 +200,9 @@ kvq_status kvq_workspace_size(const kvq_cache* cache, int32_t kmax, size_t* byte
  *            of the selected pages; zeros when a kv head has no selected page.
  *  lse       device [B][Hq] fp32 out (may be NULL): natural-log log-sum-exp of the
  *            scaled logits (-inf when nothing is selected).
- *  workspace device scratch of at least kvq_workspace_size() bytes (split-K partials).
+ *  workspace device scratch of at least kvq_workspace_size() bytes, prepared once with
+ *            kvq_workspace_init (split-K partials; the last CTA of each (b, kv head) merges
+ *            them, counted by arrival counters the call leaves at zero).  B*Hkv < 6144.
  */
 kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const int32_t* sel,
                                   const int32_t* cnt, int32_t kmax, float sm_scale, void* out,
@@ -205,7 +215,7 @@ kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const i
  *  allocate device memory at decode time, e.g. an engine that gave all device memory to
  *  its own KV page pool, or a plugin with no allocation hook.)
  *  Same arguments and results as kvq_sparse_decode_attn minus the workspace.  The split-K
- *  scratch is a static device array of kvq_noalloc_scratch_bytes() (4 MiB) inside the
+ *  scratch is a static device array of kvq_noalloc_scratch_bytes() (8 MiB) inside the
  *  library, held by every GPU that loads it until the process exits.  Allocates nothing
  *  (no cudaMalloc/cudaFree).  Returns KVQ_ERR_WORKSPACE when kvq_workspace_size() for
  *  this cache exceeds the static size.  The first call on a device looks up the array's

@@ -169,11 +169,16 @@ kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const i
   if (q == nullptr || sel == nullptr || cnt == nullptr || out == nullptr || workspace == nullptr || kmax < 1)
     return KVQ_ERR_INVALID_ARG;
   if (!aligned16(workspace) || !(sm_scale > 0.f)) return KVQ_ERR_INVALID_ARG;
-  if ((long long)c.B * c.Hkv + 1 > 8192) return KVQ_ERR_UNSUPPORTED;  // segment offsets live in shared memory
+  if ((long long)c.B * c.Hkv >= kMaxSegments) return KVQ_ERR_UNSUPPORTED;  // offsets live in shared memory
   const int n = attn_num_ctas(current_device());
   if (ws_bytes < attn_workspace_bytes(c, n)) return KVQ_ERR_WORKSPACE;
   return cuda_status(launch_attn(c, q, sel, cnt, kmax, sm_scale, out, lse, workspace, n,
                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_workspace_init(void* workspace, size_t ws_bytes, kvq_stream_t stream) {
+  if (workspace == nullptr || ws_bytes < kCounterBytes || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(workspace, 0, kCounterBytes, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 kvq_status kvq_dequant_page(const kvq_cache* cache, int32_t b, int32_t page, float* out, kvq_stream_t stream) {

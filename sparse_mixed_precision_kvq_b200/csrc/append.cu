@@ -65,6 +65,7 @@ __global__ void __launch_bounds__(128) append_kernel(DevCache c, const int32_t* 
   const int b = bg / c.Hkv, g = bg % c.Hkv;
   const int D = c.D;
   const int tid = threadIdx.x;
+  griddep_wait();
   const int P = pos[b];
   if (P < 0) return;
   if (P >= c.max_pages * kPage) {
@@ -144,6 +145,7 @@ __global__ void __launch_bounds__(128) append_kernel(DevCache c, const int32_t* 
   }
   if (ov) set_err(c.err, KVQ_DERR_FP16_RANGE);
   if (nonfinite) set_err(c.err, KVQ_DERR_NONFINITE);
+  griddep_launch_dependents();
 }
 
 // ----------------------------------------------------------------------------- build
@@ -235,13 +237,10 @@ __global__ void __launch_bounds__(128) build_kernel(DevCache c, const uint16_t* 
 cudaError_t launch_append(const DevCache& c, const int32_t* pos, const void* k_new, const void* v_new,
                           cudaStream_t s) {
   const dim3 grid(c.B * c.Hkv);
-  if (c.dtype == KVQ_DT_BF16)
-    append_kernel<true><<<grid, 128, 0, s>>>(c, pos, static_cast<const uint16_t*>(k_new),
-                                             static_cast<const uint16_t*>(v_new));
-  else
-    append_kernel<false><<<grid, 128, 0, s>>>(c, pos, static_cast<const uint16_t*>(k_new),
-                                              static_cast<const uint16_t*>(v_new));
-  return cudaGetLastError();
+  const uint16_t* kn = static_cast<const uint16_t*>(k_new);
+  const uint16_t* vn = static_cast<const uint16_t*>(v_new);
+  if (c.dtype == KVQ_DT_BF16) return launch_pdl(append_kernel<true>, grid, dim3(128), 0, s, c, pos, kn, vn);
+  return launch_pdl(append_kernel<false>, grid, dim3(128), 0, s, c, pos, kn, vn);
 }
 
 cudaError_t launch_build(const DevCache& c, const void* k_src, const void* v_src, const int64_t* cu,

@@ -7,11 +7,14 @@
 // precision before attention; no low-bit arithmetic enters the softmax.
 //
 // Work split.  The selected pages of all (b, g) are one flat list (segment bg holds
-// cnt[bg] pages); CTA i takes the contiguous slice [i*W, (i+1)*W), W = ceil(total / #CTAs),
-// so every CTA reads the same number of pages whatever the per-sequence lengths are.
-// Inside a CTA each warp takes every 8th page of a slice piece and runs its own copy
-// pipeline: lane 0 issues one bulk copy (cp.async.bulk, TMA engine) per page (K and V
-// chunks are adjacent) into the warp's shared-memory ring, completion on an mbarrier.
+// cnt[bg] pages); every warp of the grid (one CTA per SM, 8 warps each) is an
+// independent worker u that takes the contiguous slice [u*W, (u+1)*W),
+// W = ceil(total / #workers), so every warp reads the same number of pages whatever the
+// per-sequence lengths are.  A warp looks up the chunk addresses of up to 32 upcoming
+// pages at once (one per lane) and runs its own copy pipeline: lane 0 issues one bulk
+// copy (cp.async.bulk, TMA engine) per page (K and V chunks are adjacent) into the
+// warp's shared-memory ring, completion on an mbarrier.  No CTA-wide barrier is needed
+// between the prologue and the end of the CTA's pages.
 //
 // Math per page (16 tokens, the kv head's G <= 8 query heads), warp-level tensor-core
 // mma m16n8k16 with fp32 accumulation:
@@ -27,9 +30,13 @@
 // 16-bit rounding on the way to the output is the final cast.  This is the value of
 // attending fp32(code * scale + zero) up to fp32 rounding.
 //
-// Online softmax in the log2 domain; each CTA merges its warps and writes one
-// (m, l, o) partial per segment piece; combine_kernel merges the pieces of each
-// segment: M = max m_i, L = sum l_i 2^(m_i - M), o = sum o_i 2^(m_i - M) / L.
+// Online softmax in the log2 domain; each warp writes one (m, l, o) partial per segment
+// piece it covered; at the end each CTA merges its warps' partials per segment (one
+// barrier), and the last CTA to finish a segment (an atomic arrival count, reset by that
+// CTA) merges the CTA partials of the segment:
+// M = max m_i, L = sum l_i 2^(m_i - M), o = sum o_i 2^(m_i - M) / L.
+// Launched with programmatic stream serialization: the prologue up to griddepcontrol.wait
+// overlaps the previous kernel's tail.
 #include <math.h>
 
 #include "kvq_internal.cuh"
@@ -39,7 +46,7 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kRing = 16384;  // bytes of page staging per warp
+constexpr int kRing = 24576;  // bytes of page staging per warp (three 16-bit pages at D = 128)
 constexpr int kNBar = 8;      // pages in flight per warp (max)
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded pipeline wait (2 s)
 
@@ -57,8 +64,11 @@ struct AttnArgs {
   const int32_t* cnt;
   int kmax;
   float scale_log2;
-  float* ws_o;   // [slots][G][D]
+  float* wp_o;   // [wslots][G][D]  one partial per (worker warp, segment it touched)
+  float* wp_ml;  // [wslots][G][2]
+  float* ws_o;   // [slots][G][D]   one partial per (CTA, segment it touched)
   float* ws_ml;  // [slots][G][2]
+  unsigned* counters;  // [B*Hkv] CTAs finished per segment (zero between calls)
   int num_ctas;
 };
 
@@ -105,6 +115,12 @@ __device__ inline void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t byt
       : "memory");
 }
 __device__ inline void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// 2^x with the hardware approximation (relative error ~2^-22; -inf -> +0)
+__device__ inline float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 template <bool BF16>
 __device__ inline void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -267,12 +283,16 @@ template <int TIER, int D, bool BF16>
 __device__ __forceinline__ void qk_page(const unsigned char* base, int lane, const WarpState<D>& st, float (&sacc)[4]) {
   constexpr int KS = D / 16, NG = D / 32;
   if constexpr (TIER == KVQ_TIER_16) {
+    float s2[4] = {0.f, 0.f, 0.f, 0.f};  // second chain: halves the dependent-mma latency
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
       const uint4 v = *reinterpret_cast<const uint4*>(base + ((size_t)kk * 32 + lane) * 16);
       const uint32_t a[4] = {v.x, v.y, v.z, v.w};
-      mma16816<BF16>(sacc, a, st.qb[kk][0], st.qb[kk][1]);
+      if (kk & 1) mma16816<BF16>(s2, a, st.qb[kk][0], st.qb[kk][1]);
+      else mma16816<BF16>(sacc, a, st.qb[kk][0], st.qb[kk][1]);
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sacc[i] += s2[i];
   } else {
     LaneWords<TIER, D> lw;
     lw.load(base, lane);
@@ -365,12 +385,12 @@ __device__ __forceinline__ void process_page(const unsigned char* base, int tier
     pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, o));
   }
   const float mn0 = fmaxf(st.m[0], pm0), mn1 = fmaxf(st.m[1], pm1);
-  const float a0 = exp2f(st.m[0] - mn0), a1 = exp2f(st.m[1] - mn1);
+  const float a0 = ex2(st.m[0] - mn0), a1 = ex2(st.m[1] - mn1);
   float p[4];
-  p[0] = exp2f(x[0] - mn0);
-  p[1] = exp2f(x[1] - mn1);
-  p[2] = exp2f(x[2] - mn0);
-  p[3] = exp2f(x[3] - mn1);
+  p[0] = ex2(x[0] - mn0);
+  p[1] = ex2(x[1] - mn1);
+  p[2] = ex2(x[2] - mn0);
+  p[3] = ex2(x[3] - mn1);
   st.l[0] = st.l[0] * a0 + p[0] + p[2];
   st.l[1] = st.l[1] * a1 + p[1] + p[3];
   st.m[0] = mn0;
@@ -436,41 +456,137 @@ __device__ __forceinline__ void begin_segment(const AttnArgs& a, int b, int g, i
   for (int blk = 0; blk < KS; ++blk) st.o[blk][0] = st.o[blk][1] = st.o[blk][2] = st.o[blk][3] = 0.f;
 }
 
-// The sequence of pages a warp consumes: every kWarps-th page of each piece of the CTA slice.
-struct PageIter {
-  int bg, idx, end;
-  __device__ inline void normalize(const int* off, int BH, int c1, int w) {
-    while (bg < BH && idx >= end) {
-      ++bg;
-      if (bg >= BH || off[bg] >= c1) {
-        bg = BH;
-        break;
-      }
-      idx = off[bg] + w;
-      end = min(c1, off[bg + 1]);
-    }
-  }
+// Where one upcoming page lives; lane i of a warp holds the descriptor of the warp's
+// i-th next page, so the dependent loads (page list -> block table) are paid once per
+// 32 pages instead of once per page.
+struct PageDesc {
+  const unsigned char* src;
+  int tier;  // -1: skip
+  int nv;
 };
 
+// Merge partial slots [s0, s1] (stride 1) of segment bg into `dst` slot (when dst >= 0)
+// or into the output (dst < 0), with all threads of the CTA.  Loads are issued in
+// batches of 8 so the merge costs a couple of L2 round trips, not one per partial.
 template <int D, bool BF16>
-__global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a) {
+__device__ inline void merge_slots(const AttnArgs& a, uint16_t* out, float* lse, const float* src_o,
+                                   const float* src_ml, int s0, int s1, int bg, float* dst_o, float* dst_ml,
+                                   int dst) {
+  constexpr int NB = 8;
+  const DevCache& c = a.c;
+  const int G = c.G;
+  const int b = bg / c.Hkv, g = bg % c.Hkv;
+  for (int e = threadIdx.x; e < G * D; e += kThreads) {
+    const int h = e / D, d = e % D;
+    float M = -INFINITY;
+    for (int j0 = s0; j0 <= s1; j0 += NB) {
+      float mv[NB];
+#pragma unroll
+      for (int i = 0; i < NB; ++i)
+        mv[i] = (j0 + i <= s1) ? __ldcg(&src_ml[((size_t)(j0 + i) * G + h) * 2]) : -INFINITY;
+#pragma unroll
+      for (int i = 0; i < NB; ++i) M = fmaxf(M, mv[i]);
+    }
+    float o = 0.f, Ls = 0.f;
+    if (M != -INFINITY) {
+      for (int j0 = s0; j0 <= s1; j0 += NB) {
+        float2 ml[NB];
+        float ov[NB];
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+          const bool in = j0 + i <= s1;
+          ml[i] = in ? __ldcg(reinterpret_cast<const float2*>(&src_ml[((size_t)(j0 + i) * G + h) * 2]))
+                     : make_float2(-INFINITY, 0.f);
+          ov[i] = in ? __ldcg(&src_o[((size_t)(j0 + i) * G + h) * D + d]) : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+          const float f = ml[i].x == -INFINITY ? 0.f : exp2f(ml[i].x - M);
+          o += ov[i] * f;
+          Ls += ml[i].y * f;
+        }
+      }
+    }
+    if (dst >= 0) {
+      dst_o[((size_t)dst * G + h) * D + d] = o;
+      if (d == 0) {
+        dst_ml[((size_t)dst * G + h) * 2] = M;
+        dst_ml[((size_t)dst * G + h) * 2 + 1] = Ls;
+      }
+    } else {
+      const float r = Ls > 0.f ? o / Ls : 0.f;
+      const size_t oi = ((size_t)b * c.Hq + (size_t)g * G + h) * D + d;
+      if constexpr (BF16) out[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+      else out[oi] = __half_as_ushort(__float2half_rn(r));
+      if (d == 0 && lse != nullptr)
+        lse[(size_t)b * c.Hq + (size_t)g * G + h] = Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+}
+
+// Write the warp's (m, l, o) for segment bg into warp partial slot `slot`.
+template <int D>
+__device__ inline void write_warp_partial(const AttnArgs& a, WarpState<D>& st, int slot, int lane) {
   constexpr int KS = D / 16;
+  const int G = a.c.G;
+  const int g8 = lane >> 2, q4 = lane & 3;
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    st.l[0] += __shfl_xor_sync(0xffffffffu, st.l[0], o);
+    st.l[1] += __shfl_xor_sync(0xffffffffu, st.l[1], o);
+#pragma unroll
+    for (int gi = 0; gi < D / 32; ++gi) {
+      st.zacc[gi][0] += __shfl_xor_sync(0xffffffffu, st.zacc[gi][0], o);
+      st.zacc[gi][1] += __shfl_xor_sync(0xffffffffu, st.zacc[gi][1], o);
+    }
+  }
+  const int h0 = 2 * q4, h1 = 2 * q4 + 1;
+  float* wo = a.wp_o + (size_t)slot * G * D;
+#pragma unroll
+  for (int blk = 0; blk < KS; ++blk) {
+    const int d0 = 16 * blk + g8, d1 = d0 + 8, gi = blk / 2;
+    if (h0 < G) {
+      wo[h0 * D + d0] = st.o[blk][0] + st.zacc[gi][0];
+      wo[h0 * D + d1] = st.o[blk][2] + st.zacc[gi][0];
+    }
+    if (h1 < G) {
+      wo[h1 * D + d0] = st.o[blk][1] + st.zacc[gi][1];
+      wo[h1 * D + d1] = st.o[blk][3] + st.zacc[gi][1];
+    }
+  }
+  if (g8 == 0) {
+    float* wml = a.wp_ml + (size_t)slot * G * 2;
+    if (h0 < G) { wml[h0 * 2] = st.m[0]; wml[h0 * 2 + 1] = st.l[0]; }
+    if (h1 < G) { wml[h1 * 2] = st.m[1]; wml[h1 * 2 + 1] = st.l[1]; }
+  }
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t* __restrict__ out,
+                                                           float* __restrict__ lse) {
   extern __shared__ __align__(128) unsigned char smem[];
   const DevCache& c = a.c;
   const int G = c.G;
   const int BH = c.B * c.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g8 = lane >> 2, q4 = lane & 3;
+  const int nworkers = a.num_ctas * kWarps;
+  const int u = blockIdx.x * kWarps + warp;
 
   unsigned char* ring = smem + (size_t)warp * kRing;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kWarps * kRing) + warp * kNBar;
   PageMeta* pmeta = reinterpret_cast<PageMeta*>(smem + (size_t)kWarps * kRing + kWarps * kNBar * 8) + warp * kNBar;
-  float* mo = reinterpret_cast<float*>(smem + (size_t)kWarps * kRing + kWarps * kNBar * 8 +
-                                       kWarps * kNBar * sizeof(PageMeta));
-  float* mm = mo + kWarps * kMaxG * D;
-  float* ml = mm + kWarps * kMaxG;
-  int* off = reinterpret_cast<int*>(ml + kWarps * kMaxG);  // [BH + 1]
+  int* off = reinterpret_cast<int*>(smem + (size_t)kWarps * kRing + kWarps * kNBar * 8 +
+                                    kWarps * kNBar * sizeof(PageMeta));  // [BH + 1]
   __shared__ int scan_sh[kWarps + 1];
+
+  if (lane == 0) {
+    for (int i = 0; i < kNBar; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  fence_proxy_async();
+  __syncwarp();
+
+  griddep_wait();  // the page lists and the cache come from earlier kernels
 
   // segment offsets: exclusive prefix sum of the (clamped) selected counts
   {
@@ -505,57 +621,65 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a) {
     __syncthreads();
   }
   const int total = off[BH];
-  const int W = (total + a.num_ctas - 1) / a.num_ctas;
-  const int c0 = blockIdx.x * W;
-  const int c1 = min(total, c0 + W);
-  if (c0 >= c1) return;
-
-  // first segment overlapping [c0, c1)
-  int first = 0;
-  {
-    int lo = 0, hi = BH - 1;  // last bg with off[bg] <= c0
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (off[mid] <= c0) lo = mid; else hi = mid - 1;
+  const int W = (total + nworkers - 1) / nworkers;
+  // segments with nothing selected: zero output, -inf lse (every nworkers-th segment here)
+  for (int bg = u; bg < BH; bg += nworkers) {
+    if (off[bg + 1] != off[bg]) continue;
+    const int b = bg / c.Hkv, g = bg % c.Hkv;
+    for (int e = lane; e < G * D; e += 32) {
+      const int h = e / D, d = e % D;
+      out[((size_t)b * c.Hq + (size_t)g * G + h) * D + d] = 0;
+      if (d == 0 && lse != nullptr) lse[(size_t)b * c.Hq + (size_t)g * G + h] = -INFINITY;
     }
-    first = lo;
-    while (first < BH && off[first + 1] <= c0) ++first;  // skip empty segments
   }
+  const int f0 = min(total, u * W);
+  const int f1 = min(total, f0 + W);
 
-  if (lane == 0) {
-    for (int i = 0; i < kNBar; ++i) mbar_init(smem_u32(&bars[i]), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  fence_proxy_async();
-  __syncwarp();
-
-  // producer state (uniform across the warp)
-  PageIter it{first, max(c0, off[first]) + warp, min(c1, off[first + 1])};
-  it.normalize(off, BH, c1, warp);
-  int issued = 0, consumed = 0;
-  int head = 0, tail = 0;  // monotonic ring byte counters
+  int issued = 0, consumed = 0;  // pages of [f0, f1) issued / consumed
+  int head = 0, tail = 0;        // monotonic ring byte counters
+  int win_base = 0, win_n = 0;   // descriptor window: pages [f0 + win_base, f0 + win_base + win_n)
+  PageDesc my{nullptr, -1, 0};
   bool failed = false;
   const unsigned char* ring_c = ring;
 
-  auto issue_more = [&]() {
-    while (it.bg < BH && issued - consumed < kNBar) {
-      const int bg = it.bg;
+  // lane i: descriptor of page f0 + issued + i (binary search of its segment in off[])
+  auto prefetch = [&]() {
+    win_base = issued;
+    win_n = min(32, (f1 - f0) - issued);
+    my = PageDesc{nullptr, -1, 0};
+    if (lane < win_n) {
+      const int f = f0 + issued + lane;
+      int lo = 0, hi = BH - 1;  // last bg with off[bg] <= f
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= f) lo = mid; else hi = mid - 1;
+      }
+      const int bg = lo;
       const int b = bg / c.Hkv, g = bg % c.Hkv;
-      const int j = it.idx - off[bg];
-      const int p = a.sel[(size_t)bg * a.kmax + j];
-      const int L = c.seq_len[b];
+      const int p = __ldg(&a.sel[(size_t)bg * a.kmax + (f - off[bg])]);
+      const int L = __ldg(&c.seq_len[b]);
       const int P = min((L + kPage - 1) / kPage, c.max_pages);
-      int tier = -1, nv = 0;
-      const unsigned char* src = nullptr;
       if (p >= 0 && p < P) {
+        int tier;
+        const unsigned char* src;
         if (page_chunk(c, b, p, g, tier, src)) {
-          nv = min(kPage, L - p * kPage);
-        } else {
-          tier = -1;
+          my.src = src;
+          my.tier = tier;
+          my.nv = min(kPage, L - p * kPage);
         }
-      } else if (lane == 0) {
+      } else {
         set_err(c.err, KVQ_DERR_BAD_PAGE);
       }
+    }
+  };
+
+  auto issue_more = [&]() {
+    while (issued - consumed < kNBar && issued < f1 - f0) {
+      if (issued == win_base + win_n) prefetch();
+      const int k = issued - win_base;
+      const unsigned long long sp = __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my.src), k);
+      const int tier = __shfl_sync(0xffffffffu, my.tier, k);
+      const int nv = __shfl_sync(0xffffffffu, my.nv, k);
       const int bytes = tier >= 0 ? 2 * c.chunk[tier] : 0;
       int start = head;
       const int pos = head % kRing;
@@ -568,160 +692,108 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a) {
         if (bytes > 0) {
           fence_proxy_async();
           mbar_expect_tx(bar, static_cast<uint32_t>(bytes));
-          bulk_copy_g2s(smem_u32(ring + start % kRing), src, static_cast<uint32_t>(bytes), bar);
+          bulk_copy_g2s(smem_u32(ring + start % kRing), reinterpret_cast<const void*>(sp),
+                        static_cast<uint32_t>(bytes), bar);
         } else {
           mbar_arrive(bar);
         }
       }
       head = start + bytes;
       ++issued;
-      it.idx += kWarps;
-      it.normalize(off, BH, c1, warp);
     }
     __syncwarp();
   };
 
+  issue_more();  // start the copies before anything else
+
   WarpState<D> st;
-  for (int bg = first; bg < BH && off[bg] < c1; ++bg) {
-    const int pb = max(c0, off[bg]), pe = min(c1, off[bg + 1]);
-    if (pe <= pb) continue;
-    const int b = bg / c.Hkv, g = bg % c.Hkv;
-    begin_segment<D, BF16>(a, b, g, lane, st);
-    for (int idx = pb + warp; idx < pe; idx += kWarps) {
-      if (!failed) issue_more();
-      const int slot = consumed % kNBar;
-      const uint32_t parity = (consumed / kNBar) & 1;
-      if (!failed) {
-        const bool ok = mbar_wait_bounded(smem_u32(&bars[slot]), parity);
-        if (__any_sync(0xffffffffu, !ok)) {
-          failed = true;
-          if (lane == 0) set_err(c.err, KVQ_DERR_TIMEOUT);
-        }
-      }
-      if (!failed) {
-        const PageMeta pm = pmeta[slot];
-        if (pm.tier >= 0) process_page<D, BF16>(ring_c + pm.ring_off, pm.tier, pm.nv, lane, a.scale_log2, st);
-        tail = pm.end;  // everything before this page's end is free again
-      }
-      __syncwarp();
-      ++consumed;
+  int cur = -1;  // segment being accumulated
+  int bg = 0;    // segment of page f0 + k: pages are contiguous, so a forward cursor suffices
+  {
+    int lo = 0, hi = BH - 1;  // last segment starting at or before f0
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (off[mid] <= f0) lo = mid; else hi = mid - 1;
     }
-    // warp flush: finish the lane-partial sums and write the warp's state
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      st.l[0] += __shfl_xor_sync(0xffffffffu, st.l[0], o);
-      st.l[1] += __shfl_xor_sync(0xffffffffu, st.l[1], o);
-#pragma unroll
-      for (int gi = 0; gi < D / 32; ++gi) {
-        st.zacc[gi][0] += __shfl_xor_sync(0xffffffffu, st.zacc[gi][0], o);
-        st.zacc[gi][1] += __shfl_xor_sync(0xffffffffu, st.zacc[gi][1], o);
-      }
-    }
-    const int h0 = 2 * q4, h1 = 2 * q4 + 1;
-    float* mow = mo + (size_t)warp * kMaxG * D;
-#pragma unroll
-    for (int blk = 0; blk < KS; ++blk) {
-      const int d0 = 16 * blk + g8, d1 = d0 + 8, gi = blk / 2;
-      if (h0 < G) {
-        mow[h0 * D + d0] = st.o[blk][0] + st.zacc[gi][0];
-        mow[h0 * D + d1] = st.o[blk][2] + st.zacc[gi][0];
-      }
-      if (h1 < G) {
-        mow[h1 * D + d0] = st.o[blk][1] + st.zacc[gi][1];
-        mow[h1 * D + d1] = st.o[blk][3] + st.zacc[gi][1];
-      }
-    }
-    if (g8 == 0) {
-      if (h0 < G) { mm[warp * kMaxG + h0] = st.m[0]; ml[warp * kMaxG + h0] = st.l[0]; }
-      if (h1 < G) { mm[warp * kMaxG + h1] = st.m[1]; ml[warp * kMaxG + h1] = st.l[1]; }
-    }
-    __syncthreads();
-    // CTA merge of the warps -> one partial for (this CTA, bg)
-    const size_t slotp = (size_t)blockIdx.x + bg;
-    for (int e = tid; e < G * D; e += kThreads) {
-      const int h = e / D, d = e % D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mm[w * kMaxG + h]);
-      float o = 0.f, Ls = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float mw = mm[w * kMaxG + h];
-        const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-        o += mo[((size_t)w * kMaxG + h) * D + d] * f;
-        Ls += ml[w * kMaxG + h] * f;
-      }
-      a.ws_o[(slotp * G + h) * D + d] = o;
-      if (d == 0) {
-        a.ws_ml[(slotp * G + h) * 2 + 0] = M;
-        a.ws_ml[(slotp * G + h) * 2 + 1] = Ls;
-      }
-    }
-    __syncthreads();
+    bg = lo;
   }
+  for (int k = 0; k < f1 - f0; ++k) {
+    if (!failed) issue_more();
+    const int slot = consumed % kNBar;
+    const uint32_t parity = (consumed / kNBar) & 1;
+    while (off[bg + 1] <= f0 + k) ++bg;  // skip finished and empty segments
+    if (bg != cur) {
+      if (cur >= 0) write_warp_partial<D>(a, st, u + cur, lane);
+      cur = bg;
+      begin_segment<D, BF16>(a, bg / c.Hkv, bg % c.Hkv, lane, st);
+    }
+    if (!failed) {
+      const bool ok = mbar_wait_bounded(smem_u32(&bars[slot]), parity);
+      if (__any_sync(0xffffffffu, !ok)) {
+        failed = true;
+        if (lane == 0) set_err(c.err, KVQ_DERR_TIMEOUT);
+      }
+    }
+    if (!failed) {
+      const PageMeta pm = pmeta[slot];
+      if (pm.tier >= 0) process_page<D, BF16>(ring_c + pm.ring_off, pm.tier, pm.nv, lane, a.scale_log2, st);
+      tail = pm.end;  // everything before this page's end is free again
+    }
+    __syncwarp();
+    ++consumed;
+  }
+  if (cur >= 0) write_warp_partial<D>(a, st, u + cur, lane);
   // after a timeout, give copies still in flight a bounded chance to land before exit
   if (failed) {
     for (int k = consumed; k < issued; ++k) mbar_wait_bounded(smem_u32(&bars[k % kNBar]), (k / kNBar) & 1);
   }
-}
 
-// ----------------------------------------------------------------------------- combine
-template <bool BF16>
-__global__ void __launch_bounds__(256) combine_kernel(AttnArgs a, uint16_t* __restrict__ out, float* __restrict__ lse) {
-  const DevCache& c = a.c;
-  const int BH = c.B * c.Hkv;
-  const int bg = blockIdx.x;
-  const int b = bg / c.Hkv, g = bg % c.Hkv;
-  const int G = c.G, D = c.D;
-  __shared__ int s_off, s_total;
-  if (threadIdx.x < 32) {  // warp 0: this segment's offset and the grand total
-    int before = 0, tot = 0;
-    for (int i = threadIdx.x; i < BH; i += 32) {
-      const int v = min(max(a.cnt[i], 0), a.kmax);
-      tot += v;
-      if (i < bg) before += v;
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      before += __shfl_xor_sync(0xffffffffu, before, o);
-      tot += __shfl_xor_sync(0xffffffffu, tot, o);
-    }
-    if (threadIdx.x == 0) {
-      s_off = before;
-      s_total = tot;
-    }
-  }
+  // CTA pre-merge: one partial per segment this CTA touched, then the last CTA of each
+  // segment (counted arrivals; no waiting) merges those into the output.
+  __threadfence();
   __syncthreads();
-  const int n = min(max(a.cnt[bg], 0), a.kmax);
-  const int W = (s_total + a.num_ctas - 1) / a.num_ctas;
-  const int first = n > 0 ? s_off / W : 0;
-  const int last = n > 0 ? (s_off + n - 1) / W : -1;
-  for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-    const int h = e / D, d = e % D;
-    float M = -INFINITY;
-    for (int j = first; j <= last; ++j) M = fmaxf(M, a.ws_ml[(((size_t)j + bg) * G + h) * 2]);
-    float o = 0.f, Ls = 0.f;
-    if (M != -INFINITY) {
-      for (int j = first; j <= last; ++j) {
-        const size_t sl = (size_t)j + bg;
-        const float f = exp2f(a.ws_ml[(sl * G + h) * 2] - M);
-        o += a.ws_o[(sl * G + h) * D + d] * f;
-        Ls += a.ws_ml[(sl * G + h) * 2 + 1] * f;
+  const int cw = kWarps * W;  // pages per CTA
+  const int cta0 = min(total, (int)blockIdx.x * cw), cta1 = min(total, cta0 + cw);
+  __shared__ int s_last;
+  if (cta0 < cta1) {
+    int sbg = 0;
+    {
+      int lo = 0, hi = BH - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= cta0) lo = mid; else hi = mid - 1;
       }
+      sbg = lo;
     }
-    const float r = Ls > 0.f ? o / Ls : 0.f;
-    const size_t oi = ((size_t)b * c.Hq + (size_t)g * G + h) * D + d;
-    if constexpr (BF16) out[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
-    else out[oi] = __half_as_ushort(__float2half_rn(r));
-    if (d == 0 && lse != nullptr)
-      lse[(size_t)b * c.Hq + (size_t)g * G + h] = Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
+    for (; sbg < BH && off[sbg] < cta1; ++sbg) {
+      if (off[sbg + 1] <= max(cta0, off[sbg])) continue;  // empty or before the CTA
+      const int u0 = max((int)blockIdx.x * kWarps, off[sbg] / W);
+      const int u1 = min((int)blockIdx.x * kWarps + kWarps - 1, (off[sbg + 1] - 1) / W);
+      merge_slots<D, BF16>(a, out, lse, a.wp_o + (size_t)sbg * G * D, a.wp_ml + (size_t)sbg * G * 2, u0, u1, sbg,
+                           a.ws_o, a.ws_ml, (int)blockIdx.x + sbg);
+      const int n0 = off[sbg] / cw, n1 = (off[sbg + 1] - 1) / cw;
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) {
+        const unsigned old = atomicAdd(&a.counters[sbg], 1u);
+        s_last = old == static_cast<unsigned>(n1 - n0);
+        if (s_last) a.counters[sbg] = 0u;  // every CTA of this segment has arrived: reset for the next call
+      }
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        merge_slots<D, BF16>(a, out, lse, a.ws_o + (size_t)sbg * G * D, a.ws_ml + (size_t)sbg * G * 2, n0, n1, sbg,
+                             nullptr, nullptr, -1);
+      }
+      __syncthreads();
+    }
   }
+  griddep_launch_dependents();
 }
 
 template <int D>
 constexpr size_t attn_smem_fixed() {
-  return (size_t)kWarps * kRing + kWarps * kNBar * 8 + kWarps * kNBar * sizeof(PageMeta) +
-         (size_t)kWarps * kMaxG * D * 4 + 2 * kWarps * kMaxG * 4;
+  return (size_t)kWarps * kRing + kWarps * kNBar * 8 + kWarps * kNBar * sizeof(PageMeta);
 }
 
 template <int D, bool BF16>
@@ -730,11 +802,7 @@ cudaError_t launch_attn_d(const AttnArgs& a, uint16_t* out, float* lse, cudaStre
   const size_t smem = attn_smem_fixed<D>() + (size_t)(BH + 1) * 4;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  attn_kernel<D, BF16><<<a.num_ctas, kThreads, smem, s>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  combine_kernel<BF16><<<BH, 256, 0, s>>>(a, out, lse);
-  return cudaGetLastError();
+  return launch_pdl(attn_kernel<D, BF16>, dim3(a.num_ctas), dim3(kThreads), smem, s, a, out, lse);
 }
 
 }  // namespace
@@ -748,13 +816,15 @@ int attn_num_ctas(int device) {
   return sms;
 }
 
+// Workspace: [kCounterBytes] per-segment arrival counters (zero between calls, at a fixed
+// place so that any later call, whatever its shapes, finds them zero), then the warp
+// partials ([wslots][G][D] o, [wslots][G][2] (m, l); wslots = warps + B*Hkv) and the CTA
+// partials ([slots][G][D], [slots][G][2]; slots = CTAs + B*Hkv).  A warp (CTA) u that
+// covers segment bg writes slot u + bg: unique because ranges are contiguous and ordered.
 size_t attn_workspace_bytes(const DevCache& c, int num_ctas) {
-  const size_t slots = (size_t)num_ctas + (size_t)c.B * c.Hkv;
-  return slots * c.G * ((size_t)c.D + 2) * sizeof(float);
-}
-
-size_t attn_smem_bytes(int D, int BH) {
-  return (D == 128 ? attn_smem_fixed<128>() : attn_smem_fixed<64>()) + (size_t)(BH + 1) * 4;
+  const size_t BH = (size_t)c.B * c.Hkv;
+  const size_t wslots = (size_t)num_ctas * kWarps + BH, slots = (size_t)num_ctas + BH;
+  return kCounterBytes + (wslots + slots) * c.G * ((size_t)c.D + 2) * sizeof(float);
 }
 
 cudaError_t launch_attn(const DevCache& c, const void* q, const int32_t* sel, const int32_t* cnt, int kmax,
@@ -766,8 +836,12 @@ cudaError_t launch_attn(const DevCache& c, const void* q, const int32_t* sel, co
   a.cnt = cnt;
   a.kmax = kmax;
   a.scale_log2 = sm_scale * 1.4426950408889634f;
-  const size_t slots = (size_t)num_ctas + (size_t)c.B * c.Hkv;
-  a.ws_o = static_cast<float*>(ws);
+  const size_t BH = (size_t)c.B * c.Hkv;
+  const size_t wslots = (size_t)num_ctas * kWarps + BH, slots = (size_t)num_ctas + BH;
+  a.counters = static_cast<unsigned*>(ws);
+  a.wp_o = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + kCounterBytes);
+  a.wp_ml = a.wp_o + wslots * c.G * c.D;
+  a.ws_o = a.wp_ml + wslots * c.G * 2;
   a.ws_ml = a.ws_o + slots * c.G * c.D;
   a.num_ctas = num_ctas;
   uint16_t* o = static_cast<uint16_t*>(out);

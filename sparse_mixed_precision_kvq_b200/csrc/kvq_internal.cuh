@@ -15,6 +15,8 @@ constexpr int kPage = 16;       // tokens per page
 constexpr int kGroup = 32;      // channels per quantisation group
 constexpr int kMaxG = 8;        // query heads per kv head handled by one mma N-tile
 constexpr int kNumTiers = 5;
+constexpr int kMaxSegments = 6144;  // B * Hkv limit of the attention kernel (offsets in shared memory)
+constexpr size_t kCounterBytes = kMaxSegments * sizeof(unsigned);  // head of the attention workspace
 
 __host__ __device__ inline int tier_bits(int tier) {
   return tier == 0 ? 16 : tier == 1 ? 8 : tier == 2 ? 4 : tier == 3 ? 2 : 1;
@@ -101,6 +103,29 @@ __device__ inline uint16_t fp16_sat(double v, bool& ov) {
     bits = (bits & 0x8000u) | 0x7BFFu;
   }
   return bits;
+}
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream finishes; it must call
+// griddep_wait() before touching anything that kernel wrote, and calls
+// griddep_launch_dependents() once its own dependents may start launching.
+__device__ inline void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ inline void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 // Launch wrappers (defined in the .cu files).

@@ -12,10 +12,11 @@
 // Host code cannot pass the array's name to a kernel (on the host it is a stand-in, not
 // a device address), so the first call on each device looks its device address up with
 // cudaGetSymbolAddress while that device is current and caches it; make that first
-// call before any stream capture.  Every call shares the array and the split-K partials
-// are fully rewritten before they are read, so nothing needs clearing between calls, but
-// two calls whose work overlaps on the GPU (different streams, or devices sharing a
-// context) race on the scratch.
+// call before any stream capture.  Every call shares the array, which keeps the last
+// call's contents: the split-K partials are fully rewritten before they are read, and the
+// per-segment arrival counters at its head must start at zero -- they are zero when the
+// library loads and every call leaves them zero.  Two calls whose work overlaps on the
+// GPU (different streams) race on the scratch.
 #include <mutex>
 
 #include "kvq_internal.cuh"
@@ -23,7 +24,7 @@
 namespace kvq {
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = 4u << 20;  // 4 MiB
+constexpr size_t kNoAllocScratchBytes = 8u << 20;  // 8 MiB
 
 static __device__ __align__(256) unsigned char g_attn_scratch[kNoAllocScratchBytes];
 

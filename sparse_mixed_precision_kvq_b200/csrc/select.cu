@@ -69,6 +69,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(DevCache c, const f
   const int bg = blockIdx.x;
   const int b = bg / c.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  griddep_wait();
   const int L = c.seq_len[b];
   const int P = min((L + kPage - 1) / kPage, c.max_pages);
   const float* sc = scores + (size_t)bg * c.max_pages;
@@ -98,10 +99,21 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(DevCache c, const f
       for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
       __syncthreads();
       const uint32_t hmask = (shift == 24) ? 0u : (0xFFFFFFFFu << (shift + 8));
-      for (int p = tid; p < P; p += kSelThreads) {
-        const bool forced = p < ns || p >= rs;
-        const uint32_t k = keys[p];
-        if (!forced && (k & hmask) == (prefix & hmask)) atomicAdd(&hist[(k >> shift) & 255u], 1);
+      // warp-aggregated: one shared atomic per distinct bin per warp instruction (most keys
+      // share their top bytes, so plain atomics would serialise on one or two bins)
+      for (int base = warp * 32; base < P; base += kSelThreads) {
+        const int p = base + lane;
+        bool active = false;
+        uint32_t bin = 256u;
+        if (p < P && !(p < ns || p >= rs)) {
+          const uint32_t k = keys[p];
+          if ((k & hmask) == (prefix & hmask)) {
+            active = true;
+            bin = (k >> shift) & 255u;
+          }
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (active && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
       }
       __syncthreads();
       if (warp == 0) {
@@ -172,6 +184,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(DevCache c, const f
     cnt[bg] = min(total, kmax);
     if (total > kmax) set_err(c.err, KVQ_DERR_KMAX);
   }
+  griddep_launch_dependents();
 }
 
 }  // namespace
@@ -183,8 +196,7 @@ cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_sele
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  select_kernel<<<c.B * c.Hkv, kSelThreads, smem, s>>>(c, scores, prm, sel, cnt, kmax);
-  return cudaGetLastError();
+  return launch_pdl(select_kernel, dim3(c.B * c.Hkv), dim3(kSelThreads), smem, s, c, scores, prm, sel, cnt, kmax);
 }
 
 }  // namespace kvq

@@ -34,7 +34,7 @@ DERR_NONFINITE, DERR_TIMEOUT, DERR_BAD_POS = 0x10, 0x20, 0x40
 
 EXPORTS = ["kvq_chunk_bytes", "kvq_status_string", "kvq_append", "kvq_build_pages", "kvq_page_scores",
            "kvq_select_topk", "kvq_workspace_size", "kvq_sparse_decode_attn", "kvq_dequant_page",
-           "kvq_sparse_decode_attn_noalloc", "kvq_noalloc_scratch_bytes"]
+           "kvq_sparse_decode_attn_noalloc", "kvq_noalloc_scratch_bytes", "kvq_workspace_init"]
 
 
 class KvqCache(ctypes.Structure):
@@ -63,7 +63,8 @@ _lib.kvq_dequant_page.argtypes = [_P, c_int32, c_int32, c_void_p, c_void_p]
 _lib.kvq_sparse_decode_attn_noalloc.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_int32, c_float, c_void_p,
                                                 c_void_p, c_void_p]
 _lib.kvq_noalloc_scratch_bytes.argtypes, _lib.kvq_noalloc_scratch_bytes.restype = [], c_size_t
-for _f in EXPORTS[2:9] + ["kvq_sparse_decode_attn_noalloc"]:
+_lib.kvq_workspace_init.argtypes = [c_void_p, c_size_t, c_void_p]
+for _f in EXPORTS[2:9] + ["kvq_sparse_decode_attn_noalloc", "kvq_workspace_init"]:
     getattr(_lib, _f).restype = c_int32
 
 
@@ -117,6 +118,11 @@ def kvq_workspace_size(cache, kmax: int) -> int:
     n = c_size_t(0)
     _check(_lib.kvq_workspace_size(cache.ref(), kmax, ctypes.byref(n)), "kvq_workspace_size")
     return int(n.value)
+
+
+def kvq_workspace_init(workspace, stream=None):
+    _check(_lib.kvq_workspace_init(_ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                                   _stream(stream)), "kvq_workspace_init")
 
 
 def kvq_sparse_decode_attn(cache, q, sel, cnt, kmax: int, sm_scale: float, out, lse, workspace, stream=None):
@@ -265,6 +271,7 @@ class DecodeStep:
         self.lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
         nws = kvq_workspace_size(cache, self.kmax)
         self.ws = torch.empty((nws + 15) // 16 * 4, dtype=torch.float32, device=device)
+        kvq_workspace_init(self.ws)
         cache.seq_len.copy_(torch.from_numpy(w.final_lens().astype(np.int32)))
 
     def append(self):
