@@ -2,13 +2,17 @@
 """Decode-step benchmark: sparse mixed-precision paged decode attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config c1] [--impl kvq|reference]
+                    [--path fused|calls]
 
 One step = one decode step of one attention layer for the whole batch, all of it in
 libkvq kernels: append the new token (quantise + pack + summary), score every page,
 select top-k + sink + recent pages, sparse split-K attention + log-sum-exp combine.
+``--path calls`` (default) runs it as the four calls kvq_append -> kvq_page_scores ->
+kvq_select_topk -> kvq_sparse_decode_attn; ``--path fused`` as the single
+kvq_decode_step launch.
 
-Timing: W untimed steps, then K steps replayed from a CUDA graph of the four calls and
-timed on the device with CUDA events on the launching stream around each replay (L2 is
+Timing: W untimed steps, then K steps replayed from a CUDA graph of the step and timed
+on the device with CUDA events on the launching stream around each replay (L2 is
 flushed by writing a 512 MiB buffer before every timed step, outside the events).
 Per-kernel durations come from a second graph of the same step with events between the
 calls, replayed right after the timed loop.  The whole-step time is bracketed by a barrier + synchronize; with N > 1
@@ -163,38 +167,39 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
 
     for _ in range(args.warmup):
         flush.fill_(1)
-        step.run()
+        step.run_fused() if args.path == "fused" else step.run()
     torch.cuda.synchronize(dev)
     assert cache.err_bits() == 0, f"device error bits {cache.err_bits():#x}"
     sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
     nbytes = algorithmic_bytes(w, sel, cnt, tier_tbl)
 
     K = args.steps
+    fused = args.path == "fused"
+    run_step = step.run_fused if fused else step.run
+    # kernels of one step, in launch order (one callable each)
+    parts = [("decode_step", step.run_fused)] if fused else [
+        ("append", step.append), ("page_scores", step.scores_), ("select_topk", step.select),
+        ("sparse_decode_attn", step.attend)]
     # The step is replayed from CUDA graphs so the CPU never starves the GPU:
-    #  g_step: the four calls, nothing between them (programmatic launch overlap intact);
-    #  g_prof: the same calls with timing events between them (per-kernel durations).
+    #  g_step: the step's launches, nothing between them (programmatic launch overlap intact);
+    #  g_prof: the same launches with timing events between them (per-kernel durations).
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
     with torch.cuda.stream(side):
-        step.run()
+        run_step()
     stream.wait_stream(side)
     torch.cuda.synchronize(dev)
     g_step = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_step):
-        step.run()
-    pev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
+        run_step()
+    pev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(parts) + 1)]
     g_prof = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_prof):
         cs = torch.cuda.current_stream()
         pev[0].record(cs)
-        step.append()
-        pev[1].record(cs)
-        step.scores_()
-        pev[2].record(cs)
-        step.select()
-        pev[3].record(cs)
-        step.attend()
-        pev[4].record(cs)
+        for i, (_, fn) in enumerate(parts):
+            fn()
+            pev[i + 1].record(cs)
     for _ in range(3):
         flush.fill_(1)
         g_step.replay()
@@ -224,12 +229,12 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     t1 = time.time()
     # per-kernel durations: the same step with events between the kernels (one step at a time)
     KP = min(K, 300)
-    per = np.zeros((KP, 4))
+    per = np.zeros((KP, len(parts)))
     for k in range(KP):
         flush.fill_(k & 0xFF)
         g_prof.replay()
         torch.cuda.synchronize(dev)
-        per[k] = [pev[i].elapsed_time(pev[i + 1]) for i in range(4)]
+        per[k] = [pev[i].elapsed_time(pev[i + 1]) for i in range(len(parts))]
     clocks.stop()
     step_ms = np.array([e0[k].elapsed_time(e1[k]) for k in range(K)])
     total_ms = float(step_ms.sum())
@@ -279,14 +284,17 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     if rank != 0:
         return None
     peak, peak_kind = load_peaks()
-    names = ["append", "page_scores", "select_topk", "sparse_decode_attn"]
+    names = [n for n, _ in parts]
     avg = per.mean(0)
     dom = int(np.argmax(avg))
-    dom_bytes = [nbytes["append"], nbytes["score"], nbytes["select"], nbytes["attn"]][dom]
-    achieved = dom_bytes / (avg[dom] * 1e-3) / 1e9
-    files = ["append.cu", "score.cu", "select.cu", "attn.cu"]
-    tr = kernel_traffic(files[dom])
     step_bytes = nbytes["attn"] + nbytes["score"] + nbytes["select"] + nbytes["append"]
+    if fused:
+        dom_bytes, files = step_bytes, ["step.cu"]
+    else:
+        dom_bytes = [nbytes["append"], nbytes["score"], nbytes["select"], nbytes["attn"]][dom]
+        files = ["append.cu", "score.cu", "select.cu", "attn.cu"]
+    achieved = dom_bytes / (avg[dom] * 1e-3) / 1e9
+    tr = kernel_traffic(files[dom])
     line = {
         "metric": METRIC,
         "value": value,
@@ -315,9 +323,11 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
                      "traffic": None if tr is None else tr["dram_bytes_per_launch"]},
         "e2e": {"value": world * w.B / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
-        "gpu_launches": 4 * K,
-        "timing": "step: CUDA-graph replay of the 4 calls timed with events around each replay; "
-                  "kernels_ms: a second graph with events between the calls (no launch overlap)",
+        "gpu_launches": len(parts) * K,
+        "path": "kvq_decode_step (one persistent launch)" if fused else "kvq_append -> kvq_page_scores -> "
+                "kvq_select_topk -> kvq_sparse_decode_attn",
+        "timing": "step: CUDA-graph replay of the step timed with events around each replay; "
+                  "kernels_ms: a second graph with events between the launches (no launch overlap)",
         "clocks": clocks.summary(t0, t1),
     }
     if dense_ms is not None:
@@ -417,6 +427,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default="c1", choices=sorted(DESCR))
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--path", default="calls", choices=["fused", "calls"],
+                    help="one kvq_decode_step launch, or the four separate calls")
     ap.add_argument("--dense", action="store_true", help="also time attention over every page")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

@@ -8,7 +8,8 @@
  *   kvq_page_scores        score every page from its summary;
  *   kvq_select_topk        pick the top pages plus forced sink/recent pages;
  *   kvq_sparse_decode_attn attend only the selected pages (split-K + log-sum-exp combine),
- *                          unpacking and dequantising cold pages in registers.
+ *                          unpacking and dequantising cold pages in registers;
+ *   kvq_decode_step        the four above in one persistent launch (same results).
  *
  * Sources: AMASS "decode-time sparse KV-cache attention for vLLM" (amass-kv 0.1.1),
  * section "What is in the box" (per-page summary -> page score -> small selected working
@@ -182,10 +183,12 @@ kvq_status kvq_select_topk(const kvq_cache* cache, const float* scores,
 kvq_status kvq_workspace_size(const kvq_cache* cache, int32_t kmax, size_t* bytes);
 
 /*
- * kvq_workspace_init -- make a newly allocated workspace ready (zeroes its first 24 KiB,
- * the per-segment arrival counters of the split-K combine; a workspace that is all zero
- * is ready too).  Enqueued on stream.  Every kvq_sparse_decode_attn call leaves the
- * counters zero again, so this is needed once per workspace, not per call.
+ * kvq_workspace_init -- make a newly allocated workspace ready (zeroes its first 64 KiB,
+ * the arrival counters of the split-K combine and of kvq_decode_step's work queue; a
+ * workspace that is all zero is ready too).  Enqueued on stream.  Every
+ * kvq_sparse_decode_attn and kvq_decode_step call leaves the counters zero again, so
+ * this is needed once per workspace, not per call (and again after a call that flagged
+ * KVQ_DERR_TIMEOUT).  One workspace may serve both calls.
  */
 kvq_status kvq_workspace_init(void* workspace, size_t ws_bytes, kvq_stream_t stream);
 
@@ -228,6 +231,35 @@ kvq_status kvq_sparse_decode_attn_noalloc(const kvq_cache* cache, const void* q,
 
 /* Size in bytes of the static scratch used by kvq_sparse_decode_attn_noalloc. */
 size_t kvq_noalloc_scratch_bytes(void);
+
+/* Workspace bytes kvq_decode_step needs for this cache and kmax. */
+kvq_status kvq_step_workspace_size(const kvq_cache* cache, int32_t kmax, size_t* bytes);
+
+/*
+ * kvq_decode_step -- one whole decode step in one launch: kvq_append (when pos is not
+ * NULL), kvq_page_scores, kvq_select_topk and kvq_sparse_decode_attn, with the same
+ * arithmetic and the same results as those four calls made in that order (AMASS "What is
+ * in the box": score every page from its summary, attend only the selected pages; ARGUS
+ * "The One-Minute Explanation" / "Visual Architecture": the new token is written into its
+ * page's tier).  A persistent kernel streams the summaries and then the selected pages,
+ * choosing each (b, kv head)'s pages as soon as all its scores exist.
+ *  pos, k_new, v_new  as kvq_append; pos may be NULL (no append).  seq_len must already
+ *            count the appended token (pos[b] / 16 < ceil(seq_len[b] / 16), else the token
+ *            is not written and KVQ_DERR_BAD_POS is set).
+ *  q, params, sel, cnt, kmax, sm_scale, out, lse  as kvq_select_topk and
+ *            kvq_sparse_decode_attn.
+ *  scores    device [B][Hkv][max_pages] fp32 out: the page scores for p < ceil(seq_len/16)
+ *            (entries past that are not written).
+ *  workspace device scratch of at least kvq_step_workspace_size() bytes, prepared once
+ *            with kvq_workspace_init.
+ *  Returns KVQ_ERR_UNSUPPORTED when B*Hkv > 8184 or the per-CTA tables and selection keys
+ *  (4 * (3B + max_pages) bytes) leave too little shared memory for the page ring.
+ */
+kvq_status kvq_decode_step(const kvq_cache* cache, const int32_t* pos, const void* k_new,
+                           const void* v_new, const void* q, const kvq_select_params* params,
+                           float* scores, int32_t* sel, int32_t* cnt, int32_t kmax, float sm_scale,
+                           void* out, float* lse, void* workspace, size_t ws_bytes,
+                           kvq_stream_t stream);
 
 /*
  * kvq_dequant_page -- values read back from storage for one logical page (testing aid).

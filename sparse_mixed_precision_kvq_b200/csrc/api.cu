@@ -176,6 +176,34 @@ kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const i
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+kvq_status kvq_step_workspace_size(const kvq_cache* cache, int32_t kmax, size_t* bytes) {
+  DevCache c;
+  kvq_status st = to_dev(cache, c);
+  if (st != KVQ_OK) return st;
+  if (bytes == nullptr || kmax < 1) return KVQ_ERR_INVALID_ARG;
+  *bytes = step_workspace_bytes(c, kmax);
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_step(const kvq_cache* cache, const int32_t* pos, const void* k_new, const void* v_new,
+                           const void* q, const kvq_select_params* params, float* scores, int32_t* sel,
+                           int32_t* cnt, int32_t kmax, float sm_scale, void* out, float* lse, void* workspace,
+                           size_t ws_bytes, kvq_stream_t stream) {
+  DevCache c;
+  kvq_status st = to_dev(cache, c);
+  if (st != KVQ_OK) return st;
+  if (q == nullptr || params == nullptr || scores == nullptr || sel == nullptr || cnt == nullptr ||
+      out == nullptr || workspace == nullptr || kmax < 1)
+    return KVQ_ERR_INVALID_ARG;
+  if (pos != nullptr && (k_new == nullptr || v_new == nullptr)) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(workspace) || !aligned16(q) || !(sm_scale > 0.f)) return KVQ_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(c.summary) % 16 != 0) return KVQ_ERR_INVALID_ARG;
+  if (!step_supported(c)) return KVQ_ERR_UNSUPPORTED;
+  if (ws_bytes < step_workspace_bytes(c, kmax)) return KVQ_ERR_WORKSPACE;
+  return cuda_status(launch_step(c, pos, k_new, v_new, q, *params, scores, sel, cnt, kmax, sm_scale, out, lse,
+                                 workspace, attn_num_ctas(current_device()), reinterpret_cast<cudaStream_t>(stream)));
+}
+
 kvq_status kvq_workspace_init(void* workspace, size_t ws_bytes, kvq_stream_t stream) {
   if (workspace == nullptr || ws_bytes < kCounterBytes || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
   return cuda_status(cudaMemsetAsync(workspace, 0, kCounterBytes, reinterpret_cast<cudaStream_t>(stream)));

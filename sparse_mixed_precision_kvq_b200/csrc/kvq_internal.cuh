@@ -16,7 +16,9 @@ constexpr int kGroup = 32;      // channels per quantisation group
 constexpr int kMaxG = 8;        // query heads per kv head handled by one mma N-tile
 constexpr int kNumTiers = 5;
 constexpr int kMaxSegments = 6144;  // B * Hkv limit of the attention kernel (offsets in shared memory)
-constexpr size_t kCounterBytes = kMaxSegments * sizeof(unsigned);  // head of the attention workspace
+// Head of every workspace: counters that must be zero when a call starts (every call
+// leaves them zero); kvq_workspace_init zeroes it once.
+constexpr size_t kCounterBytes = 65536;
 
 __host__ __device__ inline int tier_bits(int tier) {
   return tier == 0 ? 16 : tier == 1 ? 8 : tier == 2 ? 4 : tier == 3 ? 2 : 1;
@@ -140,6 +142,11 @@ size_t attn_workspace_bytes(const DevCache& c, int num_ctas);
 int attn_num_ctas(int device);
 cudaError_t launch_attn(const DevCache& c, const void* q, const int32_t* sel, const int32_t* cnt, int kmax,
                         float sm_scale, void* out, float* lse, void* ws, int num_ctas, cudaStream_t s);
+bool step_supported(const DevCache& c);
+size_t step_workspace_bytes(const DevCache& c, int kmax);
+cudaError_t launch_step(const DevCache& c, const int32_t* pos, const void* k_new, const void* v_new,
+                        const void* q, const kvq_select_params& prm, float* scores, int32_t* sel, int32_t* cnt,
+                        int kmax, float sm_scale, void* out, float* lse, void* ws, int num_ctas, cudaStream_t s);
 cudaError_t launch_dequant(const DevCache& c, int b, int page, float* out, cudaStream_t s);
 
 }  // namespace kvq

@@ -1,0 +1,135 @@
+// Per-group quantiser of one token (warp-collective, IEEE binary64, round-half-even) and
+// the one-warp token append built on it, shared by the append, the page builder and the
+// fused decode step.
+//
+// ARGUS "Virtual Memory for Transformers", "Visual Architecture": INT8 / INT4 / INT2 /
+// 1-bit cold tiers.  Per 32-channel group: zero = fp16(min), scale =
+// fp16((max - min) / (2^b - 1)), code = clamp(rint((x - zero) / scale), 0, 2^b - 1) (0 when
+// scale == 0); 1-bit: sign (x >= 0) and magnitude fp16(sum|x| / 32) summed in channel order.
+// Every step is an IEEE binary64 operation with round-half-even, so the bytes do not depend
+// on the thread mapping.  The per-page mean-key summary (AMASS "What is in the box": a
+// tiny per-page summary) is fp16(S / n) with S the fp64 sum of the page's keys in token
+// order.
+#pragma once
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+struct QOut {
+  uint32_t code;
+  uint32_t meta;  // INT-b: scale | zero << 16 ; 1-bit: magnitude
+};
+
+// Warp-collective: lane j holds channel j of the group.
+__device__ inline QOut quant_group(double x, int tier, bool& ov) {
+  const unsigned full = 0xffffffffu;
+  if (tier == KVQ_TIER_I1) {
+    const uint32_t bit = (x >= 0.0) ? 1u : 0u;
+    const double ax = fabs(x);
+    double s = 0.0;
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) s += __shfl_sync(full, ax, j);
+    const uint16_t m = fp16_sat(s / 32.0, ov);
+    return {bit, m};
+  }
+  double lo = x, hi = x;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    lo = fmin(lo, __shfl_xor_sync(full, lo, o));
+    hi = fmax(hi, __shfl_xor_sync(full, hi, o));
+  }
+  const double qmax = static_cast<double>((1 << tier_bits(tier)) - 1);
+  const uint16_t zb = fp16_sat(lo, ov);
+  const uint16_t sb = fp16_sat((hi - lo) / qmax, ov);
+  const double zero = static_cast<double>(__half2float(__ushort_as_half(zb)));
+  const double scale = static_cast<double>(__half2float(__ushort_as_half(sb)));
+  uint32_t code = 0;
+  if (scale != 0.0) {
+    double c = rint((x - zero) / scale);
+    c = fmin(fmax(c, 0.0), qmax);
+    code = static_cast<uint32_t>(c);
+  }
+  return {code, static_cast<uint32_t>(sb) | (static_cast<uint32_t>(zb) << 16)};
+}
+
+template <bool BF16>
+__device__ inline double to_double(uint16_t v) {
+  return static_cast<double>(bits_to_float<BF16>(v));
+}
+
+// One warp writes token `pos` of sequence b, kv head g: quantises K and V into the
+// page's tier, clears a newly opened page first, and advances the open page's fp64 key
+// sum and its fp16 summary.  `patch` (nullable, D entries) receives the new summary row
+// as well.  Returns false (nothing written) if the page's block-table entry is invalid.
+// The caller has checked 0 <= pos < max_pages * 16.
+template <bool BF16>
+__device__ inline bool append_token_warp(const DevCache& c, int b, int g, int pos, const uint16_t* krow,
+                                         const uint16_t* vrow, int lane, uint16_t* patch) {
+  const int D = c.D;
+  const size_t bg = (size_t)b * c.Hkv + g;
+  const int page = pos / kPage, t = pos % kPage;
+  int tier;
+  const unsigned char* ck;
+  if (!page_chunk(c, b, page, g, tier, ck)) return false;
+  unsigned char* chunk[2] = {const_cast<unsigned char*>(ck), const_cast<unsigned char*>(ck) + c.chunk[tier]};
+  const uint16_t* row[2] = {krow, vrow};
+  bool ov = false, nonfinite = false;
+  for (int d = lane; d < D; d += 32) {  // running key sum of the open page and its summary
+    const double x = to_double<BF16>(krow[d]);
+    double* ks = c.open_ksum + bg * D + d;
+    const double S = (t == 0) ? x : (*ks + x);
+    *ks = S;
+    const uint16_t m = fp16_sat(S / static_cast<double>(t + 1), ov);
+    c.summary[(bg * c.max_pages + page) * D + d] = m;
+    if (patch != nullptr) patch[d] = m;
+  }
+  if (t == 0) {  // a newly opened page starts from zero bytes
+    uint4* p4 = reinterpret_cast<uint4*>(chunk[0]);
+    const int n16 = 2 * c.chunk[tier] / 16;
+    for (int i = lane; i < n16; i += 32) p4[i] = make_uint4(0, 0, 0, 0);
+    __syncwarp();
+  }
+  if (tier == KVQ_TIER_16) {
+#pragma unroll
+    for (int kind = 0; kind < 2; ++kind) {
+      for (int d = lane; d < D; d += 32) {
+        const uint16_t v = row[kind][d];
+        nonfinite |= !isfinite(to_double<BF16>(v));
+        int w, bit;
+        elem_pos(kind, 0, D, t, d, w, bit);
+        reinterpret_cast<uint16_t*>(chunk[kind])[2 * w + (bit >> 4)] = v;
+      }
+    }
+  } else {
+    const int ng = D / kGroup;
+    const int b_bits = tier_bits(tier);
+    const uint32_t cmask = (1u << b_bits) - 1u;
+#pragma unroll
+    for (int kind = 0; kind < 2; ++kind) {
+      unsigned char* meta = chunk[kind] + codes_bytes(tier, D);
+      for (int grp = 0; grp < ng; ++grp) {
+        const int d = grp * kGroup + lane;
+        const double x = to_double<BF16>(row[kind][d]);
+        nonfinite |= !isfinite(x);
+        const QOut q = quant_group(x, tier, ov);
+        int w, bit;
+        elem_pos(kind, tier, D, t, d, w, bit);
+        uint32_t* word = reinterpret_cast<uint32_t*>(chunk[kind]) + w;
+        atomicAnd(word, ~(cmask << bit));  // lanes of one group can share a word
+        atomicOr(word, q.code << bit);
+        if (lane == 0) {
+          if (tier == KVQ_TIER_I1)
+            reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = static_cast<uint16_t>(q.meta);
+          else
+            reinterpret_cast<uint32_t*>(meta)[t * ng + grp] = q.meta;
+        }
+      }
+    }
+  }
+  if (__any_sync(0xffffffffu, ov) && lane == 0) set_err(c.err, KVQ_DERR_FP16_RANGE);
+  if (__any_sync(0xffffffffu, nonfinite) && lane == 0) set_err(c.err, KVQ_DERR_NONFINITE);
+  return true;
+}
+
+}  // namespace kvq

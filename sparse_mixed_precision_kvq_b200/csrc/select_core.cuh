@@ -1,0 +1,367 @@
+// Per-(sequence, kv head) page selection, block-wide, shared by kvq_select_topk and the
+// fused decode step.
+//
+// AMASS "Quickstart" (budget: a fixed fraction of the pages is attended, here rounded
+// up per sequence: k = ceil(P * bp / 10000)); ARGUS "Quickstart" (sink tokens kept) and
+// "The One-Minute Explanation" (recent tokens stay hot): the first n_sink and last
+// n_recent pages are always attended, in addition to the k best other pages.  Ranking:
+// score descending, lower page index first among equal scores, NaN lowest.
+//
+// Scores are mapped to order-preserving 32-bit keys in shared memory.  The chosen
+// candidates are found exactly in two steps.  (1) A 256-bin histogram of the candidates'
+// scores, binned linearly between their minimum and maximum (NaN in a bin of its own,
+// below all others), locates the bin T that holds the k-th largest and how many of T's
+// pages are chosen; the binning is monotone in the score, so every page of a higher bin is
+// chosen and none of a lower one.  (2) The pages of bin T -- a few, for any spread-out
+// score distribution -- are ranked against each other by (key descending, page
+// ascending).  The choice is a bitmap of pages, built 32 pages per warp ballot; one
+// block scan over its words then emits the chosen pages in ascending order.  When bin T
+// holds more than kSelCand pages (heavy ties, or an infinite score range), an MSB-first
+// radix select over the keys (4 passes of 8 bits) finds the threshold key instead.
+// Ties are resolved on the keys; the binning decides nothing by itself.
+#pragma once
+
+#include <math.h>
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+// Order-preserving key of a score (larger score -> larger key); NaN -> 0 and *nan set.
+__device__ inline uint32_t order_key(float f, bool& nan) {
+  if (isnan(f)) {
+    nan = true;
+    return 0u;
+  }
+  if (f == 0.0f) f = 0.0f;  // -0 and +0 rank equal
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The split of P pages: forced pages [0, ns) and [rs, P), nC candidates, kk of them chosen.
+struct SelectSplit {
+  int ns, rs, nC, kk;
+  __host__ __device__ int count(int P) const { return (P - nC) + kk; }
+};
+
+__host__ __device__ inline SelectSplit select_split(int P, const kvq_select_params& prm) {
+  SelectSplit s;
+  s.ns = min(max(prm.n_sink, 0), P);
+  s.rs = max(P - max(prm.n_recent, 0), 0);
+  const int nF = s.ns + (P - s.rs) - max(0, s.ns - s.rs);
+  s.nC = P - nF;
+  const long long kb = prm.k_abs >= 0 ? (long long)prm.k_abs : ((long long)P * prm.k_frac_bp + 9999) / 10000;
+  const long long kb0 = kb < 0 ? 0 : kb;
+  s.kk = static_cast<int>(kb0 < s.nC ? kb0 : s.nC);
+  return s;
+}
+
+constexpr int kSelBins = 256;      // value-linear histogram bins (+1 for NaN)
+constexpr int kSelCand = 1024;     // most pages of the threshold bin ranked directly
+constexpr int kSelCandOff = 288;   // scratch: [0, 257) histogram, then candidates, then the bitmap
+constexpr int kSelBitmapOff = kSelCandOff + 2 * kSelCand;
+constexpr int kSelScratchWords = 4096;  // scratch words: bitmap of up to (4096 - 2336) * 32 pages
+constexpr int kSelMaxPages = (kSelScratchWords - kSelBitmapOff) * 32;
+
+struct SelShared {
+  int hist[256];  // radix fallback
+  int scan[33];
+  float wmin[32], wmax[32];
+  uint32_t prefix;
+  int rem;
+  int ncand;
+};
+
+// Exclusive prefix sum of one int per thread over NT threads; *total receives the sum.
+// `bar` is the block barrier.
+template <int NT, typename Bar>
+__device__ inline int sel_exclusive_scan(int v, SelShared& sh, int* total, int tid, Bar& bar) {
+  constexpr int NW = NT / 32;
+  const int lane = tid & 31, warp = tid >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh.scan[warp] = x;
+  bar();
+  if (warp == 0) {
+    int w = lane < NW ? sh.scan[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < NW) sh.scan[lane] = w;
+  }
+  bar();
+  const int before = (warp ? sh.scan[warp - 1] : 0) + x - v;
+  *total = sh.scan[NW - 1];
+  bar();
+  return before;
+}
+
+// Score of an order key (inverse of order_key; key 0 stands for NaN).
+__device__ inline float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Select among the P keys in shared memory (written, and a barrier passed, by the
+// caller); writes the chosen pages in ascending order to out[0 .. min(n, kmax)) and
+// min(n, kmax) to *cnt_out (thread 0).  Flags KVQ_DERR_KMAX if n > kmax.  `scratch` is
+// kSelScratchWords words of shared memory; P <= kSelMaxPages.
+template <int NT, typename Bar>
+__device__ inline void select_pages(const uint32_t* keys, int P, const kvq_select_params& prm, int32_t* out,
+                                    int32_t* cnt_out, int kmax, uint32_t* err, uint32_t* scratch, SelShared& sh,
+                                    int tid, Bar& bar) {
+  constexpr int NW = NT / 32;
+  constexpr int U = 4;  // words per warp in flight in the page passes
+  const int lane = tid & 31, warp = tid >> 5;
+  const SelectSplit sp = select_split(P, prm);
+  const int ns = sp.ns, rs = sp.rs, nC = sp.nC, kk = sp.kk;
+  const int nwords = (P + 31) / 32;
+  auto is_cand = [&](int p) { return p >= ns && p < rs; };
+  // f(page, valid) over all pages, page = 32 * word + lane, U words per warp at a time
+  auto pages = [&](auto&& f) {
+    for (int w0 = warp; w0 < nwords; w0 += U * NW) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int wd = w0 + u * NW;
+        const int p = 32 * wd + lane;
+        f(wd, p, wd < nwords && p < P);
+      }
+    }
+  };
+
+  // mode 0: no candidate chosen, 1: every candidate, 2: value bins + ranked bin T,
+  // 3: threshold key from the radix select (thr, need)
+  int mode = (kk == 0) ? 0 : (kk == nC ? 1 : 2);
+  int* hist = reinterpret_cast<int*>(scratch);            // [257]: bin 256 = NaN
+  uint32_t* cand = scratch + kSelCandOff;                 // [kSelCand][2] (key, page)
+  uint32_t* chosen = scratch + kSelBitmapOff;             // [nwords] bitmap of chosen pages
+  float smin = 0.f, scale = 0.f;
+  uint32_t thr = 0;
+  int need = 0;
+  auto bin_of = [](uint32_t k, float lo, float sc) -> int {
+    if (k == 0u) return 256;  // NaN
+    const float v = (key_score(k) - lo) * sc;
+    return v >= 255.f ? 255 : (v > 0.f ? static_cast<int>(v) : 0);
+  };
+  if (mode == 2) {
+    // 1) candidates' score range; clear the histogram
+    float lo = INFINITY, hi = -INFINITY;
+    pages([&](int, int p, bool valid) {
+      const uint32_t k = valid ? keys[p] : 0u;
+      if (valid && is_cand(p) && k != 0u) {
+        const float f = key_score(k);
+        lo = fminf(lo, f);
+        hi = fmaxf(hi, f);
+      }
+    });
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) {
+      sh.wmin[warp] = lo;
+      sh.wmax[warp] = hi;
+    }
+    for (int i = tid; i < 257; i += NT) hist[i] = 0;
+    if (tid == 0) sh.ncand = 0;
+    bar();
+    lo = INFINITY;
+    hi = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      lo = fminf(lo, sh.wmin[w]);
+      hi = fmaxf(hi, sh.wmax[w]);
+    }
+    smin = lo;
+    const float range = hi - lo;
+    scale = (range > 0.f && range <= 3.0e38f) ? 256.f / range : 0.f;  // 0: one bin (then the radix select)
+    if (!(scale <= 3.0e38f)) scale = 0.f;
+    // 2) histogram (shared atomics; the bins of a warp's pages are mostly distinct)
+    pages([&](int, int p, bool valid) {
+      if (valid && is_cand(p)) atomicAdd(&hist[bin_of(keys[p], smin, scale)], 1);
+    });
+    bar();
+    // 3) warp 0: bin T holding the kk-th largest (bins in rank order: 255 .. 0, then NaN)
+    if (warp == 0) {
+      int h[8], tot = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        h[i] = hist[255 - (lane * 8 + i)];
+        tot += h[i];
+      }
+      int x = tot;  // inclusive prefix over lanes
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      int cum = x - tot;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (cum < kk && kk <= cum + h[i]) {
+          sh.prefix = static_cast<uint32_t>(255 - (lane * 8 + i));
+          sh.rem = kk - cum;
+        }
+        cum += h[i];
+      }
+      if (lane == 31 && cum < kk) {  // the NaN bin
+        sh.prefix = 256u;
+        sh.rem = kk - cum;
+      }
+    }
+    bar();
+    const int T = static_cast<int>(sh.prefix);
+    const int rem = sh.rem;
+    // 4) the bitmap of pages chosen outright (forced, or a bin above T), and the pages of
+    //    bin T as (key, page) pairs
+    pages([&](int wd, int p, bool valid) {
+      const uint32_t k = valid ? keys[p] : 0u;
+      const bool c = valid && is_cand(p);
+      const int bk = c ? bin_of(k, smin, scale) : -1;
+      const bool take = valid && (!c || (bk != T && bk != 256 && (T == 256 || bk > T)));
+      const bool hit = c && bk == T;
+      const unsigned tm = __ballot_sync(0xffffffffu, take);
+      const unsigned hm = __ballot_sync(0xffffffffu, hit);
+      if (lane == 0 && wd < nwords) chosen[wd] = tm;
+      if (hm) {
+        int first = 0;
+        if (lane == 0) first = atomicAdd(&sh.ncand, __popc(hm));
+        first = __shfl_sync(0xffffffffu, first, 0);
+        if (hit) {
+          const int i = first + __popc(hm & ((1u << lane) - 1u));
+          if (i < kSelCand) {
+            cand[2 * i] = k;
+            cand[2 * i + 1] = static_cast<uint32_t>(p);
+          }
+        }
+      }
+    });
+    bar();
+    const int nc = sh.ncand;
+    if (nc <= kSelCand) {
+      // 5) rank the pages of bin T (key descending, page ascending); the first rem are chosen
+      for (int i = tid; i < nc; i += NT) {
+        const uint32_t ki = cand[2 * i], pi = cand[2 * i + 1];
+        int rank = 0;
+#pragma unroll 4
+        for (int j = 0; j < nc; ++j) {
+          const uint32_t kj = cand[2 * j], pj = cand[2 * j + 1];
+          rank += kj > ki || (kj == ki && pj < pi);
+        }
+        if (rank < rem) atomicOr(&chosen[pi >> 5], 1u << (pi & 31));
+      }
+      bar();
+    } else {
+      // heavy ties: MSB-first radix select over all candidate keys
+      mode = 3;
+      uint32_t prefix = 0;
+      int r = kk;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += NT) sh.hist[i] = 0;
+        bar();
+        const uint32_t hmask = (shift == 24) ? 0u : (0xFFFFFFFFu << (shift + 8));
+        pages([&](int, int p, bool valid) {
+          if (valid && is_cand(p)) {
+            const uint32_t k = keys[p];
+            if ((k & hmask) == (prefix & hmask)) atomicAdd(&sh.hist[(k >> shift) & 255u], 1);
+          }
+        });
+        bar();
+        if (warp == 0) {
+          int h8[8], tot = 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            h8[i] = sh.hist[lane * 8 + i];
+            tot += h8[i];
+          }
+          int suf = tot;  // sum over lanes >= lane
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_down_sync(0xffffffffu, suf, o);
+            if (lane + o < 32) suf += y;
+          }
+          int cum = suf - tot;  // keys in bins above this lane's bins
+#pragma unroll
+          for (int i = 7; i >= 0; --i) {
+            const int nxt = cum + h8[i];
+            if (cum < r && r <= nxt) {
+              sh.prefix = prefix | (static_cast<uint32_t>(lane * 8 + i) << shift);
+              sh.rem = r - cum;
+            }
+            cum = nxt;
+          }
+        }
+        bar();
+        prefix = sh.prefix;
+        r = sh.rem;
+        bar();
+      }
+      thr = prefix;
+      need = r;
+    }
+  }
+  if (mode != 2) {
+    // bitmap of the chosen pages: forced ones, plus every candidate (mode 1), none (mode
+    // 0), or those above the threshold key (mode 3; the keys equal to it come next)
+    pages([&](int wd, int p, bool valid) {
+      const bool c = valid && is_cand(p);
+      const bool take = valid && (!c || mode == 1 || (mode == 3 && keys[p] > thr));
+      const unsigned tm = __ballot_sync(0xffffffffu, take);
+      if (lane == 0 && wd < nwords) chosen[wd] = tm;
+    });
+    bar();
+  }
+  // contiguous words per thread
+  const int WPT = (nwords + NT - 1) / NT;
+  const int w_lo = min(nwords, tid * WPT), w_hi = min(nwords, w_lo + WPT);
+  if (mode == 3) {  // the keys equal to the threshold are taken in page order, `need` of them
+    auto eq_mask = [&](int wd) {
+      unsigned m = 0u;
+      for (int b = 0; b < 32; ++b) {
+        const int p = 32 * wd + b;
+        if (p < P && is_cand(p) && keys[p] == thr) m |= 1u << b;
+      }
+      return m;
+    };
+    int eq = 0;
+    for (int wd = w_lo; wd < w_hi; ++wd) eq += __popc(eq_mask(wd));
+    int tot_eq;
+    int e = sel_exclusive_scan<NT>(eq, sh, &tot_eq, tid, bar);
+    for (int wd = w_lo; wd < w_hi && e < need; ++wd) {
+      unsigned m = eq_mask(wd), add = 0u;
+      while (m && e < need) {
+        const unsigned bit = m & (0u - m);
+        add |= bit;
+        m ^= bit;
+        ++e;
+      }
+      chosen[wd] |= add;
+    }
+    bar();
+  }
+  int nsel = 0;
+  for (int wd = w_lo; wd < w_hi; ++wd) nsel += __popc(chosen[wd]);
+  int total;
+  int off = sel_exclusive_scan<NT>(nsel, sh, &total, tid, bar);
+  for (int wd = w_lo; wd < w_hi; ++wd) {
+    unsigned m = chosen[wd];
+    while (m) {
+      const int b = __ffs(m) - 1;
+      m &= m - 1u;
+      if (off < kmax) out[off] = 32 * wd + b;
+      ++off;
+    }
+  }
+  if (tid == 0) {
+    *cnt_out = min(total, kmax);
+    if (total > kmax) set_err(err, KVQ_DERR_KMAX);
+  }
+}
+
+}  // namespace kvq

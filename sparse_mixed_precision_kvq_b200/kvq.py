@@ -34,7 +34,8 @@ DERR_NONFINITE, DERR_TIMEOUT, DERR_BAD_POS = 0x10, 0x20, 0x40
 
 EXPORTS = ["kvq_chunk_bytes", "kvq_status_string", "kvq_append", "kvq_build_pages", "kvq_page_scores",
            "kvq_select_topk", "kvq_workspace_size", "kvq_sparse_decode_attn", "kvq_dequant_page",
-           "kvq_sparse_decode_attn_noalloc", "kvq_noalloc_scratch_bytes", "kvq_workspace_init"]
+           "kvq_sparse_decode_attn_noalloc", "kvq_noalloc_scratch_bytes", "kvq_workspace_init",
+           "kvq_step_workspace_size", "kvq_decode_step"]
 
 
 class KvqCache(ctypes.Structure):
@@ -64,7 +65,12 @@ _lib.kvq_sparse_decode_attn_noalloc.argtypes = [_P, c_void_p, c_void_p, c_void_p
                                                 c_void_p, c_void_p]
 _lib.kvq_noalloc_scratch_bytes.argtypes, _lib.kvq_noalloc_scratch_bytes.restype = [], c_size_t
 _lib.kvq_workspace_init.argtypes = [c_void_p, c_size_t, c_void_p]
-for _f in EXPORTS[2:9] + ["kvq_sparse_decode_attn_noalloc", "kvq_workspace_init"]:
+_lib.kvq_step_workspace_size.argtypes = [_P, c_int32, POINTER(c_size_t)]
+_lib.kvq_decode_step.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, POINTER(SelectParams), c_void_p,
+                                 c_void_p, c_void_p, c_int32, c_float, c_void_p, c_void_p, c_void_p, c_size_t,
+                                 c_void_p]
+for _f in EXPORTS[2:9] + ["kvq_sparse_decode_attn_noalloc", "kvq_workspace_init", "kvq_step_workspace_size",
+                          "kvq_decode_step"]:
     getattr(_lib, _f).restype = c_int32
 
 
@@ -129,6 +135,21 @@ def kvq_sparse_decode_attn(cache, q, sel, cnt, kmax: int, sm_scale: float, out, 
     _check(_lib.kvq_sparse_decode_attn(cache.ref(), _ptr(q), _ptr(sel), _ptr(cnt), kmax, sm_scale, _ptr(out),
                                        _ptr(lse), _ptr(workspace), int(workspace.numel() * workspace.element_size()),
                                        _stream(stream)), "kvq_sparse_decode_attn")
+
+
+def kvq_step_workspace_size(cache, kmax: int) -> int:
+    n = c_size_t(0)
+    _check(_lib.kvq_step_workspace_size(cache.ref(), kmax, ctypes.byref(n)), "kvq_step_workspace_size")
+    return int(n.value)
+
+
+def kvq_decode_step(cache, pos, k_new, v_new, q, params: SelectParams, scores, sel, cnt, kmax: int,
+                    sm_scale: float, out, lse, workspace, stream=None):
+    """The whole decode step (append if ``pos`` is not None, scores, selection, attention) in one launch."""
+    _check(_lib.kvq_decode_step(cache.ref(), _ptr(pos), _ptr(k_new), _ptr(v_new), _ptr(q), ctypes.byref(params),
+                                _ptr(scores), _ptr(sel), _ptr(cnt), kmax, sm_scale, _ptr(out), _ptr(lse),
+                                _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                                _stream(stream)), "kvq_decode_step")
 
 
 def kvq_sparse_decode_attn_noalloc(cache, q, sel, cnt, kmax: int, sm_scale: float, out, lse, stream=None):
@@ -269,7 +290,7 @@ class DecodeStep:
         self.cnt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device=device)
         self.out = torch.empty((w.B, w.Hq, w.D), dtype=dt, device=device)
         self.lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
-        nws = kvq_workspace_size(cache, self.kmax)
+        nws = max(kvq_workspace_size(cache, self.kmax), kvq_step_workspace_size(cache, self.kmax))
         self.ws = torch.empty((nws + 15) // 16 * 4, dtype=torch.float32, device=device)
         kvq_workspace_init(self.ws)
         cache.seq_len.copy_(torch.from_numpy(w.final_lens().astype(np.int32)))
@@ -293,3 +314,9 @@ class DecodeStep:
         self.scores_()
         self.select()
         self.attend()
+
+    def run_fused(self):
+        """The same step as ``run()`` in one kvq_decode_step launch."""
+        kvq_decode_step(self.cache, self.pos if self.w.append else None, self.k_new if self.w.append else None,
+                        self.v_new if self.w.append else None, self.q, self.params, self.scores, self.sel, self.cnt,
+                        self.kmax, self.w.sm_scale, self.out, self.lse, self.ws)

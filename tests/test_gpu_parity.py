@@ -41,20 +41,25 @@ def kvq():
     return k
 
 
-def _run(kvq, w):
+def _run(kvq, w, fused=False):
     cache = kvq.cache_from_workload(w)
     pre = snapshot(cache)
     step = kvq.DecodeStep(w, cache)
-    step.run()
+    step.run_fused() if fused else step.run()
     torch.cuda.synchronize()
     post = snapshot(cache)
     return cache, step, pre, post
 
 
+PATHS = ["calls", "fused"]
+
+
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("name", list(VARIANTS))
-def test_step_matches_oracle(kvq, name):
+def test_step_matches_oracle(kvq, name, path):
+    """The four calls, and the one-launch kvq_decode_step, against the oracle."""
     w = VARIANTS[name]()
-    cache, step, pre, post = _run(kvq, w)
+    cache, step, pre, post = _run(kvq, w, fused=path == "fused")
     assert cache.err_bits() == 0, hex(cache.err_bits())
     q, kn, vn = query_and_new(w)
     scores = step.scores.cpu().numpy()
@@ -79,7 +84,7 @@ def test_step_matches_oracle(kvq, name):
                 check_summary(post, sh, b, g, P)
                 assert np.array_equal(post["ksum"][b, g], sh.ksum)
             G = w.G
-            check_scores(scores[b, g], r["scores"], q[b, g * G:(g + 1) * G], sh.summary, P)
+            check_scores(scores[b, g], r["scores"], q[b, g * G:(g + 1) * G], sh.summary, P, tail=path == "calls")
             got_sel = sel[b, g, :cnt[b, g]]
             if check_selection(got_sel, r["sel"], r["scores"], w, P):
                 n_same += 1
@@ -190,12 +195,13 @@ def test_attention_isolated_random_selection(kvq, name):
                     check_output(out[b, h], r["out"][i], f"{name} b={b} h={h}", w.dtype)
 
 
-def test_edge_cases_empty_short_and_overlapping(kvq):
+@pytest.mark.parametrize("path", PATHS)
+def test_edge_cases_empty_short_and_overlapping(kvq, path):
     """Empty sequences, P < k (everything selected), sink/recent overlap, a page-aligned
     append that opens a page, and a ragged last page."""
     w = W.make("c4", B=6, Hq=8, Hkv=2, lens=np.array([0, 1, 15, 16, 40, 200]), append=True,
                n_sink=3, n_recent=3, k_abs=2, tier_fracs=ALL_TIERS)
-    cache, step, pre, post = _run(kvq, w)
+    cache, step, pre, post = _run(kvq, w, fused=path == "fused")
     assert cache.err_bits() == 0
     q, kn, vn = query_and_new(w)
     out = out_to_f64(step.out, w.dtype)
@@ -210,9 +216,10 @@ def test_edge_cases_empty_short_and_overlapping(kvq):
                 check_output(out[b, g * w.G + i], r["out"][i], f"edge b={b}", w.dtype)
 
 
-def test_empty_selection_gives_zero_output(kvq):
+@pytest.mark.parametrize("path", PATHS)
+def test_empty_selection_gives_zero_output(kvq, path):
     w = W.make("c4", B=3, Hq=8, Hkv=2, lens=np.array([0, 35, 0]), append=False)
-    cache, step, pre, post = _run(kvq, w)
+    cache, step, pre, post = _run(kvq, w, fused=path == "fused")
     out = step.out.float().cpu().numpy()
     lse = step.lse.cpu().numpy()
     assert np.all(out[0] == 0) and np.all(out[2] == 0)
@@ -251,3 +258,83 @@ def test_fp16_metadata_saturation_flag(kvq):
     sh = prepare(w, 0, 0)
     ocache.append(sh, 20, bits[0, 0], w.new_kv_bits()[1][0, 0])
     check_pages(snapshot(cache), sh, w, 0, 0, [1])
+
+
+@pytest.mark.parametrize("name", ["c2", "c4", "g2_alltiers"])
+def test_fused_step_equals_calls_and_is_deterministic(kvq, name):
+    """kvq_decode_step gives the four calls' scores and pages bit for bit, outputs within
+    the output tolerance, and the same bits on every repeat (the workspace counters are
+    back at zero after each call)."""
+    if name == "g2_alltiers":
+        w_na = W.make("c4", B=3, Hq=16, Hkv=8, lens=np.array([513, 64, 2047]), tier_fracs=ALL_TIERS, append=False)
+    else:
+        w_na = W.small(name, append=False)
+    cache = kvq.cache_from_workload(w_na)
+    step = kvq.DecodeStep(w_na, cache)
+    step.run()
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in (step.scores, step.sel, step.cnt, step.out, step.lse)]
+    outs = []
+    for _ in range(3):
+        step.scores.fill_(7.0)
+        step.sel.fill_(-3)
+        step.out.zero_()
+        step.run_fused()
+        torch.cuda.synchronize()
+        outs.append(step.out.clone())
+        cnt = step.cnt.cpu().numpy()
+        assert torch.equal(step.cnt, ref[2])
+        for b in range(w_na.B):
+            P = (int(w_na.lens[b]) + 15) // 16
+            for g in range(w_na.Hkv):
+                assert torch.equal(step.scores[b, g, :P], ref[0][b, g, :P]), (b, g)
+                assert torch.equal(step.sel[b, g, :cnt[b, g]], ref[1][b, g, :cnt[b, g]]), (b, g)
+        check_output(out_to_f64(step.out, w_na.dtype), out_to_f64(ref[3], w_na.dtype), name, w_na.dtype)
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+    assert cache.err_bits() == 0
+
+
+def test_fused_step_kmax_truncation_flag(kvq):
+    w = W.small("c1", append=False)
+    cache = kvq.cache_from_workload(w)
+    step = kvq.DecodeStep(w, cache)
+    small = 7
+    sel = torch.zeros((w.B, w.Hkv, small), dtype=torch.int32, device="cuda")
+    ws = torch.zeros(kvq.kvq_step_workspace_size(cache, small) // 4 + 4, dtype=torch.float32, device="cuda")
+    kvq.kvq_decode_step(cache, None, None, None, step.q, step.params, step.scores, sel, step.cnt, small,
+                        w.sm_scale, step.out, step.lse, ws)
+    torch.cuda.synchronize()
+    assert int(step.cnt.max()) == small
+    assert cache.err_bits() & kvq.DERR_KMAX
+    assert torch.isfinite(step.out.float()).all()
+
+
+def test_select_special_values_and_wide_ranges(kvq):
+    """Infinite scores, a range near the fp32 limit, all-equal scores, denormals and a
+    large random batch: the selection is the oracle's exactly (ties on page index)."""
+    from oracle.select import select
+    rng = np.random.default_rng(7)
+    B, Hkv, P_cap = 12, 2, 3000
+    w = W.make("c4", B=B, Hq=8, Hkv=Hkv, lens=np.full(B, 16 * P_cap), append=False)
+    cache = kvq.cache_from_workload(w)
+    sc = rng.normal(0, 3, (B, Hkv, w.max_pages)).astype(np.float32)
+    sc[0, 0, rng.integers(0, P_cap, 20)] = np.inf
+    sc[0, 1, rng.integers(0, P_cap, 20)] = -np.inf
+    sc[1, 0] = rng.choice([-3e38, 3e38, 1.0, -1.0], w.max_pages).astype(np.float32)
+    sc[1, 1] = 2.5
+    sc[2, 0] = (rng.integers(-3, 4, w.max_pages) * 1e-42).astype(np.float32)   # denormals and zeros
+    sc[2, 1] = rng.integers(0, 3, w.max_pages).astype(np.float32)              # three values only
+    sc[3, 0, ::7] = np.nan
+    for params in [(-1, 500, 1, 4), (-1, 9000, 0, 0), (37, 0, 2, 3)]:
+        prm = kvq.SelectParams(*params)
+        kmax = w.max_pages
+        scores = torch.from_numpy(sc).cuda()
+        selt = torch.full((B, Hkv, kmax), -7, dtype=torch.int32, device="cuda")
+        cntt = torch.zeros((B, Hkv), dtype=torch.int32, device="cuda")
+        kvq.kvq_select_topk(cache, scores, prm, selt, cntt, kmax)
+        got_s, got_c = selt.cpu().numpy(), cntt.cpu().numpy()
+        P = (int(w.lens[0]) + 15) // 16
+        for b in range(B):
+            for g in range(Hkv):
+                want = select(sc[b, g].astype(np.float64), P, *params)
+                assert list(got_s[b, g, :got_c[b, g]]) == list(want), (params, b, g)
