@@ -147,7 +147,7 @@ kvq_status kvq_select_topk(const kvq_cache* cache, const float* scores, const kv
   if (st != KVQ_OK) return st;
   if (scores == nullptr || params == nullptr || sel == nullptr || cnt == nullptr || kmax < 1)
     return KVQ_ERR_INVALID_ARG;
-  if ((size_t)c.max_pages * 4 > 200 * 1024) return KVQ_ERR_UNSUPPORTED;
+  if ((size_t)c.max_pages * 4 > 200 * 1024) return KVQ_ERR_UNSUPPORTED;  // keys in shared memory
   return cuda_status(launch_select(c, scores, *params, sel, cnt, kmax, reinterpret_cast<cudaStream_t>(stream)));
 }
 

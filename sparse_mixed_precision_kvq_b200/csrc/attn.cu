@@ -85,59 +85,116 @@ struct PageDesc {
 // Merge partial slots [s0, s1] (stride 1) of segment bg into `dst` slot (when dst >= 0)
 // or into the output (dst < 0), with all threads of the CTA.  Loads are issued in
 // batches of 8 so the merge costs a couple of L2 round trips, not one per partial.
-template <int D, bool BF16>
-__device__ inline void merge_slots(const AttnArgs& a, uint16_t* out, float* lse, const float* src_o,
-                                   const float* src_ml, int s0, int s1, int bg, float* dst_o, float* dst_ml,
-                                   int dst) {
-  constexpr int NB = 8;
+// Write the merged (M, L, o) of element (h, d) of segment bg: as a partial into slot `dst`
+// of (dst_o, dst_ml), or, with dst < 0, as the segment's output o / L and lse.
+template <bool BF16>
+__device__ inline void put_merged(const AttnArgs& a, uint16_t* out, float* lse, int bg, int h, int d, int D, float M,
+                                  float Ls, float o, float* dst_o, float* dst_ml, int dst) {
   const DevCache& c = a.c;
   const int G = c.G;
+  if (dst >= 0) {
+    dst_o[((size_t)dst * G + h) * D + d] = o;
+    if (d == 0) {
+      dst_ml[((size_t)dst * G + h) * 2] = M;
+      dst_ml[((size_t)dst * G + h) * 2 + 1] = Ls;
+    }
+    return;
+  }
   const int b = bg / c.Hkv, g = bg % c.Hkv;
+  const float r = Ls > 0.f ? o / Ls : 0.f;
+  const size_t oi = ((size_t)b * c.Hq + (size_t)g * G + h) * D + d;
+  if constexpr (BF16) out[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+  else out[oi] = __half_as_ushort(__float2half_rn(r));
+  if (d == 0 && lse != nullptr)
+    lse[(size_t)b * c.Hq + (size_t)g * G + h] = Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
+}
+
+// CTA merge of segment bg: warps w0..w1 of this CTA hold one partial each, in their own
+// ring (shared memory: the warp's last segment) or in their global warp slot (u + bg).
+// All of an element's partials are loaded before any is used: one memory round trip.
+template <int D, bool BF16>
+__device__ inline void cta_merge(const AttnArgs& a, uint16_t* out, float* lse, const unsigned char* rings,
+                                 const int* pseg, int bg, int w0, int w1, int dst) {
+  const int G = a.c.G;
   for (int e = threadIdx.x; e < G * D; e += kThreads) {
     const int h = e / D, d = e % D;
-    float M = -INFINITY;
-    for (int j0 = s0; j0 <= s1; j0 += NB) {
-      float mv[NB];
+    float mv[kWarps], lv[kWarps], ov[kWarps];
 #pragma unroll
-      for (int i = 0; i < NB; ++i)
-        mv[i] = (j0 + i <= s1) ? __ldcg(&src_ml[((size_t)(j0 + i) * G + h) * 2]) : -INFINITY;
-#pragma unroll
-      for (int i = 0; i < NB; ++i) M = fmaxf(M, mv[i]);
+    for (int w = 0; w < kWarps; ++w) {
+      mv[w] = -INFINITY;
+      lv[w] = 0.f;
+      ov[w] = 0.f;
+      if (w >= w0 && w <= w1) {
+        if (pseg[w] == bg) {
+          const float* sp = reinterpret_cast<const float*>(rings + (size_t)w * kRing);
+          ov[w] = sp[h * D + d];
+          mv[w] = sp[G * D + 2 * h];
+          lv[w] = sp[G * D + 2 * h + 1];
+        } else {
+          const size_t slot = (size_t)blockIdx.x * kWarps + w + bg;
+          ov[w] = __ldcg(&a.wp_o[(slot * G + h) * D + d]);
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(&a.wp_ml[(slot * G + h) * 2]));
+          mv[w] = ml.x;
+          lv[w] = ml.y;
+        }
+      }
     }
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mv[w]);
     float o = 0.f, Ls = 0.f;
     if (M != -INFINITY) {
-      for (int j0 = s0; j0 <= s1; j0 += NB) {
-        float2 ml[NB];
-        float ov[NB];
 #pragma unroll
-        for (int i = 0; i < NB; ++i) {
-          const bool in = j0 + i <= s1;
-          ml[i] = in ? __ldcg(reinterpret_cast<const float2*>(&src_ml[((size_t)(j0 + i) * G + h) * 2]))
-                     : make_float2(-INFINITY, 0.f);
-          ov[i] = in ? __ldcg(&src_o[((size_t)(j0 + i) * G + h) * D + d]) : 0.f;
-        }
-#pragma unroll
-        for (int i = 0; i < NB; ++i) {
-          const float f = ml[i].x == -INFINITY ? 0.f : exp2f(ml[i].x - M);
-          o += ov[i] * f;
-          Ls += ml[i].y * f;
-        }
+      for (int w = 0; w < kWarps; ++w) {
+        const float f = mv[w] == -INFINITY ? 0.f : exp2f(mv[w] - M);
+        o += ov[w] * f;
+        Ls += lv[w] * f;
       }
     }
-    if (dst >= 0) {
-      dst_o[((size_t)dst * G + h) * D + d] = o;
-      if (d == 0) {
-        dst_ml[((size_t)dst * G + h) * 2] = M;
-        dst_ml[((size_t)dst * G + h) * 2 + 1] = Ls;
+    put_merged<BF16>(a, out, lse, bg, h, d, D, M, Ls, o, a.ws_o, a.ws_ml, dst);
+  }
+}
+
+// Final merge of segment bg from its CTA partial slots n0 + bg .. n1 + bg into the output;
+// partials are read in batches of 8 with an online rescale (one round trip per batch).
+template <int D, bool BF16>
+__device__ inline void final_combine(const AttnArgs& a, uint16_t* out, float* lse, int bg, int n0, int n1) {
+  constexpr int NB = 8;
+  const int G = a.c.G;
+  for (int e = threadIdx.x; e < G * D; e += kThreads) {
+    const int h = e / D, d = e % D;
+    float M = -INFINITY, o = 0.f, Ls = 0.f;
+    for (int j0 = n0; j0 <= n1; j0 += NB) {
+      float mv[NB], lv[NB], ov[NB];
+#pragma unroll
+      for (int i = 0; i < NB; ++i) {
+        mv[i] = -INFINITY;
+        lv[i] = 0.f;
+        ov[i] = 0.f;
+        if (j0 + i <= n1) {
+          const size_t slot = (size_t)(j0 + i) + bg;
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(&a.ws_ml[(slot * G + h) * 2]));
+          mv[i] = ml.x;
+          lv[i] = ml.y;
+          ov[i] = __ldcg(&a.ws_o[(slot * G + h) * D + d]);
+        }
       }
-    } else {
-      const float r = Ls > 0.f ? o / Ls : 0.f;
-      const size_t oi = ((size_t)b * c.Hq + (size_t)g * G + h) * D + d;
-      if constexpr (BF16) out[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
-      else out[oi] = __half_as_ushort(__float2half_rn(r));
-      if (d == 0 && lse != nullptr)
-        lse[(size_t)b * c.Hq + (size_t)g * G + h] = Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
+      float Mn = M;
+#pragma unroll
+      for (int i = 0; i < NB; ++i) Mn = fmaxf(Mn, mv[i]);
+      if (Mn == -INFINITY) continue;
+      const float r = M == -INFINITY ? 0.f : exp2f(M - Mn);
+      o *= r;
+      Ls *= r;
+#pragma unroll
+      for (int i = 0; i < NB; ++i) {
+        const float f = mv[i] == -INFINITY ? 0.f : exp2f(mv[i] - Mn);
+        o += ov[i] * f;
+        Ls += lv[i] * f;
+      }
+      M = Mn;
     }
+    put_merged<BF16>(a, out, lse, bg, h, d, D, M, Ls, o, nullptr, nullptr, -1);
   }
 }
 
@@ -321,15 +378,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
     __syncwarp();
     ++consumed;
   }
-  if (cur >= 0) write_warp_partial<D>(G, st, a.wp_o + (size_t)(u + cur) * G * D, a.wp_ml + (size_t)(u + cur) * G * 2, lane);
+  // the last segment's partial goes to this warp's ring (every copy has been consumed),
+  // earlier ones went to the warp's global slots
+  __shared__ int s_pseg[kWarps];
+  if (cur >= 0 && !failed) {
+    float* sp = reinterpret_cast<float*>(ring);
+    write_warp_partial<D>(G, st, sp, sp + G * D, lane);
+  } else if (cur >= 0) {
+    write_warp_partial<D>(G, st, a.wp_o + (size_t)(u + cur) * G * D, a.wp_ml + (size_t)(u + cur) * G * 2, lane);
+  }
+  if (lane == 0) s_pseg[warp] = failed ? -1 : cur;
   // after a timeout, give copies still in flight a bounded chance to land before exit
   if (failed) {
     for (int k = consumed; k < issued; ++k) mbar_wait_bounded(smem_u32(&bars[k % kNBar]), (k / kNBar) & 1);
   }
 
-  // CTA pre-merge: one partial per segment this CTA touched, then the last CTA of each
-  // segment (counted arrivals; no waiting) merges those into the output.
-  __threadfence();
+  // CTA pre-merge: one partial per segment this CTA touched (written straight to the
+  // output when the segment lies inside this CTA), then the last CTA of each segment
+  // (counted arrivals; no waiting) merges those into the output.
   __syncthreads();
   const int cw = kWarps * W;  // pages per CTA
   const int cta0 = min(total, (int)blockIdx.x * cw), cta1 = min(total, cta0 + cw);
@@ -346,14 +412,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
     }
     for (; sbg < BH && off[sbg] < cta1; ++sbg) {
       if (off[sbg + 1] <= max(cta0, off[sbg])) continue;  // empty or before the CTA
-      const int u0 = max((int)blockIdx.x * kWarps, off[sbg] / W);
-      const int u1 = min((int)blockIdx.x * kWarps + kWarps - 1, (off[sbg + 1] - 1) / W);
-      merge_slots<D, BF16>(a, out, lse, a.wp_o + (size_t)sbg * G * D, a.wp_ml + (size_t)sbg * G * 2, u0, u1, sbg,
-                           a.ws_o, a.ws_ml, (int)blockIdx.x + sbg);
+      const int w0 = max((int)blockIdx.x * kWarps, off[sbg] / W) - (int)blockIdx.x * kWarps;
+      const int w1 = min((int)blockIdx.x * kWarps + kWarps - 1, (off[sbg + 1] - 1) / W) - (int)blockIdx.x * kWarps;
       const int n0 = off[sbg] / cw, n1 = (off[sbg + 1] - 1) / cw;
-      __threadfence();
+      cta_merge<D, BF16>(a, out, lse, smem, s_pseg, sbg, w0, w1, n0 == n1 ? -1 : (int)blockIdx.x + sbg);
+      if (n0 == n1) continue;  // the whole segment was in this CTA: output written
       __syncthreads();
-      if (tid == 0) {
+      if (tid == 0) {  // the barrier orders every thread's partial writes before this fence
+        __threadfence();
         const unsigned old = atomicAdd(&a.counters[sbg], 1u);
         s_last = old == static_cast<unsigned>(n1 - n0);
         if (s_last) a.counters[sbg] = 0u;  // every CTA of this segment has arrived: reset for the next call
@@ -361,8 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
       __syncthreads();
       if (s_last) {
         __threadfence();
-        merge_slots<D, BF16>(a, out, lse, a.ws_o + (size_t)sbg * G * D, a.ws_ml + (size_t)sbg * G * 2, n0, n1, sbg,
-                             nullptr, nullptr, -1);
+        final_combine<D, BF16>(a, out, lse, sbg, n0, n1);
       }
       __syncthreads();
     }

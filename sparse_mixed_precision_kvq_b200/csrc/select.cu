@@ -57,10 +57,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(DevCache c, const f
 cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_select_params& prm,
                           int32_t* sel, int32_t* cnt, int kmax, cudaStream_t s) {
   const size_t smem = (size_t)c.max_pages * sizeof(uint32_t);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
+  // static (histogram scratch) + dynamic (keys) shared memory may pass the 48 KB default
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   return launch_pdl(select_kernel, dim3(c.B * c.Hkv), dim3(kSelThreads), smem, s, c, scores, prm, sel, cnt, kmax);
 }
 

@@ -7,8 +7,8 @@
 // select_core.cuh, page_math.cuh); what changes is the schedule.
 //
 // Work units are (b, kv head) pairs u.  Each unit is cut into
-//   score items:     up to 16 ring slots of page summaries (512 pages at D = 128),
-//   attention items: up to 24 selected pages,
+//   score items:     32 ring slots of page summaries (1024 pages at D = 128),
+//   attention items: 32 selected pages,
 // and one queue orders all score items (unit by unit) before all attention items.
 // One CTA per SM takes items from the queue (an atomic counter) until it runs dry.
 //
@@ -55,14 +55,16 @@ constexpr int kCW = 8;                        // consumer warps
 constexpr int kCT = kCW * 32;                 // consumer threads
 constexpr int kStepThreads = kCT + 32;        // + the producer warp
 constexpr int kSlot = 8192;                   // ring slot bytes: one 16-bit page (K + V) at D = 128
-constexpr int kASlotsPerWarp = 2;             // score item = kCW * 2 slots
-constexpr int kBPagesPerWarp = 3;             // attention item = kCW * 3 pages
-constexpr int kBPages = kCW * kBPagesPerWarp;  // <= 32: one producer lane per page
+// Item sizes: large enough to amortise an item's fixed costs (a few dependent memory
+// round trips and consumer barriers), small enough to spread over the CTAs.
+constexpr int kASlots = 32;                   // score item: ring slots of summaries (1024 at D = 128)
+constexpr int kBPages = 32;                   // attention item: selected pages (one producer lane each)
+constexpr int kBMax = kBPages;
 constexpr int kMaxRingSlots = 24;             // data slots (a multiple of kCW: each warp owns slots w, w + 8, ...)
 constexpr int kNDesc = 64;                    // descriptor ring (a multiple of kCW, a power of two)
 constexpr int kMaxSmem = 232448 - 4096;       // 227 KB per CTA, less the static shared memory
 constexpr int kCtlWords = 16;                 // [0] item queue, [1] CTAs finished, then a_done, b_done
-static_assert(kBPages <= 32, "one producer lane per page of an attention item");
+static_assert(kBMax <= 32, "one producer lane per page of an attention item");
 
 enum : int { KIND_A = 0, KIND_B = 1, KIND_END = 2 };
 
@@ -112,15 +114,21 @@ __host__ __device__ inline int pages_of(int L, int max_pages) {
   const int P = (max(L, 0) + kPage - 1) / kPage;
   return P < max_pages ? P : max_pages;
 }
+// Score items of a unit of P pages with items of up to `as` slots (balanced split).
 template <int D>
-__host__ __device__ inline int score_items(int P) {
-  constexpr int per = kCW * kASlotsPerWarp * SummariesPerSlot<D>::value;
-  return P > 0 ? (P + per - 1) / per : 1;
+__host__ __device__ inline int score_items(int P, int as) {
+  const int nsl = (P + SummariesPerSlot<D>::value - 1) / SummariesPerSlot<D>::value;
+  return nsl > 0 ? (nsl + as - 1) / as : 1;
 }
-__host__ __device__ inline int attn_items(int P, const kvq_select_params& prm, int kmax) {
-  const int n = min(select_split(P, prm).count(P), kmax);
-  return n > 0 ? (n + kBPages - 1) / kBPages : 1;
+// Pages attended for a unit of P pages (the selection's count, clamped to kmax).
+__host__ __device__ inline int attn_pages(int P, const kvq_select_params& prm, int kmax) {
+  return min(select_split(P, prm).count(P), kmax);
 }
+__host__ __device__ inline int attn_items(int P, const kvq_select_params& prm, int kmax, int bs) {
+  const int n = attn_pages(P, prm, kmax);
+  return n > 0 ? (n + bs - 1) / bs : 1;
+}
+
 
 // last b with tab[b] <= i (tab strictly increasing, tab[0] = 0)
 __device__ inline int find_b(const int* tab, int B, int i) {
@@ -229,6 +237,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
   griddep_wait();  // the cache and the inputs come from earlier work on the stream
 
   // item tables: exclusive prefix sums over b of the items of b's Hkv units
+  constexpr int as = kASlots, bs = kBPages;
   {
     constexpr int NW = kStepThreads / 32;
     const int per = (B + kStepThreads - 1) / kStepThreads;
@@ -238,8 +247,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
       const int L = max(c.seq_len[b], 0);
       tabL[b] = L;
       const int P = pages_of(L, c.max_pages);
-      sa += score_items<D>(P) * Hkv;
-      sb += attn_items(P, a.prm, a.kmax) * Hkv;
+      sa += score_items<D>(P, as) * Hkv;
+      sb += attn_items(P, a.prm, a.kmax, bs) * Hkv;
     }
     int x = sa, y = sb;
 #pragma unroll
@@ -273,8 +282,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
       tabA[b] = ra;
       tabB[b] = rb;
       const int P = pages_of(tabL[b], c.max_pages);
-      ra += score_items<D>(P) * Hkv;
-      rb += attn_items(P, a.prm, a.kmax) * Hkv;
+      ra += score_items<D>(P, as) * Hkv;
+      rb += attn_items(P, a.prm, a.kmax, bs) * Hkv;
     }
     if (tid == 0) {
       tabA[B] = s_scan[0][NW];
@@ -327,22 +336,27 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
       if (!it.valid) return;
       if (item < totA) {
         const int b = find_b(tabA, B, item);
-        const int na = score_items<D>(pages_of(tabL[b], c.max_pages));
-        const int r = item - tabA[b];
+        const int P = pages_of(tabL[b], c.max_pages);
+        const int na = score_items<D>(P, as);
+        const int r = item - tabA[b], j = r % na;
         it.kind = KIND_A;
         it.b = b;
         it.g = r / na;
-        it.p0 = (r % na) * (kCW * kASlotsPerWarp * SP);
+        it.p0 = j * as * SP;
+        it.np = min(P, it.p0 + as * SP) - it.p0;
         it.item = item;
       } else {
         const int ib = item - totA;
         const int b = find_b(tabB, B, ib);
-        const int nb = attn_items(pages_of(tabL[b], c.max_pages), a.prm, a.kmax);
-        const int r = ib - tabB[b];
+        const int P = pages_of(tabL[b], c.max_pages);
+        const int n = attn_pages(P, a.prm, a.kmax);
+        const int nb = attn_items(P, a.prm, a.kmax, bs);
+        const int r = ib - tabB[b], j = r % nb;
         it.kind = KIND_B;
         it.b = b;
         it.g = r / nb;
-        it.p0 = (r % nb) * kBPages;  // first rank
+        it.p0 = j * bs;                          // first rank
+        it.np = max(0, min(n, it.p0 + bs) - it.p0);
         it.item = ib;
       }
       it.u = it.b * Hkv + it.g;
@@ -354,17 +368,16 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
       const int L = tabL[it.b];
       const int P = pages_of(L, c.max_pages);
       if (it.kind == KIND_A) {
-        it.np = max(0, min(P, it.p0 + kCW * kASlotsPerWarp * SP) - it.p0);
         const int nsl = (it.np + SP - 1) / SP;
         it.S = max(kCW, (nsl + kCW - 1) / kCW * kCW);
         const uint16_t* src = c.summary + ((size_t)it.u * c.max_pages + it.p0) * D;
-        if (lane < nsl)
-          bulk_prefetch_l2(src + (size_t)lane * SP * D, (uint32_t)min(SP, it.np - lane * SP) * D * 2);
+        for (int s = lane; s < nsl; s += 32)
+          bulk_prefetch_l2(src + (size_t)s * SP * D, (uint32_t)min(SP, it.np - s * SP) * D * 2);
         it.resolved = 1;
         return true;
       }
       // wait until the unit's pages are chosen (a_done = score items + 1)
-      const unsigned target = static_cast<unsigned>(score_items<D>(P)) + 1u;
+      const unsigned target = static_cast<unsigned>(score_items<D>(P, as)) + 1u;
       int ok = 1;
       if (lane == 0) {
         if (ld_acquire_gpu(&a.a_done[it.u]) < target) {
@@ -390,7 +403,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
       if (ok < 0) failed = true;
       if (ok <= 0) return false;
       const int n = min(max(__ldcg(&a.cnt[it.u]), 0), a.kmax);
-      it.np = max(0, min(n, it.p0 + kBPages) - it.p0);
+      it.np = max(0, min(n, it.p0 + it.np) - it.p0);  // the selection's own count (equal but for errors)
       it.S = max(kCW, (it.np + kCW - 1) / kCW * kCW);
       it.psrc = nullptr;
       it.tier = -1;
@@ -415,20 +428,22 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
       it.resolved = 1;
       return true;
     };
-    // Publish all positions of `it` (lane s: position s of the item).
+    // Publish all positions of `it` (lane s: positions s, s + 32, ... of the item).
     auto issue = [&](const Item& it) {
-      const int s = lane;
-      SlotDesc d;
-      if (it.kind == KIND_A) {
-        const int n = s * SP < it.np ? min(SP, it.np - s * SP) : 0;
-        d = SlotDesc{KIND_A, it.u, it.item, it.p0 + s * SP, n, 0, s >= it.S - kCW ? 1 : 0, n * D * 2,
-                     c.summary + ((size_t)it.u * c.max_pages + it.p0 + (size_t)s * SP) * D};
-      } else {
-        const bool real = s < it.np && it.tier >= 0;
-        d = SlotDesc{KIND_B, it.u, it.item, it.pg, real ? it.tier : -1, it.nv, s >= it.S - kCW ? 1 : 0,
-                     real ? 2 * c.chunk[it.tier] : 0, it.psrc};
+      for (int s0 = 0; s0 < it.S && !failed; s0 += 32) {
+        const int s = s0 + lane;
+        SlotDesc d;
+        if (it.kind == KIND_A) {
+          const int n = s * SP < it.np ? min(SP, it.np - s * SP) : 0;
+          d = SlotDesc{KIND_A, it.u, it.item, it.p0 + s * SP, n, 0, s >= it.S - kCW ? 1 : 0, n * D * 2,
+                       c.summary + ((size_t)it.u * c.max_pages + it.p0 + (size_t)s * SP) * D};
+        } else {
+          const bool real = s < it.np && it.tier >= 0;
+          d = SlotDesc{KIND_B, it.u, it.item, it.pg, real ? it.tier : -1, it.nv, s >= it.S - kCW ? 1 : 0,
+                       real ? 2 * c.chunk[it.tier] : 0, it.psrc};
+        }
+        failed = !publish(d, min(32, it.S - s0));
       }
-      failed = !publish(d, it.S);
     };
 
     Item cur, nxt;
@@ -577,7 +592,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
       if (tid == 0) {  // the barrier orders every warp's score writes before this fence
         __threadfence();
         const unsigned old = atomicAdd(&a.a_done[u], 1u);
-        s_flag = (old + 1u == static_cast<unsigned>(score_items<D>(P))) ? 1 : 0;
+        s_flag = (old + 1u == static_cast<unsigned>(score_items<D>(P, as))) ? 1 : 0;
       }
       if (!cb()) return false;
       if (s_flag) {
@@ -604,7 +619,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
       write_warp_partial<D>(G, st, mine, mine + G * D, lane);
       if (!cb()) return false;
       const int P = pages_of(tabL[b], c.max_pages);
-      const int nb = attn_items(P, a.prm, a.kmax);
+      const int nb = attn_items(P, a.prm, a.kmax, bs);
       const size_t row0 = (size_t)b * c.Hq + (size_t)g * G;
       for (int e = tid; e < G * D; e += kCT) {
         const int h = e / D, dd = e % D;

@@ -338,3 +338,21 @@ def test_select_special_values_and_wide_ranges(kvq):
             for g in range(Hkv):
                 want = select(sc[b, g].astype(np.float64), P, *params)
                 assert list(got_s[b, g, :got_c[b, g]]) == list(want), (params, b, g)
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_long_context_many_pages(kvq, path):
+    """A sequence of 8193 pages (131072 tokens + 1, as in the long-context workload): the
+    selection keeps all of its keys on chip; pages, selection and output as the oracle's."""
+    w = W.make("c3", lens=np.array([131072]), Hq=8, Hkv=2)
+    cache, step, pre, post = _run(kvq, w, fused=path == "fused")
+    assert cache.err_bits() == 0, hex(cache.err_bits())
+    q, kn, vn = query_and_new(w)
+    sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
+    out = out_to_f64(step.out, w.dtype)
+    for g in range(w.Hkv):
+        sh = prepare(w, 0, g)
+        r = oracle_step(w, sh, 0, g, q, kn, vn)
+        assert check_selection(sel[0, g, :cnt[0, g]], r["sel"], r["scores"], w, r["P"])
+        for i in range(w.G):
+            check_output(out[0, g * w.G + i], r["out"][i], f"long g={g}", w.dtype)
