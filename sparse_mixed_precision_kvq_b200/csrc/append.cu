@@ -16,22 +16,25 @@ namespace kvq {
 namespace {
 
 // ----------------------------------------------------------------------------- append
-// One warp per (b, kv head), four per CTA.
+// One CTA of four warps per (b, kv head): the summary and the page clear over all 128
+// threads, then one (kind, group) pair per warp at D = 128.
 template <bool BF16>
 __global__ void __launch_bounds__(128) append_kernel(DevCache c, const int32_t* __restrict__ pos,
                                                      const uint16_t* __restrict__ k_new,
                                                      const uint16_t* __restrict__ v_new) {
-  const int lane = threadIdx.x & 31;
-  const int bg = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bg = blockIdx.x;
+  const int b = bg / c.Hkv, g = bg % c.Hkv;
   griddep_wait();
-  if (bg < c.B * c.Hkv) {
-    const int b = bg / c.Hkv, g = bg % c.Hkv;
-    const int P = pos[b];
-    if (P >= c.max_pages * kPage) {
-      if (lane == 0) set_err(c.err, KVQ_DERR_BAD_POS);
-    } else if (P >= 0) {
-      append_token_warp<BF16>(c, b, g, P, k_new + (size_t)bg * c.D, v_new + (size_t)bg * c.D, lane, nullptr);
-    }
+  const int P = pos[b];
+  if (P >= c.max_pages * kPage) {
+    if (tid == 0) set_err(c.err, KVQ_DERR_BAD_POS);
+  } else if (P >= 0) {
+    const uint16_t* kr = k_new + (size_t)bg * c.D;
+    const uint16_t* vr = v_new + (size_t)bg * c.D;
+    const bool ok = append_phase1<BF16>(c, b, g, P, kr, tid, 128, nullptr);
+    __syncthreads();
+    if (ok) append_phase2<BF16>(c, b, g, P, kr, vr, warp, 4, lane);
   }
   griddep_launch_dependents();
 }
@@ -124,7 +127,7 @@ __global__ void __launch_bounds__(128) build_kernel(DevCache c, const uint16_t* 
 
 cudaError_t launch_append(const DevCache& c, const int32_t* pos, const void* k_new, const void* v_new,
                           cudaStream_t s) {
-  const dim3 grid((c.B * c.Hkv + 3) / 4);
+  const dim3 grid(c.B * c.Hkv);
   const uint16_t* kn = static_cast<const uint16_t*>(k_new);
   const uint16_t* vn = static_cast<const uint16_t*>(v_new);
   if (c.dtype == KVQ_DT_BF16) return launch_pdl(append_kernel<true>, grid, dim3(128), 0, s, c, pos, kn, vn);

@@ -58,24 +58,26 @@ __device__ inline double to_double(uint16_t v) {
   return static_cast<double>(bits_to_float<BF16>(v));
 }
 
-// One warp writes token `pos` of sequence b, kv head g: quantises K and V into the
-// page's tier, clears a newly opened page first, and advances the open page's fp64 key
-// sum and its fp16 summary.  `patch` (nullable, D entries) receives the new summary row
-// as well.  Returns false (nothing written) if the page's block-table entry is invalid.
-// The caller has checked 0 <= pos < max_pages * 16.
+// Token append, in two phases so that several warps can share it (the caller puts a
+// barrier over those warps between the phases):
+//  phase 1 (threads t0 = 0 .. nt-1): advance the open page's fp64 key sum and its fp16
+//          summary (`patch`, nullable, receives the new summary row too), and clear a newly
+//          opened page;
+//  phase 2 (warps w = 0 .. nw-1): quantise K and V into the page's tier, warp w taking the
+//          (kind, 32-channel group) pairs w, w + nw, ...
+// Token `pos` of sequence b, kv head g; the caller has checked 0 <= pos < max_pages * 16.
+// Both phases return false (nothing written) if the page's block-table entry is invalid.
 template <bool BF16>
-__device__ inline bool append_token_warp(const DevCache& c, int b, int g, int pos, const uint16_t* krow,
-                                         const uint16_t* vrow, int lane, uint16_t* patch) {
+__device__ inline bool append_phase1(const DevCache& c, int b, int g, int pos, const uint16_t* krow, int t0, int nt,
+                                     uint16_t* patch) {
   const int D = c.D;
   const size_t bg = (size_t)b * c.Hkv + g;
   const int page = pos / kPage, t = pos % kPage;
   int tier;
   const unsigned char* ck;
   if (!page_chunk(c, b, page, g, tier, ck)) return false;
-  unsigned char* chunk[2] = {const_cast<unsigned char*>(ck), const_cast<unsigned char*>(ck) + c.chunk[tier]};
-  const uint16_t* row[2] = {krow, vrow};
-  bool ov = false, nonfinite = false;
-  for (int d = lane; d < D; d += 32) {  // running key sum of the open page and its summary
+  bool ov = false;
+  for (int d = t0; d < D; d += nt) {  // running key sum of the open page and its summary
     const double x = to_double<BF16>(krow[d]);
     double* ks = c.open_ksum + bg * D + d;
     const double S = (t == 0) ? x : (*ks + x);
@@ -84,52 +86,63 @@ __device__ inline bool append_token_warp(const DevCache& c, int b, int g, int po
     c.summary[(bg * c.max_pages + page) * D + d] = m;
     if (patch != nullptr) patch[d] = m;
   }
+  if (ov) set_err(c.err, KVQ_DERR_FP16_RANGE);
   if (t == 0) {  // a newly opened page starts from zero bytes
-    uint4* p4 = reinterpret_cast<uint4*>(chunk[0]);
+    uint4* p4 = reinterpret_cast<uint4*>(const_cast<unsigned char*>(ck));
     const int n16 = 2 * c.chunk[tier] / 16;
-    for (int i = lane; i < n16; i += 32) p4[i] = make_uint4(0, 0, 0, 0);
-    __syncwarp();
+    for (int i = t0; i < n16; i += nt) p4[i] = make_uint4(0, 0, 0, 0);
   }
-  if (tier == KVQ_TIER_16) {
-#pragma unroll
-    for (int kind = 0; kind < 2; ++kind) {
-      for (int d = lane; d < D; d += 32) {
-        const uint16_t v = row[kind][d];
-        nonfinite |= !isfinite(to_double<BF16>(v));
-        int w, bit;
-        elem_pos(kind, 0, D, t, d, w, bit);
-        reinterpret_cast<uint16_t*>(chunk[kind])[2 * w + (bit >> 4)] = v;
-      }
+  return true;
+}
+
+template <bool BF16>
+__device__ inline bool append_phase2(const DevCache& c, int b, int g, int pos, const uint16_t* krow,
+                                     const uint16_t* vrow, int w, int nw, int lane) {
+  const int D = c.D;
+  const int page = pos / kPage, t = pos % kPage;
+  int tier;
+  const unsigned char* ck;
+  if (!page_chunk(c, b, page, g, tier, ck)) return false;
+  bool ov = false, nonfinite = false;
+  const int ng = D / kGroup;
+  for (int gi = w; gi < 2 * ng; gi += nw) {
+    const int kind = gi / ng, grp = gi % ng;
+    const int d = grp * kGroup + lane;
+    unsigned char* chunk = const_cast<unsigned char*>(ck) + (kind ? c.chunk[tier] : 0);
+    const uint16_t v = (kind ? vrow : krow)[d];
+    const double x = to_double<BF16>(v);
+    nonfinite |= !isfinite(x);
+    int wd, bit;
+    elem_pos(kind, tier, D, t, d, wd, bit);
+    if (tier == KVQ_TIER_16) {
+      reinterpret_cast<uint16_t*>(chunk)[2 * wd + (bit >> 4)] = v;
+      continue;
     }
-  } else {
-    const int ng = D / kGroup;
-    const int b_bits = tier_bits(tier);
-    const uint32_t cmask = (1u << b_bits) - 1u;
-#pragma unroll
-    for (int kind = 0; kind < 2; ++kind) {
-      unsigned char* meta = chunk[kind] + codes_bytes(tier, D);
-      for (int grp = 0; grp < ng; ++grp) {
-        const int d = grp * kGroup + lane;
-        const double x = to_double<BF16>(row[kind][d]);
-        nonfinite |= !isfinite(x);
-        const QOut q = quant_group(x, tier, ov);
-        int w, bit;
-        elem_pos(kind, tier, D, t, d, w, bit);
-        uint32_t* word = reinterpret_cast<uint32_t*>(chunk[kind]) + w;
-        atomicAnd(word, ~(cmask << bit));  // lanes of one group can share a word
-        atomicOr(word, q.code << bit);
-        if (lane == 0) {
-          if (tier == KVQ_TIER_I1)
-            reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = static_cast<uint16_t>(q.meta);
-          else
-            reinterpret_cast<uint32_t*>(meta)[t * ng + grp] = q.meta;
-        }
-      }
+    const QOut q = quant_group(x, tier, ov);
+    const uint32_t cmask = (1u << tier_bits(tier)) - 1u;
+    uint32_t* word = reinterpret_cast<uint32_t*>(chunk) + wd;
+    atomicAnd(word, ~(cmask << bit));  // lanes of one group can share a word
+    atomicOr(word, q.code << bit);
+    if (lane == 0) {
+      unsigned char* meta = chunk + codes_bytes(tier, D);
+      if (tier == KVQ_TIER_I1)
+        reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = static_cast<uint16_t>(q.meta);
+      else
+        reinterpret_cast<uint32_t*>(meta)[t * ng + grp] = q.meta;
     }
   }
   if (__any_sync(0xffffffffu, ov) && lane == 0) set_err(c.err, KVQ_DERR_FP16_RANGE);
   if (__any_sync(0xffffffffu, nonfinite) && lane == 0) set_err(c.err, KVQ_DERR_NONFINITE);
   return true;
+}
+
+// One warp does both phases.
+template <bool BF16>
+__device__ inline bool append_token_warp(const DevCache& c, int b, int g, int pos, const uint16_t* krow,
+                                         const uint16_t* vrow, int lane, uint16_t* patch) {
+  const bool ok = append_phase1<BF16>(c, b, g, pos, krow, lane, 32, patch);
+  __syncwarp();
+  return ok && append_phase2<BF16>(c, b, g, pos, krow, vrow, 0, 1, lane);
 }
 
 }  // namespace kvq
