@@ -146,6 +146,29 @@ def kernel_traffic(kernel_file: str):
     return e
 
 
+# ----------------------------------------------------------------------------- ranks
+def rank_workload(config: str, rank: int, batch=None):
+    """Rank r's batch: the workload's shapes with its own seeds (independent sequences per
+    rank: weak scaling, nothing exchanged on the data path)."""
+    from sparse_mixed_precision_kvq_b200 import workloads as W
+    base = W.make(config)
+    over = {} if batch is None else dict(B=batch)
+    if batch is not None and config != "c4":
+        over["lens"] = np.resize(base.lens, batch)
+    return W.make(config, seed=base.seed + 1000 * rank, **over)
+
+
+def max_over_ranks(x: float, device) -> float:
+    """The largest x over all ranks of the process group (plain value with one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def run_kvq(args, rank: int, world: int, local_rank: int):
     import torch
@@ -155,10 +178,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    over = {} if args.batch is None else dict(B=args.batch)
-    if args.batch is not None and args.config != "c4":
-        over["lens"] = np.resize(W.make(args.config).lens, args.batch)
-    w = W.make(args.config, seed=W.make(args.config).seed + 1000 * rank, **over)
+    w = rank_workload(args.config, rank, args.batch)
     cache = kvq.cache_from_workload(w, device=dev)
     step = kvq.DecodeStep(w, cache, device=dev)
     tier_tbl, _, _ = w.slot_map()
@@ -237,11 +257,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
         per[k] = [pev[i].elapsed_time(pev[i + 1]) for i in range(len(parts))]
     clocks.stop()
     step_ms = np.array([e0[k].elapsed_time(e1[k]) for k in range(K)])
-    total_ms = float(step_ms.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(step_ms.sum()), dev)
     ms_per_step = total_ms / K
     tokens = world * w.B * K
     value = tokens / (total_ms / 1e3)
@@ -267,11 +283,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
         lse_h.copy_(step.lse, non_blocking=True)
         e_end[k].record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = float(np.mean([e_start[k].elapsed_time(e_end[k]) for k in range(KE)]))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(float(np.mean([e_start[k].elapsed_time(e_end[k]) for k in range(KE)])), dev)
     h2d = pin["q"].numel() * 2 + (pin["k"].numel() * 2 * 2 if w.append else 0)
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
     del g_prof, g_step
