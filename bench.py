@@ -187,7 +187,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
 
     for _ in range(args.warmup):
         flush.fill_(1)
-        step.run_fused() if args.path == "fused" else step.run()
+        {"fused": step.run_fused, "two": step.run_two, "calls": step.run}[args.path]()
     torch.cuda.synchronize(dev)
     assert cache.err_bits() == 0, f"device error bits {cache.err_bits():#x}"
     sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
@@ -195,11 +195,12 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
 
     K = args.steps
     fused = args.path == "fused"
-    run_step = step.run_fused if fused else step.run
+    run_step = {"fused": step.run_fused, "two": step.run_two, "calls": step.run}[args.path]
     # kernels of one step, in launch order (one callable each)
-    parts = [("decode_step", step.run_fused)] if fused else [
-        ("append", step.append), ("page_scores", step.scores_), ("select_topk", step.select),
-        ("sparse_decode_attn", step.attend)]
+    parts = {"fused": [("decode_step", step.run_fused)],
+             "two": [("score_select", step.score_select), ("sparse_decode_attn", step.attend)],
+             "calls": [("append", step.append), ("page_scores", step.scores_), ("select_topk", step.select),
+                       ("sparse_decode_attn", step.attend)]}[args.path]
     # The step is replayed from CUDA graphs so the CPU never starves the GPU:
     #  g_step: the step's launches, nothing between them (programmatic launch overlap intact);
     #  g_prof: the same launches with timing events between them (per-kernel durations).
@@ -302,6 +303,9 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     step_bytes = nbytes["attn"] + nbytes["score"] + nbytes["select"] + nbytes["append"]
     if fused:
         dom_bytes, files = step_bytes, ["step.cu"]
+    elif args.path == "two":
+        dom_bytes = [nbytes["score"] + nbytes["select"] + nbytes["append"], nbytes["attn"]][dom]
+        files = ["score.cu", "attn.cu"]
     else:
         dom_bytes = [nbytes["append"], nbytes["score"], nbytes["select"], nbytes["attn"]][dom]
         files = ["append.cu", "score.cu", "select.cu", "attn.cu"]
@@ -336,8 +340,9 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
         "e2e": {"value": world * w.B / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
         "gpu_launches": len(parts) * K,
-        "path": "kvq_decode_step (one persistent launch)" if fused else "kvq_append -> kvq_page_scores -> "
-                "kvq_select_topk -> kvq_sparse_decode_attn",
+        "path": {"fused": "kvq_decode_step (one persistent launch)",
+                 "two": "kvq_score_select -> kvq_sparse_decode_attn",
+                 "calls": "kvq_append -> kvq_page_scores -> kvq_select_topk -> kvq_sparse_decode_attn"}[args.path],
         "timing": "step: CUDA-graph replay of the step timed with events around each replay; "
                   "kernels_ms: a second graph with events between the launches (no launch overlap)",
         "clocks": clocks.summary(t0, t1),
@@ -439,8 +444,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default="c1", choices=sorted(DESCR))
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
-    ap.add_argument("--path", default="calls", choices=["fused", "calls"],
-                    help="one kvq_decode_step launch, or the four separate calls")
+    ap.add_argument("--path", default="calls", choices=["calls", "two", "fused"],
+                    help="the four separate calls, kvq_score_select + attention, or one kvq_decode_step launch")
     ap.add_argument("--dense", action="store_true", help="also time attention over every page")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

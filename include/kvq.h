@@ -9,6 +9,7 @@
  *   kvq_select_topk        pick the top pages plus forced sink/recent pages;
  *   kvq_sparse_decode_attn attend only the selected pages (split-K + log-sum-exp combine),
  *                          unpacking and dequantising cold pages in registers;
+ *   kvq_score_select       the first three in one launch (same results);
  *   kvq_decode_step        the four above in one persistent launch (same results).
  *
  * Sources: AMASS "decode-time sparse KV-cache attention for vLLM" (amass-kv 0.1.1),
@@ -231,6 +232,21 @@ kvq_status kvq_sparse_decode_attn_noalloc(const kvq_cache* cache, const void* q,
 
 /* Size in bytes of the static scratch used by kvq_sparse_decode_attn_noalloc. */
 size_t kvq_noalloc_scratch_bytes(void);
+
+/*
+ * kvq_score_select -- kvq_append (when pos is not NULL), kvq_page_scores and
+ * kvq_select_topk in one launch, with the same results (AMASS "What is in the box":
+ * score every page from its summary, keep the best).  The warp that scores the tile of a
+ * sequence's appended token writes the token first; the CTA that finishes the last score
+ * tile of a (b, kv head) selects its pages.  Arguments as those three calls; workspace:
+ * any kvq workspace of at least 64 KiB prepared with kvq_workspace_init (per-(b, kv head)
+ * tile counters at its head; the call leaves them zero).  B*Hkv <= 8192,
+ * max_pages <= 51200.
+ */
+kvq_status kvq_score_select(const kvq_cache* cache, const int32_t* pos, const void* k_new,
+                            const void* v_new, const void* q, const kvq_select_params* params,
+                            float* scores, int32_t* sel, int32_t* cnt, int32_t kmax, void* workspace,
+                            size_t ws_bytes, kvq_stream_t stream);
 
 /* Workspace bytes kvq_decode_step needs for this cache and kmax. */
 kvq_status kvq_step_workspace_size(const kvq_cache* cache, int32_t kmax, size_t* bytes);

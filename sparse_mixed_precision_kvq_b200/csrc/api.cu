@@ -176,6 +176,25 @@ kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const i
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+kvq_status kvq_score_select(const kvq_cache* cache, const int32_t* pos, const void* k_new, const void* v_new,
+                            const void* q, const kvq_select_params* params, float* scores, int32_t* sel,
+                            int32_t* cnt, int32_t kmax, void* workspace, size_t ws_bytes, kvq_stream_t stream) {
+  DevCache c;
+  kvq_status st = to_dev(cache, c);
+  if (st != KVQ_OK) return st;
+  if (q == nullptr || params == nullptr || scores == nullptr || sel == nullptr || cnt == nullptr ||
+      workspace == nullptr || kmax < 1)
+    return KVQ_ERR_INVALID_ARG;
+  if (pos != nullptr && (k_new == nullptr || v_new == nullptr)) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
+  if ((long long)c.B * c.Hkv > (long long)(kCounterBytes / 4 - kScoreSelectCounterWord)) return KVQ_ERR_UNSUPPORTED;
+  if ((size_t)c.max_pages * 4 > 200 * 1024) return KVQ_ERR_UNSUPPORTED;  // keys in shared memory
+  if (ws_bytes < kCounterBytes) return KVQ_ERR_WORKSPACE;
+  unsigned* done = static_cast<unsigned*>(workspace) + kScoreSelectCounterWord;
+  return cuda_status(launch_score_select(c, pos, k_new, v_new, q, *params, scores, sel, cnt, kmax, done,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 kvq_status kvq_step_workspace_size(const kvq_cache* cache, int32_t kmax, size_t* bytes) {
   DevCache c;
   kvq_status st = to_dev(cache, c);

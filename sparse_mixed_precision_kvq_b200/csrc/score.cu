@@ -11,7 +11,9 @@
 #include <math.h>
 
 #include "kvq_internal.cuh"
+#include "quant.cuh"
 #include "score_tile.cuh"
+#include "select_core.cuh"
 
 namespace kvq {
 namespace {
@@ -27,79 +29,166 @@ __device__ inline void load_tile(const uint16_t* sbase, int tile, int P, int lan
     const int p = tile * 16 + g8 + 8 * r;
     const uint4* src = reinterpret_cast<const uint4*>(sbase + (size_t)p * D + CW * q4);
 #pragma unroll
-    for (int i = 0; i < CW / 8; ++i) av[r][i] = p < P ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < CW / 8; ++i) av[r][i] = p < P ? __ldcg(src + i) : make_uint4(0, 0, 0, 0);
   }
 }
 
+// Extra work of the fused form (kvq_score_select): the token append before the scores
+// and the selection after them.
+struct ScoreSelect {
+  const int32_t* pos;  // nullable: no append
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  kvq_select_params prm;
+  int32_t* sel;
+  int32_t* cnt;
+  int kmax;
+  unsigned* done;  // [B * Hkv] tiles scored per (b, g) (zero between calls)
+};
+
 // Grid of 2 CTAs per SM; warp w takes the contiguous run of 16-page tiles
 // [w * per, (w + 1) * per) of the flat list (b, g, tile), loading the next tile while
-// the current one is multiplied.
-template <int D, bool BF16>
+// the current one is multiplied.  FUSED: the warp that owns the tile of a (b, g)'s
+// appended token writes the token first (so that tile is read after the new summary row
+// is stored); after its tiles, the CTA counts them on each (b, g) it touched, and the CTA
+// that completes a (b, g) selects its pages (select_core.cuh) from the scores in L2.
+template <int D, bool BF16, bool FUSED>
 __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, const uint16_t* __restrict__ q,
                                                                     float* __restrict__ scores, int tiles_per_bg,
-                                                                    int per) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                                                                    int per, ScoreSelect f) {
+  extern __shared__ __align__(16) uint32_t sel_smem[];  // FUSED: keys [max_pages], then the scratch
+  __shared__ SelShared sel_sh;
+  __shared__ int s_unit;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, q4 = lane & 3;
   const int total = c.B * c.Hkv * tiles_per_bg;
   const int i0 = (blockIdx.x * kScoreWarps + warp) * per;
   const int i1 = min(total, i0 + per);
   griddep_wait();
-  if (i0 >= i1) return;
 
-  QFrag<D, BF16> qf;
-  int cur_bg = -1, P = 0;
-  float* out = nullptr;
-  bool bad = false;
-  uint4 av0[2][D / 32], av1[2][D / 32];  // double buffer (compile-time indexed)
-
-  // where tile item i lives
-  auto tile_src = [&](int i, int& Pn) -> const uint16_t* {
-    const int bg = i / tiles_per_bg;
-    const int L = c.seq_len[bg / c.Hkv];
-    Pn = min((L + kPage - 1) / kPage, c.max_pages);
-    return c.summary + (size_t)bg * c.max_pages * D;
-  };
-  auto compute = [&](int i, const uint4 (&av)[2][D / 32]) {
-    const int bg = i / tiles_per_bg, tile = i % tiles_per_bg;
-    if (bg != cur_bg) {  // new (b, g): its query fragments (hi + lo)
-      cur_bg = bg;
+  if (FUSED && f.pos != nullptr && i0 < i1) {  // appends whose page lies in this warp's tiles
+    for (int bg = i0 / tiles_per_bg; bg <= (i1 - 1) / tiles_per_bg; ++bg) {
       const int b = bg / c.Hkv, g = bg % c.Hkv;
-      const int L = c.seq_len[b];
-      P = min((L + kPage - 1) / kPage, c.max_pages);
-      out = scores + (size_t)bg * c.max_pages;
-      qf.load(q, c.Hq, c.G, b, g, lane, bad);
+      const int ps = f.pos[b];
+      if (ps < 0) continue;
+      if (ps >= c.max_pages * kPage) {
+        if (lane == 0 && g == 0 && bg * tiles_per_bg >= i0) set_err(c.err, KVQ_DERR_BAD_POS);
+        continue;
+      }
+      const int it = bg * tiles_per_bg + (ps / kPage) / 16;
+      if (it < i0 || it >= i1) continue;
+      append_token_warp<BF16>(c, b, g, ps, f.k_new + (size_t)bg * D, f.v_new + (size_t)bg * D, lane, nullptr);
+      __syncwarp();
     }
-    float m0, m1;
-    tile_scores<D, BF16>(av, qf, c.G, lane, m0, m1);
-    if (q4 == 0) {
-      const int p0 = tile * 16 + g8, p1 = p0 + 8;
-      if (p0 < c.max_pages) out[p0] = p0 < P ? m0 : -INFINITY;
-      if (p1 < c.max_pages) out[p1] = p1 < P ? m1 : -INFINITY;
-    }
-  };
-
-  int Pn;
-  const uint16_t* src = tile_src(i0, Pn);
-  load_tile<D>(src, i0 % tiles_per_bg, Pn, lane, av0);
-  for (int i = i0; i < i1; i += 2) {
-    if (i + 1 < i1) {  // next tile into the odd buffer, then the even tile's math
-      src = tile_src(i + 1, Pn);
-      load_tile<D>(src, (i + 1) % tiles_per_bg, Pn, lane, av1);
-    }
-    compute(i, av0);
-    if (i + 1 >= i1) break;
-    if (i + 2 < i1) {
-      src = tile_src(i + 2, Pn);
-      load_tile<D>(src, (i + 2) % tiles_per_bg, Pn, lane, av0);
-    }
-    compute(i + 1, av1);
   }
-  if (bad) set_err(c.err, KVQ_DERR_FP16_RANGE);
+
+  if (i0 < i1) {
+    QFrag<D, BF16> qf;
+    int cur_bg = -1, P = 0;
+    float* out = nullptr;
+    bool bad = false;
+    uint4 av0[2][D / 32], av1[2][D / 32];  // double buffer (compile-time indexed)
+
+    // where tile item i lives
+    auto tile_src = [&](int i, int& Pn) -> const uint16_t* {
+      const int bg = i / tiles_per_bg;
+      const int L = c.seq_len[bg / c.Hkv];
+      Pn = min((L + kPage - 1) / kPage, c.max_pages);
+      return c.summary + (size_t)bg * c.max_pages * D;
+    };
+    auto compute = [&](int i, const uint4 (&av)[2][D / 32]) {
+      const int bg = i / tiles_per_bg, tile = i % tiles_per_bg;
+      if (bg != cur_bg) {  // new (b, g): its query fragments (hi + lo)
+        cur_bg = bg;
+        const int b = bg / c.Hkv, g = bg % c.Hkv;
+        const int L = c.seq_len[b];
+        P = min((L + kPage - 1) / kPage, c.max_pages);
+        out = scores + (size_t)bg * c.max_pages;
+        qf.load(q, c.Hq, c.G, b, g, lane, bad);
+      }
+      float m0, m1;
+      tile_scores<D, BF16>(av, qf, c.G, lane, m0, m1);
+      if (q4 == 0) {
+        const int p0 = tile * 16 + g8, p1 = p0 + 8;
+        if (p0 < c.max_pages) out[p0] = p0 < P ? m0 : -INFINITY;
+        if (p1 < c.max_pages) out[p1] = p1 < P ? m1 : -INFINITY;
+      }
+    };
+
+    int Pn;
+    const uint16_t* src = tile_src(i0, Pn);
+    load_tile<D>(src, i0 % tiles_per_bg, Pn, lane, av0);
+    for (int i = i0; i < i1; i += 2) {
+      if (i + 1 < i1) {  // next tile into the odd buffer, then the even tile's math
+        src = tile_src(i + 1, Pn);
+        load_tile<D>(src, (i + 1) % tiles_per_bg, Pn, lane, av1);
+      }
+      compute(i, av0);
+      if (i + 1 >= i1) break;
+      if (i + 2 < i1) {
+        src = tile_src(i + 2, Pn);
+        load_tile<D>(src, (i + 2) % tiles_per_bg, Pn, lane, av0);
+      }
+      compute(i + 1, av1);
+    }
+    if (bad) set_err(c.err, KVQ_DERR_FP16_RANGE);
+  }
+
+  if constexpr (FUSED) {
+    // count this CTA's tiles on each (b, g) it touched; the CTA completing one selects it
+    const int c0 = min(total, (int)blockIdx.x * kScoreWarps * per);
+    const int c1 = min(total, c0 + kScoreWarps * per);
+    __syncthreads();
+    if (c0 < c1) {
+      for (int bg = c0 / tiles_per_bg; bg <= (c1 - 1) / tiles_per_bg; ++bg) {
+        if (tid == 0) {  // the barrier orders every warp's score writes before this fence
+          const int n = min(c1, (bg + 1) * tiles_per_bg) - max(c0, bg * tiles_per_bg);
+          __threadfence();
+          const unsigned old = atomicAdd(&f.done[bg], static_cast<unsigned>(n));
+          s_unit = (old + static_cast<unsigned>(n) == static_cast<unsigned>(tiles_per_bg)) ? bg : -1;
+          if (s_unit >= 0) f.done[bg] = 0u;  // complete: free for the next call
+        }
+        __syncthreads();
+        if (s_unit == bg) {
+          __threadfence();
+          const int L = c.seq_len[bg / c.Hkv];
+          const int P = min((L + kPage - 1) / kPage, c.max_pages);
+          const float* sc = scores + (size_t)bg * c.max_pages;
+          uint32_t* keys = sel_smem;
+          bool nan_seen = false;
+          for (int p0 = tid; p0 < P; p0 += 4 * kScoreWarps * 32) {  // four loads in flight per thread
+            float v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int p = p0 + j * kScoreWarps * 32;
+              v[j] = p < P ? __ldcg(sc + p) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int p = p0 + j * kScoreWarps * 32;
+              if (p < P) keys[p] = order_key(v[j], nan_seen);
+            }
+          }
+          if (nan_seen) set_err(c.err, KVQ_DERR_NAN_SCORE);
+          __syncthreads();
+          struct SyncBar {
+            __device__ bool operator()() const {
+              __syncthreads();
+              return true;
+            }
+          } bar;
+          select_pages<kScoreWarps * 32>(keys, P, f.prm, f.sel + (size_t)bg * f.kmax, f.cnt + bg, f.kmax, c.err,
+                                         sel_smem + (c.max_pages + 3) / 4 * 4, sel_sh, tid, bar);
+        }
+        __syncthreads();
+      }
+    }
+  }
   griddep_launch_dependents();
 }
 
-template <int D, bool BF16>
-cudaError_t launch_d(const DevCache& c, const void* q, float* scores, cudaStream_t s) {
+template <int D, bool BF16, bool FUSED>
+cudaError_t launch_d(const DevCache& c, const void* q, float* scores, const ScoreSelect& f, cudaStream_t s) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
   const int tiles_per_bg = (c.max_pages + 15) / 16;
@@ -108,8 +197,15 @@ cudaError_t launch_d(const DevCache& c, const void* q, float* scores, cudaStream
   const long long warps = blocks_max * kScoreWarps;
   const int per = (int)((total + warps - 1) / warps);
   const long long blocks = (total + (long long)per * kScoreWarps - 1) / ((long long)per * kScoreWarps);
-  return launch_pdl(score_kernel<D, BF16>, dim3((unsigned)blocks), dim3(kScoreWarps * 32), 0, s, c,
-                    static_cast<const uint16_t*>(q), scores, tiles_per_bg, per);
+  size_t smem = 0;
+  if (FUSED) {
+    smem = ((size_t)(c.max_pages + 3) / 4 * 4 + kSelScratchWords) * sizeof(uint32_t);
+    const cudaError_t e =
+        cudaFuncSetAttribute(score_kernel<D, BF16, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_pdl(score_kernel<D, BF16, FUSED>, dim3((unsigned)blocks), dim3(kScoreWarps * 32), smem, s, c,
+                    static_cast<const uint16_t*>(q), scores, tiles_per_bg, per, f);
 }
 
 }  // namespace
@@ -117,8 +213,21 @@ cudaError_t launch_d(const DevCache& c, const void* q, float* scores, cudaStream
 cudaError_t launch_scores(const DevCache& c, const void* q, float* scores, cudaStream_t s) {
   if (c.G > kMaxG) return cudaErrorInvalidValue;
   const bool bf = c.dtype == KVQ_DT_BF16;
-  if (c.D == 128) return bf ? launch_d<128, true>(c, q, scores, s) : launch_d<128, false>(c, q, scores, s);
-  if (c.D == 64) return bf ? launch_d<64, true>(c, q, scores, s) : launch_d<64, false>(c, q, scores, s);
+  const ScoreSelect f{};
+  if (c.D == 128) return bf ? launch_d<128, true, false>(c, q, scores, f, s) : launch_d<128, false, false>(c, q, scores, f, s);
+  if (c.D == 64) return bf ? launch_d<64, true, false>(c, q, scores, f, s) : launch_d<64, false, false>(c, q, scores, f, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_score_select(const DevCache& c, const int32_t* pos, const void* k_new, const void* v_new,
+                                const void* q, const kvq_select_params& prm, float* scores, int32_t* sel,
+                                int32_t* cnt, int kmax, unsigned* done, cudaStream_t s) {
+  if (c.G > kMaxG) return cudaErrorInvalidValue;
+  const bool bf = c.dtype == KVQ_DT_BF16;
+  const ScoreSelect f{pos, static_cast<const uint16_t*>(k_new), static_cast<const uint16_t*>(v_new), prm, sel, cnt,
+                      kmax, done};
+  if (c.D == 128) return bf ? launch_d<128, true, true>(c, q, scores, f, s) : launch_d<128, false, true>(c, q, scores, f, s);
+  if (c.D == 64) return bf ? launch_d<64, true, true>(c, q, scores, f, s) : launch_d<64, false, true>(c, q, scores, f, s);
   return cudaErrorInvalidValue;
 }
 

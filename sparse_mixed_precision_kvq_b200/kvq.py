@@ -35,7 +35,7 @@ DERR_NONFINITE, DERR_TIMEOUT, DERR_BAD_POS = 0x10, 0x20, 0x40
 EXPORTS = ["kvq_chunk_bytes", "kvq_status_string", "kvq_append", "kvq_build_pages", "kvq_page_scores",
            "kvq_select_topk", "kvq_workspace_size", "kvq_sparse_decode_attn", "kvq_dequant_page",
            "kvq_sparse_decode_attn_noalloc", "kvq_noalloc_scratch_bytes", "kvq_workspace_init",
-           "kvq_step_workspace_size", "kvq_decode_step"]
+           "kvq_step_workspace_size", "kvq_decode_step", "kvq_score_select"]
 
 
 class KvqCache(ctypes.Structure):
@@ -69,8 +69,10 @@ _lib.kvq_step_workspace_size.argtypes = [_P, c_int32, POINTER(c_size_t)]
 _lib.kvq_decode_step.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, POINTER(SelectParams), c_void_p,
                                  c_void_p, c_void_p, c_int32, c_float, c_void_p, c_void_p, c_void_p, c_size_t,
                                  c_void_p]
+_lib.kvq_score_select.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, POINTER(SelectParams), c_void_p,
+                                  c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]
 for _f in EXPORTS[2:9] + ["kvq_sparse_decode_attn_noalloc", "kvq_workspace_init", "kvq_step_workspace_size",
-                          "kvq_decode_step"]:
+                          "kvq_decode_step", "kvq_score_select"]:
     getattr(_lib, _f).restype = c_int32
 
 
@@ -150,6 +152,15 @@ def kvq_decode_step(cache, pos, k_new, v_new, q, params: SelectParams, scores, s
                                 _ptr(scores), _ptr(sel), _ptr(cnt), kmax, sm_scale, _ptr(out), _ptr(lse),
                                 _ptr(workspace), int(workspace.numel() * workspace.element_size()),
                                 _stream(stream)), "kvq_decode_step")
+
+
+def kvq_score_select(cache, pos, k_new, v_new, q, params: SelectParams, scores, sel, cnt, kmax: int, workspace,
+                     stream=None):
+    """kvq_append (if ``pos`` is not None) + kvq_page_scores + kvq_select_topk in one launch."""
+    _check(_lib.kvq_score_select(cache.ref(), _ptr(pos), _ptr(k_new), _ptr(v_new), _ptr(q), ctypes.byref(params),
+                                 _ptr(scores), _ptr(sel), _ptr(cnt), kmax, _ptr(workspace),
+                                 int(workspace.numel() * workspace.element_size()), _stream(stream)),
+           "kvq_score_select")
 
 
 def kvq_sparse_decode_attn_noalloc(cache, q, sel, cnt, kmax: int, sm_scale: float, out, lse, stream=None):
@@ -313,6 +324,16 @@ class DecodeStep:
         self.append()
         self.scores_()
         self.select()
+        self.attend()
+
+    def score_select(self):
+        kvq_score_select(self.cache, self.pos if self.w.append else None, self.k_new if self.w.append else None,
+                         self.v_new if self.w.append else None, self.q, self.params, self.scores, self.sel, self.cnt,
+                         self.kmax, self.ws)
+
+    def run_two(self):
+        """The same step as ``run()`` in two launches: kvq_score_select, kvq_sparse_decode_attn."""
+        self.score_select()
         self.attend()
 
     def run_fused(self):

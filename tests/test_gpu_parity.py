@@ -45,21 +45,27 @@ def _run(kvq, w, fused=False):
     cache = kvq.cache_from_workload(w)
     pre = snapshot(cache)
     step = kvq.DecodeStep(w, cache)
-    step.run_fused() if fused else step.run()
+    if fused == "two":
+        step.run_two()
+    elif fused:
+        step.run_fused()
+    else:
+        step.run()
     torch.cuda.synchronize()
     post = snapshot(cache)
     return cache, step, pre, post
 
 
-PATHS = ["calls", "fused"]
+PATHS = ["calls", "fused", "two"]
 
 
 @pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("name", list(VARIANTS))
 def test_step_matches_oracle(kvq, name, path):
-    """The four calls, and the one-launch kvq_decode_step, against the oracle."""
+    """The four calls, the two-launch kvq_score_select + attention, and the one-launch
+    kvq_decode_step, against the oracle."""
     w = VARIANTS[name]()
-    cache, step, pre, post = _run(kvq, w, fused=path == "fused")
+    cache, step, pre, post = _run(kvq, w, fused={"calls": False, "fused": True, "two": "two"}[path])
     assert cache.err_bits() == 0, hex(cache.err_bits())
     q, kn, vn = query_and_new(w)
     scores = step.scores.cpu().numpy()
@@ -84,7 +90,7 @@ def test_step_matches_oracle(kvq, name, path):
                 check_summary(post, sh, b, g, P)
                 assert np.array_equal(post["ksum"][b, g], sh.ksum)
             G = w.G
-            check_scores(scores[b, g], r["scores"], q[b, g * G:(g + 1) * G], sh.summary, P, tail=path == "calls")
+            check_scores(scores[b, g], r["scores"], q[b, g * G:(g + 1) * G], sh.summary, P, tail=path != "fused")
             got_sel = sel[b, g, :cnt[b, g]]
             if check_selection(got_sel, r["sel"], r["scores"], w, P):
                 n_same += 1
@@ -201,7 +207,7 @@ def test_edge_cases_empty_short_and_overlapping(kvq, path):
     append that opens a page, and a ragged last page."""
     w = W.make("c4", B=6, Hq=8, Hkv=2, lens=np.array([0, 1, 15, 16, 40, 200]), append=True,
                n_sink=3, n_recent=3, k_abs=2, tier_fracs=ALL_TIERS)
-    cache, step, pre, post = _run(kvq, w, fused=path == "fused")
+    cache, step, pre, post = _run(kvq, w, fused={"calls": False, "fused": True, "two": "two"}[path])
     assert cache.err_bits() == 0
     q, kn, vn = query_and_new(w)
     out = out_to_f64(step.out, w.dtype)
@@ -219,7 +225,7 @@ def test_edge_cases_empty_short_and_overlapping(kvq, path):
 @pytest.mark.parametrize("path", PATHS)
 def test_empty_selection_gives_zero_output(kvq, path):
     w = W.make("c4", B=3, Hq=8, Hkv=2, lens=np.array([0, 35, 0]), append=False)
-    cache, step, pre, post = _run(kvq, w, fused=path == "fused")
+    cache, step, pre, post = _run(kvq, w, fused={"calls": False, "fused": True, "two": "two"}[path])
     out = step.out.float().cpu().numpy()
     lse = step.lse.cpu().numpy()
     assert np.all(out[0] == 0) and np.all(out[2] == 0)
@@ -345,7 +351,7 @@ def test_long_context_many_pages(kvq, path):
     """A sequence of 8193 pages (131072 tokens + 1, as in the long-context workload): the
     selection keeps all of its keys on chip; pages, selection and output as the oracle's."""
     w = W.make("c3", lens=np.array([131072]), Hq=8, Hkv=2)
-    cache, step, pre, post = _run(kvq, w, fused=path == "fused")
+    cache, step, pre, post = _run(kvq, w, fused={"calls": False, "fused": True, "two": "two"}[path])
     assert cache.err_bits() == 0, hex(cache.err_bits())
     q, kn, vn = query_and_new(w)
     sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
@@ -356,3 +362,28 @@ def test_long_context_many_pages(kvq, path):
         assert check_selection(sel[0, g, :cnt[0, g]], r["sel"], r["scores"], w, r["P"])
         for i in range(w.G):
             check_output(out[0, g * w.G + i], r["out"][i], f"long g={g}", w.dtype)
+
+
+@pytest.mark.parametrize("name", ["c1", "c4", "g2_alltiers"])
+def test_score_select_equals_calls(kvq, name):
+    """kvq_score_select (append + scores + selection in one launch) leaves the same cache
+    bytes, scores, selection and (through the same attention call) outputs as the calls."""
+    w = VARIANTS[name]()
+    outs = []
+    for two in (False, True):
+        cache = kvq.cache_from_workload(w)
+        step = kvq.DecodeStep(w, cache)
+        step.run_two() if two else step.run()
+        torch.cuda.synchronize()
+        outs.append((snapshot(cache), step.scores.clone(), step.sel.clone(), step.cnt.clone(), step.out.clone()))
+        assert cache.err_bits() == 0, hex(cache.err_bits())
+    (s0, sc0, sel0, cnt0, o0), (s1, sc1, sel1, cnt1, o1) = outs
+    for t, (p0, p1) in enumerate(zip(s0["pools"], s1["pools"])):
+        assert (p0 is None) == (p1 is None) and (p0 is None or np.array_equal(p0, p1)), t
+    for k in ("bt", "summary", "ksum"):
+        assert np.array_equal(s0[k], s1[k]), k
+    assert torch.equal(sc0, sc1) and torch.equal(cnt0, cnt1) and torch.equal(o0, o1)
+    c = cnt0.cpu().numpy()
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            assert torch.equal(sel0[b, g, :c[b, g]], sel1[b, g, :c[b, g]])
