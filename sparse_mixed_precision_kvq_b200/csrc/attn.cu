@@ -198,7 +198,7 @@ __device__ inline void final_combine(const AttnArgs& a, uint16_t* out, float* ls
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool ONLY16>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t* __restrict__ out,
                                                            float* __restrict__ lse) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
     }
     if (!failed) {
       const PageMeta pm = pmeta[slot];
-      if (pm.tier >= 0) process_page<D, BF16>(ring_c + pm.ring_off, pm.tier, pm.nv, lane, a.scale_log2, st);
+      if (pm.tier >= 0) process_page<D, BF16, ONLY16>(ring_c + pm.ring_off, pm.tier, pm.nv, lane, a.scale_log2, st);
       tail = pm.end;  // everything before this page's end is free again
     }
     __syncwarp();
@@ -440,13 +440,22 @@ constexpr size_t attn_smem_fixed() {
   return (size_t)kWarps * kRing + kWarps * kNBar * 8 + kWarps * kNBar * sizeof(PageMeta);
 }
 
-template <int D, bool BF16>
-cudaError_t launch_attn_d(const AttnArgs& a, uint16_t* out, float* lse, cudaStream_t s) {
+template <int D, bool BF16, bool ONLY16>
+cudaError_t launch_attn_v(const AttnArgs& a, uint16_t* out, float* lse, cudaStream_t s) {
   const int BH = a.c.B * a.c.Hkv;
   const size_t smem = attn_smem_fixed<D>() + (size_t)(BH + 1) * 4;
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(attn_kernel<D, BF16, ONLY16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_kernel<D, BF16>, dim3(a.num_ctas), dim3(kThreads), smem, s, a, out, lse);
+  return launch_pdl(attn_kernel<D, BF16, ONLY16>, dim3(a.num_ctas), dim3(kThreads), smem, s, a, out, lse);
+}
+
+// A cache whose only pool is the 16-bit one runs the 16-bit-only kernel.
+template <int D, bool BF16>
+cudaError_t launch_attn_d(const AttnArgs& a, uint16_t* out, float* lse, cudaStream_t s) {
+  bool only16 = true;
+  for (int t = 1; t < kNumTiers; ++t) only16 = only16 && a.c.pool[t] == nullptr;
+  return only16 ? launch_attn_v<D, BF16, true>(a, out, lse, s) : launch_attn_v<D, BF16, false>(a, out, lse, s);
 }
 
 }  // namespace

@@ -239,17 +239,24 @@ __device__ __forceinline__ void pv_page(const unsigned char* base, int lane, War
   }
 }
 
-template <int D, bool BF16>
+// ONLY16: the cache has 16-bit pages only (no code for the other tiers is generated, which
+// keeps the kernel's instruction footprint small).
+template <int D, bool BF16, bool ONLY16 = false>
 __device__ __forceinline__ void process_page(const unsigned char* base, int tier, int nv, int lane, float scale_log2,
                                     WarpState<D>& st) {
   constexpr int KS = D / 16, NG = D / 32;
   float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-  switch (tier) {
-    case KVQ_TIER_16: qk_page<KVQ_TIER_16, D, BF16>(base, lane, st, sacc); break;
-    case KVQ_TIER_I8: qk_page<KVQ_TIER_I8, D, BF16>(base, lane, st, sacc); break;
-    case KVQ_TIER_I4: qk_page<KVQ_TIER_I4, D, BF16>(base, lane, st, sacc); break;
-    case KVQ_TIER_I2: qk_page<KVQ_TIER_I2, D, BF16>(base, lane, st, sacc); break;
-    default: qk_page<KVQ_TIER_I1, D, BF16>(base, lane, st, sacc); break;
+  if constexpr (ONLY16) {
+    tier = KVQ_TIER_16;
+    qk_page<KVQ_TIER_16, D, BF16>(base, lane, st, sacc);
+  } else {
+    switch (tier) {
+      case KVQ_TIER_16: qk_page<KVQ_TIER_16, D, BF16>(base, lane, st, sacc); break;
+      case KVQ_TIER_I8: qk_page<KVQ_TIER_I8, D, BF16>(base, lane, st, sacc); break;
+      case KVQ_TIER_I4: qk_page<KVQ_TIER_I4, D, BF16>(base, lane, st, sacc); break;
+      case KVQ_TIER_I2: qk_page<KVQ_TIER_I2, D, BF16>(base, lane, st, sacc); break;
+      default: qk_page<KVQ_TIER_I1, D, BF16>(base, lane, st, sacc); break;
+    }
   }
   const int t0 = lane >> 2, t1 = t0 + 8;
   float x[4];
@@ -287,6 +294,10 @@ __device__ __forceinline__ void process_page(const unsigned char* base, int tier
     st.zacc[gi][1] *= a1;
   }
   const unsigned char* vbase = base + chunk_bytes(tier, D);
+  if constexpr (ONLY16) {
+    pv_page<KVQ_TIER_16, D, BF16>(vbase, lane, st, p);
+    return;
+  }
   switch (tier) {
     case KVQ_TIER_16: pv_page<KVQ_TIER_16, D, BF16>(vbase, lane, st, p); break;
     case KVQ_TIER_I8: pv_page<KVQ_TIER_I8, D, BF16>(vbase, lane, st, p); break;
