@@ -14,8 +14,6 @@
 namespace kvq {
 namespace {
 
-constexpr int kSelThreads = 512;
-
 struct SyncBar {
   __device__ bool operator()() const {
     __syncthreads();
@@ -23,9 +21,11 @@ struct SyncBar {
   }
 };
 
-__global__ void __launch_bounds__(kSelThreads) select_kernel(DevCache c, const float* __restrict__ scores,
-                                                             kvq_select_params prm, int32_t* __restrict__ sel,
-                                                             int32_t* __restrict__ cnt, int kmax) {
+// NT threads per (b, g): 512, or 1024 when a few long sequences leave most SMs idle.
+template <int NT>
+__global__ void __launch_bounds__(NT) select_kernel(DevCache c, const float* __restrict__ scores,
+                                                   kvq_select_params prm, int32_t* __restrict__ sel,
+                                                   int32_t* __restrict__ cnt, int kmax) {
   extern __shared__ uint32_t keys[];  // [max_pages]
   __shared__ SelShared sh;
   __shared__ uint32_t scratch[kSelScratchWords];
@@ -37,30 +37,40 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(DevCache c, const f
   const int P = min((L + kPage - 1) / kPage, c.max_pages);
   const float* sc = scores + (size_t)bg * c.max_pages;
   bool nan_seen = false;
-  for (int p0 = tid; p0 < P; p0 += 4 * kSelThreads) {  // four loads in flight per thread
+  for (int p0 = tid; p0 < P; p0 += 4 * NT) {  // four loads in flight per thread
     float v[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = p0 + j * kSelThreads < P ? sc[p0 + j * kSelThreads] : 0.f;
+    for (int j = 0; j < 4; ++j) v[j] = p0 + j * NT < P ? sc[p0 + j * NT] : 0.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-      if (p0 + j * kSelThreads < P) keys[p0 + j * kSelThreads] = order_key(v[j], nan_seen);
+      if (p0 + j * NT < P) keys[p0 + j * NT] = order_key(v[j], nan_seen);
   }
   if (nan_seen) set_err(c.err, KVQ_DERR_NAN_SCORE);
   __syncthreads();
   SyncBar bar;
-  select_pages<kSelThreads>(keys, P, prm, sel + (size_t)bg * kmax, cnt + bg, kmax, c.err, scratch, sh, tid, bar);
+  select_pages<NT>(keys, P, prm, sel + (size_t)bg * kmax, cnt + bg, kmax, c.err, scratch, sh, tid, bar);
   griddep_launch_dependents();
+}
+
+template <int NT>
+cudaError_t launch_select_t(const DevCache& c, const float* scores, const kvq_select_params& prm, int32_t* sel,
+                            int32_t* cnt, int kmax, cudaStream_t s) {
+  const size_t smem = (size_t)c.max_pages * sizeof(uint32_t);
+  // static (histogram scratch) + dynamic (keys) shared memory may pass the 48 KB default
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(select_kernel<NT>, dim3(c.B * c.Hkv), dim3(NT), smem, s, c, scores, prm, sel, cnt, kmax);
 }
 
 }  // namespace
 
 cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_select_params& prm,
                           int32_t* sel, int32_t* cnt, int kmax, cudaStream_t s) {
-  const size_t smem = (size_t)c.max_pages * sizeof(uint32_t);
-  // static (histogram scratch) + dynamic (keys) shared memory may pass the 48 KB default
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(select_kernel, dim3(c.B * c.Hkv), dim3(kSelThreads), smem, s, c, scores, prm, sel, cnt, kmax);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  const bool wide = (long long)c.B * c.Hkv * 4 <= attn_num_ctas(dev) && c.max_pages >= 4096;
+  return wide ? launch_select_t<1024>(c, scores, prm, sel, cnt, kmax, s)
+              : launch_select_t<512>(c, scores, prm, sel, cnt, kmax, s);
 }
 
 }  // namespace kvq

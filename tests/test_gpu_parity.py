@@ -315,12 +315,14 @@ def test_fused_step_kmax_truncation_flag(kvq):
     assert torch.isfinite(step.out.float()).all()
 
 
-def test_select_special_values_and_wide_ranges(kvq):
+@pytest.mark.parametrize("P_cap", [3000, 5000])
+def test_select_special_values_and_wide_ranges(kvq, P_cap):
     """Infinite scores, a range near the fp32 limit, all-equal scores, denormals and a
-    large random batch: the selection is the oracle's exactly (ties on page index)."""
+    large random batch: the selection is the oracle's exactly (ties on page index).
+    5000 pages for 24 (b, kv head) pairs runs the 1024-thread selection."""
     from oracle.select import select
     rng = np.random.default_rng(7)
-    B, Hkv, P_cap = 12, 2, 3000
+    B, Hkv = 12, 2
     w = W.make("c4", B=B, Hq=8, Hkv=Hkv, lens=np.full(B, 16 * P_cap), append=False)
     cache = kvq.cache_from_workload(w)
     sc = rng.normal(0, 3, (B, Hkv, w.max_pages)).astype(np.float32)
