@@ -60,3 +60,72 @@ def kth_margin(scores: np.ndarray, P: int, k_abs: int, k_frac_bp: int, n_sink: i
     s = np.sort(c)[::-1]
     a, b = s[k - 1], s[k]
     return float((a - b) / max(abs(a), abs(b), 1e-30))
+
+
+# ----------------------------------------------------------------------------- coverage
+# AMASS "Quickstart" (``coverage=0.95``: the nucleus variant of the selection).  The pages
+# do not give the mass estimate; the plainest reading, used here: a page's attention mass
+# is estimated from its score as ``n_p * exp(sm_scale * s_p)`` (n_p = the page's valid
+# tokens, the score standing in for each token's logit), normalised over all pages of the
+# (sequence, kv head).  The forced pages are attended and count as covered; candidates are
+# then added by estimated mass (larger first, lower page index first on ties) until the
+# covered mass reaches ``coverage`` of the total.  A NaN score has mass 0.
+
+def page_masses(scores: np.ndarray, P: int, L: int, sm_scale: float) -> np.ndarray:
+    """Estimated mass of pages 0..P-1 (fp64), relative to the largest score's page."""
+    s = np.asarray(scores[:P], dtype=np.float64)
+    n = np.full(P, 16.0)
+    if P:
+        n[P - 1] = float(L - 16 * (P - 1))
+    finite = s[~np.isnan(s)]
+    if finite.size == 0:
+        return np.zeros(P)
+    smax = float(finite.max())
+    m = np.zeros(P)
+    for p in range(P):
+        if not math.isnan(s[p]):
+            m[p] = n[p] * math.exp(sm_scale * (s[p] - smax))
+    return m
+
+
+def select_coverage(scores: np.ndarray, P: int, L: int, sm_scale: float, coverage: float, n_sink: int,
+                    n_recent: int) -> np.ndarray:
+    """Coverage selection of one (sequence, kv head), ascending, int64."""
+    F = forced_pages(P, n_sink, n_recent)
+    m = page_masses(scores, P, L, sm_scale)
+    total = math.fsum(m)
+    covered = math.fsum(m[p] for p in F)
+    target = coverage * total
+    order = sorted((p for p in range(P) if p not in F), key=lambda p: (-m[p], p))
+    chosen = []
+    for p in order:
+        if covered >= target:
+            break
+        chosen.append(p)
+        covered += m[p]
+    return np.array(sorted(F | set(chosen)), dtype=np.int64)
+
+
+def coverage_margin(scores: np.ndarray, P: int, L: int, sm_scale: float, coverage: float, n_sink: int,
+                    n_recent: int) -> float:
+    """How far the coverage cut is from being decided otherwise: the smaller of the relative
+    gap between the last chosen and the first unchosen candidate masses and the relative
+    distance of the covered mass (before the last chosen page) from the target."""
+    F = forced_pages(P, n_sink, n_recent)
+    m = page_masses(scores, P, L, sm_scale)
+    total = math.fsum(m)
+    target = coverage * total
+    order = sorted((p for p in range(P) if p not in F), key=lambda p: (-m[p], p))
+    covered = math.fsum(m[p] for p in F)
+    k = 0
+    while k < len(order) and covered < target:
+        covered += m[order[k]]
+        k += 1
+    out = math.inf
+    if 0 < k < len(order):
+        a, b = m[order[k - 1]], m[order[k]]
+        out = min(out, (a - b) / max(a, 1e-300))
+    if total > 0:
+        before = covered - (m[order[k - 1]] if k else 0.0)
+        out = min(out, abs(target - before) / total, abs(covered - target) / total)
+    return float(out)
