@@ -180,7 +180,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     torch.cuda.set_device(dev)
     w = rank_workload(args.config, rank, args.batch)
     cache = kvq.cache_from_workload(w, device=dev)
-    step = kvq.DecodeStep(w, cache, device=dev)
+    step = kvq.DecodeStep(w, cache, device=dev, coverage=args.coverage)
     tier_tbl, _, _ = w.slot_map()
     flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -327,6 +327,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
         "config": {"workload": f"{args.config}: {DESCR[args.config]}", "batch_per_gpu": w.B,
                    "context": int(w.lens.max()), "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
                    "selected_pages": int(cnt.sum()),
+                   "selection": "budget" if args.coverage is None else f"coverage {args.coverage}",
                    "l2": f"flushed ({args.flush_mib} MiB write) before every timed step",
                    "parallelism": f"replicas x{world} (independent batches)"},
         "step_hbm": {"bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3) / 1e9,
@@ -444,6 +445,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default="c1", choices=sorted(DESCR))
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--coverage", type=float, default=None,
+                    help="coverage (nucleus) selection at this mass fraction instead of the workload's budget "
+                         "(four-call path only)")
     ap.add_argument("--path", default="calls", choices=["calls", "two", "fused"],
                     help="the four separate calls, kvq_score_select + attention, or one kvq_decode_step launch")
     ap.add_argument("--dense", action="store_true", help="also time attention over every page")
@@ -454,6 +458,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.coverage is not None and args.path != "calls":
+        ap.error("--coverage runs on the four-call path")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

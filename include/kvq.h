@@ -118,6 +118,11 @@ typedef struct {
   int32_t k_frac_bp;  /* fraction in basis points: k = ceil(P * k_frac_bp / 10000) per sequence */
   int32_t n_sink;     /* first n_sink pages always attended (in addition to k) */
   int32_t n_recent;   /* last n_recent pages always attended (in addition to k) */
+  int32_t coverage_ppm; /* > 0: coverage selection instead of k (AMASS "Quickstart" coverage):
+                           the fewest best pages whose estimated mass, with the forced pages',
+                           reaches coverage_ppm / 1e6 of the total; mass of page p estimated
+                           as n_p * exp(sm_scale * s_p), n_p its valid tokens; ties: lower page */
+  float sm_scale;     /* softmax scale of the mass estimate (coverage only) */
 } kvq_select_params;
 
 /* Bytes of one chunk (one page, one kv head, K or V) of a tier; 0 for a bad tier/D. */
@@ -175,6 +180,8 @@ kvq_status kvq_page_scores(const kvq_cache* cache, const void* q, float* scores,
  *          (score descending, lower page index first on ties, NaN lowest), ascending.
  *  cnt     device [B][Hkv] int32 out: entries written to sel (<= kmax).
  *  kmax    row length of sel; a longer selection is truncated and flagged.
+ *  With params->coverage_ppm > 0 the k best are replaced by the coverage choice; the
+ *  candidates of a sequence (pages minus forced ones) must number at most 8192.
  */
 kvq_status kvq_select_topk(const kvq_cache* cache, const float* scores,
                            const kvq_select_params* params, int32_t* sel, int32_t* cnt,
@@ -243,6 +250,7 @@ size_t kvq_noalloc_scratch_bytes(void);
  * tile counters at its head; the call leaves them zero).  B*Hkv <= 8192,
  * max_pages <= 51200.
  */
+/* (coverage selection is not supported here: KVQ_ERR_UNSUPPORTED) */
 kvq_status kvq_score_select(const kvq_cache* cache, const int32_t* pos, const void* k_new,
                             const void* v_new, const void* q, const kvq_select_params* params,
                             float* scores, int32_t* sel, int32_t* cnt, int32_t kmax, void* workspace,
@@ -268,7 +276,8 @@ kvq_status kvq_step_workspace_size(const kvq_cache* cache, int32_t kmax, size_t*
  *            (entries past that are not written).
  *  workspace device scratch of at least kvq_step_workspace_size() bytes, prepared once
  *            with kvq_workspace_init.
- *  Returns KVQ_ERR_UNSUPPORTED when B*Hkv > 8184 or the per-CTA tables and selection keys
+ *  Returns KVQ_ERR_UNSUPPORTED for coverage selection, when B*Hkv > 8184, or when the
+ *  per-CTA tables and selection keys
  *  (4 * (3B + max_pages) bytes) leave too little shared memory for the page ring.
  */
 kvq_status kvq_decode_step(const kvq_cache* cache, const int32_t* pos, const void* k_new,

@@ -148,6 +148,11 @@ kvq_status kvq_select_topk(const kvq_cache* cache, const float* scores, const kv
   if (scores == nullptr || params == nullptr || sel == nullptr || cnt == nullptr || kmax < 1)
     return KVQ_ERR_INVALID_ARG;
   if ((size_t)c.max_pages * 4 > 200 * 1024) return KVQ_ERR_UNSUPPORTED;  // keys in shared memory
+  if (params->coverage_ppm > 0) {
+    if (params->coverage_ppm > 1000000 || !(params->sm_scale > 0.f)) return KVQ_ERR_INVALID_ARG;
+    const int n = coverage_sort_size(c, *params);
+    if (n == 0 || ((size_t)c.max_pages + 1) / 2 * 8 + (size_t)n * 12 > 200 * 1024) return KVQ_ERR_UNSUPPORTED;
+  }
   return cuda_status(launch_select(c, scores, *params, sel, cnt, kmax, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -187,6 +192,7 @@ kvq_status kvq_score_select(const kvq_cache* cache, const int32_t* pos, const vo
     return KVQ_ERR_INVALID_ARG;
   if (pos != nullptr && (k_new == nullptr || v_new == nullptr)) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
+  if (params->coverage_ppm > 0) return KVQ_ERR_UNSUPPORTED;
   if ((long long)c.B * c.Hkv > (long long)(kCounterBytes / 4 - kScoreSelectCounterWord)) return KVQ_ERR_UNSUPPORTED;
   if ((size_t)c.max_pages * 4 > 200 * 1024) return KVQ_ERR_UNSUPPORTED;  // keys in shared memory
   if (ws_bytes < kCounterBytes) return KVQ_ERR_WORKSPACE;
@@ -216,6 +222,7 @@ kvq_status kvq_decode_step(const kvq_cache* cache, const int32_t* pos, const voi
     return KVQ_ERR_INVALID_ARG;
   if (pos != nullptr && (k_new == nullptr || v_new == nullptr)) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(workspace) || !aligned16(q) || !(sm_scale > 0.f)) return KVQ_ERR_INVALID_ARG;
+  if (params->coverage_ppm > 0) return KVQ_ERR_UNSUPPORTED;
   if (reinterpret_cast<uintptr_t>(c.summary) % 16 != 0) return KVQ_ERR_INVALID_ARG;
   if (!step_supported(c)) return KVQ_ERR_UNSUPPORTED;
   if (ws_bytes < step_workspace_bytes(c, kmax)) return KVQ_ERR_WORKSPACE;

@@ -142,6 +142,7 @@ cudaError_t launch_score_select(const DevCache& c, const int32_t* pos, const voi
 constexpr size_t kScoreSelectCounterWord = 8192;  // workspace word of the per-(b, g) tile counters
 cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_select_params& prm,
                           int32_t* sel, int32_t* cnt, int kmax, cudaStream_t s);
+int coverage_sort_size(const DevCache& c, const kvq_select_params& prm);
 size_t attn_workspace_bytes(const DevCache& c, int num_ctas);
 int attn_num_ctas(int device);
 cudaError_t launch_attn(const DevCache& c, const void* q, const int32_t* sel, const int32_t* cnt, int kmax,

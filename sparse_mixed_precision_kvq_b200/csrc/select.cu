@@ -25,8 +25,9 @@ struct SyncBar {
 template <int NT>
 __global__ void __launch_bounds__(NT) select_kernel(DevCache c, const float* __restrict__ scores,
                                                    kvq_select_params prm, int32_t* __restrict__ sel,
-                                                   int32_t* __restrict__ cnt, int kmax) {
-  extern __shared__ uint32_t keys[];  // [max_pages]
+                                                   int32_t* __restrict__ cnt, int kmax, int ncov) {
+  // keys [max_pages, rounded to 2 words]; coverage: then mass keys [ncov] (u64), pages [ncov]
+  extern __shared__ __align__(16) uint32_t keys[];
   __shared__ SelShared sh;
   __shared__ uint32_t scratch[kSelScratchWords];
   const int bg = blockIdx.x;
@@ -48,29 +49,47 @@ __global__ void __launch_bounds__(NT) select_kernel(DevCache c, const float* __r
   if (nan_seen) set_err(c.err, KVQ_DERR_NAN_SCORE);
   __syncthreads();
   SyncBar bar;
-  select_pages<NT>(keys, P, prm, sel + (size_t)bg * kmax, cnt + bg, kmax, c.err, scratch, sh, tid, bar);
+  if (prm.coverage_ppm > 0) {
+    unsigned long long* mkey = reinterpret_cast<unsigned long long*>(keys + (c.max_pages + 1) / 2 * 2);
+    uint32_t* mpage = reinterpret_cast<uint32_t*>(mkey + ncov);
+    select_coverage<NT>(keys, P, L, prm, mkey, mpage, scratch + kSelBitmapOff, sel + (size_t)bg * kmax, cnt + bg,
+                        kmax, c.err, sh, tid, bar);
+  } else {
+    select_pages<NT>(keys, P, prm, sel + (size_t)bg * kmax, cnt + bg, kmax, c.err, scratch, sh, tid, bar);
+  }
   griddep_launch_dependents();
 }
 
 template <int NT>
 cudaError_t launch_select_t(const DevCache& c, const float* scores, const kvq_select_params& prm, int32_t* sel,
-                            int32_t* cnt, int kmax, cudaStream_t s) {
-  const size_t smem = (size_t)c.max_pages * sizeof(uint32_t);
+                            int32_t* cnt, int kmax, int ncov, cudaStream_t s) {
+  const size_t smem = (size_t)(c.max_pages + 1) / 2 * 2 * sizeof(uint32_t) + (size_t)ncov * 12;
   // static (histogram scratch) + dynamic (keys) shared memory may pass the 48 KB default
   cudaError_t e = cudaFuncSetAttribute(select_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(select_kernel<NT>, dim3(c.B * c.Hkv), dim3(NT), smem, s, c, scores, prm, sel, cnt, kmax);
+  return launch_pdl(select_kernel<NT>, dim3(c.B * c.Hkv), dim3(NT), smem, s, c, scores, prm, sel, cnt, kmax, ncov);
 }
 
 }  // namespace
+
+// Sort slots coverage selection needs: a power of two >= the candidates of the longest
+// possible sequence (max_pages minus the forced pages); 0 if above kCovMaxCand.
+int coverage_sort_size(const DevCache& c, const kvq_select_params& prm) {
+  const int forced = max(prm.n_sink, 0) + max(prm.n_recent, 0);
+  const int nc = max(1, c.max_pages - min(forced, c.max_pages));
+  int n = 1;
+  while (n < nc) n <<= 1;
+  return n <= kCovMaxCand ? n : 0;
+}
 
 cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_select_params& prm,
                           int32_t* sel, int32_t* cnt, int kmax, cudaStream_t s) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
   const bool wide = (long long)c.B * c.Hkv * 4 <= attn_num_ctas(dev) && c.max_pages >= 4096;
-  return wide ? launch_select_t<1024>(c, scores, prm, sel, cnt, kmax, s)
-              : launch_select_t<512>(c, scores, prm, sel, cnt, kmax, s);
+  const int ncov = prm.coverage_ppm > 0 ? coverage_sort_size(c, prm) : 0;
+  return wide ? launch_select_t<1024>(c, scores, prm, sel, cnt, kmax, ncov, s)
+              : launch_select_t<512>(c, scores, prm, sel, cnt, kmax, ncov, s);
 }
 
 }  // namespace kvq

@@ -67,6 +67,7 @@ struct SelShared {
   int hist[256];  // radix fallback
   int scan[33];
   float wmin[32], wmax[32];
+  double dsum[33];
   uint32_t prefix;
   int rem;
   int ncand;
@@ -105,6 +106,32 @@ __device__ inline int sel_exclusive_scan(int v, SelShared& sh, int* total, int t
 // Score of an order key (inverse of order_key; key 0 stands for NaN).
 __device__ inline float key_score(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Write the pages of a bitmap (nwords words) in ascending order to out[0 .. min(n, kmax)),
+// min(n, kmax) to *cnt_out (thread 0); flags KVQ_DERR_KMAX if n > kmax.
+template <int NT, typename Bar>
+__device__ inline void emit_chosen(const uint32_t* chosen, int nwords, int32_t* out, int32_t* cnt_out, int kmax,
+                                   uint32_t* err, SelShared& sh, int tid, Bar& bar) {
+  const int WPT = (nwords + NT - 1) / NT;  // contiguous words per thread
+  const int w_lo = min(nwords, tid * WPT), w_hi = min(nwords, w_lo + WPT);
+  int nsel = 0;
+  for (int wd = w_lo; wd < w_hi; ++wd) nsel += __popc(chosen[wd]);
+  int total;
+  int off = sel_exclusive_scan<NT>(nsel, sh, &total, tid, bar);
+  for (int wd = w_lo; wd < w_hi; ++wd) {
+    unsigned m = chosen[wd];
+    while (m) {
+      const int b = __ffs(m) - 1;
+      m &= m - 1u;
+      if (off < kmax) out[off] = 32 * wd + b;
+      ++off;
+    }
+  }
+  if (tid == 0) {
+    *cnt_out = min(total, kmax);
+    if (total > kmax) set_err(err, KVQ_DERR_KMAX);
+  }
 }
 
 // Select among the P keys in shared memory (written, and a barrier passed, by the
@@ -345,23 +372,157 @@ __device__ inline void select_pages(const uint32_t* keys, int P, const kvq_selec
     }
     bar();
   }
-  int nsel = 0;
-  for (int wd = w_lo; wd < w_hi; ++wd) nsel += __popc(chosen[wd]);
-  int total;
-  int off = sel_exclusive_scan<NT>(nsel, sh, &total, tid, bar);
-  for (int wd = w_lo; wd < w_hi; ++wd) {
-    unsigned m = chosen[wd];
-    while (m) {
-      const int b = __ffs(m) - 1;
-      m &= m - 1u;
-      if (off < kmax) out[off] = 32 * wd + b;
-      ++off;
+  emit_chosen<NT>(chosen, nwords, out, cnt_out, kmax, err, sh, tid, bar);
+}
+
+// ----------------------------------------------------------------------------- coverage
+// AMASS "Quickstart" (coverage = 0.95, the nucleus variant of the selection).  A page's
+// attention mass is estimated from its score as n_p * exp(sm_scale * (s_p - s_max)) (fp64;
+// n_p its valid tokens; NaN -> 0); the forced pages count as covered, and candidates are
+// added by mass (larger first, lower page first on ties) until the covered mass reaches
+// coverage * the total.  The candidates are sorted in shared memory (bitonic, N a power of
+// two >= their count), the sorted masses scanned (fp64), and the chosen pages emitted
+// through the same bitmap as the top-k selection.
+
+constexpr int kCovMaxCand = 8192;  // candidates one CTA sorts in shared memory
+
+// Sum of one double per thread (fixed tree: the same order in every call).
+template <int NT, typename Bar>
+__device__ inline double sel_block_sum(double v, SelShared& sh, int tid, Bar& bar) {
+  constexpr int NW = NT / 32;
+  const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) sh.dsum[warp] = v;
+  bar();
+  double t = 0.0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) t += sh.dsum[w];
+  bar();
+  return t;
+}
+
+// Inclusive prefix sums of the doubles a[0..n) in place, contiguous chunks per thread.
+template <int NT, typename Bar>
+__device__ inline void sel_prefix_sum(double* a, int n, SelShared& sh, int tid, Bar& bar) {
+  const int lane = tid & 31, warp = tid >> 5;
+  const int per = (n + NT - 1) / NT;
+  const int lo = min(n, tid * per), hi = min(n, lo + per);
+  double run = 0.0;
+  for (int i = lo; i < hi; ++i) run += a[i];
+  double x = run;  // inclusive scan over threads
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh.dsum[warp] = x;
+  bar();
+  double before = x - run;
+  for (int w = 0; w < warp; ++w) before += sh.dsum[w];
+  for (int i = lo; i < hi; ++i) {
+    before += a[i];
+    a[i] = before;
+  }
+  bar();
+}
+
+// keys: the P order keys (scores) in shared memory; mkey/mpage: 2 * kCovMaxCand words
+// and kCovMaxCand words of shared memory; chosen: the bitmap area (ceil(P / 32) words).
+template <int NT, typename Bar>
+__device__ inline void select_coverage(const uint32_t* keys, int P, int L, const kvq_select_params& prm,
+                                       unsigned long long* mkey, uint32_t* mpage, uint32_t* chosen, int32_t* out,
+                                       int32_t* cnt_out, int kmax, uint32_t* err, SelShared& sh, int tid, Bar& bar) {
+  constexpr int NW = NT / 32;
+  const int lane = tid & 31, warp = tid >> 5;
+  const SelectSplit sp = select_split(P, prm);
+  const int ns = sp.ns, rs = sp.rs, nC = sp.nC;
+  auto is_cand = [&](int p) { return p >= ns && p < rs; };
+  const int nwords = (P + 31) / 32;
+  // 1) largest finite score
+  float hi = -INFINITY;
+  for (int p = tid; p < P; p += NT)
+    if (keys[p] != 0u) hi = fmaxf(hi, key_score(keys[p]));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  if (lane == 0) sh.wmax[warp] = hi;
+  bar();
+  float smax = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) smax = fmaxf(smax, sh.wmax[w]);
+  const double scale = static_cast<double>(prm.sm_scale);
+  auto mass = [&](int p) -> double {
+    const uint32_t k = keys[p];
+    if (k == 0u || !(smax > -INFINITY)) return 0.0;
+    const double n = p == P - 1 ? static_cast<double>(L - kPage * (P - 1)) : static_cast<double>(kPage);
+    return n * exp(scale * (static_cast<double>(key_score(k)) - static_cast<double>(smax)));
+  };
+  // 2) the candidates' (mass, page) in sort slots 0..nC-1, padding after; the totals
+  int N = 1;
+  while (N < nC) N <<= 1;
+  double tot = 0.0, forced = 0.0;
+  for (int p = tid; p < P; p += NT) {
+    const double m = mass(p);
+    tot += m;
+    if (!is_cand(p)) forced += m;
+  }
+  for (int i = tid; i < N; i += NT) {
+    if (i < nC) {  // the candidates are the pages ns .. rs - 1
+      mkey[i] = static_cast<unsigned long long>(__double_as_longlong(mass(ns + i)));
+      mpage[i] = static_cast<uint32_t>(ns + i);
+    } else {
+      mkey[i] = 0ull;
+      mpage[i] = 0x7FFFFFFFu;
     }
   }
-  if (tid == 0) {
-    *cnt_out = min(total, kmax);
-    if (total > kmax) set_err(err, KVQ_DERR_KMAX);
+  for (int i = tid; i < nwords; i += NT) chosen[i] = 0u;
+  const double total = sel_block_sum<NT>(tot, sh, tid, bar);
+  const double fsum = sel_block_sum<NT>(forced, sh, tid, bar);
+  const double need = static_cast<double>(prm.coverage_ppm) * 1e-6 * total - fsum;
+  int kstar = 0;
+  if (need > 0.0 && nC > 0) {
+    // 3) bitonic sort: mass descending, then page ascending (masses are >= 0: their bits
+    //    order like the values)
+    for (int size = 2; size <= N; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int t = tid; t < N / 2; t += NT) {
+          const int i = 2 * t - (t & (stride - 1));
+          const int j = i + stride;
+          const bool down = (i & size) == 0;  // this run sorts "first before" (descending)
+          const unsigned long long ki = mkey[i], kj = mkey[j];
+          const uint32_t pi = mpage[i], pj = mpage[j];
+          const bool j_first = kj > ki || (kj == ki && pj < pi);
+          if (j_first == down) {
+            mkey[i] = kj;
+            mkey[j] = ki;
+            mpage[i] = pj;
+            mpage[j] = pi;
+          }
+        }
+        bar();
+      }
+    }
+    // 4) prefix sums of the sorted masses; the cut is the first prefix reaching `need`
+    double* pre = reinterpret_cast<double*>(mkey);
+    for (int i = tid; i < nC; i += NT) pre[i] = __longlong_as_double(static_cast<long long>(mkey[i]));
+    bar();
+    sel_prefix_sum<NT>(pre, nC, sh, tid, bar);
+    if (tid == 0) sh.rem = nC;
+    bar();
+    for (int i = tid; i < nC; i += NT)
+      if (pre[i] >= need && (i == 0 || pre[i - 1] < need)) sh.rem = i + 1;
+    bar();
+    kstar = sh.rem;
+    for (int i = tid; i < kstar; i += NT) {
+      const uint32_t p = mpage[i];
+      atomicOr(&chosen[p >> 5], 1u << (p & 31));
+    }
   }
+  // 5) forced pages
+  for (int p = tid; p < P; p += NT)
+    if (!is_cand(p)) atomicOr(&chosen[p >> 5], 1u << (p & 31));
+  bar();
+  emit_chosen<NT>(chosen, nwords, out, cnt_out, kmax, err, sh, tid, bar);
 }
 
 }  // namespace kvq

@@ -47,7 +47,8 @@ class KvqCache(ctypes.Structure):
 
 
 class SelectParams(ctypes.Structure):
-    _fields_ = [("k_abs", c_int32), ("k_frac_bp", c_int32), ("n_sink", c_int32), ("n_recent", c_int32)]
+    _fields_ = [("k_abs", c_int32), ("k_frac_bp", c_int32), ("n_sink", c_int32), ("n_recent", c_int32),
+                ("coverage_ppm", c_int32), ("sm_scale", c_float)]
 
 
 _P = POINTER(KvqCache)
@@ -272,8 +273,11 @@ def cache_from_workload(w, device="cuda", threads: int = 8):
     return cache
 
 
-def select_params(w) -> SelectParams:
-    return SelectParams(w.k_abs, w.k_frac_bp, w.n_sink, w.n_recent)
+def select_params(w, coverage=None) -> SelectParams:
+    """The workload's budget selection, or coverage selection at ``coverage`` (0..1)."""
+    if coverage is None:
+        return SelectParams(w.k_abs, w.k_frac_bp, w.n_sink, w.n_recent)
+    return SelectParams(-1, 0, w.n_sink, w.n_recent, int(round(coverage * 1e6)), w.sm_scale)
 
 
 class DecodeStep:
@@ -283,7 +287,7 @@ class DecodeStep:
     kvq_select_topk -> kvq_sparse_decode_attn, all on the current stream.
     """
 
-    def __init__(self, w, cache: PagedCache, device="cuda"):
+    def __init__(self, w, cache: PagedCache, device="cuda", coverage=None):
         import torch
         self.w, self.cache = w, cache
         dt = cache.tdtype
@@ -294,8 +298,8 @@ class DecodeStep:
             self.k_new = torch.from_numpy(kn.view(np.int16)).to(device).view(dt)
             self.v_new = torch.from_numpy(vn.view(np.int16)).to(device).view(dt)
             self.pos = torch.from_numpy(np.asarray(w.lens, dtype=np.int32)).to(device)
-        self.kmax = w.kmax()
-        self.params = select_params(w)
+        self.kmax = w.kmax() if coverage is None else w.max_pages
+        self.params = select_params(w, coverage)
         self.scores = torch.empty((w.B, w.Hkv, w.max_pages), dtype=torch.float32, device=device)
         self.sel = torch.zeros((w.B, w.Hkv, self.kmax), dtype=torch.int32, device=device)
         self.cnt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device=device)

@@ -389,3 +389,75 @@ def test_score_select_equals_calls(kvq, name):
     for b in range(w.B):
         for g in range(w.Hkv):
             assert torch.equal(sel0[b, g, :c[b, g]], sel1[b, g, :c[b, g]])
+
+
+@pytest.mark.parametrize("P_cap", [700, 5000])
+def test_coverage_selection_matches_oracle(kvq, P_cap):
+    """Coverage (nucleus) selection: the GPU set is the oracle's wherever the cut is not
+    within rounding of another decision (ties, NaNs, partial last pages, every coverage)."""
+    from oracle.select import coverage_margin, select_coverage
+    rng = np.random.default_rng(P_cap)
+    B, Hkv = 12, 2
+    lens = rng.integers(1, 16 * P_cap + 1, B)
+    lens[0] = 16 * P_cap
+    w = W.make("c4", B=B, Hq=8, Hkv=Hkv, lens=lens, append=False)
+    cache = kvq.cache_from_workload(w)
+    sc = rng.normal(0, 3, (B, Hkv, w.max_pages)).astype(np.float32)
+    sc[1] = np.round(sc[1])           # ties
+    sc[2, 0, ::5] = np.nan
+    sc[3] = 1.5                       # every page the same score
+    checked = 0
+    for cov, scale, ns, nr in [(0.95, 0.088, 1, 4), (0.5, 0.3, 0, 0), (0.99, 0.05, 2, 1), (1.0, 1.0, 0, 2),
+                               (0.9, 0.088, 0, 0)]:
+        prm = kvq.SelectParams(-1, 0, ns, nr, int(round(cov * 1e6)), scale)
+        kmax = w.max_pages
+        selt = torch.full((B, Hkv, kmax), -7, dtype=torch.int32, device="cuda")
+        cntt = torch.zeros((B, Hkv), dtype=torch.int32, device="cuda")
+        cache.err.zero_()
+        kvq.kvq_select_topk(cache, torch.from_numpy(sc).cuda(), prm, selt, cntt, kmax)
+        got_s, got_c = selt.cpu().numpy(), cntt.cpu().numpy()
+        for b in range(B):
+            L = int(w.lens[b])
+            P = (L + 15) // 16
+            for g in range(Hkv):
+                want = select_coverage(sc[b, g].astype(np.float64), P, L, scale, int(round(cov * 1e6)) * 1e-6, ns, nr)
+                got = list(got_s[b, g, :got_c[b, g]])
+                if coverage_margin(sc[b, g].astype(np.float64), P, L, scale, cov, ns, nr) > 1e-5:
+                    assert got == list(want), (cov, scale, b, g, len(got), len(want))
+                    checked += 1
+                else:
+                    assert abs(len(got) - len(want)) <= 1
+        assert not (cache.err_bits() & ~kvq.DERR_NAN_SCORE)
+    assert checked >= 40
+
+
+def test_coverage_step_through_attention(kvq):
+    """A whole step with coverage selection: the pages chosen and the attention over them
+    match the oracle's."""
+    from oracle.select import coverage_margin, select_coverage
+    w = W.small("c1")
+    cache = kvq.cache_from_workload(w)
+    step = kvq.DecodeStep(w, cache)
+    step.params = kvq.SelectParams(-1, 0, w.n_sink, w.n_recent, 900000, w.sm_scale)
+    step.kmax = w.max_pages
+    step.sel = torch.zeros((w.B, w.Hkv, step.kmax), dtype=torch.int32, device="cuda")
+    step.ws = torch.zeros(max(kvq.kvq_workspace_size(cache, step.kmax), 1 << 16) // 4 + 4, dtype=torch.float32,
+                          device="cuda")
+    step.run()
+    torch.cuda.synchronize()
+    assert cache.err_bits() == 0, hex(cache.err_bits())
+    q, kn, vn = query_and_new(w)
+    sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
+    out = out_to_f64(step.out, w.dtype)
+    scores = step.scores.cpu().numpy()
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            sh = prepare(w, b, g)
+            r0 = oracle_step(w, prepare(w, b, g), b, g, q, kn, vn)
+            L, P = int(w.final_lens()[b]), r0["P"]
+            want = select_coverage(r0["scores"], P, L, w.sm_scale, 0.9, w.n_sink, w.n_recent)
+            if coverage_margin(r0["scores"], P, L, w.sm_scale, 0.9, w.n_sink, w.n_recent) > 1e-4:
+                assert list(sel[b, g, :cnt[b, g]]) == list(want)
+            r = oracle_step(w, sh, b, g, q, kn, vn, sel=sel[b, g, :cnt[b, g]].astype(np.int64))
+            for i in range(w.G):
+                check_output(out[b, g * w.G + i], r["out"][i], f"coverage b={b}", w.dtype)
