@@ -187,7 +187,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
 
     for _ in range(args.warmup):
         flush.fill_(1)
-        {"fused": step.run_fused, "two": step.run_two, "calls": step.run}[args.path]()
+        {"fused": step.run_fused, "two": step.run_two, "three": step.run_three, "calls": step.run}[args.path]()
     torch.cuda.synchronize(dev)
     assert cache.err_bits() == 0, f"device error bits {cache.err_bits():#x}"
     sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
@@ -195,10 +195,12 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
 
     K = args.steps
     fused = args.path == "fused"
-    run_step = {"fused": step.run_fused, "two": step.run_two, "calls": step.run}[args.path]
+    run_step = {"fused": step.run_fused, "two": step.run_two, "three": step.run_three, "calls": step.run}[args.path]
     # kernels of one step, in launch order (one callable each)
     parts = {"fused": [("decode_step", step.run_fused)],
              "two": [("score_select", step.score_select), ("sparse_decode_attn", step.attend)],
+             "three": [("append_scores", step.append_scores), ("select_topk", step.select),
+                       ("sparse_decode_attn", step.attend)],
              "calls": [("append", step.append), ("page_scores", step.scores_), ("select_topk", step.select),
                        ("sparse_decode_attn", step.attend)]}[args.path]
     # The step is replayed from CUDA graphs so the CPU never starves the GPU:
@@ -306,6 +308,9 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     elif args.path == "two":
         dom_bytes = [nbytes["score"] + nbytes["select"] + nbytes["append"], nbytes["attn"]][dom]
         files = ["score.cu", "attn.cu"]
+    elif args.path == "three":
+        dom_bytes = [nbytes["score"] + nbytes["append"], nbytes["select"], nbytes["attn"]][dom]
+        files = ["score.cu", "select.cu", "attn.cu"]
     else:
         dom_bytes = [nbytes["append"], nbytes["score"], nbytes["select"], nbytes["attn"]][dom]
         files = ["append.cu", "score.cu", "select.cu", "attn.cu"]
@@ -343,6 +348,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
         "gpu_launches": len(parts) * K,
         "path": {"fused": "kvq_decode_step (one persistent launch)",
                  "two": "kvq_score_select -> kvq_sparse_decode_attn",
+                 "three": "kvq_append_scores -> kvq_select_topk -> kvq_sparse_decode_attn",
                  "calls": "kvq_append -> kvq_page_scores -> kvq_select_topk -> kvq_sparse_decode_attn"}[args.path],
         "timing": "step: CUDA-graph replay of the step timed with events around each replay; "
                   "kernels_ms: a second graph with events between the launches (no launch overlap)",
@@ -448,8 +454,9 @@ def main():
     ap.add_argument("--coverage", type=float, default=None,
                     help="coverage (nucleus) selection at this mass fraction instead of the workload's budget "
                          "(four-call path only)")
-    ap.add_argument("--path", default="calls", choices=["calls", "two", "fused"],
-                    help="the four separate calls, kvq_score_select + attention, or one kvq_decode_step launch")
+    ap.add_argument("--path", default="calls", choices=["calls", "three", "two", "fused"],
+                    help="the four separate calls; kvq_append_scores + select + attention; kvq_score_select + "
+                         "attention; or one kvq_decode_step launch")
     ap.add_argument("--dense", action="store_true", help="also time attention over every page")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

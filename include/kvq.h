@@ -9,6 +9,7 @@
  *   kvq_select_topk        pick the top pages plus forced sink/recent pages;
  *   kvq_sparse_decode_attn attend only the selected pages (split-K + log-sum-exp combine),
  *                          unpacking and dequantising cold pages in registers;
+ *   kvq_append_scores      the first two in one launch (same results);
  *   kvq_score_select       the first three in one launch (same results);
  *   kvq_decode_step        the four above in one persistent launch (same results).
  *
@@ -250,6 +251,14 @@ size_t kvq_noalloc_scratch_bytes(void);
  * tile counters at its head; the call leaves them zero).  B*Hkv <= 8192,
  * max_pages <= 51200.
  */
+/*
+ * kvq_append_scores -- kvq_append followed by kvq_page_scores in one launch, with the same
+ * results: the warp that scores the tile of a sequence's appended token writes the token
+ * first.  Arguments as those two calls (pos, k_new, v_new required).
+ */
+kvq_status kvq_append_scores(const kvq_cache* cache, const int32_t* pos, const void* k_new,
+                             const void* v_new, const void* q, float* scores, kvq_stream_t stream);
+
 /* (coverage selection is not supported here: KVQ_ERR_UNSUPPORTED) */
 kvq_status kvq_score_select(const kvq_cache* cache, const int32_t* pos, const void* k_new,
                             const void* v_new, const void* q, const kvq_select_params* params,

@@ -181,6 +181,16 @@ kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const i
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+kvq_status kvq_append_scores(const kvq_cache* cache, const int32_t* pos, const void* k_new, const void* v_new,
+                             const void* q, float* scores, kvq_stream_t stream) {
+  DevCache c;
+  kvq_status st = to_dev(cache, c);
+  if (st != KVQ_OK) return st;
+  if (pos == nullptr || k_new == nullptr || v_new == nullptr || q == nullptr || scores == nullptr || !aligned16(q))
+    return KVQ_ERR_INVALID_ARG;
+  return cuda_status(launch_append_scores(c, pos, k_new, v_new, q, scores, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 kvq_status kvq_score_select(const kvq_cache* cache, const int32_t* pos, const void* k_new, const void* v_new,
                             const void* q, const kvq_select_params* params, float* scores, int32_t* sel,
                             int32_t* cnt, int32_t kmax, void* workspace, size_t ws_bytes, kvq_stream_t stream) {

@@ -139,6 +139,8 @@ cudaError_t launch_scores(const DevCache& c, const void* q, float* scores, cudaS
 cudaError_t launch_score_select(const DevCache& c, const int32_t* pos, const void* k_new, const void* v_new,
                                 const void* q, const kvq_select_params& prm, float* scores, int32_t* sel,
                                 int32_t* cnt, int kmax, unsigned* done, cudaStream_t s);
+cudaError_t launch_append_scores(const DevCache& c, const int32_t* pos, const void* k_new, const void* v_new,
+                                 const void* q, float* scores, cudaStream_t s);
 constexpr size_t kScoreSelectCounterWord = 8192;  // workspace word of the per-(b, g) tile counters
 cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_select_params& prm,
                           int32_t* sel, int32_t* cnt, int kmax, cudaStream_t s);

@@ -48,15 +48,19 @@ struct ScoreSelect {
 
 // Grid of 2 CTAs per SM; warp w takes the contiguous run of 16-page tiles
 // [w * per, (w + 1) * per) of the flat list (b, g, tile), loading the next tile while
-// the current one is multiplied.  FUSED: the warp that owns the tile of a (b, g)'s
-// appended token writes the token first (so that tile is read after the new summary row
-// is stored); after its tiles, the CTA counts them on each (b, g) it touched, and the CTA
-// that completes a (b, g) selects its pages (select_core.cuh) from the scores in L2.
-template <int D, bool BF16, bool FUSED>
+// the current one is multiplied.
+// MODE 1 (kvq_append_scores) and 2 (kvq_score_select): the warp that owns the tile of a
+// (b, g)'s appended token writes the token first (so that tile is read after the new
+// summary row is stored).  MODE 2: after its tiles, the CTA counts them on each (b, g) it
+// touched, and the CTA that completes a (b, g) selects its pages (select_core.cuh) from
+// the scores in L2.
+enum { SCORES = 0, APPEND_SCORES = 1, APPEND_SCORES_SELECT = 2 };
+
+template <int D, bool BF16, int MODE>
 __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, const uint16_t* __restrict__ q,
                                                                     float* __restrict__ scores, int tiles_per_bg,
                                                                     int per, ScoreSelect f) {
-  extern __shared__ __align__(16) uint32_t sel_smem[];  // FUSED: keys [max_pages], then the scratch
+  extern __shared__ __align__(16) uint32_t sel_smem[];  // MODE 2: keys [max_pages], then the scratch
   __shared__ SelShared sel_sh;
   __shared__ int s_unit;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -66,7 +70,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
   const int i1 = min(total, i0 + per);
   griddep_wait();
 
-  if (FUSED && f.pos != nullptr && i0 < i1) {  // appends whose page lies in this warp's tiles
+  if (MODE != SCORES && f.pos != nullptr && i0 < i1) {  // appends whose page lies in this warp's tiles
     for (int bg = i0 / tiles_per_bg; bg <= (i1 - 1) / tiles_per_bg; ++bg) {
       const int b = bg / c.Hkv, g = bg % c.Hkv;
       const int ps = f.pos[b];
@@ -134,7 +138,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
     if (bad) set_err(c.err, KVQ_DERR_FP16_RANGE);
   }
 
-  if constexpr (FUSED) {
+  if constexpr (MODE == APPEND_SCORES_SELECT) {
     // count this CTA's tiles on each (b, g) it touched; the CTA completing one selects it
     const int c0 = min(total, (int)blockIdx.x * kScoreWarps * per);
     const int c1 = min(total, c0 + kScoreWarps * per);
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
   griddep_launch_dependents();
 }
 
-template <int D, bool BF16, bool FUSED>
+template <int D, bool BF16, int MODE>
 cudaError_t launch_d(const DevCache& c, const void* q, float* scores, const ScoreSelect& f, cudaStream_t s) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
@@ -198,13 +202,13 @@ cudaError_t launch_d(const DevCache& c, const void* q, float* scores, const Scor
   const int per = (int)((total + warps - 1) / warps);
   const long long blocks = (total + (long long)per * kScoreWarps - 1) / ((long long)per * kScoreWarps);
   size_t smem = 0;
-  if (FUSED) {
+  if (MODE == APPEND_SCORES_SELECT) {
     smem = ((size_t)(c.max_pages + 3) / 4 * 4 + kSelScratchWords) * sizeof(uint32_t);
     const cudaError_t e =
-        cudaFuncSetAttribute(score_kernel<D, BF16, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(score_kernel<D, BF16, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(score_kernel<D, BF16, FUSED>, dim3((unsigned)blocks), dim3(kScoreWarps * 32), smem, s, c,
+  return launch_pdl(score_kernel<D, BF16, MODE>, dim3((unsigned)blocks), dim3(kScoreWarps * 32), smem, s, c,
                     static_cast<const uint16_t*>(q), scores, tiles_per_bg, per, f);
 }
 
@@ -214,8 +218,8 @@ cudaError_t launch_scores(const DevCache& c, const void* q, float* scores, cudaS
   if (c.G > kMaxG) return cudaErrorInvalidValue;
   const bool bf = c.dtype == KVQ_DT_BF16;
   const ScoreSelect f{};
-  if (c.D == 128) return bf ? launch_d<128, true, false>(c, q, scores, f, s) : launch_d<128, false, false>(c, q, scores, f, s);
-  if (c.D == 64) return bf ? launch_d<64, true, false>(c, q, scores, f, s) : launch_d<64, false, false>(c, q, scores, f, s);
+  if (c.D == 128) return bf ? launch_d<128, true, SCORES>(c, q, scores, f, s) : launch_d<128, false, SCORES>(c, q, scores, f, s);
+  if (c.D == 64) return bf ? launch_d<64, true, SCORES>(c, q, scores, f, s) : launch_d<64, false, SCORES>(c, q, scores, f, s);
   return cudaErrorInvalidValue;
 }
 
@@ -226,8 +230,27 @@ cudaError_t launch_score_select(const DevCache& c, const int32_t* pos, const voi
   const bool bf = c.dtype == KVQ_DT_BF16;
   const ScoreSelect f{pos, static_cast<const uint16_t*>(k_new), static_cast<const uint16_t*>(v_new), prm, sel, cnt,
                       kmax, done};
-  if (c.D == 128) return bf ? launch_d<128, true, true>(c, q, scores, f, s) : launch_d<128, false, true>(c, q, scores, f, s);
-  if (c.D == 64) return bf ? launch_d<64, true, true>(c, q, scores, f, s) : launch_d<64, false, true>(c, q, scores, f, s);
+  if (c.D == 128)
+    return bf ? launch_d<128, true, APPEND_SCORES_SELECT>(c, q, scores, f, s)
+              : launch_d<128, false, APPEND_SCORES_SELECT>(c, q, scores, f, s);
+  if (c.D == 64)
+    return bf ? launch_d<64, true, APPEND_SCORES_SELECT>(c, q, scores, f, s)
+              : launch_d<64, false, APPEND_SCORES_SELECT>(c, q, scores, f, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_append_scores(const DevCache& c, const int32_t* pos, const void* k_new, const void* v_new,
+                                 const void* q, float* scores, cudaStream_t s) {
+  if (c.G > kMaxG) return cudaErrorInvalidValue;
+  const bool bf = c.dtype == KVQ_DT_BF16;
+  ScoreSelect f{};
+  f.pos = pos;
+  f.k_new = static_cast<const uint16_t*>(k_new);
+  f.v_new = static_cast<const uint16_t*>(v_new);
+  if (c.D == 128)
+    return bf ? launch_d<128, true, APPEND_SCORES>(c, q, scores, f, s) : launch_d<128, false, APPEND_SCORES>(c, q, scores, f, s);
+  if (c.D == 64)
+    return bf ? launch_d<64, true, APPEND_SCORES>(c, q, scores, f, s) : launch_d<64, false, APPEND_SCORES>(c, q, scores, f, s);
   return cudaErrorInvalidValue;
 }
 

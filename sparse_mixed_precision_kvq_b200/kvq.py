@@ -35,7 +35,7 @@ DERR_NONFINITE, DERR_TIMEOUT, DERR_BAD_POS = 0x10, 0x20, 0x40
 EXPORTS = ["kvq_chunk_bytes", "kvq_status_string", "kvq_append", "kvq_build_pages", "kvq_page_scores",
            "kvq_select_topk", "kvq_workspace_size", "kvq_sparse_decode_attn", "kvq_dequant_page",
            "kvq_sparse_decode_attn_noalloc", "kvq_noalloc_scratch_bytes", "kvq_workspace_init",
-           "kvq_step_workspace_size", "kvq_decode_step", "kvq_score_select"]
+           "kvq_step_workspace_size", "kvq_decode_step", "kvq_score_select", "kvq_append_scores"]
 
 
 class KvqCache(ctypes.Structure):
@@ -72,8 +72,9 @@ _lib.kvq_decode_step.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, POI
                                  c_void_p]
 _lib.kvq_score_select.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, POINTER(SelectParams), c_void_p,
                                   c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]
+_lib.kvq_append_scores.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
 for _f in EXPORTS[2:9] + ["kvq_sparse_decode_attn_noalloc", "kvq_workspace_init", "kvq_step_workspace_size",
-                          "kvq_decode_step", "kvq_score_select"]:
+                          "kvq_decode_step", "kvq_score_select", "kvq_append_scores"]:
     getattr(_lib, _f).restype = c_int32
 
 
@@ -153,6 +154,12 @@ def kvq_decode_step(cache, pos, k_new, v_new, q, params: SelectParams, scores, s
                                 _ptr(scores), _ptr(sel), _ptr(cnt), kmax, sm_scale, _ptr(out), _ptr(lse),
                                 _ptr(workspace), int(workspace.numel() * workspace.element_size()),
                                 _stream(stream)), "kvq_decode_step")
+
+
+def kvq_append_scores(cache, pos, k_new, v_new, q, scores, stream=None):
+    """kvq_append + kvq_page_scores in one launch."""
+    _check(_lib.kvq_append_scores(cache.ref(), _ptr(pos), _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(scores),
+                                  _stream(stream)), "kvq_append_scores")
 
 
 def kvq_score_select(cache, pos, k_new, v_new, q, params: SelectParams, scores, sel, cnt, kmax: int, workspace,
@@ -334,6 +341,18 @@ class DecodeStep:
         kvq_score_select(self.cache, self.pos if self.w.append else None, self.k_new if self.w.append else None,
                          self.v_new if self.w.append else None, self.q, self.params, self.scores, self.sel, self.cnt,
                          self.kmax, self.ws)
+
+    def append_scores(self):
+        if self.w.append:
+            kvq_append_scores(self.cache, self.pos, self.k_new, self.v_new, self.q, self.scores)
+        else:
+            self.scores_()
+
+    def run_three(self):
+        """The same step as ``run()`` in three launches: kvq_append_scores, select, attention."""
+        self.append_scores()
+        self.select()
+        self.attend()
 
     def run_two(self):
         """The same step as ``run()`` in two launches: kvq_score_select, kvq_sparse_decode_attn."""

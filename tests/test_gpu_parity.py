@@ -47,6 +47,8 @@ def _run(kvq, w, fused=False):
     step = kvq.DecodeStep(w, cache)
     if fused == "two":
         step.run_two()
+    elif fused == "three":
+        step.run_three()
     elif fused:
         step.run_fused()
     else:
@@ -56,7 +58,7 @@ def _run(kvq, w, fused=False):
     return cache, step, pre, post
 
 
-PATHS = ["calls", "fused", "two"]
+PATHS = ["calls", "fused", "two", "three"]
 
 
 @pytest.mark.parametrize("path", PATHS)
@@ -65,7 +67,7 @@ def test_step_matches_oracle(kvq, name, path):
     """The four calls, the two-launch kvq_score_select + attention, and the one-launch
     kvq_decode_step, against the oracle."""
     w = VARIANTS[name]()
-    cache, step, pre, post = _run(kvq, w, fused={"calls": False, "fused": True, "two": "two"}[path])
+    cache, step, pre, post = _run(kvq, w, fused={"calls": False, "fused": True, "two": "two", "three": "three"}[path])
     assert cache.err_bits() == 0, hex(cache.err_bits())
     q, kn, vn = query_and_new(w)
     scores = step.scores.cpu().numpy()
@@ -207,7 +209,7 @@ def test_edge_cases_empty_short_and_overlapping(kvq, path):
     append that opens a page, and a ragged last page."""
     w = W.make("c4", B=6, Hq=8, Hkv=2, lens=np.array([0, 1, 15, 16, 40, 200]), append=True,
                n_sink=3, n_recent=3, k_abs=2, tier_fracs=ALL_TIERS)
-    cache, step, pre, post = _run(kvq, w, fused={"calls": False, "fused": True, "two": "two"}[path])
+    cache, step, pre, post = _run(kvq, w, fused={"calls": False, "fused": True, "two": "two", "three": "three"}[path])
     assert cache.err_bits() == 0
     q, kn, vn = query_and_new(w)
     out = out_to_f64(step.out, w.dtype)
@@ -225,7 +227,7 @@ def test_edge_cases_empty_short_and_overlapping(kvq, path):
 @pytest.mark.parametrize("path", PATHS)
 def test_empty_selection_gives_zero_output(kvq, path):
     w = W.make("c4", B=3, Hq=8, Hkv=2, lens=np.array([0, 35, 0]), append=False)
-    cache, step, pre, post = _run(kvq, w, fused={"calls": False, "fused": True, "two": "two"}[path])
+    cache, step, pre, post = _run(kvq, w, fused={"calls": False, "fused": True, "two": "two", "three": "three"}[path])
     out = step.out.float().cpu().numpy()
     lse = step.lse.cpu().numpy()
     assert np.all(out[0] == 0) and np.all(out[2] == 0)
@@ -353,7 +355,7 @@ def test_long_context_many_pages(kvq, path):
     """A sequence of 8193 pages (131072 tokens + 1, as in the long-context workload): the
     selection keeps all of its keys on chip; pages, selection and output as the oracle's."""
     w = W.make("c3", lens=np.array([131072]), Hq=8, Hkv=2)
-    cache, step, pre, post = _run(kvq, w, fused={"calls": False, "fused": True, "two": "two"}[path])
+    cache, step, pre, post = _run(kvq, w, fused={"calls": False, "fused": True, "two": "two", "three": "three"}[path])
     assert cache.err_bits() == 0, hex(cache.err_bits())
     q, kn, vn = query_and_new(w)
     sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
@@ -368,27 +370,29 @@ def test_long_context_many_pages(kvq, path):
 
 @pytest.mark.parametrize("name", ["c1", "c4", "g2_alltiers"])
 def test_score_select_equals_calls(kvq, name):
-    """kvq_score_select (append + scores + selection in one launch) leaves the same cache
-    bytes, scores, selection and (through the same attention call) outputs as the calls."""
+    """kvq_score_select (append + scores + selection in one launch) and kvq_append_scores
+    leave the same cache bytes, scores, selection and (through the same attention call)
+    outputs as the four calls."""
     w = VARIANTS[name]()
     outs = []
-    for two in (False, True):
+    for how in ("calls", "two", "three"):
         cache = kvq.cache_from_workload(w)
         step = kvq.DecodeStep(w, cache)
-        step.run_two() if two else step.run()
+        {"calls": step.run, "two": step.run_two, "three": step.run_three}[how]()
         torch.cuda.synchronize()
         outs.append((snapshot(cache), step.scores.clone(), step.sel.clone(), step.cnt.clone(), step.out.clone()))
         assert cache.err_bits() == 0, hex(cache.err_bits())
-    (s0, sc0, sel0, cnt0, o0), (s1, sc1, sel1, cnt1, o1) = outs
-    for t, (p0, p1) in enumerate(zip(s0["pools"], s1["pools"])):
-        assert (p0 is None) == (p1 is None) and (p0 is None or np.array_equal(p0, p1)), t
-    for k in ("bt", "summary", "ksum"):
-        assert np.array_equal(s0[k], s1[k]), k
-    assert torch.equal(sc0, sc1) and torch.equal(cnt0, cnt1) and torch.equal(o0, o1)
-    c = cnt0.cpu().numpy()
-    for b in range(w.B):
-        for g in range(w.Hkv):
-            assert torch.equal(sel0[b, g, :c[b, g]], sel1[b, g, :c[b, g]])
+    (s0, sc0, sel0, cnt0, o0) = outs[0]
+    for (s1, sc1, sel1, cnt1, o1) in outs[1:]:
+        for t, (p0, p1) in enumerate(zip(s0["pools"], s1["pools"])):
+            assert (p0 is None) == (p1 is None) and (p0 is None or np.array_equal(p0, p1)), t
+        for k in ("bt", "summary", "ksum"):
+            assert np.array_equal(s0[k], s1[k]), k
+        assert torch.equal(sc0, sc1) and torch.equal(cnt0, cnt1) and torch.equal(o0, o1)
+        c = cnt0.cpu().numpy()
+        for b in range(w.B):
+            for g in range(w.Hkv):
+                assert torch.equal(sel0[b, g, :c[b, g]], sel1[b, g, :c[b, g]])
 
 
 @pytest.mark.parametrize("P_cap", [700, 5000])
