@@ -142,3 +142,23 @@ def page_bytes(sh: SeqHead, p: int, kind: str) -> np.ndarray:
     pay = (sh.kcodes if kind == "k" else sh.vcodes)[s:s + n]
     meta = (sh.kmeta if kind == "k" else sh.vmeta)[s:s + n]
     return pack_chunk(kind, tier, sh.D, n, pay, meta)
+
+
+def requantize(sh: SeqHead, p: int, new_tier: int):
+    """Tier demotion (ARGUS "Visual Architecture": pages move down the cascade as they cool).
+
+    Reading: the page's values as read back from its current tier (the 16-bit values, or
+    ``fp32(c*scale + zero)``, or ``+-m``) are quantised again, token by token and group by
+    group, with the same quantiser into ``new_tier`` (a b-bit tier).  The summary, built
+    from the keys as they arrived, is unchanged.
+    """
+    assert new_tier != TIER_F16, "demotion goes to a b-bit tier"
+    s = slice(p * T, max(p * T, min(sh.L, p * T + T)))
+    for t in range(s.start, s.stop):
+        qk = quantise_token(sh.khat[t].copy(), new_tier)
+        qv = quantise_token(sh.vhat[t].copy(), new_tier)
+        sh.khat[t], sh.vhat[t] = qk["xhat"], qv["xhat"]
+        sh.kcodes[t], sh.vcodes[t] = qk["codes"], qv["codes"]
+        sh.kmeta[t], sh.vmeta[t] = qk["meta"], qv["meta"]
+        sh.overflow |= bool(np.any(qk["overflow"]) or np.any(qv["overflow"]))
+    sh.tiers[p] = new_tier
