@@ -356,6 +356,9 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     }
     if dense_ms is not None:
         line["dense_all_pages_ms"] = dense_ms
+    if args.demote is not None:
+        del step, cache
+        line["demotion"] = time_demotion(w, args.demote, flush, stream, dev, peak, peak_kind)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
     return line
@@ -385,6 +388,50 @@ def time_dense(w, cache, step, flush, stream, dev, reps=20):
         if r >= 3:
             ts.append(a.elapsed_time(b_))
     return float(np.mean(ts))
+
+
+def time_demotion(w, tier: int, flush, stream, dev, peak: float, peak_kind: str, reps: int = 20):
+    """kvq_requantize_pages over every prefilled page outside the sink and recent windows
+    whose tier is above ``tier``, into spare slots of a fresh cache (the block table is
+    put back, outside the timed region, before every repetition)."""
+    import torch
+    from sparse_mixed_precision_kvq_b200 import kvq
+    tier_tbl, _, counts = w.slot_map()
+    items = []
+    nxt = list(counts)
+    for b in range(w.B):
+        P0 = w.pages_before(b)
+        for p in range(w.n_sink, P0 - w.n_recent):
+            if tier_tbl[b, p] < tier:
+                items.append((b, p, int(np.uint32((tier << 29) | nxt[tier]).view(np.int32))))
+                nxt[tier] += 1
+    spare = [n - c for n, c in zip(nxt, counts)]
+    cache = kvq.cache_from_workload(w, device=dev, spare=spare)
+    it = torch.tensor(items, dtype=torch.int32, device=dev)
+    bt0 = cache.block_table.clone()
+    cb = np.array([2 * kvq.kvq_chunk_bytes(t, w.D) for t in range(5)], dtype=np.int64)
+    src = np.array([tier_tbl[b, p] for b, p, _ in items], dtype=np.int64)
+    nbytes = int(w.Hkv * (cb[src].sum() + len(items) * cb[tier])) + len(items) * (12 + 8)
+    ts = []
+    for r in range(reps + 3):
+        cache.block_table.copy_(bt0)
+        flush.fill_(r & 0xFF)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        kvq.kvq_requantize_pages(cache, it)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        if r >= 3:
+            ts.append(a.elapsed_time(b_))
+    assert cache.err_bits() == 0, f"device error bits {cache.err_bits():#x}"
+    ms = float(np.mean(ts))
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"op": "kvq_requantize_pages (re-encode + block-table switch: two launches)",
+            "pages": len(items), "kv_heads": w.Hkv, "to_tier": tier,
+            "from_tiers": {int(t): int((src == t).sum()) for t in np.unique(src)},
+            "ms": ms, "bytes": nbytes, "pages_per_s": len(items) / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "peak_kind": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"}}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -458,6 +505,9 @@ def main():
                     help="the four separate calls; kvq_append_scores + select + attention; kvq_score_select + "
                          "attention; or one kvq_decode_step launch")
     ap.add_argument("--dense", action="store_true", help="also time attention over every page")
+    ap.add_argument("--demote", type=int, default=None, choices=[1, 2, 3, 4],
+                    help="also time kvq_requantize_pages moving the workload's pages outside the sink and "
+                         "recent windows down to this tier (1 int8, 2 int4, 3 int2, 4 1-bit)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling runs)")

@@ -296,6 +296,27 @@ kvq_status kvq_decode_step(const kvq_cache* cache, const int32_t* pos, const voi
                            kvq_stream_t stream);
 
 /*
+ * kvq_requantize_pages -- tier demotion: move pages to a lower-precision tier.
+ * (ARGUS "Virtual Memory for Transformers", "Visual Architecture": pages cool down the
+ *  cascade FP16 -> INT8 -> INT4 -> INT2 -> 1-bit.)
+ *  items  device [n][3] int32: (b, page, new block-table entry (tier << 29) | slot).
+ *  For every item, each kv head's K and V values of the page are read back from the
+ *  current tier (the 16-bit value, fp32(c*scale+zero) or +-m, as kvq_dequant_page) and
+ *  quantised again with kvq_append's quantiser into the new entry's tier and slot, token
+ *  slots past seq_len zero; then block_table[b][page] = new entry.  The page summary and
+ *  open_ksum are unchanged (they follow the keys as they arrived), so later appends to an
+ *  open page continue in the new tier.
+ *  The new tier must be a quantised one (1..4) and the new (tier, slot) must differ from
+ *  the current one; an item that is out of range, names a page without tokens, has an
+ *  invalid current or new entry, or aliases its own slot is skipped with
+ *  KVQ_DERR_BAD_PAGE.  The caller owns slot allocation: new slots must not be referenced
+ *  by any block-table entry, one item per (b, page), and the old slot may be reused once
+ *  the call's work on the stream is complete.  Two kernel launches; n == 0 is a no-op.
+ */
+kvq_status kvq_requantize_pages(const kvq_cache* cache, const int32_t* items, int32_t n,
+                                kvq_stream_t stream);
+
+/*
  * kvq_dequant_page -- values read back from storage for one logical page (testing aid).
  *  out device [Hkv][2][16][D] fp32: for each kv head, K then V, every token slot: the
  *  16-bit value, fp32(c * scale + zero), or +-m, per the page's tier.

@@ -15,31 +15,9 @@ __global__ void dequant_kernel(DevCache c, int b, int page, float* __restrict__ 
   const unsigned char* ck;
   if (!page_chunk(c, b, page, g, tier, ck)) return;
   const unsigned char* chunk = ck + (size_t)kind * c.chunk[tier];
-  const int ng = D / kGroup;
   for (int e = threadIdx.x; e < kPage * D; e += blockDim.x) {
     const int t = e / D, d = e % D;
-    int w, bit;
-    elem_pos(kind, tier, D, t, d, w, bit);
-    const uint32_t word = reinterpret_cast<const uint32_t*>(chunk)[w];
-    float v;
-    if (tier == KVQ_TIER_16) {
-      const uint16_t x = static_cast<uint16_t>(word >> bit);
-      v = c.dtype == KVQ_DT_BF16 ? bits_to_float<true>(x) : bits_to_float<false>(x);
-    } else {
-      const int bits = tier_bits(tier);
-      const uint32_t code = (word >> bit) & ((1u << bits) - 1u);
-      const unsigned char* meta = chunk + codes_bytes(tier, D);
-      if (tier == KVQ_TIER_I1) {
-        const float m = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(meta)[t * ng + d / kGroup]));
-        v = code ? m : -m;
-      } else {
-        const uint32_t mw = reinterpret_cast<const uint32_t*>(meta)[t * ng + d / kGroup];
-        const float scale = __half2float(__ushort_as_half(static_cast<uint16_t>(mw & 0xFFFFu)));
-        const float zero = __half2float(__ushort_as_half(static_cast<uint16_t>(mw >> 16)));
-        v = fmaf(static_cast<float>(code), scale, zero);
-      }
-    }
-    out[(((size_t)g * 2 + kind) * kPage + t) * D + d] = v;
+    out[(((size_t)g * 2 + kind) * kPage + t) * D + d] = load_value(chunk, kind, tier, D, c.dtype == KVQ_DT_BF16, t, d);
   }
 }
 
@@ -243,6 +221,15 @@ kvq_status kvq_decode_step(const kvq_cache* cache, const int32_t* pos, const voi
 kvq_status kvq_workspace_init(void* workspace, size_t ws_bytes, kvq_stream_t stream) {
   if (workspace == nullptr || ws_bytes < kCounterBytes || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
   return cuda_status(cudaMemsetAsync(workspace, 0, kCounterBytes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_requantize_pages(const kvq_cache* cache, const int32_t* items, int32_t n, kvq_stream_t stream) {
+  DevCache c;
+  kvq_status st = to_dev(cache, c);
+  if (st != KVQ_OK) return st;
+  if (n < 0 || (n > 0 && items == nullptr)) return KVQ_ERR_INVALID_ARG;
+  if (n == 0) return KVQ_OK;
+  return cuda_status(launch_requantize(c, items, n, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 kvq_status kvq_dequant_page(const kvq_cache* cache, int32_t b, int32_t page, float* out, kvq_stream_t stream) {

@@ -123,6 +123,90 @@ __global__ void __launch_bounds__(128) build_kernel(DevCache c, const uint16_t* 
   if (nonfinite) set_err(c.err, KVQ_DERR_NONFINITE);
 }
 
+// Tier demotion (ARGUS "Virtual Memory for Transformers", "Visual Architecture": pages
+// move down the cascade of tiers as they cool).  Item i = (b, page, new entry): the page's
+// tokens are read back from their current tier and quantised again, per token and
+// 32-channel group, into the new entry's b-bit tier and slot; a second launch then points
+// the block table at the new slot.  Both launches decide an item's validity the same way,
+// from a block table that only the second one changes: b and page in range, the page
+// holds tokens, the current entry is valid, and the new entry is a b-bit tier slot other
+// than the current one.
+__device__ inline bool requant_item(const DevCache& c, const int32_t* items, int i, int& b, int& p, uint32_t& oe,
+                                    uint32_t& ne, int& n) {
+  b = items[3 * i];
+  p = items[3 * i + 1];
+  ne = static_cast<uint32_t>(items[3 * i + 2]);
+  if (b < 0 || b >= c.B || p < 0 || p >= c.max_pages) return false;
+  n = min(kPage, c.seq_len[b] - p * kPage);
+  if (n <= 0) return false;
+  oe = static_cast<uint32_t>(c.block_table[(size_t)b * c.max_pages + p]);
+  const int ot = static_cast<int>(oe >> 29), nt = static_cast<int>(ne >> 29);
+  const long long os = oe & 0x1FFFFFFFu, ns = ne & 0x1FFFFFFFu;
+  if (ot >= kNumTiers || c.pool[ot] == nullptr || os >= c.pool_slots[ot]) return false;
+  if (nt < 1 || nt >= kNumTiers || c.pool[nt] == nullptr || ns >= c.pool_slots[nt]) return false;
+  return !(nt == ot && ns == os);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(128) requant_kernel(DevCache c, const int32_t* __restrict__ items) {
+  const int g = blockIdx.y, tid = threadIdx.x;
+  int b, p, n;
+  uint32_t oe, ne;
+  if (!requant_item(c, items, blockIdx.x, b, p, oe, ne, n)) {
+    if (g == 0 && tid == 0) set_err(c.err, KVQ_DERR_BAD_PAGE);
+    return;
+  }
+  const int D = c.D, ot = static_cast<int>(oe >> 29), nt = static_cast<int>(ne >> 29);
+  const int OB = c.chunk[ot], NB = c.chunk[nt];
+  const unsigned char* src = c.pool[ot] + ((size_t)(oe & 0x1FFFFFFFu) * c.Hkv + g) * 2 * (size_t)OB;
+  unsigned char* dst = c.pool[nt] + ((size_t)(ne & 0x1FFFFFFFu) * c.Hkv + g) * 2 * (size_t)NB;
+
+  __shared__ __align__(16) uint32_t old_words[2048];   // current K and V chunks (<= 8 KB)
+  __shared__ __align__(16) uint32_t words[2][1024];    // new chunk images (<= 4 KB each)
+  for (int k = tid; k < 2 * OB / 16; k += blockDim.x)
+    reinterpret_cast<uint4*>(old_words)[k] = __ldcg(reinterpret_cast<const uint4*>(src) + k);
+  for (int k = tid; k < 2 * 1024; k += blockDim.x) (&words[0][0])[k] = 0u;
+  __syncthreads();
+
+  const int warp = tid >> 5, lane = tid & 31, ng = D / kGroup;
+  bool ov = false, nonfinite = false;
+  for (int gi = warp; gi < 2 * n * ng; gi += 4) {
+    const int kind = gi / (n * ng), rem = gi % (n * ng), t = rem / ng, grp = rem % ng;
+    const int d = grp * kGroup + lane;
+    const unsigned char* oc = reinterpret_cast<const unsigned char*>(old_words) + kind * OB;
+    const double x = static_cast<double>(load_value(oc, kind, ot, D, BF16, t, d));
+    nonfinite |= !isfinite(x);
+    const QOut q = quant_group(x, nt, ov);
+    int w, bit;
+    elem_pos(kind, nt, D, t, d, w, bit);
+    atomicOr(&words[kind][w], q.code << bit);
+    if (lane == 0) {
+      unsigned char* meta = reinterpret_cast<unsigned char*>(words[kind]) + codes_bytes(nt, D);
+      if (nt == KVQ_TIER_I1)
+        reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = static_cast<uint16_t>(q.meta);
+      else
+        reinterpret_cast<uint32_t*>(meta)[t * ng + grp] = q.meta;
+    }
+  }
+  __syncthreads();
+  for (int kind = 0; kind < 2; ++kind) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(words[kind]);
+    uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)kind * NB);
+    for (int k = tid; k < NB / 16; k += blockDim.x) d4[k] = s4[k];
+  }
+  if (ov) set_err(c.err, KVQ_DERR_FP16_RANGE);
+  if (nonfinite) set_err(c.err, KVQ_DERR_NONFINITE);
+}
+
+__global__ void requant_commit_kernel(DevCache c, const int32_t* __restrict__ items, int n_items) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_items) return;
+  int b, p, n;
+  uint32_t oe, ne;
+  if (requant_item(c, items, i, b, p, oe, ne, n))
+    const_cast<int32_t*>(c.block_table)[(size_t)b * c.max_pages + p] = static_cast<int32_t>(ne);
+}
+
 }  // namespace
 
 cudaError_t launch_append(const DevCache& c, const int32_t* pos, const void* k_new, const void* v_new,
@@ -143,6 +227,16 @@ cudaError_t launch_build(const DevCache& c, const void* k_src, const void* v_src
   else
     build_kernel<false><<<grid, 128, 0, s>>>(c, static_cast<const uint16_t*>(k_src),
                                              static_cast<const uint16_t*>(v_src), cu, src_tokens);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_requantize(const DevCache& c, const int32_t* items, int n, cudaStream_t s) {
+  const dim3 grid(n, c.Hkv);
+  if (c.dtype == KVQ_DT_BF16) requant_kernel<true><<<grid, 128, 0, s>>>(c, items);
+  else requant_kernel<false><<<grid, 128, 0, s>>>(c, items);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  requant_commit_kernel<<<(n + 255) / 256, 256, 0, s>>>(c, items, n);
   return cudaGetLastError();
 }
 

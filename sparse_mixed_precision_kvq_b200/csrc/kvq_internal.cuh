@@ -96,6 +96,29 @@ __device__ inline float bits_to_float(uint16_t v) {
   else return __half2float(__ushort_as_half(v));
 }
 
+// Value read back from storage for element (t, d) of a K (kind 0) or V (kind 1) chunk:
+// the 16-bit value, fp32(c * scale + zero) with one rounding, or +-m.
+__device__ inline float load_value(const unsigned char* chunk, int kind, int tier, int D, bool bf16, int t, int d) {
+  int w, bit;
+  elem_pos(kind, tier, D, t, d, w, bit);
+  const uint32_t word = reinterpret_cast<const uint32_t*>(chunk)[w];
+  if (tier == 0) {
+    const uint16_t x = static_cast<uint16_t>(word >> bit);
+    return bf16 ? bits_to_float<true>(x) : bits_to_float<false>(x);
+  }
+  const int ng = D / kGroup;
+  const uint32_t code = (word >> bit) & ((1u << tier_bits(tier)) - 1u);
+  const unsigned char* meta = chunk + codes_bytes(tier, D);
+  if (tier == 4) {
+    const float m = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(meta)[t * ng + d / kGroup]));
+    return code ? m : -m;
+  }
+  const uint32_t mw = reinterpret_cast<const uint32_t*>(meta)[t * ng + d / kGroup];
+  const float scale = __half2float(__ushort_as_half(static_cast<uint16_t>(mw & 0xFFFFu)));
+  const float zero = __half2float(__ushort_as_half(static_cast<uint16_t>(mw >> 16)));
+  return fmaf(static_cast<float>(code), scale, zero);
+}
+
 // fp16 round-half-even of a double, saturating at +-65504 (flag in *ov).
 __device__ inline uint16_t fp16_sat(double v, bool& ov) {
   __half h = __double2half(v);
@@ -155,5 +178,6 @@ cudaError_t launch_step(const DevCache& c, const int32_t* pos, const void* k_new
                         const void* q, const kvq_select_params& prm, float* scores, int32_t* sel, int32_t* cnt,
                         int kmax, float sm_scale, void* out, float* lse, void* ws, int num_ctas, cudaStream_t s);
 cudaError_t launch_dequant(const DevCache& c, int b, int page, float* out, cudaStream_t s);
+cudaError_t launch_requantize(const DevCache& c, const int32_t* items, int n, cudaStream_t s);
 
 }  // namespace kvq

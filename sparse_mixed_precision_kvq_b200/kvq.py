@@ -35,7 +35,8 @@ DERR_NONFINITE, DERR_TIMEOUT, DERR_BAD_POS = 0x10, 0x20, 0x40
 EXPORTS = ["kvq_chunk_bytes", "kvq_status_string", "kvq_append", "kvq_build_pages", "kvq_page_scores",
            "kvq_select_topk", "kvq_workspace_size", "kvq_sparse_decode_attn", "kvq_dequant_page",
            "kvq_sparse_decode_attn_noalloc", "kvq_noalloc_scratch_bytes", "kvq_workspace_init",
-           "kvq_step_workspace_size", "kvq_decode_step", "kvq_score_select", "kvq_append_scores"]
+           "kvq_step_workspace_size", "kvq_decode_step", "kvq_score_select", "kvq_append_scores",
+           "kvq_requantize_pages"]
 
 
 class KvqCache(ctypes.Structure):
@@ -73,8 +74,9 @@ _lib.kvq_decode_step.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, POI
 _lib.kvq_score_select.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, POINTER(SelectParams), c_void_p,
                                   c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]
 _lib.kvq_append_scores.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
+_lib.kvq_requantize_pages.argtypes = [_P, c_void_p, c_int32, c_void_p]
 for _f in EXPORTS[2:9] + ["kvq_sparse_decode_attn_noalloc", "kvq_workspace_init", "kvq_step_workspace_size",
-                          "kvq_decode_step", "kvq_score_select", "kvq_append_scores"]:
+                          "kvq_decode_step", "kvq_score_select", "kvq_append_scores", "kvq_requantize_pages"]:
     getattr(_lib, _f).restype = c_int32
 
 
@@ -186,6 +188,13 @@ def kvq_dequant_page(cache, b: int, page: int, out, stream=None):
     _check(_lib.kvq_dequant_page(cache.ref(), b, page, _ptr(out), _stream(stream)), "kvq_dequant_page")
 
 
+def kvq_requantize_pages(cache, items, stream=None):
+    """``items``: device int32 tensor [n, 3] of (b, page, new block-table entry)."""
+    n = 0 if items is None else int(items.shape[0])
+    _check(_lib.kvq_requantize_pages(cache.ref(), _ptr(items) if n else None, n, _stream(stream)),
+           "kvq_requantize_pages")
+
+
 # ------------------------------------------------------------------------- allocation
 def encode_block_table(tier_tbl: np.ndarray, slot_tbl: np.ndarray) -> np.ndarray:
     """(tier << 29) | slot as int32; unused entries (tier < 0) get an invalid tier (7)."""
@@ -245,14 +254,17 @@ class PagedCache:
         return tier, self.pools[tier][o:o + cb]
 
 
-def cache_from_workload(w, device="cuda", threads: int = 8):
+def cache_from_workload(w, device="cuda", threads: int = 8, spare=None):
     """Allocate a cache for workload ``w`` and store its prefilled context with kvq_build_pages.
 
     After the call ``seq_len`` holds the prefilled lengths (before the step's append).
+    ``spare`` (optional, per tier) adds free slots after the used ones of each pool.
     """
     import torch
     from concurrent.futures import ThreadPoolExecutor
     tier_tbl, slot_tbl, counts = w.slot_map()
+    if spare is not None:
+        counts = [int(c) + int(x) for c, x in zip(counts, spare)]
     cache = PagedCache(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.dtype, counts, device)
     cache.block_table.copy_(torch.from_numpy(encode_block_table(tier_tbl, slot_tbl)))
     lens = np.asarray(w.lens, dtype=np.int64)

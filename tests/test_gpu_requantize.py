@@ -1,0 +1,147 @@
+"""Tier demotion on the GPU (kvq_requantize_pages) vs the oracle's ``requantize``.
+
+Every page of every (sequence, kv head) is compared bit for bit after a seeded mix of
+demotions (each page to a random lower tier, partial last pages included), then a whole
+decode step (append into a demoted open page, scores, selection, attention) runs on the
+demoted cache and is compared with the oracle's step on the demoted oracle cache.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import cache as ocache
+from oracle.step import prepare
+from sparse_mixed_precision_kvq_b200 import workloads as W
+from tests.parity_helpers import (check_output, check_pages, check_selection, oracle_step, out_to_f64,
+                                  query_and_new, snapshot)
+
+pytestmark = pytest.mark.gpu
+
+ALL_TIERS = {W.TIER_F16: 0.2, W.TIER_I8: 0.2, W.TIER_I4: 0.2, W.TIER_I2: 0.2, W.TIER_I1: 0.2}
+CASES = {
+    "bf16_d128": lambda: W.make("c1", B=2, Hq=16, Hkv=4, lens=np.array([700, 333]), tier_fracs=ALL_TIERS,
+                                k_frac_bp=2000),
+    "f16_d64": lambda: W.make("c0", B=2, lens=np.array([1000, 77]), append=True, tier_fracs=ALL_TIERS),
+}
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    from sparse_mixed_precision_kvq_b200 import kvq as k
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return k
+
+
+def demotion_plan(w, seed=7, frac=0.6):
+    """(b, page, new tier) for a seeded subset of the prefilled pages, each to a lower tier;
+    the last prefilled page of every sequence is always in the plan (when it can move)."""
+    rng = np.random.default_rng(seed)
+    plan = []
+    for b in range(w.B):
+        tiers = w.tiers(b)
+        P0 = w.pages_before(b)
+        for p in range(P0):
+            t = int(tiers[p])
+            if t == W.TIER_I1 or (p != P0 - 1 and rng.random() > frac):
+                continue
+            plan.append((b, p, int(rng.integers(max(t, W.TIER_F16) + 1, W.TIER_I1 + 1))))
+    return plan
+
+
+def apply_plan(kvq, w, plan):
+    """Cache with spare slots, demoted on the GPU; returns (cache, items, new entries)."""
+    spare = [0] * 5
+    for _, _, t in plan:
+        spare[t] += 1
+    _, _, counts = w.slot_map()
+    cache = kvq.cache_from_workload(w, spare=spare)
+    nxt = list(counts)
+    items = []
+    for b, p, t in plan:
+        items.append((b, p, int(np.uint32((t << 29) | nxt[t]).view(np.int32))))
+        nxt[t] += 1
+    it = torch.tensor(items, dtype=torch.int32, device="cuda")
+    kvq.kvq_requantize_pages(cache, it)
+    torch.cuda.synchronize()
+    return cache, items
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_requantized_pages_match_the_oracle(kvq, name):
+    w = CASES[name]()
+    plan = demotion_plan(w)
+    assert len(plan) > 10
+    cache, items = apply_plan(kvq, w, plan)
+    assert cache.err_bits() == 0, hex(cache.err_bits())
+    snap = snapshot(cache)
+    for b, p, e in items:
+        assert int(snap["bt"][b, p]) == e
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            sh = prepare(w, b, g)
+            for bb, p, t in plan:
+                if bb == b:
+                    ocache.requantize(sh, p, t)
+            check_pages(snap, sh, w, b, g, range(w.pages_before(b)))
+            assert np.array_equal(snap["summary"][b, g, :sh.P], sh.summary_bits[:sh.P])
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_decode_step_on_a_demoted_cache(kvq, name):
+    w = CASES[name]()
+    plan = demotion_plan(w, seed=11)
+    cache, _ = apply_plan(kvq, w, plan)
+    step = kvq.DecodeStep(w, cache)
+    step.run()
+    torch.cuda.synchronize()
+    assert cache.err_bits() == 0, hex(cache.err_bits())
+    snap = snapshot(cache)
+    q, kn, vn = query_and_new(w)
+    out = out_to_f64(step.out, w.dtype)
+    sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
+    scores = step.scores.cpu().numpy()
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            sh = prepare(w, b, g)
+            for bb, p, t in plan:
+                if bb == b:
+                    ocache.requantize(sh, p, t)
+            r = oracle_step(w, sh, b, g, q, kn, vn)
+            check_pages(snap, sh, w, b, g, range(sh.P))  # the append wrote into the demoted tier
+            if not check_selection(sel[b, g, :cnt[b, g]], r["sel"], scores[b, g], w, sh.P):
+                continue
+            for i in range(w.G):
+                check_output(out[b, g * w.G + i], r["out"][i], f"b={b} g={g} h={i}", w.dtype)
+
+
+def test_invalid_items_are_skipped_with_an_error_bit(kvq):
+    w = CASES["f16_d64"]()
+    cache = kvq.cache_from_workload(w, spare=[0, 1, 1, 1, 1])
+    bt0 = cache.block_table.clone()
+    pools0 = [None if p is None else p.clone() for p in cache.pools]
+    _, _, counts = w.slot_map()
+    e = int(bt0[0, 5].item()) & 0xFFFFFFFF
+    tier, slot = e >> 29, e & 0x1FFFFFFF
+
+    def ent(t, s):
+        return int(np.uint32((t << 29) | s).view(np.int32))
+
+    bad = [
+        (0, 5, ent(tier, slot)),                   # its own slot
+        (0, 5, ent(0, counts[0])),                 # the 16-bit tier is not a demotion target
+        (0, 5, ent(2, counts[2] + 5)),             # slot past the pool
+        (2, 0, ent(2, counts[2])),                 # sequence out of range
+        (1, w.max_pages, ent(2, counts[2])),       # page out of range
+        (1, 10, ent(2, counts[2])),                # a page holding no tokens (77 tokens: pages 0..4)
+        (0, 3, ent(6, 0)),                         # no such tier
+    ]
+    kvq.kvq_requantize_pages(cache, torch.tensor(bad, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    assert cache.err_bits() == 0x1
+    assert torch.equal(cache.block_table, bt0)
+    for a, b0 in zip(cache.pools, pools0):
+        assert (a is None) == (b0 is None) and (a is None or torch.equal(a, b0))
+    cache.err.zero_()
+    kvq.kvq_requantize_pages(cache, None)        # n == 0: nothing launched
+    torch.cuda.synchronize()
+    assert cache.err_bits() == 0 and torch.equal(cache.block_table, bt0)

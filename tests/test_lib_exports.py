@@ -36,6 +36,34 @@ def test_binding_mirrors_the_header():
         assert callable(getattr(kvq, n))
 
 
+def _param_counts():
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for name, params in re.findall(r"\b(kvq_[a-z_]+)\s*\(([^)]*)\)\s*;", src):
+        params = params.strip()
+        out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_every_binding_declares_its_argument_types():
+    """Without argtypes ctypes passes a Python int as a C int, which would truncate a
+    device pointer; every entry point must declare one ctypes type per header parameter,
+    and a pointer-sized type wherever the header takes a pointer."""
+    from sparse_mixed_precision_kvq_b200 import kvq
+    counts = _param_counts()
+    assert sorted(counts) == _declared()
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    for n in kvq.EXPORTS:
+        at = getattr(kvq._lib, n).argtypes
+        assert at is not None and len(at) == counts[n], n
+        params = re.search(n + r"\s*\(([^)]*)\)", src).group(1).strip()
+        if params in ("", "void"):
+            continue
+        for decl, ty in zip(params.split(","), at):
+            if "*" in decl or "stream" in decl:
+                assert ctypes.sizeof(ty) == 8, (n, decl)
+
+
 def test_host_helpers_without_gpu():
     from sparse_mixed_precision_kvq_b200 import kvq
     assert [2 * kvq.kvq_chunk_bytes(t, 128) for t in range(5)] == [8192, 4608, 2560, 1536, 768]
