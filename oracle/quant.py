@@ -8,6 +8,8 @@ ARGUS ("Virtual Memory for Transformers", sections "The One-Minute Explanation" 
 quantiser, so this file takes the plainest affine reading and fixes every rounding:
 
 * a group is 32 consecutive channels of one token of one head (K or V alike);
+* ``lo`` and ``hi`` are the group's min and max as values: a zero extreme is +0 (the
+  signs of the zeros in a group do not change its bytes);
 * INT-b (b in {8, 4, 2}) is asymmetric min/max with a float zero offset:
   ``zero = fp16(lo)``, ``scale = fp16((hi - lo) / (2^b - 1))``,
   ``c = clamp(rint((x - zero) / scale), 0, 2^b - 1)`` (0 when scale == 0), and the
@@ -39,8 +41,8 @@ def quantise_int(x: np.ndarray, bits: int):
     x = np.asarray(x, dtype=np.float64)
     assert x.shape[-1] == GROUP
     qmax = float((1 << bits) - 1)
-    lo = x.min(axis=-1)
-    hi = x.max(axis=-1)
+    lo = x.min(axis=-1) + 0.0   # a zero extreme is +0 whatever the signs of the zeros
+    hi = x.max(axis=-1) + 0.0
     zero, zero_bits, ov0 = fp16_rne_sat(lo)
     scale, scale_bits, ov1 = fp16_rne_sat((hi - lo) / qmax)
     safe = np.where(scale == 0.0, 1.0, scale)

@@ -39,6 +39,8 @@ __device__ inline QOut quant_group(double x, int tier, bool& ov) {
     lo = fmin(lo, __shfl_xor_sync(full, lo, o));
     hi = fmax(hi, __shfl_xor_sync(full, hi, o));
   }
+  lo += 0.0;  // a zero extreme is +0, whichever zero the reduction met first
+  hi += 0.0;
   const double qmax = static_cast<double>((1 << tier_bits(tier)) - 1);
   const uint16_t zb = fp16_sat(lo, ov);
   const uint16_t sb = fp16_sat((hi - lo) / qmax, ov);

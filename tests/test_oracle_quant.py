@@ -87,6 +87,29 @@ def test_constant_group_is_exact():
             assert np.all(dequant_int(codes, scale, zero) == v)
 
 
+def test_zero_extremes_are_positive_zero():
+    """The signs of zeros do not change a group's bytes: a zero min gives zero = +0, and
+    an all-zero group (any mix of +0 and -0) gives scale = +0 and zero = +0."""
+    pos = np.abs(np.linspace(0.0, 3.0, GROUP))
+    for order in (1, -1):
+        x = pos.copy()
+        x[0] = -0.0
+        x[5] = 0.0
+        x = x[::order][None]
+        for bits in (2, 4, 8):
+            *_, sb, zb, _ = quantise_int(x, bits)
+            assert int(zb[0]) == 0x0000 and int(sb[0]) != 0
+            want = quantise_int(np.abs(x), bits)
+            assert np.array_equal(quantise_int(x, bits)[0], want[0])
+    z = np.zeros((1, GROUP))
+    z[0, ::3] = -0.0
+    for bits in (2, 4, 8):
+        *_, sb, zb, _ = quantise_int(z, bits)
+        assert int(sb[0]) == 0 and int(zb[0]) == 0
+        *_, sb, zb, _ = quantise_int(-np.zeros((1, GROUP)), bits)
+        assert int(sb[0]) == 0 and int(zb[0]) == 0
+
+
 @pytest.mark.parametrize("bits", [2, 4, 8])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 def test_roundtrip_bound(bits, dtype):
