@@ -16,6 +16,7 @@ import numpy as np
 from .attention import attend, token_index
 from .cache import SeqHead, append, build
 from .fp import bits16_to_f64
+from .quad import quad_scores
 from .score import page_scores
 from .select import select
 
@@ -27,18 +28,26 @@ def prepare(w, b: int, g: int) -> SeqHead:
 
 
 def step_pair(w, sh: SeqHead, b: int, g: int, q: np.ndarray, k_new=None, v_new=None,
-              sel=None) -> dict:
+              sel=None, quad=None) -> dict:
     """Run the step for one (b, g) on a prepared cache (mutated by the append).
 
     ``q`` is the fp64 query ``[Hq, D]`` of sequence b.  ``sel`` (optional) replaces
-    the selection by a given page list, for testing attention on its own.
+    the selection by a given page list, for testing attention on its own.  ``quad``
+    (optional, an ``oracle.quad.QuadState`` of the same pair) switches the page score
+    to the quad score; the append then also advances its state.
     """
     if w.append:
-        append(sh, int(w.lens[b]), k_new, v_new)
+        pos = int(w.lens[b])
+        append(sh, pos, k_new, v_new)
+        if quad is not None:
+            quad.append(pos, sh.korig[pos])
     P = sh.P
     G = w.G
     qg = q[g * G:(g + 1) * G]
-    scores = page_scores(qg, sh.summary, P, w.max_pages)
+    if quad is None:
+        scores = page_scores(qg, sh.summary, P, w.max_pages)
+    else:
+        scores = quad_scores(qg, sh.summary, quad.lam, quad.basis, w.sm_scale, P, w.max_pages)
     chosen = select(scores, P, w.k_abs, w.k_frac_bp, w.n_sink, w.n_recent)
     use = chosen if sel is None else np.asarray(sel, dtype=np.int64)
     idx = token_index(use, sh.L)

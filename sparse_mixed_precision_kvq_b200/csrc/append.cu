@@ -1,4 +1,5 @@
-// Quantise-and-pack: kvq_append (one token per sequence) and kvq_build_pages (whole pages).
+// Quantise-and-pack: kvq_append (one token per sequence), kvq_build_pages (whole pages) and
+// kvq_requantize_pages (tier demotion of whole pages).
 //
 // Tiers after ARGUS "Virtual Memory for Transformers", "The One-Minute Explanation" and
 // "Visual Architecture": 16-bit hot pages; INT8, INT4 (two per byte), INT2 (four per
@@ -9,6 +10,8 @@
 // operation with round-half-even, so the bytes do not depend on the thread mapping.
 // The per-page mean-key summary (AMASS "What is in the box": a tiny per-page summary)
 // is fp16(S / n) with S the fp64 sum of the page's keys in token order.
+#include <utility>
+
 #include "kvq_internal.cuh"
 #include "quant.cuh"
 
@@ -147,7 +150,163 @@ __device__ inline bool requant_item(const DevCache& c, const int32_t* items, int
   return !(nt == ot && ns == os);
 }
 
-template <bool BF16>
+// Re-quantiser of one (page, kv head), 128 threads, in three phases over shared memory:
+//  A  decode the current chunk word by word into fp32 values vals[j][group], group =
+//     (kind * 16 + t) * (D / 32) + d / 32 and j = d % 32 (one row per channel of a group,
+//     so that phase B reads without bank conflicts);
+//  B  one thread per (kind, token, 32-channel group): the group's min and max, its fp16
+//     zero and scale in fp64 as quant_group computes them, then each code from an fp32
+//     quotient; a quotient within 1e-4 of a rounding tie (or not finite) is recomputed
+//     exactly in fp64.  Away from ties both round to the same integer: the fp32 quotient
+//     is within 3 * 2^-24 relative of the exact one, i.e. within 5e-5 where the clamp to
+//     [0, 2^b - 1] does not decide the code.  Code bytes go to shared memory, metadata
+//     straight to the new chunk;
+//  C  one thread per word of the new codes area gathers its codes: one store per word.
+constexpr int kRqGroups = 2 * kPage * 128 / kGroup;  // groups per (page, kv head), D <= 128
+
+template <int OT, int KIND, int D, bool BF16, bool FULL, int I>
+__device__ inline void rq_decode_word(const uint32_t* chunk, int W0, int n, float (*vals)[kRqGroups + 1]) {
+  constexpr int ng = D / kGroup;
+  const unsigned char* meta = reinterpret_cast<const unsigned char*>(chunk) + codes_bytes(OT, D);
+  const uint32_t word = chunk[W0 + 128 * I];
+  word_elems_at<OT, KIND, D, I>(W0, [&](int t, int d, int sh) {
+    if (!FULL && t >= n) return;
+    float v;
+    if constexpr (OT == KVQ_TIER_16) {
+      v = bits_to_float<BF16>(static_cast<uint16_t>(word >> sh));
+    } else {
+      const uint32_t code = (word >> sh) & ((1u << tier_bits(OT)) - 1u);
+      if constexpr (OT == KVQ_TIER_I1) {
+        const float m = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(meta)[t * ng + (d >> 5)]));
+        v = code ? m : -m;
+      } else {
+        const uint32_t mw = reinterpret_cast<const uint32_t*>(meta)[t * ng + (d >> 5)];
+        v = fmaf(static_cast<float>(code), __half2float(__ushort_as_half(static_cast<uint16_t>(mw & 0xFFFFu))),
+                 __half2float(__ushort_as_half(static_cast<uint16_t>(mw >> 16))));
+      }
+    }
+    vals[d & 31][(KIND * kPage + t) * ng + (d >> 5)] = v;
+  });
+}
+
+// Thread W0 (< 128) decodes words W0, W0 + 128, ... of the K then the V codes area.
+template <int OT, int KIND, int D, bool BF16, bool FULL, int... Is>
+__device__ inline void rq_decode_kind(const uint32_t* chunk, int n, float (*vals)[kRqGroups + 1],
+                                      std::integer_sequence<int, Is...>) {
+  constexpr int wpk = codes_bytes(OT, D) / 4;
+  const int W0 = threadIdx.x;
+  ((W0 + 128 * Is < wpk ? rq_decode_word<OT, KIND, D, BF16, FULL, Is>(chunk, W0, n, vals) : void()), ...);
+}
+
+template <int OT, int D, bool BF16>
+__device__ inline void rq_decode(const uint32_t* oldw, int n, float (*vals)[kRqGroups + 1]) {
+  constexpr int wpk = codes_bytes(OT, D) / 4, cw = chunk_bytes(OT, D) / 4;
+  using Seq = std::make_integer_sequence<int, (wpk + 127) / 128>;
+  if (n == kPage) {  // a full page: no token-range test per element
+    rq_decode_kind<OT, 0, D, BF16, true>(oldw, n, vals, Seq{});
+    rq_decode_kind<OT, 1, D, BF16, true>(oldw + cw, n, vals, Seq{});
+  } else {
+    rq_decode_kind<OT, 0, D, BF16, false>(oldw, n, vals, Seq{});
+    rq_decode_kind<OT, 1, D, BF16, false>(oldw + cw, n, vals, Seq{});
+  }
+}
+
+template <int NT, int D>
+__device__ inline void rq_quant(int gid, int n, const float (*vals)[kRqGroups + 1], unsigned char* codes8,
+                                unsigned char* dst, bool& ov, bool& nonfinite) {
+  constexpr int ng = D / kGroup, NB = chunk_bytes(NT, D);
+  const int kind = gid / (kPage * ng), t = (gid / ng) % kPage, grp = gid % ng;
+  uint4* crow = reinterpret_cast<uint4*>(codes8 + (kind * kPage + t) * D + grp * kGroup);
+  unsigned char* meta = dst + kind * NB + codes_bytes(NT, D);
+  if (t >= n) {  // token slot past the sequence: zero codes and metadata
+    crow[0] = crow[1] = make_uint4(0, 0, 0, 0);
+    if constexpr (NT == KVQ_TIER_I1) reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = 0;
+    else reinterpret_cast<uint32_t*>(meta)[t * ng + grp] = 0u;
+    return;
+  }
+  float v[kGroup];
+#pragma unroll
+  for (int j = 0; j < kGroup; ++j) v[j] = vals[j][gid];
+  uint32_t packed[kGroup / 4];
+  if constexpr (NT == KVQ_TIER_I1) {
+    double s = 0.0;
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) s += fabs(static_cast<double>(v[j]));
+    nonfinite |= !isfinite(s);  // an infinite or NaN value makes the sum so
+#pragma unroll
+    for (int k = 0; k < kGroup / 4; ++k) {
+      packed[k] = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) packed[k] |= (v[4 * k + i] >= 0.0f ? 1u : 0u) << (8 * i);
+    }
+    reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = fp16_sat(s / 32.0, ov);
+  } else {
+    constexpr int qmax = (1 << tier_bits(NT)) - 1;
+    float lo = v[0], hi = v[0];
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) {
+      lo = fminf(lo, v[j]);
+      hi = fmaxf(hi, v[j]);
+    }
+    const double lod = static_cast<double>(lo) + 0.0, hid = static_cast<double>(hi) + 0.0;
+    const uint16_t zb = fp16_sat(lod, ov);
+    const uint16_t sb = fp16_sat((hid - lod) / static_cast<double>(qmax), ov);
+    const float zf = __half2float(__ushort_as_half(zb)), sf = __half2float(__ushort_as_half(sb));
+    const float inv = 1.0f / sf;
+    if (sf == 0.0f) {  // constant group (min/max skip NaN: check the values)
+#pragma unroll
+      for (int j = 0; j < kGroup; ++j) nonfinite |= !isfinite(v[j]);
+#pragma unroll
+      for (int k = 0; k < kGroup / 4; ++k) packed[k] = 0;
+    } else {
+#pragma unroll
+      for (int k = 0; k < kGroup / 4; ++k) {
+        packed[k] = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float x = v[4 * k + i];
+          const float q = (x - zf) * inv;
+          float c = rintf(q);
+          if (!(fabsf(q - c) < 0.4999f)) {  // near a tie, or not finite (every non-finite x lands here)
+            nonfinite |= !isfinite(x);
+            c = static_cast<float>(
+                rint((static_cast<double>(x) - static_cast<double>(zf)) / static_cast<double>(sf)));
+          }
+          // clamp to [0, qmax] (fmaxf maps NaN to 0); the codes of a word do not overlap
+          packed[k] += min(__float2uint_rn(fmaxf(c, 0.0f)), static_cast<uint32_t>(qmax)) << (8 * i);
+        }
+      }
+    }
+    reinterpret_cast<uint32_t*>(meta)[t * ng + grp] = static_cast<uint32_t>(sb) | (static_cast<uint32_t>(zb) << 16);
+  }
+  crow[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  crow[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+}
+
+template <int NT, int KIND, int D, int I>
+__device__ inline void rq_pack_word(const unsigned char* codes8, uint32_t* d32, int W0) {
+  uint32_t acc = 0;
+  word_elems_at<NT, KIND, D, I>(W0, [&](int t, int d, int sh) { acc |= static_cast<uint32_t>(codes8[t * D + d]) << sh; });
+  d32[W0 + 128 * I] = acc;
+}
+
+template <int NT, int KIND, int D, int... Is>
+__device__ inline void rq_pack_kind(const unsigned char* codes8, uint32_t* d32, std::integer_sequence<int, Is...>) {
+  constexpr int wpk = codes_bytes(NT, D) / 4;
+  const int W0 = threadIdx.x;
+  ((W0 + 128 * Is < wpk ? rq_pack_word<NT, KIND, D, Is>(codes8, d32, W0) : void()), ...);
+}
+
+template <int NT, int D>
+__device__ inline void rq_pack(const unsigned char* codes8, unsigned char* dst) {
+  constexpr int wpk = codes_bytes(NT, D) / 4, cw = chunk_bytes(NT, D) / 4;
+  using Seq = std::make_integer_sequence<int, (wpk + 127) / 128>;
+  uint32_t* d32 = reinterpret_cast<uint32_t*>(dst);
+  rq_pack_kind<NT, 0, D>(codes8, d32, Seq{});
+  rq_pack_kind<NT, 1, D>(codes8 + kPage * D, d32 + cw, Seq{});
+}
+
+template <bool BF16, int D>
 __global__ void __launch_bounds__(128) requant_kernel(DevCache c, const int32_t* __restrict__ items) {
   const int g = blockIdx.y, tid = threadIdx.x;
   int b, p, n;
@@ -156,43 +315,40 @@ __global__ void __launch_bounds__(128) requant_kernel(DevCache c, const int32_t*
     if (g == 0 && tid == 0) set_err(c.err, KVQ_DERR_BAD_PAGE);
     return;
   }
-  const int D = c.D, ot = static_cast<int>(oe >> 29), nt = static_cast<int>(ne >> 29);
-  const int OB = c.chunk[ot], NB = c.chunk[nt];
+  const int ot = static_cast<int>(oe >> 29), nt = static_cast<int>(ne >> 29);
+  const int OB = chunk_bytes(ot, D), NB = chunk_bytes(nt, D);
   const unsigned char* src = c.pool[ot] + ((size_t)(oe & 0x1FFFFFFFu) * c.Hkv + g) * 2 * (size_t)OB;
   unsigned char* dst = c.pool[nt] + ((size_t)(ne & 0x1FFFFFFFu) * c.Hkv + g) * 2 * (size_t)NB;
 
-  __shared__ __align__(16) uint32_t old_words[2048];   // current K and V chunks (<= 8 KB)
-  __shared__ __align__(16) uint32_t words[2][1024];    // new chunk images (<= 4 KB each)
+  __shared__ __align__(16) uint32_t old_words[2 * chunk_bytes(KVQ_TIER_16, 128) / 4];
+  __shared__ float vals[kGroup][kRqGroups + 1];
+  __shared__ __align__(16) unsigned char codes8[2 * kPage * 128];
   for (int k = tid; k < 2 * OB / 16; k += blockDim.x)
     reinterpret_cast<uint4*>(old_words)[k] = __ldcg(reinterpret_cast<const uint4*>(src) + k);
-  for (int k = tid; k < 2 * 1024; k += blockDim.x) (&words[0][0])[k] = 0u;
   __syncthreads();
-
-  const int warp = tid >> 5, lane = tid & 31, ng = D / kGroup;
+  switch (ot) {
+    case 0: rq_decode<0, D, BF16>(old_words, n, vals); break;
+    case 1: rq_decode<1, D, BF16>(old_words, n, vals); break;
+    case 2: rq_decode<2, D, BF16>(old_words, n, vals); break;
+    case 3: rq_decode<3, D, BF16>(old_words, n, vals); break;
+    default: rq_decode<4, D, BF16>(old_words, n, vals); break;
+  }
+  __syncthreads();
   bool ov = false, nonfinite = false;
-  for (int gi = warp; gi < 2 * n * ng; gi += 4) {
-    const int kind = gi / (n * ng), rem = gi % (n * ng), t = rem / ng, grp = rem % ng;
-    const int d = grp * kGroup + lane;
-    const unsigned char* oc = reinterpret_cast<const unsigned char*>(old_words) + kind * OB;
-    const double x = static_cast<double>(load_value(oc, kind, ot, D, BF16, t, d));
-    nonfinite |= !isfinite(x);
-    const QOut q = quant_group(x, nt, ov);
-    int w, bit;
-    elem_pos(kind, nt, D, t, d, w, bit);
-    atomicOr(&words[kind][w], q.code << bit);
-    if (lane == 0) {
-      unsigned char* meta = reinterpret_cast<unsigned char*>(words[kind]) + codes_bytes(nt, D);
-      if (nt == KVQ_TIER_I1)
-        reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = static_cast<uint16_t>(q.meta);
-      else
-        reinterpret_cast<uint32_t*>(meta)[t * ng + grp] = q.meta;
+  if (tid < 2 * kPage * (D / kGroup)) {
+    switch (nt) {
+      case 1: rq_quant<1, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
+      case 2: rq_quant<2, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
+      case 3: rq_quant<3, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
+      default: rq_quant<4, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
     }
   }
   __syncthreads();
-  for (int kind = 0; kind < 2; ++kind) {
-    const uint4* s4 = reinterpret_cast<const uint4*>(words[kind]);
-    uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)kind * NB);
-    for (int k = tid; k < NB / 16; k += blockDim.x) d4[k] = s4[k];
+  switch (nt) {
+    case 1: rq_pack<1, D>(codes8, dst); break;
+    case 2: rq_pack<2, D>(codes8, dst); break;
+    case 3: rq_pack<3, D>(codes8, dst); break;
+    default: rq_pack<4, D>(codes8, dst); break;
   }
   if (ov) set_err(c.err, KVQ_DERR_FP16_RANGE);
   if (nonfinite) set_err(c.err, KVQ_DERR_NONFINITE);
@@ -232,8 +388,14 @@ cudaError_t launch_build(const DevCache& c, const void* k_src, const void* v_src
 
 cudaError_t launch_requantize(const DevCache& c, const int32_t* items, int n, cudaStream_t s) {
   const dim3 grid(n, c.Hkv);
-  if (c.dtype == KVQ_DT_BF16) requant_kernel<true><<<grid, 128, 0, s>>>(c, items);
-  else requant_kernel<false><<<grid, 128, 0, s>>>(c, items);
+  const bool bf = c.dtype == KVQ_DT_BF16;
+  if (c.D == 128) {
+    if (bf) requant_kernel<true, 128><<<grid, 128, 0, s>>>(c, items);
+    else requant_kernel<false, 128><<<grid, 128, 0, s>>>(c, items);
+  } else {
+    if (bf) requant_kernel<true, 64><<<grid, 128, 0, s>>>(c, items);
+    else requant_kernel<false, 64><<<grid, 128, 0, s>>>(c, items);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   requant_commit_kernel<<<(n + 255) / 256, 256, 0, s>>>(c, items, n);
