@@ -113,8 +113,10 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- bytes
-def algorithmic_bytes(w, sel: np.ndarray, cnt: np.ndarray, tier_tbl: np.ndarray):
-    """Bytes the step must move: (attention, scores, select, append) per launch."""
+def algorithmic_bytes(w, sel: np.ndarray, cnt: np.ndarray, tier_tbl: np.ndarray, quad_rank: int = 0):
+    """Bytes the step must move: (attention, scores, select, append) per launch; with the
+    quad score the scores also read r' fp16 eigenvalues per page and the append updates
+    the open page's sums and eigenvalues."""
     from sparse_mixed_precision_kvq_b200.kvq import kvq_chunk_bytes
     cb = np.array([2 * kvq_chunk_bytes(t, w.D) for t in range(5)], dtype=np.int64)
     attn = 0
@@ -125,9 +127,11 @@ def algorithmic_bytes(w, sel: np.ndarray, cnt: np.ndarray, tier_tbl: np.ndarray)
     q_bytes = w.B * w.Hq * w.D * 2
     attn += q_bytes + w.B * w.Hq * w.D * 2 + int(cnt.sum()) * 4          # q, out, page list
     P = np.array([w.pages_after(b) for b in range(w.B)])
-    score = int(P.sum()) * w.Hkv * w.D * 2 + q_bytes + w.B * w.Hkv * w.max_pages * 4
+    score = int(P.sum()) * w.Hkv * (w.D + quad_rank) * 2 + q_bytes + w.B * w.Hkv * w.max_pages * 4
     select = w.B * w.Hkv * w.max_pages * 4 + int(cnt.sum()) * 4
     append = w.B * w.Hkv * w.D * 2 * 2 if w.append else 0
+    if w.append and quad_rank:
+        append += w.B * w.Hkv * (w.D * 2 + quad_rank * (4 * 8 + 2))  # key, sums read + written, lambda
     return dict(attn=attn, score=score, select=select, append=append)
 
 
@@ -179,8 +183,12 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = rank_workload(args.config, rank, args.batch)
-    cache = kvq.cache_from_workload(w, device=dev)
-    step = kvq.DecodeStep(w, cache, device=dev, coverage=args.coverage)
+    quad_rank = args.quad_rank if args.score == "quad" else 0
+    basis = None
+    if quad_rank:
+        basis = np.stack([w.quad_basis(g, quad_rank, "law") for g in range(w.Hkv)])
+    cache = kvq.cache_from_workload(w, device=dev, quad_basis=basis)
+    step = kvq.DecodeStep(w, cache, device=dev, coverage=args.coverage, quad=bool(quad_rank))
     tier_tbl, _, _ = w.slot_map()
     flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -191,7 +199,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize(dev)
     assert cache.err_bits() == 0, f"device error bits {cache.err_bits():#x}"
     sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
-    nbytes = algorithmic_bytes(w, sel, cnt, tier_tbl)
+    nbytes = algorithmic_bytes(w, sel, cnt, tier_tbl, quad_rank)
 
     K = args.steps
     fused = args.path == "fused"
@@ -313,7 +321,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
         files = ["score.cu", "select.cu", "attn.cu"]
     else:
         dom_bytes = [nbytes["append"], nbytes["score"], nbytes["select"], nbytes["attn"]][dom]
-        files = ["append.cu", "score.cu", "select.cu", "attn.cu"]
+        files = ["append.cu", "quad.cu" if quad_rank else "score.cu", "select.cu", "attn.cu"]
     achieved = dom_bytes / (avg[dom] * 1e-3) / 1e9
     tr = kernel_traffic(files[dom])
     line = {
@@ -333,6 +341,8 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
                    "context": int(w.lens.max()), "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
                    "selected_pages": int(cnt.sum()),
                    "selection": "budget" if args.coverage is None else f"coverage {args.coverage}",
+                   "page_score": "mean-key" if not quad_rank else
+                   f"quad (rank {quad_rank}, basis: eigenvectors of the key law's covariance)",
                    "l2": f"flushed ({args.flush_mib} MiB write) before every timed step",
                    "parallelism": f"replicas x{world} (independent batches)"},
         "step_hbm": {"bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3) / 1e9,
@@ -345,7 +355,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
                      "traffic": None if tr is None else tr["dram_bytes_per_launch"]},
         "e2e": {"value": world * w.B / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
-        "gpu_launches": len(parts) * K,
+        "gpu_launches": (len(parts) + (1 if quad_rank and w.append else 0)) * K,
         "path": {"fused": "kvq_decode_step (one persistent launch)",
                  "two": "kvq_score_select -> kvq_sparse_decode_attn",
                  "three": "kvq_append_scores -> kvq_select_topk -> kvq_sparse_decode_attn",
@@ -504,6 +514,9 @@ def main():
     ap.add_argument("--path", default="calls", choices=["calls", "three", "two", "fused"],
                     help="the four separate calls; kvq_append_scores + select + attention; kvq_score_select + "
                          "attention; or one kvq_decode_step launch")
+    ap.add_argument("--score", default="mean", choices=["mean", "quad"],
+                    help="page score: the mean-key score, or the quad (Gaussian-MGF) score (four-call path only)")
+    ap.add_argument("--quad-rank", type=int, default=16, help="r' of the quad score (8, 16, 24 or 32)")
     ap.add_argument("--dense", action="store_true", help="also time attention over every page")
     ap.add_argument("--demote", type=int, default=None, choices=[1, 2, 3, 4],
                     help="also time kvq_requantize_pages moving the workload's pages outside the sink and "
@@ -517,6 +530,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.coverage is not None and args.path != "calls":
         ap.error("--coverage runs on the four-call path")
+    if args.score == "quad" and args.path != "calls":
+        ap.error("--score quad runs on the four-call path")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

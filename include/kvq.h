@@ -296,6 +296,47 @@ kvq_status kvq_decode_step(const kvq_cache* cache, const int32_t* pos, const voi
                            kvq_stream_t stream);
 
 /*
+ * quad page score (AMASS "decode-time sparse KV-cache attention for vLLM", "What is in the
+ * box", Stage A: a quadratic Gaussian-MGF page score from a tiny per-page summary holding
+ * r' eigenvalues per page).  The pages give no formula, rank or basis; this library reads
+ * it as follows.  Keys of page p ~ N(mu_p, Sigma_p); with the caller's orthonormal basis
+ * rows u_1..u_r' of a kv head, page p keeps lambda[p][i] = u_i^T Sigma_p u_i (the (1/n)
+ * variance of the page's keys, as they arrived, along u_i), and its score for query head h
+ * is log E[exp(s q_h.k)] ~= s q_h.kbar_p + 1/2 s^2 sum_i lambda[p][i] (u_i.q_h)^2 (kbar_p
+ * the fp16 mean-key summary), maximised over the kv head's query heads.
+ * State arithmetic (fp64, no fused multiply-add, so built and appended pages agree bit for
+ * bit): y_i = sum_d u[i][d] k[d] in channel order; per page S1_i = sum_t y_i, S2_i =
+ * sum_t y_i^2 in token order; lambda = fp16(max(S2/n - (S1/n)^2, 0)), saturating (flagged).
+ */
+typedef struct {
+  int32_t rank;        /* r', a multiple of 8 in [8, 32] */
+  int32_t reserved;
+  const float* basis;  /* device [Hkv][rank][D] fp32, the basis rows of each kv head (caller-owned) */
+  uint16_t* lambda;    /* device [B][Hkv][max_pages][rank] fp16 bits */
+  double* open_sums;   /* device [B][Hkv][2][rank]: S1 then S2 of each sequence's open page */
+} kvq_quad;
+
+/* kvq_quad_build -- quad state of a prefilled context (same inputs as kvq_build_pages):
+ *  lambda of every page holding tokens, and the open page's sums (zero when the last page
+ *  is full).  Pages past seq_len are not written. */
+kvq_status kvq_quad_build(const kvq_cache* cache, const kvq_quad* quad, const void* k_src,
+                          const int64_t* cu_seqlens, int64_t src_tokens, kvq_stream_t stream);
+
+/* kvq_quad_append -- advance the quad state by one token per sequence (same pos and k_new
+ *  as kvq_append; pos < 0 skips, pos >= max_pages*16 sets KVQ_DERR_BAD_POS): the open
+ *  page's sums restart at a page boundary, and lambda[pos/16] is refreshed. */
+kvq_status kvq_quad_append(const kvq_cache* cache, const kvq_quad* quad, const int32_t* pos,
+                           const void* k_new, kvq_stream_t stream);
+
+/* kvq_quad_page_scores -- scores[b][g][p] = max over h in the group of
+ *  sm_scale * q_h.kbar_p + 0.5 * sm_scale^2 * sum_i lambda[b][g][p][i] * (u_i.q_h)^2,
+ *  fp32, for p < ceil(seq_len[b]/16), -inf for the remaining pages (layouts as
+ *  kvq_page_scores; q must be 16-byte aligned).  Feed the result to kvq_select_topk; for
+ *  coverage selection pass sm_scale = 1 there (the score already carries the scale). */
+kvq_status kvq_quad_page_scores(const kvq_cache* cache, const kvq_quad* quad, const void* q,
+                                float sm_scale, float* scores, kvq_stream_t stream);
+
+/*
  * kvq_requantize_pages -- tier demotion: move pages to a lower-precision tier.
  * (ARGUS "Virtual Memory for Transformers", "Visual Architecture": pages cool down the
  *  cascade FP16 -> INT8 -> INT4 -> INT2 -> 1-bit.)

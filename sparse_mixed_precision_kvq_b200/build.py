@@ -4,8 +4,8 @@
 
 Each ``csrc/*.cu`` is compiled to an object with
 ``-gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`` (no fast-math; the
-quantise-and-pack unit also gets ``-fmad=false`` so its fp64 metadata math is a fixed
-sequence of IEEE operations), then linked into ``lib/libkvq.so`` with the static CUDA
+quantise-and-pack and quad-state units also get ``-fmad=false`` so their fp64 metadata
+math is a fixed sequence of IEEE operations), then linked into ``lib/libkvq.so`` with the static CUDA
 runtime.  Rebuilds only when a source or header is newer than the library.
 """
 from __future__ import annotations
@@ -27,7 +27,7 @@ OBJDIR = os.path.join(ROOT, "_build")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
-PER_FILE = {"append.cu": ["-fmad=false"]}
+PER_FILE = {"append.cu": ["-fmad=false"], "quad.cu": ["-fmad=false"]}
 
 
 def nvcc() -> str:

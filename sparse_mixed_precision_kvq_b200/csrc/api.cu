@@ -63,6 +63,19 @@ kvq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_E
 
 bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
 
+kvq_status to_quad(const kvq_quad* k, DevQuad& q) {
+  if (k == nullptr || k->basis == nullptr || k->lambda == nullptr || k->open_sums == nullptr)
+    return KVQ_ERR_INVALID_ARG;
+  if (k->rank < 8 || k->rank > kMaxQuadRank || k->rank % 8 != 0) return KVQ_ERR_UNSUPPORTED;
+  if (!aligned16(k->basis) || !aligned16(k->lambda) || reinterpret_cast<uintptr_t>(k->open_sums) % 8 != 0)
+    return KVQ_ERR_INVALID_ARG;
+  q.rank = k->rank;
+  q.basis = k->basis;
+  q.lambda = k->lambda;
+  q.open = k->open_sums;
+  return KVQ_OK;
+}
+
 int current_device() {
   int d = 0;
   if (cudaGetDevice(&d) != cudaSuccess) d = 0;
@@ -221,6 +234,39 @@ kvq_status kvq_decode_step(const kvq_cache* cache, const int32_t* pos, const voi
 kvq_status kvq_workspace_init(void* workspace, size_t ws_bytes, kvq_stream_t stream) {
   if (workspace == nullptr || ws_bytes < kCounterBytes || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
   return cuda_status(cudaMemsetAsync(workspace, 0, kCounterBytes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_quad_build(const kvq_cache* cache, const kvq_quad* quad, const void* k_src,
+                          const int64_t* cu_seqlens, int64_t src_tokens, kvq_stream_t stream) {
+  DevCache c;
+  DevQuad q;
+  kvq_status st = to_dev(cache, c);
+  if (st == KVQ_OK) st = to_quad(quad, q);
+  if (st != KVQ_OK) return st;
+  if (k_src == nullptr || cu_seqlens == nullptr || src_tokens < 0) return KVQ_ERR_INVALID_ARG;
+  return cuda_status(launch_quad_build(c, q, k_src, cu_seqlens, src_tokens, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_quad_append(const kvq_cache* cache, const kvq_quad* quad, const int32_t* pos, const void* k_new,
+                           kvq_stream_t stream) {
+  DevCache c;
+  DevQuad q;
+  kvq_status st = to_dev(cache, c);
+  if (st == KVQ_OK) st = to_quad(quad, q);
+  if (st != KVQ_OK) return st;
+  if (pos == nullptr || k_new == nullptr) return KVQ_ERR_INVALID_ARG;
+  return cuda_status(launch_quad_append(c, q, pos, k_new, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_quad_page_scores(const kvq_cache* cache, const kvq_quad* quad, const void* q, float sm_scale,
+                                float* scores, kvq_stream_t stream) {
+  DevCache c;
+  DevQuad qd;
+  kvq_status st = to_dev(cache, c);
+  if (st == KVQ_OK) st = to_quad(quad, qd);
+  if (st != KVQ_OK) return st;
+  if (q == nullptr || scores == nullptr || !aligned16(q) || !(sm_scale > 0.0f)) return KVQ_ERR_INVALID_ARG;
+  return cuda_status(launch_quad_scores(c, qd, q, sm_scale, scores, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 kvq_status kvq_requantize_pages(const kvq_cache* cache, const int32_t* items, int32_t n, kvq_stream_t stream) {

@@ -20,14 +20,23 @@ constexpr int kMaxSegments = 6144;  // B * Hkv limit of the attention kernel (of
 // leaves them zero); kvq_workspace_init zeroes it once.
 constexpr size_t kCounterBytes = 65536;
 
-__host__ __device__ inline int tier_bits(int tier) {
+__host__ __device__ constexpr int tier_bits(int tier) {
   return tier == 0 ? 16 : tier == 1 ? 8 : tier == 2 ? 4 : tier == 3 ? 2 : 1;
 }
-__host__ __device__ inline int codes_bytes(int tier, int D) { return kPage * D * tier_bits(tier) / 8; }
-__host__ __device__ inline int meta_bytes(int tier, int D) {
+__host__ __device__ constexpr int codes_bytes(int tier, int D) { return kPage * D * tier_bits(tier) / 8; }
+__host__ __device__ constexpr int meta_bytes(int tier, int D) {
   return tier == 0 ? 0 : kPage * (D / kGroup) * (tier == 4 ? 2 : 4);
 }
-__host__ __device__ inline int chunk_bytes(int tier, int D) { return codes_bytes(tier, D) + meta_bytes(tier, D); }
+__host__ __device__ constexpr int chunk_bytes(int tier, int D) { return codes_bytes(tier, D) + meta_bytes(tier, D); }
+
+// quad page-score state (see kvq_quad in kvq.h).
+constexpr int kMaxQuadRank = 32;
+struct DevQuad {
+  int rank;
+  const float* basis;
+  uint16_t* lambda;
+  double* open;
+};
 
 // Everything a kernel needs to locate pages (copied by value into kernel parameters).
 struct DevCache {
@@ -69,6 +78,76 @@ __host__ __device__ inline void elem_pos(int kind, int tier, int D, int t, int d
   const int pw = nw < 4 ? nw : 4;
   word = ((w / pw) * 32 + lam) * pw + (w % pw);
   bit = b * j + 16 * h;
+}
+
+// Token t and channel c (0..15 within the 16-channel block) of fragment lane `lam`,
+// register `r`, half `h` of a K (KIND 0) or V (KIND 1) chunk: the inverse of elem_pos.
+template <int KIND>
+__host__ __device__ constexpr void frag_tc(int lam, int r, int h, int& t, int& c) {
+  if (KIND == 0) {
+    t = 8 * (r & 1) + (lam >> 2);
+    c = 8 * (r >> 1) + 2 * (lam & 3) + h;
+  } else {
+    c = 8 * (r & 1) + (lam >> 2);
+    t = 8 * (r >> 1) + 2 * (lam & 3) + h;
+  }
+}
+
+// Every element stored in word W of a chunk's codes area: f(t, d, shift) for each, shift
+// being the bit offset of its code (16-bit tier: of its value) in the word.
+template <int TIER, int KIND, int D, typename F>
+__host__ __device__ inline void word_elems(int W, F&& f) {
+  if constexpr (TIER == 0) {
+    const int kk = W >> 7, lam = (W >> 2) & 31, r = W & 3;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      int t = 0, c = 0;
+      frag_tc<KIND>(lam, r, h, t, c);
+      f(t, 16 * kk + c, 16 * h);
+    }
+  } else {
+    constexpr int b = tier_bits(TIER), ppw = 16 / b, nw = D * b / 64, pw = nw < 4 ? nw : 4;
+    const int lam = (W / pw) & 31, w = (W / (32 * pw)) * pw + W % pw;
+#pragma unroll
+    for (int j = 0; j < ppw; ++j) {
+      const int R = w * ppw + j, kk = R >> 2, r = R & 3;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        int t = 0, c = 0;
+        frag_tc<KIND>(lam, r, h, t, c);
+        f(t, 16 * kk + c, b * j + 16 * h);
+      }
+    }
+  }
+}
+
+// word_elems for word W = W0 + 128 * i of a chunk's codes area (0 <= W0 < 128, i a
+// compile-time constant after unrolling): the position inside the word's 128-word block
+// fixes lam, r and the pair index modulo 4, so only a constant offset depends on i.
+template <int TIER, int KIND, int D, int I, typename F>
+__host__ __device__ inline void word_elems_at(int W0, F&& f) {
+  if constexpr (TIER == 0) {
+    const int lam = (W0 >> 2) & 31, r = W0 & 3;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      int t = 0, c = 0;
+      frag_tc<KIND>(lam, r, h, t, c);
+      f(t, 16 * I + c, 16 * h);
+    }
+  } else {
+    constexpr int b = tier_bits(TIER), ppw = 16 / b, nw = D * b / 64, pw = nw < 4 ? nw : 4;
+    const int lam = (W0 / pw) & 31, w = (W0 / (32 * pw)) * pw + W0 % pw + 4 * I;
+#pragma unroll
+    for (int j = 0; j < ppw; ++j) {
+      const int R = w * ppw + j, kk = R >> 2, r = R & 3;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        int t = 0, c = 0;
+        frag_tc<KIND>(lam, r, h, t, c);
+        f(t, 16 * kk + c, b * j + 16 * h);
+      }
+    }
+  }
 }
 
 __device__ inline void set_err(uint32_t* err, uint32_t bits) {
@@ -179,5 +258,11 @@ cudaError_t launch_step(const DevCache& c, const int32_t* pos, const void* k_new
                         int kmax, float sm_scale, void* out, float* lse, void* ws, int num_ctas, cudaStream_t s);
 cudaError_t launch_dequant(const DevCache& c, int b, int page, float* out, cudaStream_t s);
 cudaError_t launch_requantize(const DevCache& c, const int32_t* items, int n, cudaStream_t s);
+cudaError_t launch_quad_build(const DevCache& c, const DevQuad& qd, const void* k_src, const int64_t* cu,
+                              int64_t src_tokens, cudaStream_t s);
+cudaError_t launch_quad_append(const DevCache& c, const DevQuad& qd, const int32_t* pos, const void* k_new,
+                               cudaStream_t s);
+cudaError_t launch_quad_scores(const DevCache& c, const DevQuad& qd, const void* q, float sm_scale, float* scores,
+                               cudaStream_t s);
 
 }  // namespace kvq

@@ -1,0 +1,289 @@
+// quad page score: kvq_quad_build, kvq_quad_append and kvq_quad_page_scores.
+//
+// AMASS "decode-time sparse KV-cache attention for vLLM", "What is in the box", Stage A:
+// a quadratic, Gaussian-MGF page score built from a tiny per-page summary that keeps r'
+// eigenvalues per page.  Reading (the page gives no formula, rank or basis): with the
+// caller's orthonormal basis rows u_i of a kv head, page p keeps
+// lambda[p][i] = u_i^T Sigma_p u_i, the (1/n) variance of its keys along u_i, and scores
+//   max_h  s q_h.kbar_p + 1/2 s^2 sum_i lambda[p][i] (u_i.q_h)^2,
+// the log of the Gaussian moment-generating function E[exp(s q.k)] for k ~ N(kbar_p,
+// Sigma_p) restricted to the basis.
+//
+// State arithmetic is IEEE fp64 without fused multiply-add (this unit is compiled with
+// -fmad=false): y_i = sum_d u[i][d] k[d] in channel order, S1 = sum_t y and S2 = sum_t y^2
+// in token order, lambda = fp16(max(S2/n - (S1/n)^2, 0)); a page built at once and a page
+// grown token by token hold the same bits.  The score is fp32: the q.kbar part on the
+// tensor core exactly as kvq_page_scores (score_tile.cuh), the quadratic part on the CUDA
+// cores from (u_i.q_h)^2 computed once per (sequence, kv head) and warp.
+#include <math.h>
+
+#include "kvq_internal.cuh"
+#include "ptx.cuh"
+#include "score_tile.cuh"
+
+namespace kvq {
+namespace {
+
+template <bool BF16>
+__device__ inline double key_f64(uint16_t v) {
+  return static_cast<double>(bits_to_float<BF16>(v));
+}
+
+__device__ inline uint16_t quad_lambda(double s1, double s2, int n, bool& ov) {
+  const double m = s1 / static_cast<double>(n);
+  double v = s2 / static_cast<double>(n) - m * m;
+  v = v > 0.0 ? v : 0.0;
+  return fp16_sat(v, ov);
+}
+
+// One CTA per (page, sequence * kv head) of the prefilled context.
+template <bool BF16>
+__global__ void __launch_bounds__(256) quad_build_kernel(DevCache c, DevQuad qd, const uint16_t* __restrict__ ksrc,
+                                                         const int64_t* __restrict__ cu, int64_t src_tokens) {
+  const int p = blockIdx.x, bg = blockIdx.y;
+  const int b = bg / c.Hkv, g = bg % c.Hkv;
+  const int D = c.D, r = qd.rank, tid = threadIdx.x;
+  const int L = c.seq_len[b];
+  const int P = (L + kPage - 1) / kPage;
+  if (p >= P || p >= c.max_pages) return;
+  const int n = min(kPage, L - p * kPage);
+  const int64_t row0 = cu[b] + (int64_t)p * kPage;
+  if (row0 < 0 || row0 + n > src_tokens) {
+    if (tid == 0) set_err(c.err, KVQ_DERR_BAD_POS);
+    return;
+  }
+  __shared__ float ub[kMaxQuadRank * 128];  // basis rows of kv head g
+  __shared__ uint16_t kb[kPage * 128];      // the page's keys
+  __shared__ double ys[kPage][kMaxQuadRank + 1];
+  for (int i = tid; i < r * D; i += blockDim.x) ub[i] = qd.basis[(size_t)g * r * D + i];
+  for (int i = tid; i < n * D; i += blockDim.x) {
+    const int t = i / D, d = i % D;
+    kb[i] = ksrc[((size_t)g * src_tokens + (size_t)(row0 + t)) * D + d];
+  }
+  __syncthreads();
+  for (int e = tid; e < n * r; e += blockDim.x) {
+    const int t = e / r, i = e % r;
+    double y = 0.0;
+    for (int d = 0; d < D; ++d) y = y + static_cast<double>(ub[i * D + d]) * key_f64<BF16>(kb[t * D + d]);
+    ys[t][i] = y;
+  }
+  __syncthreads();
+  if (tid < r) {
+    double s1 = 0.0, s2 = 0.0;
+    for (int t = 0; t < n; ++t) {
+      const double y = ys[t][tid];
+      s1 = s1 + y;
+      s2 = s2 + y * y;
+    }
+    bool ov = false;
+    qd.lambda[((size_t)bg * c.max_pages + p) * r + tid] = quad_lambda(s1, s2, n, ov);
+    if (p == P - 1) {
+      double* o = qd.open + (size_t)bg * 2 * r;
+      o[tid] = (L % kPage) ? s1 : 0.0;
+      o[r + tid] = (L % kPage) ? s2 : 0.0;
+    }
+    if (ov) set_err(c.err, KVQ_DERR_FP16_RANGE);
+  }
+}
+
+// One warp per (sequence, kv head); lane i < r owns basis row i.
+template <bool BF16>
+__global__ void __launch_bounds__(32) quad_append_kernel(DevCache c, DevQuad qd, const int32_t* __restrict__ pos,
+                                                         const uint16_t* __restrict__ k_new) {
+  const int bg = blockIdx.x, b = bg / c.Hkv, g = bg % c.Hkv, lane = threadIdx.x;
+  const int D = c.D, r = qd.rank;
+  griddep_wait();
+  const int ps = pos[b];
+  if (ps >= 0 && ps >= c.max_pages * kPage) {
+    if (lane == 0 && g == 0) set_err(c.err, KVQ_DERR_BAD_POS);
+  } else if (ps >= 0 && lane < r) {
+    const int p = ps / kPage, t = ps % kPage;
+    const float* u = qd.basis + ((size_t)g * r + lane) * D;
+    const uint16_t* k = k_new + (size_t)bg * D;
+    double y = 0.0;
+    for (int d = 0; d < D; ++d) y = y + static_cast<double>(u[d]) * key_f64<BF16>(k[d]);
+    double* o = qd.open + (size_t)bg * 2 * r;
+    const double s1 = t == 0 ? y : o[lane] + y;
+    const double s2 = t == 0 ? y * y : o[r + lane] + y * y;
+    o[lane] = s1;
+    o[r + lane] = s2;
+    bool ov = false;
+    qd.lambda[((size_t)bg * c.max_pages + p) * r + lane] = quad_lambda(s1, s2, t + 1, ov);
+    if (ov) set_err(c.err, KVQ_DERR_FP16_RANGE);
+  }
+  griddep_launch_dependents();
+}
+
+constexpr int kQuadWarps = 8;
+
+template <int D>
+__device__ inline void quad_load_tile(const uint16_t* sbase, const uint16_t* lbase, int r, int tile, int P, int lane,
+                                      uint4 (&av)[2][D / 32], uint4 (&lv)[2][kMaxQuadRank / 8]) {
+  constexpr int CW = D / 4;
+  const int g8 = lane >> 2, q4 = lane & 3;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int p = tile * 16 + g8 + 8 * h;
+    const uint4* src = reinterpret_cast<const uint4*>(sbase + (size_t)p * D + CW * q4);
+#pragma unroll
+    for (int i = 0; i < CW / 8; ++i) av[h][i] = p < P ? __ldcg(src + i) : make_uint4(0, 0, 0, 0);
+    const uint4* ls = reinterpret_cast<const uint4*>(lbase + (size_t)p * r);
+#pragma unroll
+    for (int k = 0; k < kMaxQuadRank / 8; ++k) lv[h][k] = (p < P && 8 * k < r) ? __ldcg(ls + k) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Warp w takes tiles [w * per, (w + 1) * per) of the flat list (b, g, 16-page tile), as
+// kvq_page_scores does, loading the next tile (summary rows and lambda rows) while the
+// current one is multiplied; the two buffers take more registers than two CTAs per SM
+// leave, so one CTA of 8 warps runs per SM.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kQuadWarps * 32, 1)
+    quad_score_kernel(DevCache c, DevQuad qd, const uint16_t* __restrict__ q, float sm_scale,
+                      float* __restrict__ scores, int tiles_per_bg, int per) {
+  __shared__ float zs[kQuadWarps][kMaxG][kMaxQuadRank];  // (u_i . q_h)^2 of the warp's current (b, g)
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g8 = lane >> 2, q4 = lane & 3;
+  const int r = qd.rank;
+  const int total = c.B * c.Hkv * tiles_per_bg;
+  const int i0 = (blockIdx.x * kQuadWarps + warp) * per;
+  const int i1 = min(total, i0 + per);
+  griddep_wait();
+  if (i0 < i1) {
+    const float c1 = sm_scale, c2 = 0.5f * sm_scale * sm_scale;
+    QFrag<D, BF16> qf;
+    int cur_bg = -1, P = 0;
+    float* out = nullptr;
+    bool bad = false;
+    uint4 av0[2][D / 32], av1[2][D / 32];
+    uint4 lv0[2][kMaxQuadRank / 8], lv1[2][kMaxQuadRank / 8];
+
+    auto load = [&](int i, uint4 (&av)[2][D / 32], uint4 (&lv)[2][kMaxQuadRank / 8]) {
+      const int bg = i / tiles_per_bg;
+      const int L = c.seq_len[bg / c.Hkv];
+      const int Pn = min((L + kPage - 1) / kPage, c.max_pages);
+      quad_load_tile<D>(c.summary + (size_t)bg * c.max_pages * D, qd.lambda + (size_t)bg * c.max_pages * r, r,
+                        i % tiles_per_bg, Pn, lane, av, lv);
+    };
+    auto compute = [&](int i, const uint4 (&av)[2][D / 32], const uint4 (&lv)[2][kMaxQuadRank / 8]) {
+      const int bg = i / tiles_per_bg, tile = i % tiles_per_bg;
+      if (bg != cur_bg) {  // new (b, g): query fragments and (u_i . q_h)^2
+        cur_bg = bg;
+        const int b = bg / c.Hkv, g = bg % c.Hkv;
+        const int L = c.seq_len[b];
+        P = min((L + kPage - 1) / kPage, c.max_pages);
+        out = scores + (size_t)bg * c.max_pages;
+        qf.load(q, c.Hq, c.G, b, g, lane, bad);
+        __syncwarp();
+        for (int h = 0; h < kMaxG; ++h) {
+          float z = 0.0f;
+          if (h < c.G && lane < r) {
+            const float4* u = reinterpret_cast<const float4*>(qd.basis + ((size_t)g * r + lane) * D);
+            const uint2* qh = reinterpret_cast<const uint2*>(q + ((size_t)b * c.Hq + (size_t)g * c.G + h) * D);
+#pragma unroll 4
+            for (int d4 = 0; d4 < D / 4; ++d4) {
+              const float4 uv = u[d4];
+              const uint2 qv = qh[d4];
+              z = fmaf(uv.x, bits_to_float<BF16>(static_cast<uint16_t>(qv.x & 0xFFFFu)), z);
+              z = fmaf(uv.y, bits_to_float<BF16>(static_cast<uint16_t>(qv.x >> 16)), z);
+              z = fmaf(uv.z, bits_to_float<BF16>(static_cast<uint16_t>(qv.y & 0xFFFFu)), z);
+              z = fmaf(uv.w, bits_to_float<BF16>(static_cast<uint16_t>(qv.y >> 16)), z);
+            }
+          }
+          zs[warp][h][lane] = z * z;
+        }
+        __syncwarp();
+      }
+      float v[4];
+      tile_head_dots<D, BF16>(av, qf, v);
+      float qs[4] = {0.f, 0.f, 0.f, 0.f};
+      const float* z0 = zs[warp][(2 * q4) & (kMaxG - 1)];
+      const float* z1 = zs[warp][(2 * q4 + 1) & (kMaxG - 1)];
+#pragma unroll
+      for (int k = 0; k < kMaxQuadRank / 8; ++k) {
+        if (8 * k < r) {
+          const uint32_t w0[4] = {lv[0][k].x, lv[0][k].y, lv[0][k].z, lv[0][k].w};
+          const uint32_t w1[4] = {lv[1][k].x, lv[1][k].y, lv[1][k].z, lv[1][k].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 l0 = __half22float2(*reinterpret_cast<const __half2*>(&w0[e]));
+            const float2 l1 = __half22float2(*reinterpret_cast<const __half2*>(&w1[e]));
+            const int i = 8 * k + 2 * e;
+            qs[0] = fmaf(l0.x, z0[i], fmaf(l0.y, z0[i + 1], qs[0]));
+            qs[1] = fmaf(l0.x, z1[i], fmaf(l0.y, z1[i + 1], qs[1]));
+            qs[2] = fmaf(l1.x, z0[i], fmaf(l1.y, z0[i + 1], qs[2]));
+            qs[3] = fmaf(l1.x, z1[i], fmaf(l1.y, z1[i + 1], qs[3]));
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = c1 * v[j] + c2 * qs[j];
+      float m0, m1;
+      heads_max(v, c.G, lane, m0, m1);
+      if (q4 == 0) {
+        const int p0 = tile * 16 + g8, p1 = p0 + 8;
+        if (p0 < c.max_pages) out[p0] = p0 < P ? m0 : -INFINITY;
+        if (p1 < c.max_pages) out[p1] = p1 < P ? m1 : -INFINITY;
+      }
+    };
+
+    load(i0, av0, lv0);
+    for (int i = i0; i < i1; i += 2) {
+      if (i + 1 < i1) load(i + 1, av1, lv1);
+      compute(i, av0, lv0);
+      if (i + 1 >= i1) break;
+      if (i + 2 < i1) load(i + 2, av0, lv0);
+      compute(i + 1, av1, lv1);
+    }
+    if (bad) set_err(c.err, KVQ_DERR_FP16_RANGE);
+  }
+  griddep_launch_dependents();
+}
+
+template <int D, bool BF16>
+cudaError_t launch_quad_scores_d(const DevCache& c, const DevQuad& qd, const void* q, float sm_scale, float* scores,
+                                 cudaStream_t s) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  const int tiles_per_bg = (c.max_pages + 15) / 16;
+  const long long total = (long long)c.B * c.Hkv * tiles_per_bg;
+  const long long warps = (long long)attn_num_ctas(dev) * kQuadWarps;  // one CTA per SM (registers)
+  const int per = (int)((total + warps - 1) / warps);
+  const long long blocks = (total + (long long)per * kQuadWarps - 1) / ((long long)per * kQuadWarps);
+  return launch_pdl(quad_score_kernel<D, BF16>, dim3((unsigned)blocks), dim3(kQuadWarps * 32), 0, s, c, qd,
+                    static_cast<const uint16_t*>(q), sm_scale, scores, tiles_per_bg, per);
+}
+
+}  // namespace
+
+cudaError_t launch_quad_build(const DevCache& c, const DevQuad& qd, const void* k_src, const int64_t* cu,
+                              int64_t src_tokens, cudaStream_t s) {
+  const dim3 grid(c.max_pages, c.B * c.Hkv);
+  const uint16_t* k = static_cast<const uint16_t*>(k_src);
+  if (c.dtype == KVQ_DT_BF16) quad_build_kernel<true><<<grid, 256, 0, s>>>(c, qd, k, cu, src_tokens);
+  else quad_build_kernel<false><<<grid, 256, 0, s>>>(c, qd, k, cu, src_tokens);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quad_append(const DevCache& c, const DevQuad& qd, const int32_t* pos, const void* k_new,
+                               cudaStream_t s) {
+  const uint16_t* k = static_cast<const uint16_t*>(k_new);
+  const dim3 grid(c.B * c.Hkv);
+  if (c.dtype == KVQ_DT_BF16) return launch_pdl(quad_append_kernel<true>, grid, dim3(32), 0, s, c, qd, pos, k);
+  return launch_pdl(quad_append_kernel<false>, grid, dim3(32), 0, s, c, qd, pos, k);
+}
+
+cudaError_t launch_quad_scores(const DevCache& c, const DevQuad& qd, const void* q, float sm_scale, float* scores,
+                               cudaStream_t s) {
+  if (c.G > kMaxG) return cudaErrorInvalidValue;
+  const bool bf = c.dtype == KVQ_DT_BF16;
+  if (c.D == 128)
+    return bf ? launch_quad_scores_d<128, true>(c, qd, q, sm_scale, scores, s)
+              : launch_quad_scores_d<128, false>(c, qd, q, sm_scale, scores, s);
+  if (c.D == 64)
+    return bf ? launch_quad_scores_d<64, true>(c, qd, q, sm_scale, scores, s)
+              : launch_quad_scores_d<64, false>(c, qd, q, sm_scale, scores, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kvq

@@ -79,14 +79,11 @@ __device__ inline void load_tile_rows(const uint16_t* rows, int lane, uint4 (&av
   }
 }
 
-// Scores of the tile's rows g8 (m0) and g8 + 8 (m1): max over the G heads, NaN-propagating;
-// the result is valid in every lane of the row's quad.
+// Dot products of the tile's rows with the lane's two query heads: v[0] = (page g8, head
+// 2q4), v[1] = (g8, 2q4 + 1), v[2] = (g8 + 8, 2q4), v[3] = (g8 + 8, 2q4 + 1).
 template <int D, bool BF16>
-__device__ inline void tile_scores(const uint4 (&av)[2][D / 32], const QFrag<D, BF16>& qf, int G, int lane,
-                                   float& m0, float& m1) {
+__device__ inline void tile_head_dots(const uint4 (&av)[2][D / 32], const QFrag<D, BF16>& qf, float (&v)[4]) {
   constexpr int KS = D / 16;
-  const int q4 = lane & 3;
-  const bool h0ok = 2 * q4 < G, h1ok = 2 * q4 + 1 < G;
   float ch[4] = {0.f, 0.f, 0.f, 0.f}, cl[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int kk = 0; kk < KS; ++kk) {
@@ -98,16 +95,32 @@ __device__ inline void tile_scores(const uint4 (&av)[2][D / 32], const QFrag<D, 
     mma16816<false>(ch, a, qf.bh[kk][0], qf.bh[kk][1]);
     if constexpr (BF16) mma16816<false>(cl, a, qf.bl[kk][0], qf.bl[kk][1]);
   }
-  // c: (page g8, head 2q4), (g8, 2q4+1), (g8 + 8, 2q4), (g8 + 8, 2q4+1)
-  const float v0 = h0ok ? ch[0] + cl[0] : -INFINITY, v1 = h1ok ? ch[1] + cl[1] : -INFINITY;
-  const float v2 = h0ok ? ch[2] + cl[2] : -INFINITY, v3 = h1ok ? ch[3] + cl[3] : -INFINITY;
-  m0 = nanmax(v0, v1);
-  m1 = nanmax(v2, v3);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) v[j] = ch[j] + cl[j];
+}
+
+// Max over the lane's valid heads of values laid out as tile_head_dots's, then over the
+// quad (NaN-propagating): m0 for row g8, m1 for row g8 + 8, valid in every lane of the quad.
+__device__ inline void heads_max(const float (&v)[4], int G, int lane, float& m0, float& m1) {
+  const int q4 = lane & 3;
+  const bool h0ok = 2 * q4 < G, h1ok = 2 * q4 + 1 < G;
+  m0 = nanmax(h0ok ? v[0] : -INFINITY, h1ok ? v[1] : -INFINITY);
+  m1 = nanmax(h0ok ? v[2] : -INFINITY, h1ok ? v[3] : -INFINITY);
 #pragma unroll
   for (int o = 1; o <= 2; o <<= 1) {
     m0 = nanmax(m0, __shfl_xor_sync(0xffffffffu, m0, o));
     m1 = nanmax(m1, __shfl_xor_sync(0xffffffffu, m1, o));
   }
+}
+
+// Scores of the tile's rows g8 (m0) and g8 + 8 (m1): max over the G heads, NaN-propagating;
+// the result is valid in every lane of the row's quad.
+template <int D, bool BF16>
+__device__ inline void tile_scores(const uint4 (&av)[2][D / 32], const QFrag<D, BF16>& qf, int G, int lane,
+                                   float& m0, float& m1) {
+  float v[4];
+  tile_head_dots<D, BF16>(av, qf, v);
+  heads_max(v, G, lane, m0, m1);
 }
 
 }  // namespace kvq

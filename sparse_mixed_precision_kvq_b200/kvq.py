@@ -36,7 +36,7 @@ EXPORTS = ["kvq_chunk_bytes", "kvq_status_string", "kvq_append", "kvq_build_page
            "kvq_select_topk", "kvq_workspace_size", "kvq_sparse_decode_attn", "kvq_dequant_page",
            "kvq_sparse_decode_attn_noalloc", "kvq_noalloc_scratch_bytes", "kvq_workspace_init",
            "kvq_step_workspace_size", "kvq_decode_step", "kvq_score_select", "kvq_append_scores",
-           "kvq_requantize_pages"]
+           "kvq_requantize_pages", "kvq_quad_build", "kvq_quad_append", "kvq_quad_page_scores"]
 
 
 class KvqCache(ctypes.Structure):
@@ -52,7 +52,13 @@ class SelectParams(ctypes.Structure):
                 ("coverage_ppm", c_int32), ("sm_scale", c_float)]
 
 
+class KvqQuad(ctypes.Structure):
+    _fields_ = [("rank", c_int32), ("reserved", c_int32), ("basis", c_void_p), ("lambda_", c_void_p),
+                ("open_sums", c_void_p)]
+
+
 _P = POINTER(KvqCache)
+_PQ = POINTER(KvqQuad)
 _lib.kvq_chunk_bytes.argtypes, _lib.kvq_chunk_bytes.restype = [c_int32, c_int32], c_size_t
 _lib.kvq_status_string.argtypes, _lib.kvq_status_string.restype = [c_int32], c_char_p
 _lib.kvq_append.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p]
@@ -75,8 +81,12 @@ _lib.kvq_score_select.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, PO
                                   c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]
 _lib.kvq_append_scores.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
 _lib.kvq_requantize_pages.argtypes = [_P, c_void_p, c_int32, c_void_p]
+_lib.kvq_quad_build.argtypes = [_P, _PQ, c_void_p, c_void_p, c_int64, c_void_p]
+_lib.kvq_quad_append.argtypes = [_P, _PQ, c_void_p, c_void_p, c_void_p]
+_lib.kvq_quad_page_scores.argtypes = [_P, _PQ, c_void_p, c_float, c_void_p, c_void_p]
 for _f in EXPORTS[2:9] + ["kvq_sparse_decode_attn_noalloc", "kvq_workspace_init", "kvq_step_workspace_size",
-                          "kvq_decode_step", "kvq_score_select", "kvq_append_scores", "kvq_requantize_pages"]:
+                          "kvq_decode_step", "kvq_score_select", "kvq_append_scores", "kvq_requantize_pages",
+                          "kvq_quad_build", "kvq_quad_append", "kvq_quad_page_scores"]:
     getattr(_lib, _f).restype = c_int32
 
 
@@ -195,6 +205,20 @@ def kvq_requantize_pages(cache, items, stream=None):
            "kvq_requantize_pages")
 
 
+def kvq_quad_build(cache, quad, k_src, cu_seqlens, stream=None):
+    _check(_lib.kvq_quad_build(cache.ref(), quad.ref(), _ptr(k_src), _ptr(cu_seqlens), int(k_src.shape[1]),
+                               _stream(stream)), "kvq_quad_build")
+
+
+def kvq_quad_append(cache, quad, pos, k_new, stream=None):
+    _check(_lib.kvq_quad_append(cache.ref(), quad.ref(), _ptr(pos), _ptr(k_new), _stream(stream)), "kvq_quad_append")
+
+
+def kvq_quad_page_scores(cache, quad, q, sm_scale: float, scores, stream=None):
+    _check(_lib.kvq_quad_page_scores(cache.ref(), quad.ref(), _ptr(q), float(sm_scale), _ptr(scores),
+                                     _stream(stream)), "kvq_quad_page_scores")
+
+
 # ------------------------------------------------------------------------- allocation
 def encode_block_table(tier_tbl: np.ndarray, slot_tbl: np.ndarray) -> np.ndarray:
     """(tier << 29) | slot as int32; unused entries (tier < 0) get an invalid tier (7)."""
@@ -226,6 +250,7 @@ class PagedCache:
         self.summary = torch.zeros((B, Hkv, max_pages, D), dtype=torch.float16, device=dev)
         self.open_ksum = torch.zeros((B, Hkv, D), dtype=torch.float64, device=dev)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.quad = None  # a QuadState when the quad page score is maintained
         self._s = KvqCache()
         s = self._s
         s.B, s.Hq, s.Hkv, s.D, s.page_size, s.max_pages = B, Hq, Hkv, D, 16, max_pages
@@ -254,11 +279,34 @@ class PagedCache:
         return tier, self.pools[tier][o:o + cb]
 
 
-def cache_from_workload(w, device="cuda", threads: int = 8, spare=None):
+class QuadState:
+    """Device buffers of the quad page-score state of a cache and its ``kvq_quad`` struct.
+
+    ``basis``: fp32 ``[Hkv, rank, D]`` (host array or tensor), copied to the device."""
+
+    def __init__(self, cache: PagedCache, basis):
+        import torch
+        b = torch.as_tensor(np.asarray(basis, dtype=np.float32)).to(cache.device).contiguous()
+        self.rank = int(b.shape[1])
+        self.basis = b
+        self.lam = torch.zeros((cache.B, cache.Hkv, cache.max_pages, self.rank), dtype=torch.float16,
+                               device=cache.device)
+        self.open = torch.zeros((cache.B, cache.Hkv, 2, self.rank), dtype=torch.float64, device=cache.device)
+        self._s = KvqQuad()
+        self._s.rank = self.rank
+        self._s.basis, self._s.lambda_, self._s.open_sums = _ptr(self.basis), _ptr(self.lam), _ptr(self.open)
+
+    def ref(self):
+        return ctypes.byref(self._s)
+
+
+def cache_from_workload(w, device="cuda", threads: int = 8, spare=None, quad_basis=None):
     """Allocate a cache for workload ``w`` and store its prefilled context with kvq_build_pages.
 
     After the call ``seq_len`` holds the prefilled lengths (before the step's append).
     ``spare`` (optional, per tier) adds free slots after the used ones of each pool.
+    ``quad_basis`` (optional, fp32 ``[Hkv, rank, D]``) also builds the quad page-score state
+    (``cache.quad``) from the same keys with kvq_quad_build.
     """
     import torch
     from concurrent.futures import ThreadPoolExecutor
@@ -287,6 +335,10 @@ def cache_from_workload(w, device="cuda", threads: int = 8, spare=None):
             vsrc[g, s:e].copy_(torch.from_numpy(vb.view(np.int16)))
     cu_t = torch.from_numpy(cu).to(device)
     kvq_build_pages(cache, ksrc, vsrc, cu_t)
+    cache.quad = None
+    if quad_basis is not None:
+        cache.quad = QuadState(cache, quad_basis)
+        kvq_quad_build(cache, cache.quad, ksrc, cu_t)
     torch.cuda.synchronize(device)
     del ksrc, vsrc
     return cache
@@ -303,10 +355,12 @@ class DecodeStep:
     """The buffers and calls of one decode step of workload ``w`` on ``cache``.
 
     ``run()`` enqueues: kvq_append (if the workload appends) -> kvq_page_scores ->
-    kvq_select_topk -> kvq_sparse_decode_attn, all on the current stream.
+    kvq_select_topk -> kvq_sparse_decode_attn, all on the current stream.  With
+    ``quad=True`` (the cache built with a quad basis) the page score is the quad score:
+    kvq_append -> kvq_quad_append -> kvq_quad_page_scores -> select -> attention.
     """
 
-    def __init__(self, w, cache: PagedCache, device="cuda", coverage=None):
+    def __init__(self, w, cache: PagedCache, device="cuda", coverage=None, quad=False):
         import torch
         self.w, self.cache = w, cache
         dt = cache.tdtype
@@ -318,7 +372,12 @@ class DecodeStep:
             self.v_new = torch.from_numpy(vn.view(np.int16)).to(device).view(dt)
             self.pos = torch.from_numpy(np.asarray(w.lens, dtype=np.int32)).to(device)
         self.kmax = w.kmax() if coverage is None else w.max_pages
+        self.quad = cache.quad if quad else None
+        if quad:
+            assert self.quad is not None, "the cache has no quad state (cache_from_workload(quad_basis=...))"
         self.params = select_params(w, coverage)
+        if quad and coverage is not None:
+            self.params.sm_scale = 1.0  # the quad score already carries the softmax scale
         self.scores = torch.empty((w.B, w.Hkv, w.max_pages), dtype=torch.float32, device=device)
         self.sel = torch.zeros((w.B, w.Hkv, self.kmax), dtype=torch.int32, device=device)
         self.cnt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device=device)
@@ -332,9 +391,14 @@ class DecodeStep:
     def append(self):
         if self.w.append:
             kvq_append(self.cache, self.pos, self.k_new, self.v_new)
+            if self.quad is not None:
+                kvq_quad_append(self.cache, self.quad, self.pos, self.k_new)
 
     def scores_(self):
-        kvq_page_scores(self.cache, self.q, self.scores)
+        if self.quad is not None:
+            kvq_quad_page_scores(self.cache, self.quad, self.q, self.w.sm_scale, self.scores)
+        else:
+            kvq_page_scores(self.cache, self.q, self.scores)
 
     def select(self):
         kvq_select_topk(self.cache, self.scores, self.params, self.sel, self.cnt, self.kmax)
@@ -350,11 +414,13 @@ class DecodeStep:
         self.attend()
 
     def score_select(self):
+        assert self.quad is None, "the fused launches score pages with the mean-key score"
         kvq_score_select(self.cache, self.pos if self.w.append else None, self.k_new if self.w.append else None,
                          self.v_new if self.w.append else None, self.q, self.params, self.scores, self.sel, self.cnt,
                          self.kmax, self.ws)
 
     def append_scores(self):
+        assert self.quad is None, "the fused launches score pages with the mean-key score"
         if self.w.append:
             kvq_append_scores(self.cache, self.pos, self.k_new, self.v_new, self.q, self.scores)
         else:
@@ -373,6 +439,7 @@ class DecodeStep:
 
     def run_fused(self):
         """The same step as ``run()`` in one kvq_decode_step launch."""
+        assert self.quad is None, "the fused launches score pages with the mean-key score"
         kvq_decode_step(self.cache, self.pos if self.w.append else None, self.k_new if self.w.append else None,
                         self.v_new if self.w.append else None, self.q, self.params, self.scores, self.sel, self.cnt,
                         self.kmax, self.w.sm_scale, self.out, self.lse, self.ws)

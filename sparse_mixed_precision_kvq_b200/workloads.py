@@ -41,7 +41,7 @@ TIER_F16, TIER_I8, TIER_I4, TIER_I2, TIER_I1 = 0, 1, 2, 3, 4
 N_TIERS = 5
 
 # stream tags (part of the seed key of each random stream)
-_S_KEY, _S_VAL, _S_Q, _S_KNEW, _S_VNEW, _S_OUTL, _S_PLANT, _S_TIER, _S_SLOT, _S_LEN = range(10)
+_S_KEY, _S_VAL, _S_Q, _S_KNEW, _S_VNEW, _S_OUTL, _S_PLANT, _S_TIER, _S_SLOT, _S_LEN, _S_QUAD = range(11)
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -138,6 +138,23 @@ class Workload:
             return np.zeros(0, dtype=np.int64)
         r = _rng(self.seed, _S_OUTL, g)
         return np.sort(r.choice(self.D, size=self.outlier_channels, replace=False))
+
+    def quad_basis(self, g: int, rank: int, kind: str = "law") -> np.ndarray:
+        """Basis rows of kv head g for the quad page score, fp32 ``[rank, D]``.
+
+        ``law``: unit vectors along the channels of largest key variance under this
+        workload's key law (its outlier channels, then the others in index order) -- the
+        eigenvectors of the law's diagonal covariance.  ``random``: a seeded random
+        orthonormal set (QR of a Gaussian matrix)."""
+        if kind == "random":
+            a = _rng(self.seed, _S_QUAD, g).standard_normal((self.D, self.D))
+            qm, _ = np.linalg.qr(a)
+            return np.ascontiguousarray(qm[:, :rank].T).astype(np.float32)
+        first = [int(c) for c in self.outlier_idx(g)]
+        chans = (first + [c for c in range(self.D) if c not in first])[:rank]
+        u = np.zeros((rank, self.D), dtype=np.float32)
+        u[np.arange(rank), chans] = 1.0
+        return u
 
     def query_bits(self) -> np.ndarray:
         """q [B, Hq, D] as 16-bit patterns of the workload dtype."""

@@ -105,7 +105,8 @@ def query_and_new(w):
     return q, kn, vn
 
 
-def oracle_step(w, sh, b: int, g: int, q, kn, vn, sel=None):
-    """Run the oracle step on a prepared (b, g) cache (mutates it by the append)."""
+def oracle_step(w, sh, b: int, g: int, q, kn, vn, sel=None, quad=None):
+    """Run the oracle step on a prepared (b, g) cache (mutates it by the append); ``quad``
+    (an ``oracle.quad.QuadState``) scores pages with the quad score."""
     return step_pair(w, sh, b, g, q[b], None if kn is None else kn[b, g], None if vn is None else vn[b, g],
-                     sel=sel)
+                     sel=sel, quad=quad)

@@ -145,3 +145,56 @@ def test_invalid_items_are_skipped_with_an_error_bit(kvq):
     kvq.kvq_requantize_pages(cache, None)        # n == 0: nothing launched
     torch.cuda.synchronize()
     assert cache.err_bits() == 0 and torch.equal(cache.block_table, bt0)
+
+
+def _tie_values(D, L, seed=3):
+    """fp16 K/V rows [L, D] whose 32-channel groups put the exact quotients of the target
+    tiers on rounding ties (x = k + 1/2 with lo = 0 and hi = 2^b - 1, so scale = 1 and
+    zero = 0), mixed with random groups, signed zeros and constant groups."""
+    rng = np.random.default_rng(seed)
+    x = rng.normal(0, 2, (2, L, D))
+    for t in range(L):
+        qmax = (255, 15, 3)[(t // 16) % 3]
+        for kind in range(2):
+            g0 = x[kind, t, :32]
+            g0[:] = (np.arange(32) % (qmax + 1)) + 0.5
+            g0[g0 > qmax] = qmax
+            g0[0], g0[1] = 0.0, qmax
+            if t % 4 == 1:
+                x[kind, t, 32:64] = 0.0
+                x[kind, t, 32:64:3] = -0.0          # a constant group of mixed signed zeros
+            if t % 4 == 2:
+                x[kind, t, 32:40] = -0.0            # a zero minimum of either sign
+                x[kind, t, 40:64] = np.abs(x[kind, t, 40:64])
+    return x.astype(np.float16).view(np.uint16)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_requantize_rounding_ties_and_signed_zeros(kvq, D):
+    """Page p (16-bit) moves to int8, int4, int2 in turn: every tie group takes the exact
+    fp64 route and rounds half to even; then int8 -> int2 and int4 -> 1-bit."""
+    L, Hkv = 40, 2
+    bits = [_tie_values(D, L, seed=g) for g in range(Hkv)]
+    cache = kvq.PagedCache(1, 2 * Hkv, Hkv, D, 3, "f16", [3, 3, 3, 3, 3], "cuda")
+    cache.block_table.copy_(torch.from_numpy(kvq.encode_block_table(np.zeros((1, 3), np.int64),
+                                                                    np.arange(3)[None])))
+    cache.seq_len.fill_(L)
+    k = torch.from_numpy(np.stack([b_[0] for b_ in bits]).view(np.int16)).cuda()
+    v = torch.from_numpy(np.stack([b_[1] for b_ in bits]).view(np.int16)).cuda()
+    kvq.kvq_build_pages(cache, k, v, torch.tensor([0, L], dtype=torch.int64, device="cuda"))
+
+    def ent(t, s):
+        return int(np.uint32((t << 29) | s).view(np.int32))
+
+    heads = [ocache.build(b_[0], b_[1], "f16", np.zeros(3, np.int64)) for b_ in bits]
+    for plan in ([(0, 1, 0), (1, 2, 0), (2, 3, 0)], [(0, 3, 1), (1, 4, 1)]):
+        items = torch.tensor([(0, p, ent(t, s)) for p, t, s in plan], dtype=torch.int32, device="cuda")
+        kvq.kvq_requantize_pages(cache, items)
+        torch.cuda.synchronize()
+        for sh in heads:
+            for p, t, _ in plan:
+                ocache.requantize(sh, p, t)
+        assert cache.err_bits() == 0, hex(cache.err_bits())
+        snap = snapshot(cache)
+        for g, sh in enumerate(heads):
+            check_pages(snap, sh, W.make("c0", Hq=2 * Hkv, Hkv=Hkv, D=D, lens=np.array([L])), 0, g, range(3))

@@ -83,3 +83,26 @@ def test_invalid_arguments_rejected_on_host():
     assert st == 1          # null pointers
     c.Hq = 24               # G = 12 > 8
     assert kvq._lib.kvq_append(ctypes.byref(c), None, None, None, None) == 2
+
+
+def test_quad_arguments_rejected_on_host():
+    """Every case fails its host-side check before anything is enqueued (no device needed)."""
+    from sparse_mixed_precision_kvq_b200 import kvq
+    c = kvq.KvqCache()
+    c.B, c.Hq, c.Hkv, c.D, c.page_size, c.max_pages, c.dtype = 1, 8, 2, 64, 16, 4, 1
+    c.block_table = c.seq_len = c.summary = c.open_ksum = c.err_word = 4096
+    c.pool[0], c.pool_slots[0] = 4096, 4
+    qd = kvq.KvqQuad()
+    qd.rank, qd.basis, qd.lambda_, qd.open_sums = 12, 4096, 4096, 4096
+    ref, qref = ctypes.byref(c), ctypes.byref(qd)
+    assert kvq._lib.kvq_quad_page_scores(ref, qref, 4096, 0.1, 4096, None) == 2      # rank 12: unsupported
+    qd.rank = 40
+    assert kvq._lib.kvq_quad_append(ref, qref, 4096, 4096, None) == 2                # rank 40 > 32
+    qd.rank = 16
+    assert kvq._lib.kvq_quad_page_scores(ref, qref, 4096, 0.0, 4096, None) == 1      # sm_scale 0
+    assert kvq._lib.kvq_quad_page_scores(ref, qref, 4100, 0.1, 4096, None) == 1      # q not 16-byte aligned
+    assert kvq._lib.kvq_quad_page_scores(ref, None, 4096, 0.1, 4096, None) == 1      # no quad state
+    qd.lambda_ = 4104
+    assert kvq._lib.kvq_quad_build(ref, qref, 4096, 4096, 16, None) == 1             # lambda not 16-byte aligned
+    qd.lambda_, qd.basis = 4096, None
+    assert kvq._lib.kvq_quad_append(ref, qref, 4096, 4096, None) == 1                # no basis
