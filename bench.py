@@ -318,7 +318,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
         files = ["score.cu", "attn.cu"]
     elif args.path == "three":
         dom_bytes = [nbytes["score"] + nbytes["append"], nbytes["select"], nbytes["attn"]][dom]
-        files = ["score.cu", "select.cu", "attn.cu"]
+        files = ["quad.cu" if quad_rank else "score.cu", "select.cu", "attn.cu"]
     else:
         dom_bytes = [nbytes["append"], nbytes["score"], nbytes["select"], nbytes["attn"]][dom]
         files = ["append.cu", "quad.cu" if quad_rank else "score.cu", "select.cu", "attn.cu"]
@@ -355,7 +355,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
                      "traffic": None if tr is None else tr["dram_bytes_per_launch"]},
         "e2e": {"value": world * w.B / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
-        "gpu_launches": (len(parts) + (1 if quad_rank and w.append else 0)) * K,
+        "gpu_launches": (len(parts) + (1 if quad_rank and w.append and args.path == "calls" else 0)) * K,
         "path": {"fused": "kvq_decode_step (one persistent launch)",
                  "two": "kvq_score_select -> kvq_sparse_decode_attn",
                  "three": "kvq_append_scores -> kvq_select_topk -> kvq_sparse_decode_attn",
@@ -515,7 +515,7 @@ def main():
                     help="the four separate calls; kvq_append_scores + select + attention; kvq_score_select + "
                          "attention; or one kvq_decode_step launch")
     ap.add_argument("--score", default="mean", choices=["mean", "quad"],
-                    help="page score: the mean-key score, or the quad (Gaussian-MGF) score (four-call path only)")
+                    help="page score: the mean-key score, or the quad (Gaussian-MGF) score (--path calls or three)")
     ap.add_argument("--quad-rank", type=int, default=16, help="r' of the quad score (8, 16, 24 or 32)")
     ap.add_argument("--dense", action="store_true", help="also time attention over every page")
     ap.add_argument("--demote", type=int, default=None, choices=[1, 2, 3, 4],
@@ -530,8 +530,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.coverage is not None and args.path != "calls":
         ap.error("--coverage runs on the four-call path")
-    if args.score == "quad" and args.path != "calls":
-        ap.error("--score quad runs on the four-call path")
+    if args.score == "quad" and args.path not in ("calls", "three"):
+        ap.error("--score quad runs on the four-call or the three-call path")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

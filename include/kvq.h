@@ -336,6 +336,13 @@ kvq_status kvq_quad_append(const kvq_cache* cache, const kvq_quad* quad, const i
 kvq_status kvq_quad_page_scores(const kvq_cache* cache, const kvq_quad* quad, const void* q,
                                 float sm_scale, float* scores, kvq_stream_t stream);
 
+/* kvq_quad_append_scores -- kvq_append + kvq_quad_append + kvq_quad_page_scores in one
+ *  launch, with the same results (the warp that scores the tile holding a sequence's new
+ *  token writes the token and its quad state first).  pos, k_new, v_new as kvq_append. */
+kvq_status kvq_quad_append_scores(const kvq_cache* cache, const kvq_quad* quad, const int32_t* pos,
+                                  const void* k_new, const void* v_new, const void* q, float sm_scale,
+                                  float* scores, kvq_stream_t stream);
+
 /*
  * kvq_requantize_pages -- tier demotion: move pages to a lower-precision tier.
  * (ARGUS "Virtual Memory for Transformers", "Visual Architecture": pages cool down the

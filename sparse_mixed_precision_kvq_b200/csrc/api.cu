@@ -266,7 +266,22 @@ kvq_status kvq_quad_page_scores(const kvq_cache* cache, const kvq_quad* quad, co
   if (st == KVQ_OK) st = to_quad(quad, qd);
   if (st != KVQ_OK) return st;
   if (q == nullptr || scores == nullptr || !aligned16(q) || !(sm_scale > 0.0f)) return KVQ_ERR_INVALID_ARG;
-  return cuda_status(launch_quad_scores(c, qd, q, sm_scale, scores, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(
+      launch_quad_scores(c, qd, q, sm_scale, scores, nullptr, nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_quad_append_scores(const kvq_cache* cache, const kvq_quad* quad, const int32_t* pos,
+                                  const void* k_new, const void* v_new, const void* q, float sm_scale, float* scores,
+                                  kvq_stream_t stream) {
+  DevCache c;
+  DevQuad qd;
+  kvq_status st = to_dev(cache, c);
+  if (st == KVQ_OK) st = to_quad(quad, qd);
+  if (st != KVQ_OK) return st;
+  if (pos == nullptr || k_new == nullptr || v_new == nullptr) return KVQ_ERR_INVALID_ARG;
+  if (q == nullptr || scores == nullptr || !aligned16(q) || !(sm_scale > 0.0f)) return KVQ_ERR_INVALID_ARG;
+  return cuda_status(launch_quad_scores(c, qd, q, sm_scale, scores, pos, k_new, v_new,
+                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
 kvq_status kvq_requantize_pages(const kvq_cache* cache, const int32_t* items, int32_t n, kvq_stream_t stream) {

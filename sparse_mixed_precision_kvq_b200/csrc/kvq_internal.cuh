@@ -263,6 +263,6 @@ cudaError_t launch_quad_build(const DevCache& c, const DevQuad& qd, const void* 
 cudaError_t launch_quad_append(const DevCache& c, const DevQuad& qd, const int32_t* pos, const void* k_new,
                                cudaStream_t s);
 cudaError_t launch_quad_scores(const DevCache& c, const DevQuad& qd, const void* q, float sm_scale, float* scores,
-                               cudaStream_t s);
+                               const int32_t* pos, const void* k_new, const void* v_new, cudaStream_t s);
 
 }  // namespace kvq

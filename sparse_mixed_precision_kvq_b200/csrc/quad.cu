@@ -1,4 +1,6 @@
-// quad page score: kvq_quad_build, kvq_quad_append and kvq_quad_page_scores.
+// quad page score: kvq_quad_build, kvq_quad_append, kvq_quad_page_scores and
+// kvq_quad_append_scores (the token append, the quad state update and the scores in one
+// launch).
 //
 // AMASS "decode-time sparse KV-cache attention for vLLM", "What is in the box", Stage A:
 // a quadratic, Gaussian-MGF page score built from a tiny per-page summary that keeps r'
@@ -19,6 +21,7 @@
 
 #include "kvq_internal.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 #include "score_tile.cuh"
 
 namespace kvq {
@@ -86,39 +89,119 @@ __global__ void __launch_bounds__(256) quad_build_kernel(DevCache c, DevQuad qd,
   }
 }
 
-// One warp per (sequence, kv head); lane i < r owns basis row i.
+// One warp: token `pos` (0 <= pos < max_pages * 16) of sequence b, kv head g, key `krow`,
+// joins the quad state; lane i < r owns basis row i.
+template <bool BF16>
+__device__ inline void quad_append_warp(const DevCache& c, const DevQuad& qd, int bg, int g, int ps,
+                                        const uint16_t* krow, int lane) {
+  const int D = c.D, r = qd.rank;
+  if (lane >= r) return;
+  const int p = ps / kPage, t = ps % kPage;
+  const float* u = qd.basis + ((size_t)g * r + lane) * D;
+  double y = 0.0;
+  for (int d = 0; d < D; ++d) y = y + static_cast<double>(u[d]) * key_f64<BF16>(krow[d]);
+  double* o = qd.open + (size_t)bg * 2 * r;
+  const double s1 = t == 0 ? y : o[lane] + y;
+  const double s2 = t == 0 ? y * y : o[r + lane] + y * y;
+  o[lane] = s1;
+  o[r + lane] = s2;
+  bool ov = false;
+  qd.lambda[((size_t)bg * c.max_pages + p) * r + lane] = quad_lambda(s1, s2, t + 1, ov);
+  if (ov) set_err(c.err, KVQ_DERR_FP16_RANGE);
+}
+
+// One warp per (sequence, kv head).
 template <bool BF16>
 __global__ void __launch_bounds__(32) quad_append_kernel(DevCache c, DevQuad qd, const int32_t* __restrict__ pos,
                                                          const uint16_t* __restrict__ k_new) {
   const int bg = blockIdx.x, b = bg / c.Hkv, g = bg % c.Hkv, lane = threadIdx.x;
-  const int D = c.D, r = qd.rank;
   griddep_wait();
   const int ps = pos[b];
   if (ps >= 0 && ps >= c.max_pages * kPage) {
     if (lane == 0 && g == 0) set_err(c.err, KVQ_DERR_BAD_POS);
-  } else if (ps >= 0 && lane < r) {
-    const int p = ps / kPage, t = ps % kPage;
-    const float* u = qd.basis + ((size_t)g * r + lane) * D;
-    const uint16_t* k = k_new + (size_t)bg * D;
-    double y = 0.0;
-    for (int d = 0; d < D; ++d) y = y + static_cast<double>(u[d]) * key_f64<BF16>(k[d]);
-    double* o = qd.open + (size_t)bg * 2 * r;
-    const double s1 = t == 0 ? y : o[lane] + y;
-    const double s2 = t == 0 ? y * y : o[r + lane] + y * y;
-    o[lane] = s1;
-    o[r + lane] = s2;
-    bool ov = false;
-    qd.lambda[((size_t)bg * c.max_pages + p) * r + lane] = quad_lambda(s1, s2, t + 1, ov);
-    if (ov) set_err(c.err, KVQ_DERR_FP16_RANGE);
+  } else if (ps >= 0) {
+    quad_append_warp<BF16>(c, qd, bg, g, ps, k_new + (size_t)bg * c.D, lane);
   }
   griddep_launch_dependents();
 }
 
+// zs[h][i] = (u_i . q_h)^2 for the G query heads of kv head g (fp32): the lanes split the
+// channels (D/32 each), so every load of a basis row or query row is coalesced and all of
+// them are in flight at once; a butterfly over the warp sums each product.
+template <int D, bool BF16>
+__device__ inline void quad_qterms(const DevQuad& qd, const uint16_t* qg, int G, int g, int lane,
+                                   float (*zs)[kMaxQuadRank]) {
+  constexpr int CPL = D / 32;  // channels per lane: 4 (D = 128) or 2 (D = 64)
+  static_assert(CPL == 4 || CPL == 2, "D is 64 or 128");
+  float qv[kMaxG][CPL];
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) {
+    uint32_t w[CPL / 2];
+    if (h < G) {
+      if constexpr (CPL == 4) {
+        const uint2 x = *reinterpret_cast<const uint2*>(qg + (size_t)h * D + CPL * lane);
+        w[0] = x.x;
+        w[1] = x.y;
+      } else {
+        w[0] = *reinterpret_cast<const uint32_t*>(qg + (size_t)h * D + CPL * lane);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < CPL / 2; ++j) w[j] = 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < CPL / 2; ++j) {
+      qv[h][2 * j] = bits_to_float<BF16>(static_cast<uint16_t>(w[j] & 0xFFFFu));
+      qv[h][2 * j + 1] = bits_to_float<BF16>(static_cast<uint16_t>(w[j] >> 16));
+    }
+  }
+  const float* ub = qd.basis + (size_t)g * qd.rank * D + CPL * lane;
+  for (int i0 = 0; i0 < qd.rank; i0 += 8) {  // 8 basis rows at a time, all loads in flight
+    float u[8][CPL];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if constexpr (CPL == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(ub + (size_t)(i0 + k) * D);
+        u[k][0] = x.x, u[k][1] = x.y, u[k][2] = x.z, u[k][3] = x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(ub + (size_t)(i0 + k) * D);
+        u[k][0] = x.x, u[k][1] = x.y;
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+      if (h < G) {  // warp-uniform
+        float p[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          p[k] = 0.0f;
+#pragma unroll
+          for (int j = 0; j < CPL; ++j) p[k] = fmaf(u[k][j], qv[h][j], p[k]);
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) p[k] += __shfl_xor_sync(0xffffffffu, p[k], o);
+        }
+        if (lane < 8) {
+          float z = p[0];
+#pragma unroll
+          for (int k = 1; k < 8; ++k) z = lane == k ? p[k] : z;
+          zs[h][i0 + lane] = z * z;
+        }
+      } else if (lane < 8) {
+        zs[h][i0 + lane] = 0.0f;
+      }
+    }
+  }
+  __syncwarp();
+}
+
 constexpr int kQuadWarps = 8;
 
-template <int D>
-__device__ inline void quad_load_tile(const uint16_t* sbase, const uint16_t* lbase, int r, int tile, int P, int lane,
-                                      uint4 (&av)[2][D / 32], uint4 (&lv)[2][kMaxQuadRank / 8]) {
+template <int D, int RK>
+__device__ inline void quad_load_tile(const uint16_t* sbase, const uint16_t* lbase, int tile, int P, int lane,
+                                      uint4 (&av)[2][D / 32], uint4 (&lv)[2][RK]) {
   constexpr int CW = D / 4;
   const int g8 = lane >> 2, q4 = lane & 3;
 #pragma unroll
@@ -127,9 +210,9 @@ __device__ inline void quad_load_tile(const uint16_t* sbase, const uint16_t* lba
     const uint4* src = reinterpret_cast<const uint4*>(sbase + (size_t)p * D + CW * q4);
 #pragma unroll
     for (int i = 0; i < CW / 8; ++i) av[h][i] = p < P ? __ldcg(src + i) : make_uint4(0, 0, 0, 0);
-    const uint4* ls = reinterpret_cast<const uint4*>(lbase + (size_t)p * r);
+    const uint4* ls = reinterpret_cast<const uint4*>(lbase + (size_t)p * 8 * RK);
 #pragma unroll
-    for (int k = 0; k < kMaxQuadRank / 8; ++k) lv[h][k] = (p < P && 8 * k < r) ? __ldcg(ls + k) : make_uint4(0, 0, 0, 0);
+    for (int k = 0; k < RK; ++k) lv[h][k] = p < P ? __ldcg(ls + k) : make_uint4(0, 0, 0, 0);
   }
 }
 
@@ -137,10 +220,19 @@ __device__ inline void quad_load_tile(const uint16_t* sbase, const uint16_t* lba
 // kvq_page_scores does, loading the next tile (summary rows and lambda rows) while the
 // current one is multiplied; the two buffers take more registers than two CTAs per SM
 // leave, so one CTA of 8 warps runs per SM.
-template <int D, bool BF16>
+// With `ap.pos` set (kvq_quad_append_scores) the warp that owns the tile of a (b, g)'s
+// appended token first writes the token into the cache (quantise, pack, summary) and the
+// quad state, so that tile is read after both are stored.
+struct QuadAppend {
+  const int32_t* pos;  // nullable: no append
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+};
+
+template <int D, bool BF16, int RK>
 __global__ void __launch_bounds__(kQuadWarps * 32, 1)
     quad_score_kernel(DevCache c, DevQuad qd, const uint16_t* __restrict__ q, float sm_scale,
-                      float* __restrict__ scores, int tiles_per_bg, int per) {
+                      float* __restrict__ scores, int tiles_per_bg, int per, QuadAppend ap) {
   __shared__ float zs[kQuadWarps][kMaxG][kMaxQuadRank];  // (u_i . q_h)^2 of the warp's current (b, g)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, q4 = lane & 3;
@@ -149,6 +241,22 @@ __global__ void __launch_bounds__(kQuadWarps * 32, 1)
   const int i0 = (blockIdx.x * kQuadWarps + warp) * per;
   const int i1 = min(total, i0 + per);
   griddep_wait();
+  if (ap.pos != nullptr && i0 < i1) {  // appends whose page lies in this warp's tiles
+    for (int bg = i0 / tiles_per_bg; bg <= (i1 - 1) / tiles_per_bg; ++bg) {
+      const int b = bg / c.Hkv, g = bg % c.Hkv;
+      const int ps = ap.pos[b];
+      if (ps < 0) continue;
+      if (ps >= c.max_pages * kPage) {
+        if (lane == 0 && g == 0 && bg * tiles_per_bg >= i0) set_err(c.err, KVQ_DERR_BAD_POS);
+        continue;
+      }
+      const int it = bg * tiles_per_bg + (ps / kPage) / 16;
+      if (it < i0 || it >= i1) continue;
+      append_token_warp<BF16>(c, b, g, ps, ap.k_new + (size_t)bg * D, ap.v_new + (size_t)bg * D, lane, nullptr);
+      quad_append_warp<BF16>(c, qd, bg, g, ps, ap.k_new + (size_t)bg * D, lane);
+      __syncwarp();
+    }
+  }
   if (i0 < i1) {
     const float c1 = sm_scale, c2 = 0.5f * sm_scale * sm_scale;
     QFrag<D, BF16> qf;
@@ -156,16 +264,16 @@ __global__ void __launch_bounds__(kQuadWarps * 32, 1)
     float* out = nullptr;
     bool bad = false;
     uint4 av0[2][D / 32], av1[2][D / 32];
-    uint4 lv0[2][kMaxQuadRank / 8], lv1[2][kMaxQuadRank / 8];
+    uint4 lv0[2][RK], lv1[2][RK];
 
-    auto load = [&](int i, uint4 (&av)[2][D / 32], uint4 (&lv)[2][kMaxQuadRank / 8]) {
+    auto load = [&](int i, uint4 (&av)[2][D / 32], uint4 (&lv)[2][RK]) {
       const int bg = i / tiles_per_bg;
       const int L = c.seq_len[bg / c.Hkv];
       const int Pn = min((L + kPage - 1) / kPage, c.max_pages);
-      quad_load_tile<D>(c.summary + (size_t)bg * c.max_pages * D, qd.lambda + (size_t)bg * c.max_pages * r, r,
-                        i % tiles_per_bg, Pn, lane, av, lv);
+      quad_load_tile<D, RK>(c.summary + (size_t)bg * c.max_pages * D, qd.lambda + (size_t)bg * c.max_pages * r,
+                            i % tiles_per_bg, Pn, lane, av, lv);
     };
-    auto compute = [&](int i, const uint4 (&av)[2][D / 32], const uint4 (&lv)[2][kMaxQuadRank / 8]) {
+    auto compute = [&](int i, const uint4 (&av)[2][D / 32], const uint4 (&lv)[2][RK]) {
       const int bg = i / tiles_per_bg, tile = i % tiles_per_bg;
       if (bg != cur_bg) {  // new (b, g): query fragments and (u_i . q_h)^2
         cur_bg = bg;
@@ -174,24 +282,7 @@ __global__ void __launch_bounds__(kQuadWarps * 32, 1)
         P = min((L + kPage - 1) / kPage, c.max_pages);
         out = scores + (size_t)bg * c.max_pages;
         qf.load(q, c.Hq, c.G, b, g, lane, bad);
-        __syncwarp();
-        for (int h = 0; h < kMaxG; ++h) {
-          float z = 0.0f;
-          if (h < c.G && lane < r) {
-            const float4* u = reinterpret_cast<const float4*>(qd.basis + ((size_t)g * r + lane) * D);
-            const uint2* qh = reinterpret_cast<const uint2*>(q + ((size_t)b * c.Hq + (size_t)g * c.G + h) * D);
-#pragma unroll 4
-            for (int d4 = 0; d4 < D / 4; ++d4) {
-              const float4 uv = u[d4];
-              const uint2 qv = qh[d4];
-              z = fmaf(uv.x, bits_to_float<BF16>(static_cast<uint16_t>(qv.x & 0xFFFFu)), z);
-              z = fmaf(uv.y, bits_to_float<BF16>(static_cast<uint16_t>(qv.x >> 16)), z);
-              z = fmaf(uv.z, bits_to_float<BF16>(static_cast<uint16_t>(qv.y & 0xFFFFu)), z);
-              z = fmaf(uv.w, bits_to_float<BF16>(static_cast<uint16_t>(qv.y >> 16)), z);
-            }
-          }
-          zs[warp][h][lane] = z * z;
-        }
+        quad_qterms<D, BF16>(qd, q + ((size_t)b * c.Hq + (size_t)g * c.G) * D, c.G, g, lane, zs[warp]);
         __syncwarp();
       }
       float v[4];
@@ -200,8 +291,8 @@ __global__ void __launch_bounds__(kQuadWarps * 32, 1)
       const float* z0 = zs[warp][(2 * q4) & (kMaxG - 1)];
       const float* z1 = zs[warp][(2 * q4 + 1) & (kMaxG - 1)];
 #pragma unroll
-      for (int k = 0; k < kMaxQuadRank / 8; ++k) {
-        if (8 * k < r) {
+      for (int k = 0; k < RK; ++k) {
+        {
           const uint32_t w0[4] = {lv[0][k].x, lv[0][k].y, lv[0][k].z, lv[0][k].w};
           const uint32_t w1[4] = {lv[1][k].x, lv[1][k].y, lv[1][k].z, lv[1][k].w};
 #pragma unroll
@@ -240,9 +331,9 @@ __global__ void __launch_bounds__(kQuadWarps * 32, 1)
   griddep_launch_dependents();
 }
 
-template <int D, bool BF16>
-cudaError_t launch_quad_scores_d(const DevCache& c, const DevQuad& qd, const void* q, float sm_scale, float* scores,
-                                 cudaStream_t s) {
+template <int D, bool BF16, int RK>
+cudaError_t launch_quad_scores_r(const DevCache& c, const DevQuad& qd, const void* q, float sm_scale, float* scores,
+                                 const QuadAppend& ap, cudaStream_t s) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
   const int tiles_per_bg = (c.max_pages + 15) / 16;
@@ -250,8 +341,20 @@ cudaError_t launch_quad_scores_d(const DevCache& c, const DevQuad& qd, const voi
   const long long warps = (long long)attn_num_ctas(dev) * kQuadWarps;  // one CTA per SM (registers)
   const int per = (int)((total + warps - 1) / warps);
   const long long blocks = (total + (long long)per * kQuadWarps - 1) / ((long long)per * kQuadWarps);
-  return launch_pdl(quad_score_kernel<D, BF16>, dim3((unsigned)blocks), dim3(kQuadWarps * 32), 0, s, c, qd,
-                    static_cast<const uint16_t*>(q), sm_scale, scores, tiles_per_bg, per);
+  return launch_pdl(quad_score_kernel<D, BF16, RK>, dim3((unsigned)blocks), dim3(kQuadWarps * 32), 0, s, c, qd,
+                    static_cast<const uint16_t*>(q), sm_scale, scores, tiles_per_bg, per, ap);
+}
+
+template <int D, bool BF16>
+cudaError_t launch_quad_scores_d(const DevCache& c, const DevQuad& qd, const void* q, float sm_scale, float* scores,
+                                 const QuadAppend& ap, cudaStream_t s) {
+  switch (qd.rank / 8) {
+    case 1: return launch_quad_scores_r<D, BF16, 1>(c, qd, q, sm_scale, scores, ap, s);
+    case 2: return launch_quad_scores_r<D, BF16, 2>(c, qd, q, sm_scale, scores, ap, s);
+    case 3: return launch_quad_scores_r<D, BF16, 3>(c, qd, q, sm_scale, scores, ap, s);
+    case 4: return launch_quad_scores_r<D, BF16, 4>(c, qd, q, sm_scale, scores, ap, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -274,15 +377,16 @@ cudaError_t launch_quad_append(const DevCache& c, const DevQuad& qd, const int32
 }
 
 cudaError_t launch_quad_scores(const DevCache& c, const DevQuad& qd, const void* q, float sm_scale, float* scores,
-                               cudaStream_t s) {
+                               const int32_t* pos, const void* k_new, const void* v_new, cudaStream_t s) {
   if (c.G > kMaxG) return cudaErrorInvalidValue;
   const bool bf = c.dtype == KVQ_DT_BF16;
+  const QuadAppend ap{pos, static_cast<const uint16_t*>(k_new), static_cast<const uint16_t*>(v_new)};
   if (c.D == 128)
-    return bf ? launch_quad_scores_d<128, true>(c, qd, q, sm_scale, scores, s)
-              : launch_quad_scores_d<128, false>(c, qd, q, sm_scale, scores, s);
+    return bf ? launch_quad_scores_d<128, true>(c, qd, q, sm_scale, scores, ap, s)
+              : launch_quad_scores_d<128, false>(c, qd, q, sm_scale, scores, ap, s);
   if (c.D == 64)
-    return bf ? launch_quad_scores_d<64, true>(c, qd, q, sm_scale, scores, s)
-              : launch_quad_scores_d<64, false>(c, qd, q, sm_scale, scores, s);
+    return bf ? launch_quad_scores_d<64, true>(c, qd, q, sm_scale, scores, ap, s)
+              : launch_quad_scores_d<64, false>(c, qd, q, sm_scale, scores, ap, s);
   return cudaErrorInvalidValue;
 }
 

@@ -36,7 +36,8 @@ EXPORTS = ["kvq_chunk_bytes", "kvq_status_string", "kvq_append", "kvq_build_page
            "kvq_select_topk", "kvq_workspace_size", "kvq_sparse_decode_attn", "kvq_dequant_page",
            "kvq_sparse_decode_attn_noalloc", "kvq_noalloc_scratch_bytes", "kvq_workspace_init",
            "kvq_step_workspace_size", "kvq_decode_step", "kvq_score_select", "kvq_append_scores",
-           "kvq_requantize_pages", "kvq_quad_build", "kvq_quad_append", "kvq_quad_page_scores"]
+           "kvq_requantize_pages", "kvq_quad_build", "kvq_quad_append", "kvq_quad_page_scores",
+           "kvq_quad_append_scores"]
 
 
 class KvqCache(ctypes.Structure):
@@ -84,9 +85,10 @@ _lib.kvq_requantize_pages.argtypes = [_P, c_void_p, c_int32, c_void_p]
 _lib.kvq_quad_build.argtypes = [_P, _PQ, c_void_p, c_void_p, c_int64, c_void_p]
 _lib.kvq_quad_append.argtypes = [_P, _PQ, c_void_p, c_void_p, c_void_p]
 _lib.kvq_quad_page_scores.argtypes = [_P, _PQ, c_void_p, c_float, c_void_p, c_void_p]
+_lib.kvq_quad_append_scores.argtypes = [_P, _PQ, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_void_p, c_void_p]
 for _f in EXPORTS[2:9] + ["kvq_sparse_decode_attn_noalloc", "kvq_workspace_init", "kvq_step_workspace_size",
                           "kvq_decode_step", "kvq_score_select", "kvq_append_scores", "kvq_requantize_pages",
-                          "kvq_quad_build", "kvq_quad_append", "kvq_quad_page_scores"]:
+                          "kvq_quad_build", "kvq_quad_append", "kvq_quad_page_scores", "kvq_quad_append_scores"]:
     getattr(_lib, _f).restype = c_int32
 
 
@@ -217,6 +219,11 @@ def kvq_quad_append(cache, quad, pos, k_new, stream=None):
 def kvq_quad_page_scores(cache, quad, q, sm_scale: float, scores, stream=None):
     _check(_lib.kvq_quad_page_scores(cache.ref(), quad.ref(), _ptr(q), float(sm_scale), _ptr(scores),
                                      _stream(stream)), "kvq_quad_page_scores")
+
+
+def kvq_quad_append_scores(cache, quad, pos, k_new, v_new, q, sm_scale: float, scores, stream=None):
+    _check(_lib.kvq_quad_append_scores(cache.ref(), quad.ref(), _ptr(pos), _ptr(k_new), _ptr(v_new), _ptr(q),
+                                       float(sm_scale), _ptr(scores), _stream(stream)), "kvq_quad_append_scores")
 
 
 # ------------------------------------------------------------------------- allocation
@@ -420,8 +427,10 @@ class DecodeStep:
                          self.kmax, self.ws)
 
     def append_scores(self):
-        assert self.quad is None, "the fused launches score pages with the mean-key score"
-        if self.w.append:
+        if self.w.append and self.quad is not None:
+            kvq_quad_append_scores(self.cache, self.quad, self.pos, self.k_new, self.v_new, self.q, self.w.sm_scale,
+                                   self.scores)
+        elif self.w.append:
             kvq_append_scores(self.cache, self.pos, self.k_new, self.v_new, self.q, self.scores)
         else:
             self.scores_()

@@ -142,3 +142,28 @@ def test_quad_scores_differ_from_the_plain_score(kvq):
     assert np.array_equal(fin, np.isfinite(bq))
     assert np.all(bq[fin] >= a[fin] - 1e-4 * np.abs(a[fin]) - 1e-6)   # the added term is >= 0
     assert np.mean(bq[fin] > a[fin] + 1e-6) > 0.9
+
+
+@pytest.mark.parametrize("name", ["c1_r16_random", "c4_r24_random"])
+def test_fused_quad_append_scores_equals_the_separate_calls(kvq, name):
+    """kvq_quad_append_scores (one launch) -> select -> attention gives the bytes, state,
+    scores and outputs of kvq_append -> kvq_quad_append -> kvq_quad_page_scores -> ..."""
+    mk, rank, kind = CASES[name]
+    w = mk()
+    basis = _basis(w, rank, kind)
+    res = []
+    for path in ("calls", "three"):
+        cache = kvq.cache_from_workload(w, quad_basis=basis)
+        step = kvq.DecodeStep(w, cache, quad=True)
+        step.run() if path == "calls" else step.run_three()
+        torch.cuda.synchronize()
+        assert cache.err_bits() == 0, hex(cache.err_bits())
+        res.append(dict(scores=step.scores.cpu().numpy(), sel=step.sel.cpu().numpy(), cnt=step.cnt.cpu().numpy(),
+                        out=step.out.cpu().view(torch.int16).numpy(), lam=cache.quad.lam.cpu().numpy().view(np.uint16),
+                        open=cache.quad.open.cpu().numpy(), summary=cache.summary.cpu().numpy().view(np.uint16),
+                        pools=[None if p is None else p.cpu().numpy() for p in cache.pools]))
+    a, b = res
+    for key in ("scores", "sel", "cnt", "out", "lam", "open", "summary"):
+        assert np.array_equal(a[key], b[key]), key
+    for pa, pb in zip(a["pools"], b["pools"]):
+        assert (pa is None) == (pb is None) and (pa is None or np.array_equal(pa, pb))
