@@ -15,8 +15,8 @@
 // -fmad=false): y_i = sum_d u[i][d] k[d] in channel order, S1 = sum_t y and S2 = sum_t y^2
 // in token order, lambda = fp16(max(S2/n - (S1/n)^2, 0)); a page built at once and a page
 // grown token by token hold the same bits.  The score is fp32: the q.kbar part on the
-// tensor core exactly as kvq_page_scores (score_tile.cuh), the quadratic part on the CUDA
-// cores from (u_i.q_h)^2 computed once per (sequence, kv head) and warp.
+// tensor core exactly as kvq_page_scores (score_tile.cuh), (u_i.q_h)^2 on the tensor core
+// once per (sequence, kv head) and warp, the quadratic sum on the CUDA cores.
 #include <math.h>
 
 #include "kvq_internal.cuh"
@@ -90,16 +90,23 @@ __global__ void __launch_bounds__(256) quad_build_kernel(DevCache c, DevQuad qd,
 }
 
 // One warp: token `pos` (0 <= pos < max_pages * 16) of sequence b, kv head g, key `krow`,
-// joins the quad state; lane i < r owns basis row i.
-template <bool BF16>
+// joins the quad state; lane i < r owns basis row i.  The dot product is a sequential fp64
+// chain over the channels; the basis row and the key are fetched 8 channels ahead of it.
+template <int D, bool BF16>
 __device__ inline void quad_append_warp(const DevCache& c, const DevQuad& qd, int bg, int g, int ps,
                                         const uint16_t* krow, int lane) {
-  const int D = c.D, r = qd.rank;
+  const int r = qd.rank;
   if (lane >= r) return;
   const int p = ps / kPage, t = ps % kPage;
-  const float* u = qd.basis + ((size_t)g * r + lane) * D;
+  const float4* u4 = reinterpret_cast<const float4*>(qd.basis + ((size_t)g * r + lane) * D);
   double y = 0.0;
-  for (int d = 0; d < D; ++d) y = y + static_cast<double>(u[d]) * key_f64<BF16>(krow[d]);
+#pragma unroll
+  for (int c8 = 0; c8 < D / 8; ++c8) {
+    const float4 ua = u4[2 * c8], ub = u4[2 * c8 + 1];
+    const float uu[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y = y + static_cast<double>(uu[j]) * key_f64<BF16>(krow[8 * c8 + j]);
+  }
   double* o = qd.open + (size_t)bg * 2 * r;
   const double s1 = t == 0 ? y : o[lane] + y;
   const double s2 = t == 0 ? y * y : o[r + lane] + y * y;
@@ -111,7 +118,7 @@ __device__ inline void quad_append_warp(const DevCache& c, const DevQuad& qd, in
 }
 
 // One warp per (sequence, kv head).
-template <bool BF16>
+template <int D, bool BF16>
 __global__ void __launch_bounds__(32) quad_append_kernel(DevCache c, DevQuad qd, const int32_t* __restrict__ pos,
                                                          const uint16_t* __restrict__ k_new) {
   const int bg = blockIdx.x, b = bg / c.Hkv, g = bg % c.Hkv, lane = threadIdx.x;
@@ -120,78 +127,62 @@ __global__ void __launch_bounds__(32) quad_append_kernel(DevCache c, DevQuad qd,
   if (ps >= 0 && ps >= c.max_pages * kPage) {
     if (lane == 0 && g == 0) set_err(c.err, KVQ_DERR_BAD_POS);
   } else if (ps >= 0) {
-    quad_append_warp<BF16>(c, qd, bg, g, ps, k_new + (size_t)bg * c.D, lane);
+    quad_append_warp<D, BF16>(c, qd, bg, g, ps, k_new + (size_t)bg * D, lane);
   }
   griddep_launch_dependents();
 }
 
-// zs[h][i] = (u_i . q_h)^2 for the G query heads of kv head g (fp32): the lanes split the
-// channels (D/32 each), so every load of a basis row or query row is coalesced and all of
-// them are in flight at once; a butterfly over the warp sums each product.
+// zs[h][i] = (u_i . q_h)^2 for the query heads of kv head g, on the tensor core: A = 16
+// basis rows (fp32 split into fp16 hi + lo parts) in the permuted channel order of the
+// score tile (lane (g8, q4) loads channels [D/4 q4, D/4 q4 + D/4) of rows g8 and g8 + 8 as
+// 16-byte loads), B = the query fragments already in registers (hi + lo), fp32
+// accumulation: u_hi q_hi + u_lo q_hi + u_hi q_lo, all products exact.  Rows past the rank
+// load as zero; heads past G are zero rows of B, so their terms are 0.
+__device__ inline void split_f32x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 hf = __half22float2(h);
+  const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
 template <int D, bool BF16>
-__device__ inline void quad_qterms(const DevQuad& qd, const uint16_t* qg, int G, int g, int lane,
+__device__ inline void quad_qterms(const DevQuad& qd, const QFrag<D, BF16>& qf, int g, int lane,
                                    float (*zs)[kMaxQuadRank]) {
-  constexpr int CPL = D / 32;  // channels per lane: 4 (D = 128) or 2 (D = 64)
-  static_assert(CPL == 4 || CPL == 2, "D is 64 or 128");
-  float qv[kMaxG][CPL];
+  constexpr int KS = D / 16, CW = D / 4;
+  const int g8 = lane >> 2, q4 = lane & 3;
+  const float* ub = qd.basis + (size_t)g * qd.rank * D + CW * q4;
+  for (int m0 = 0; m0 < qd.rank; m0 += 16) {
+    const int i0 = m0 + g8, i1 = m0 + g8 + 8;
+    const bool ok0 = i0 < qd.rank, ok1 = i1 < qd.rank;
+    const float4* s0 = reinterpret_cast<const float4*>(ub + (size_t)i0 * D);
+    const float4* s1 = reinterpret_cast<const float4*>(ub + (size_t)i1 * D);
+    float4 x0[KS], x1[KS];
 #pragma unroll
-  for (int h = 0; h < kMaxG; ++h) {
-    uint32_t w[CPL / 2];
-    if (h < G) {
-      if constexpr (CPL == 4) {
-        const uint2 x = *reinterpret_cast<const uint2*>(qg + (size_t)h * D + CPL * lane);
-        w[0] = x.x;
-        w[1] = x.y;
-      } else {
-        w[0] = *reinterpret_cast<const uint32_t*>(qg + (size_t)h * D + CPL * lane);
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < CPL / 2; ++j) w[j] = 0u;
+    for (int kk = 0; kk < KS; ++kk) {
+      x0[kk] = ok0 ? s0[kk] : make_float4(0.f, 0.f, 0.f, 0.f);
+      x1[kk] = ok1 ? s1[kk] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    float cacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int j = 0; j < CPL / 2; ++j) {
-      qv[h][2 * j] = bits_to_float<BF16>(static_cast<uint16_t>(w[j] & 0xFFFFu));
-      qv[h][2 * j + 1] = bits_to_float<BF16>(static_cast<uint16_t>(w[j] >> 16));
+    for (int kk = 0; kk < KS; ++kk) {
+      uint32_t ah[4], al[4];
+      split_f32x2(x0[kk].x, x0[kk].y, ah[0], al[0]);
+      split_f32x2(x1[kk].x, x1[kk].y, ah[1], al[1]);
+      split_f32x2(x0[kk].z, x0[kk].w, ah[2], al[2]);
+      split_f32x2(x1[kk].z, x1[kk].w, ah[3], al[3]);
+      mma16816<false>(cacc, ah, qf.bh[kk][0], qf.bh[kk][1]);
+      mma16816<false>(cacc, al, qf.bh[kk][0], qf.bh[kk][1]);
+      if constexpr (BF16) mma16816<false>(cacc, ah, qf.bl[kk][0], qf.bl[kk][1]);
     }
-  }
-  const float* ub = qd.basis + (size_t)g * qd.rank * D + CPL * lane;
-  for (int i0 = 0; i0 < qd.rank; i0 += 8) {  // 8 basis rows at a time, all loads in flight
-    float u[8][CPL];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if constexpr (CPL == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(ub + (size_t)(i0 + k) * D);
-        u[k][0] = x.x, u[k][1] = x.y, u[k][2] = x.z, u[k][3] = x.w;
-      } else {
-        const float2 x = *reinterpret_cast<const float2*>(ub + (size_t)(i0 + k) * D);
-        u[k][0] = x.x, u[k][1] = x.y;
-      }
+    // cacc: (row i0, head 2 q4), (i0, 2 q4 + 1), (i1, 2 q4), (i1, 2 q4 + 1)
+    if (ok0) {
+      zs[2 * q4][i0] = cacc[0] * cacc[0];
+      zs[2 * q4 + 1][i0] = cacc[1] * cacc[1];
     }
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h) {
-      if (h < G) {  // warp-uniform
-        float p[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          p[k] = 0.0f;
-#pragma unroll
-          for (int j = 0; j < CPL; ++j) p[k] = fmaf(u[k][j], qv[h][j], p[k]);
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) p[k] += __shfl_xor_sync(0xffffffffu, p[k], o);
-        }
-        if (lane < 8) {
-          float z = p[0];
-#pragma unroll
-          for (int k = 1; k < 8; ++k) z = lane == k ? p[k] : z;
-          zs[h][i0 + lane] = z * z;
-        }
-      } else if (lane < 8) {
-        zs[h][i0 + lane] = 0.0f;
-      }
+    if (ok1) {
+      zs[2 * q4][i1] = cacc[2] * cacc[2];
+      zs[2 * q4 + 1][i1] = cacc[3] * cacc[3];
     }
   }
   __syncwarp();
@@ -253,7 +244,7 @@ __global__ void __launch_bounds__(kQuadWarps * 32, 1)
       const int it = bg * tiles_per_bg + (ps / kPage) / 16;
       if (it < i0 || it >= i1) continue;
       append_token_warp<BF16>(c, b, g, ps, ap.k_new + (size_t)bg * D, ap.v_new + (size_t)bg * D, lane, nullptr);
-      quad_append_warp<BF16>(c, qd, bg, g, ps, ap.k_new + (size_t)bg * D, lane);
+      quad_append_warp<D, BF16>(c, qd, bg, g, ps, ap.k_new + (size_t)bg * D, lane);
       __syncwarp();
     }
   }
@@ -282,7 +273,7 @@ __global__ void __launch_bounds__(kQuadWarps * 32, 1)
         P = min((L + kPage - 1) / kPage, c.max_pages);
         out = scores + (size_t)bg * c.max_pages;
         qf.load(q, c.Hq, c.G, b, g, lane, bad);
-        quad_qterms<D, BF16>(qd, q + ((size_t)b * c.Hq + (size_t)g * c.G) * D, c.G, g, lane, zs[warp]);
+        quad_qterms<D, BF16>(qd, qf, g, lane, zs[warp]);
         __syncwarp();
       }
       float v[4];
@@ -372,8 +363,12 @@ cudaError_t launch_quad_append(const DevCache& c, const DevQuad& qd, const int32
                                cudaStream_t s) {
   const uint16_t* k = static_cast<const uint16_t*>(k_new);
   const dim3 grid(c.B * c.Hkv);
-  if (c.dtype == KVQ_DT_BF16) return launch_pdl(quad_append_kernel<true>, grid, dim3(32), 0, s, c, qd, pos, k);
-  return launch_pdl(quad_append_kernel<false>, grid, dim3(32), 0, s, c, qd, pos, k);
+  const bool bf = c.dtype == KVQ_DT_BF16;
+  if (c.D == 128)
+    return bf ? launch_pdl(quad_append_kernel<128, true>, grid, dim3(32), 0, s, c, qd, pos, k)
+              : launch_pdl(quad_append_kernel<128, false>, grid, dim3(32), 0, s, c, qd, pos, k);
+  return bf ? launch_pdl(quad_append_kernel<64, true>, grid, dim3(32), 0, s, c, qd, pos, k)
+            : launch_pdl(quad_append_kernel<64, false>, grid, dim3(32), 0, s, c, qd, pos, k);
 }
 
 cudaError_t launch_quad_scores(const DevCache& c, const DevQuad& qd, const void* q, float sm_scale, float* scores,
