@@ -41,7 +41,7 @@ import functools
 
 import numpy as np
 
-from .quant import TIER_F16, TIER_I1, TIER_BITS
+from .quant import TIER_F16, TIER_F8, TIER_I1, TIER_BITS
 
 T = 16
 
@@ -53,7 +53,7 @@ def codes_bytes(tier: int, D: int) -> int:
 def meta_bytes(tier: int, D: int) -> int:
     if tier == TIER_F16:
         return 0
-    return T * (D // 32) * (2 if tier == TIER_I1 else 4)
+    return T * (D // 32) * (2 if tier in (TIER_I1, TIER_F8) else 4)
 
 
 def chunk_bytes(tier: int, D: int) -> int:
@@ -114,7 +114,7 @@ def pack_chunk(kind: str, tier: int, D: int, n_valid: int, payload: np.ndarray,
     out = [words.astype(np.uint32).view(np.uint8)]
     if tier != TIER_F16:
         G = D // 32
-        if tier == TIER_I1:
+        if tier in (TIER_I1, TIER_F8):
             m = np.zeros((T, G), dtype=np.uint16)
             m[:n_valid] = np.asarray(meta, dtype=np.uint16)[:n_valid]
         else:
@@ -135,6 +135,6 @@ def unpack_chunk(kind: str, tier: int, D: int, data: np.ndarray):
     meta = None
     if tier != TIER_F16:
         G = D // 32
-        dt = np.uint16 if tier == TIER_I1 else np.uint32
+        dt = np.uint16 if tier in (TIER_I1, TIER_F8) else np.uint32
         meta = data[cb:].view(dt).reshape(T, G)
     return payload.astype(np.int64), meta

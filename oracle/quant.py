@@ -3,8 +3,8 @@
 Test infrastructure only (see ``oracle/__init__.py``).
 
 ARGUS ("Virtual Memory for Transformers", sections "The One-Minute Explanation" and
-"Visual Architecture") lists the cold tiers INT8, INT4 (two codes per byte), INT2
-(four per byte) and 1-bit (eight signs per byte).  The pages do not fix the
+"Visual Architecture") lists the tier cascade FP16 -> FP8 -> INT8 -> INT4 (two codes per
+byte) -> INT2 (four per byte) -> 1-bit (eight signs per byte).  The pages do not fix the
 quantiser, so this file takes the plainest affine reading and fixes every rounding:
 
 * a group is 32 consecutive channels of one token of one head (K or V alike);
@@ -16,7 +16,10 @@ quantiser, so this file takes the plainest affine reading and fixes every roundi
   value read back is ``fp32(c * scale + zero)`` with one rounding;
 * 1-bit keeps the sign (``x >= 0`` -> +, so -0 -> +) and one magnitude per group,
   ``m = fp16(sum_j |x_j| / 32)`` (the L2-optimal alpha for ``alpha * sign(x)``), read
-  back as ``+m`` or ``-m``.
+  back as ``+m`` or ``-m``;
+* FP8 is e4m3 with one fp16 scale per group, ``scale = fp16(amax / 448)`` (448 the
+  largest e4m3 value), ``code = e4m3(x / scale)`` rounded half to even with saturation,
+  read back as ``e4m3(code) * scale``.
 
 All intermediate steps are IEEE binary64 with round-half-even; fp16 results that
 would overflow saturate to +-65504 and are reported.
@@ -28,8 +31,57 @@ import numpy as np
 from .fp import fp16_rne_sat, f32_rne, two_sum_exact
 
 GROUP = 32
-TIER_F16, TIER_I8, TIER_I4, TIER_I2, TIER_I1 = 0, 1, 2, 3, 4
-TIER_BITS = {TIER_F16: 16, TIER_I8: 8, TIER_I4: 4, TIER_I2: 2, TIER_I1: 1}
+TIER_F16, TIER_I8, TIER_I4, TIER_I2, TIER_I1, TIER_F8 = 0, 1, 2, 3, 4, 5
+TIER_BITS = {TIER_F16: 16, TIER_I8: 8, TIER_I4: 4, TIER_I2: 2, TIER_I1: 1, TIER_F8: 8}
+E4M3_MAX = 448.0
+
+
+def e4m3_value(code: np.ndarray) -> np.ndarray:
+    """Value of an FP8 e4m3 code (OCP 8-bit float, 'fn' variant): sign, 4 exponent bits
+    (bias 7), 3 mantissa bits; exponent 0 holds the subnormals m * 2^-9; 0x7F / 0xFF are
+    NaN and there is no infinity (the largest finite value is 0x7E = 448)."""
+    c = np.asarray(code, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * 2.0 ** (e.astype(np.float64) - 7.0))
+    mag = np.where((c & 0x7F) == 0x7F, np.nan, mag)
+    return sign * mag
+
+
+def e4m3_rne(v: np.ndarray) -> np.ndarray:
+    """Code of the e4m3 value nearest to ``v`` (fp64), ties to the even code, magnitudes
+    beyond 448 saturating to 448, the sign of ``v`` kept (so -0 -> 0x80); NaN -> 0x7F."""
+    v = np.asarray(v, dtype=np.float64)
+    grid = e4m3_value(np.arange(0x7F))                    # the 127 finite magnitudes, ascending
+    a = np.minimum(np.abs(v), E4M3_MAX)
+    hi = np.searchsorted(grid, a, side="left")            # first grid value >= a
+    hi = np.clip(hi, 0, 0x7E)
+    lo = np.clip(hi - 1, 0, 0x7E)
+    dlo, dhi = a - grid[lo], grid[hi] - a
+    pick = np.where(dlo < dhi, lo, np.where(dhi < dlo, hi, np.where(lo % 2 == 0, lo, hi)))
+    pick = np.where(a == grid[hi], hi, pick)
+    code = pick | np.where(np.signbit(v), 0x80, 0)
+    return np.where(np.isnan(v), 0x7F, code).astype(np.int64)
+
+
+def quantise_fp8(x: np.ndarray):
+    """FP8 tier of groups ``x[..., 32]``: ``scale = fp16(amax / 448)`` (amax the largest
+    magnitude, a zero amax is +0), ``code = e4m3(x / scale)`` (fp64 quotient, then one
+    round-half-even to e4m3 with saturation; all codes 0 when scale == 0); read back as
+    ``e4m3(code) * scale`` (exact in fp32).  Returns ``(codes, scale, scale_bits, overflow)``."""
+    x = np.asarray(x, dtype=np.float64)
+    assert x.shape[-1] == GROUP
+    amax = np.abs(x).max(axis=-1) + 0.0
+    scale, scale_bits, ov = fp16_rne_sat(amax / E4M3_MAX)
+    safe = np.where(scale == 0.0, 1.0, scale)
+    codes = e4m3_rne(x / safe[..., None])
+    codes = np.where((scale == 0.0)[..., None], 0, codes)
+    return codes, scale, scale_bits, ov
+
+
+def dequant_fp8(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    return e4m3_value(codes) * scale[..., None]
 
 
 def quantise_int(x: np.ndarray, bits: int):
@@ -101,6 +153,10 @@ def quantise_token(x: np.ndarray, tier: int):
     if tier == TIER_F16:
         return dict(codes=None, meta=None, xhat=x.copy(), overflow=np.zeros(x.shape[:-1], bool))
     g = x.reshape(*x.shape[:-1], D // GROUP, GROUP)
+    if tier == TIER_F8:
+        codes, scale, sbits, ov = quantise_fp8(g)
+        return dict(codes=codes.reshape(x.shape), meta=sbits.astype(np.uint32),
+                    xhat=dequant_fp8(codes, scale).reshape(x.shape), overflow=ov.any(axis=-1))
     if tier == TIER_I1:
         bits, m, m_bits, ov = quantise_sign(g)
         xhat = dequant_sign(bits, m)

@@ -9,7 +9,7 @@ from oracle.layout import T, _positions, chunk_bytes, codes_bytes, pack_chunk, u
 from oracle.quant import TIER_BITS
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden")
-ALL = [(kind, tier, D) for kind in "kv" for tier in range(5) for D in (64, 128)]
+ALL = [(kind, tier, D) for kind in "kv" for tier in range(6) for D in (64, 128)]
 
 
 def test_hand_derived_positions():
@@ -51,7 +51,7 @@ def test_pack_unpack_roundtrip(kind, tier, D):
     hi = 1 << b
     for n_valid in (T, 5, 1):
         pay = rng.integers(0, hi, (n_valid, D))
-        meta = rng.integers(0, 1 << (16 if tier == 4 else 32), (n_valid, D // 32), dtype=np.uint64)
+        meta = rng.integers(0, 1 << (16 if tier in (4, 5) else 32), (n_valid, D // 32), dtype=np.uint64)
         data = pack_chunk(kind, tier, D, n_valid, pay, meta if tier else None)
         assert data.size == chunk_bytes(tier, D)
         p2, m2 = unpack_chunk(kind, tier, D, data)
@@ -63,8 +63,8 @@ def test_pack_unpack_roundtrip(kind, tier, D):
 
 
 def test_chunk_sizes_d128():
-    # K+V bytes per (page, kv head): 16-bit 8192, int8 4608, int4 2560, int2 1536, 1-bit 768
-    assert [2 * chunk_bytes(t, 128) for t in range(5)] == [8192, 4608, 2560, 1536, 768]
-    for t in range(5):
+    # K+V bytes per (page, kv head): 16-bit 8192, int8 4608, int4 2560, int2 1536, 1-bit 768, fp8 4352
+    assert [2 * chunk_bytes(t, 128) for t in range(6)] == [8192, 4608, 2560, 1536, 768, 4352]
+    for t in range(6):
         for D in (64, 128):
             assert chunk_bytes(t, D) % 16 == 0
