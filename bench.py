@@ -118,7 +118,7 @@ def algorithmic_bytes(w, sel: np.ndarray, cnt: np.ndarray, tier_tbl: np.ndarray,
     quad score the scores also read r' fp16 eigenvalues per page and the append updates
     the open page's sums and eigenvalues."""
     from sparse_mixed_precision_kvq_b200.kvq import kvq_chunk_bytes
-    cb = np.array([2 * kvq_chunk_bytes(t, w.D) for t in range(5)], dtype=np.int64)
+    cb = np.array([2 * kvq_chunk_bytes(t, w.D) for t in range(6)], dtype=np.int64)
     attn = 0
     for b in range(w.B):
         for g in range(w.Hkv):
@@ -400,9 +400,12 @@ def time_dense(w, cache, step, flush, stream, dev, reps=20):
     return float(np.mean(ts))
 
 
+CASCADE = [0, 5, 1, 2, 3, 4]  # tiers from hot to cold: 16-bit, fp8, int8, int4, int2, 1-bit
+
+
 def time_demotion(w, tier: int, flush, stream, dev, peak: float, peak_kind: str, reps: int = 20):
     """kvq_requantize_pages over every prefilled page outside the sink and recent windows
-    whose tier is above ``tier``, into spare slots of a fresh cache (the block table is
+    whose tier is hotter than ``tier``, into spare slots of a fresh cache (the block table is
     put back, outside the timed region, before every repetition)."""
     import torch
     from sparse_mixed_precision_kvq_b200 import kvq
@@ -412,14 +415,14 @@ def time_demotion(w, tier: int, flush, stream, dev, peak: float, peak_kind: str,
     for b in range(w.B):
         P0 = w.pages_before(b)
         for p in range(w.n_sink, P0 - w.n_recent):
-            if tier_tbl[b, p] < tier:
+            if CASCADE.index(int(tier_tbl[b, p])) < CASCADE.index(tier):  # hotter than the target
                 items.append((b, p, int(np.uint32((tier << 29) | nxt[tier]).view(np.int32))))
                 nxt[tier] += 1
     spare = [n - c for n, c in zip(nxt, counts)]
     cache = kvq.cache_from_workload(w, device=dev, spare=spare)
     it = torch.tensor(items, dtype=torch.int32, device=dev)
     bt0 = cache.block_table.clone()
-    cb = np.array([2 * kvq.kvq_chunk_bytes(t, w.D) for t in range(5)], dtype=np.int64)
+    cb = np.array([2 * kvq.kvq_chunk_bytes(t, w.D) for t in range(6)], dtype=np.int64)
     src = np.array([tier_tbl[b, p] for b, p, _ in items], dtype=np.int64)
     nbytes = int(w.Hkv * (cb[src].sum() + len(items) * cb[tier])) + len(items) * (12 + 8)
     ts = []
@@ -518,9 +521,9 @@ def main():
                     help="page score: the mean-key score, or the quad (Gaussian-MGF) score (--path calls or three)")
     ap.add_argument("--quad-rank", type=int, default=16, help="r' of the quad score (8, 16, 24 or 32)")
     ap.add_argument("--dense", action="store_true", help="also time attention over every page")
-    ap.add_argument("--demote", type=int, default=None, choices=[1, 2, 3, 4],
+    ap.add_argument("--demote", type=int, default=None, choices=[1, 2, 3, 4, 5],
                     help="also time kvq_requantize_pages moving the workload's pages outside the sink and "
-                         "recent windows down to this tier (1 int8, 2 int4, 3 int2, 4 1-bit)")
+                         "recent windows to this tier (1 int8, 2 int4, 3 int2, 4 1-bit, 5 fp8)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling runs)")

@@ -87,7 +87,9 @@ typedef enum {
   KVQ_TIER_I8 = 1, /* 8-bit codes, per-32-channel fp16 scale/zero */
   KVQ_TIER_I4 = 2, /* 4-bit codes, two per byte */
   KVQ_TIER_I2 = 3, /* 2-bit codes, four per byte */
-  KVQ_TIER_I1 = 4  /* sign bits, eight per byte, per-32-channel fp16 magnitude */
+  KVQ_TIER_I1 = 4, /* sign bits, eight per byte, per-32-channel fp16 magnitude */
+  KVQ_TIER_F8 = 5  /* FP8 e4m3 codes, per-32-channel fp16 scale = fp16(amax/448),
+                      code = e4m3(x/scale) round-half-even, saturating (ARGUS cascade FP16 -> FP8 -> INT8) */
 } kvq_tier;
 
 /* device error-word bits */
@@ -107,8 +109,8 @@ typedef struct {
   int32_t reserved;
   int32_t* block_table;    /* device [B][max_pages] */
   int32_t* seq_len;        /* device [B] */
-  void* pool[5];           /* device, per tier (NULL if unused) */
-  int64_t pool_slots[5];   /* slots in each pool */
+  void* pool[6];           /* device, per tier (NULL if unused) */
+  int64_t pool_slots[6];   /* slots in each pool */
   uint16_t* summary;       /* device [B][Hkv][max_pages][D] fp16 bits */
   double* open_ksum;       /* device [B][Hkv][D] */
   uint32_t* err_word;      /* device, 1 word */

@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(128) build_kernel(DevCache c, const uint16_t* 
       atomicOr(&words[kind][w], q.code << bit);
       if (lane == 0) {
         unsigned char* meta = reinterpret_cast<unsigned char*>(words[kind]) + codes_bytes(tier, D);
-        if (tier == KVQ_TIER_I1)
+        if (tier == KVQ_TIER_I1 || tier == KVQ_TIER_F8)
           reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = static_cast<uint16_t>(q.meta);
         else
           reinterpret_cast<uint32_t*>(meta)[t * ng + grp] = q.meta;
@@ -179,6 +179,9 @@ __device__ inline void rq_decode_word(const uint32_t* chunk, int W0, int n, floa
       if constexpr (OT == KVQ_TIER_I1) {
         const float m = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(meta)[t * ng + (d >> 5)]));
         v = code ? m : -m;
+      } else if constexpr (OT == KVQ_TIER_F8) {
+        v = e4m3_to_float(code) *
+            __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(meta)[t * ng + (d >> 5)]));
       } else {
         const uint32_t mw = reinterpret_cast<const uint32_t*>(meta)[t * ng + (d >> 5)];
         v = fmaf(static_cast<float>(code), __half2float(__ushort_as_half(static_cast<uint16_t>(mw & 0xFFFFu))),
@@ -220,7 +223,7 @@ __device__ inline void rq_quant(int gid, int n, const float (*vals)[kRqGroups + 
   unsigned char* meta = dst + kind * NB + codes_bytes(NT, D);
   if (t >= n) {  // token slot past the sequence: zero codes and metadata
     crow[0] = crow[1] = make_uint4(0, 0, 0, 0);
-    if constexpr (NT == KVQ_TIER_I1) reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = 0;
+    if constexpr (NT == KVQ_TIER_I1 || NT == KVQ_TIER_F8) reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = 0;
     else reinterpret_cast<uint32_t*>(meta)[t * ng + grp] = 0u;
     return;
   }
@@ -228,7 +231,26 @@ __device__ inline void rq_quant(int gid, int n, const float (*vals)[kRqGroups + 
 #pragma unroll
   for (int j = 0; j < kGroup; ++j) v[j] = vals[j][gid];
   uint32_t packed[kGroup / 4];
-  if constexpr (NT == KVQ_TIER_I1) {
+  if constexpr (NT == KVQ_TIER_F8) {  // scale fp16(amax / 448), code e4m3(x / scale) from the fp64 quotient
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    const uint16_t sb = fp16_sat(static_cast<double>(amax) / 448.0, ov);
+    const double sc = static_cast<double>(__half2float(__ushort_as_half(sb)));
+#pragma unroll
+    for (int k = 0; k < kGroup / 4; ++k) {
+      packed[k] = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float x = v[4 * k + i];
+        nonfinite |= !isfinite(x);
+        const uint32_t code =
+            sc != 0.0 ? __nv_cvt_double_to_fp8(static_cast<double>(x) / sc, __NV_SATFINITE, __NV_E4M3) : 0u;
+        packed[k] |= code << (8 * i);
+      }
+    }
+    reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = sb;
+  } else if constexpr (NT == KVQ_TIER_I1) {
     double s = 0.0;
 #pragma unroll
     for (int j = 0; j < kGroup; ++j) s += fabs(static_cast<double>(v[j]));
@@ -331,7 +353,8 @@ __global__ void __launch_bounds__(128) requant_kernel(DevCache c, const int32_t*
     case 1: rq_decode<1, D, BF16>(old_words, n, vals); break;
     case 2: rq_decode<2, D, BF16>(old_words, n, vals); break;
     case 3: rq_decode<3, D, BF16>(old_words, n, vals); break;
-    default: rq_decode<4, D, BF16>(old_words, n, vals); break;
+    case 4: rq_decode<4, D, BF16>(old_words, n, vals); break;
+    default: rq_decode<5, D, BF16>(old_words, n, vals); break;
   }
   __syncthreads();
   bool ov = false, nonfinite = false;
@@ -340,7 +363,8 @@ __global__ void __launch_bounds__(128) requant_kernel(DevCache c, const int32_t*
       case 1: rq_quant<1, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
       case 2: rq_quant<2, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
       case 3: rq_quant<3, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
-      default: rq_quant<4, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
+      case 4: rq_quant<4, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
+      default: rq_quant<5, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
     }
   }
   __syncthreads();
@@ -348,7 +372,8 @@ __global__ void __launch_bounds__(128) requant_kernel(DevCache c, const int32_t*
     case 1: rq_pack<1, D>(codes8, dst); break;
     case 2: rq_pack<2, D>(codes8, dst); break;
     case 3: rq_pack<3, D>(codes8, dst); break;
-    default: rq_pack<4, D>(codes8, dst); break;
+    case 4: rq_pack<4, D>(codes8, dst); break;
+    default: rq_pack<5, D>(codes8, dst); break;
   }
   if (ov) set_err(c.err, KVQ_DERR_FP16_RANGE);
   if (nonfinite) set_err(c.err, KVQ_DERR_NONFINITE);

@@ -4,6 +4,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -14,18 +15,18 @@ namespace kvq {
 constexpr int kPage = 16;       // tokens per page
 constexpr int kGroup = 32;      // channels per quantisation group
 constexpr int kMaxG = 8;        // query heads per kv head handled by one mma N-tile
-constexpr int kNumTiers = 5;
+constexpr int kNumTiers = 6;
 constexpr int kMaxSegments = 6144;  // B * Hkv limit of the attention kernel (offsets in shared memory)
 // Head of every workspace: counters that must be zero when a call starts (every call
 // leaves them zero); kvq_workspace_init zeroes it once.
 constexpr size_t kCounterBytes = 65536;
 
 __host__ __device__ constexpr int tier_bits(int tier) {
-  return tier == 0 ? 16 : tier == 1 ? 8 : tier == 2 ? 4 : tier == 3 ? 2 : 1;
+  return tier == 0 ? 16 : tier == 1 ? 8 : tier == 2 ? 4 : tier == 3 ? 2 : tier == 4 ? 1 : 8;
 }
 __host__ __device__ constexpr int codes_bytes(int tier, int D) { return kPage * D * tier_bits(tier) / 8; }
 __host__ __device__ constexpr int meta_bytes(int tier, int D) {
-  return tier == 0 ? 0 : kPage * (D / kGroup) * (tier == 4 ? 2 : 4);
+  return tier == 0 ? 0 : kPage * (D / kGroup) * ((tier == 4 || tier == 5) ? 2 : 4);
 }
 __host__ __device__ constexpr int chunk_bytes(int tier, int D) { return codes_bytes(tier, D) + meta_bytes(tier, D); }
 
@@ -175,6 +176,11 @@ __device__ inline float bits_to_float(uint16_t v) {
   else return __half2float(__ushort_as_half(v));
 }
 
+// FP8 e4m3 code -> float (exact, NaN codes -> NaN).
+__device__ inline float e4m3_to_float(uint32_t code) {
+  return __half2float(__half(__nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E4M3)));
+}
+
 // Value read back from storage for element (t, d) of a K (kind 0) or V (kind 1) chunk:
 // the 16-bit value, fp32(c * scale + zero) with one rounding, or +-m.
 __device__ inline float load_value(const unsigned char* chunk, int kind, int tier, int D, bool bf16, int t, int d) {
@@ -191,6 +197,10 @@ __device__ inline float load_value(const unsigned char* chunk, int kind, int tie
   if (tier == 4) {
     const float m = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(meta)[t * ng + d / kGroup]));
     return code ? m : -m;
+  }
+  if (tier == 5) {  // e4m3 value times the group's fp16 scale (exact in fp32)
+    const float sc = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(meta)[t * ng + d / kGroup]));
+    return e4m3_to_float(code) * sc;
   }
   const uint32_t mw = reinterpret_cast<const uint32_t*>(meta)[t * ng + d / kGroup];
   const float scale = __half2float(__ushort_as_half(static_cast<uint16_t>(mw & 0xFFFFu)));

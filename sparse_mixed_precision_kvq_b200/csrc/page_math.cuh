@@ -10,7 +10,8 @@
 // and the per-group affine map is applied around the mma with z' = zero + 2^(b-1)*scale:
 // for K, S += scale_t * (codes . q) + z'_t * sum(q over the group); for V, P^T is scaled
 // per token by the group's scale before the mma and sum_t z'_t * p_t is accumulated on
-// the side.  P^T enters the tensor core as a 16-bit hi + lo pair (two mmas), so the only
+// the side.  FP8 (e4m3) pages convert their codes exactly to fp16 / bf16 and have no zero
+// offset (S += scale_t * (codes . q); V: P^T scaled per token).  P^T enters the tensor core as a 16-bit hi + lo pair (two mmas), so the only
 // 16-bit rounding on the way to the output is the final cast.  Online softmax runs in
 // the log2 domain.
 #pragma once
@@ -62,9 +63,24 @@ __device__ inline uint32_t sub2(uint32_t x, uint32_t y, bool bf16) {
 // j of lane word w (1-bit: +-1).  Centring keeps the tensor-core term and the separate
 // zero term small, so the 16-bit rounding of the other operand is not amplified by
 // cancellation between them.
+// FP8 e4m3 byte -> fp32, exact: the byte's exponent and mantissa placed in an fp32
+// pattern, then scaled by 2^(127 - 7); e4m3 subnormals land on fp32 subnormals, so the
+// product is exact for them too (NaN codes, from non-finite input, come out as 480).
+__device__ inline float e4m3_bits_to_f32(uint32_t b) {
+  return __uint_as_float(((b & 0x80u) << 24) | ((b & 0x7Fu) << 20)) * 0x1p120f;
+}
+
 template <int TIER, bool BF16>
 __device__ inline uint32_t code_pair(uint32_t w, int j) {
-  if constexpr (TIER == KVQ_TIER_I1) {
+  if constexpr (TIER == KVQ_TIER_F8) {  // e4m3 bytes j and j + 2: exact in fp16 and bf16
+    if constexpr (BF16) {
+      return pack2<true>(e4m3_bits_to_f32(w >> (8 * j)), e4m3_bits_to_f32(w >> (16 + 8 * j)));
+    } else {
+      const uint32_t x2 = __byte_perm(w, 0u, static_cast<uint32_t>(j | ((j + 2) << 4) | 0x4400));
+      const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(x2), __NV_E4M3);
+      return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+    }
+  } else if constexpr (TIER == KVQ_TIER_I1) {
     const uint32_t neg1 = BF16 ? 0xBF80BF80u : 0xBC00BC00u;  // (-1, -1)
     return ((w << (15 - j)) & 0x80008000u) ^ neg1;              // bit set -> +1
   } else if constexpr (TIER == KVQ_TIER_I8 && BF16) {
@@ -85,7 +101,8 @@ __device__ inline uint32_t code_pair(uint32_t w, int j) {
 // Lane words of a b-bit codes area (NW words per lane, stored in pieces of PW words).
 template <int TIER, int D>
 struct LaneWords {
-  static constexpr int b = TIER == KVQ_TIER_I8 ? 8 : TIER == KVQ_TIER_I4 ? 4 : TIER == KVQ_TIER_I2 ? 2 : 1;
+  static constexpr int b = (TIER == KVQ_TIER_I8 || TIER == KVQ_TIER_F8) ? 8 : TIER == KVQ_TIER_I4 ? 4
+                           : TIER == KVQ_TIER_I2 ? 2 : 1;
   static constexpr int NW = D * b / 64;
   static constexpr int PW = NW < 4 ? NW : 4;
   static constexpr int PPW = 16 / b;  // register pairs per word
@@ -117,7 +134,8 @@ struct LaneWords {
 };
 
 // Per-token metadata of one chunk for the lane's two token rows t0 = g8, t1 = g8 + 8:
-// the scale s and the zero offset of the centred codes, z + 2^(b-1) * s (1-bit: m, 0).
+// the scale s and the zero offset of the centred codes, z + 2^(b-1) * s (1-bit: m, 0;
+// FP8: the scale, 0).
 template <int TIER, int D>
 __device__ __forceinline__ void load_meta(const unsigned char* meta, int t0, float (&s)[2][D / 32],
                                           float (&z)[2][D / 32]) {
@@ -126,7 +144,7 @@ __device__ __forceinline__ void load_meta(const unsigned char* meta, int t0, flo
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int t = t0 + 8 * i;
-    if constexpr (TIER == KVQ_TIER_I1) {
+    if constexpr (TIER == KVQ_TIER_I1 || TIER == KVQ_TIER_F8) {
       const uint16_t* m = reinterpret_cast<const uint16_t*>(meta) + t * NG;
 #pragma unroll
       for (int gi = 0; gi < NG; ++gi) {
@@ -186,10 +204,17 @@ __device__ __forceinline__ void qk_page(const unsigned char* base, int lane, con
         lw.template frag<BF16>(2 * gi + h, a);
         mma16816<BF16>(acc, a, st.qb[2 * gi + h][0], st.qb[2 * gi + h][1]);
       }
-      sacc[0] += s[0][gi] * acc[0] + z[0][gi] * st.qs[gi][0];
-      sacc[1] += s[0][gi] * acc[1] + z[0][gi] * st.qs[gi][1];
-      sacc[2] += s[1][gi] * acc[2] + z[1][gi] * st.qs[gi][0];
-      sacc[3] += s[1][gi] * acc[3] + z[1][gi] * st.qs[gi][1];
+      if constexpr (TIER == KVQ_TIER_F8) {  // no zero offset
+        sacc[0] += s[0][gi] * acc[0];
+        sacc[1] += s[0][gi] * acc[1];
+        sacc[2] += s[1][gi] * acc[2];
+        sacc[3] += s[1][gi] * acc[3];
+      } else {
+        sacc[0] += s[0][gi] * acc[0] + z[0][gi] * st.qs[gi][0];
+        sacc[1] += s[0][gi] * acc[1] + z[0][gi] * st.qs[gi][1];
+        sacc[2] += s[1][gi] * acc[2] + z[1][gi] * st.qs[gi][0];
+        sacc[3] += s[1][gi] * acc[3] + z[1][gi] * st.qs[gi][1];
+      }
     }
   }
 }
@@ -231,7 +256,7 @@ __device__ __forceinline__ void pv_page(const unsigned char* base, int lane, War
         mma16816<true>(st.o[2 * gi + h], a, b0h, b1h);
         mma16816<true>(st.o[2 * gi + h], a, b0l, b1l);
       }
-      if constexpr (TIER != KVQ_TIER_I1) {
+      if constexpr (TIER != KVQ_TIER_I1 && TIER != KVQ_TIER_F8) {
         st.zacc[gi][0] += z[0][gi] * p[0] + z[1][gi] * p[2];
         st.zacc[gi][1] += z[0][gi] * p[1] + z[1][gi] * p[3];
       }
@@ -255,7 +280,8 @@ __device__ __forceinline__ void process_page(const unsigned char* base, int tier
       case KVQ_TIER_I8: qk_page<KVQ_TIER_I8, D, BF16>(base, lane, st, sacc); break;
       case KVQ_TIER_I4: qk_page<KVQ_TIER_I4, D, BF16>(base, lane, st, sacc); break;
       case KVQ_TIER_I2: qk_page<KVQ_TIER_I2, D, BF16>(base, lane, st, sacc); break;
-      default: qk_page<KVQ_TIER_I1, D, BF16>(base, lane, st, sacc); break;
+      case KVQ_TIER_I1: qk_page<KVQ_TIER_I1, D, BF16>(base, lane, st, sacc); break;
+      default: qk_page<KVQ_TIER_F8, D, BF16>(base, lane, st, sacc); break;
     }
   }
   const int t0 = lane >> 2, t1 = t0 + 8;
@@ -303,7 +329,8 @@ __device__ __forceinline__ void process_page(const unsigned char* base, int tier
     case KVQ_TIER_I8: pv_page<KVQ_TIER_I8, D, BF16>(vbase, lane, st, p); break;
     case KVQ_TIER_I4: pv_page<KVQ_TIER_I4, D, BF16>(vbase, lane, st, p); break;
     case KVQ_TIER_I2: pv_page<KVQ_TIER_I2, D, BF16>(vbase, lane, st, p); break;
-    default: pv_page<KVQ_TIER_I1, D, BF16>(vbase, lane, st, p); break;
+    case KVQ_TIER_I1: pv_page<KVQ_TIER_I1, D, BF16>(vbase, lane, st, p); break;
+    default: pv_page<KVQ_TIER_F8, D, BF16>(vbase, lane, st, p); break;
   }
 }
 

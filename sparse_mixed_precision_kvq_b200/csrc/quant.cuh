@@ -3,7 +3,8 @@
 // fused decode step.
 //
 // ARGUS "Virtual Memory for Transformers", "Visual Architecture": INT8 / INT4 / INT2 /
-// 1-bit cold tiers.  Per 32-channel group: zero = fp16(min), scale =
+// 1-bit cold tiers (and FP8 e4m3: scale = fp16(max|x| / 448), code = e4m3(x / scale)
+// rounded half to even with saturation).  Per 32-channel group: zero = fp16(min), scale =
 // fp16((max - min) / (2^b - 1)), code = clamp(rint((x - zero) / scale), 0, 2^b - 1) (0 when
 // scale == 0); 1-bit: sign (x >= 0) and magnitude fp16(sum|x| / 32) summed in channel order.
 // Every step is an IEEE binary64 operation with round-half-even, so the bytes do not depend
@@ -32,6 +33,16 @@ __device__ inline QOut quant_group(double x, int tier, bool& ov) {
     for (int j = 0; j < kGroup; ++j) s += __shfl_sync(full, ax, j);
     const uint16_t m = fp16_sat(s / 32.0, ov);
     return {bit, m};
+  }
+  if (tier == KVQ_TIER_F8) {  // e4m3 with scale fp16(amax / 448), round-half-even, saturating
+    double a = fabs(x);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) a = fmax(a, __shfl_xor_sync(full, a, o));
+    a += 0.0;
+    const uint16_t sb = fp16_sat(a / 448.0, ov);
+    const double scale = static_cast<double>(__half2float(__ushort_as_half(sb)));
+    const uint32_t code = scale != 0.0 ? __nv_cvt_double_to_fp8(x / scale, __NV_SATFINITE, __NV_E4M3) : 0u;
+    return {code, sb};
   }
   double lo = x, hi = x;
 #pragma unroll
@@ -127,7 +138,7 @@ __device__ inline bool append_phase2(const DevCache& c, int b, int g, int pos, c
     atomicOr(word, q.code << bit);
     if (lane == 0) {
       unsigned char* meta = chunk + codes_bytes(tier, D);
-      if (tier == KVQ_TIER_I1)
+      if (tier == KVQ_TIER_I1 || tier == KVQ_TIER_F8)
         reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = static_cast<uint16_t>(q.meta);
       else
         reinterpret_cast<uint32_t*>(meta)[t * ng + grp] = q.meta;

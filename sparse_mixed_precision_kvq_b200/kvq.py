@@ -25,7 +25,7 @@ if not os.path.exists(LIB_PATH):
         "`python -m sparse_mixed_precision_kvq_b200.build` (there is no CPU fallback)")
 _lib = ctypes.CDLL(LIB_PATH)
 
-TIER_16, TIER_I8, TIER_I4, TIER_I2, TIER_I1 = 0, 1, 2, 3, 4
+TIER_16, TIER_I8, TIER_I4, TIER_I2, TIER_I1, TIER_F8 = 0, 1, 2, 3, 4, 5
 DT_F16, DT_BF16 = 0, 1
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "workspace too small", 4: "CUDA error"}
 
@@ -43,8 +43,8 @@ EXPORTS = ["kvq_chunk_bytes", "kvq_status_string", "kvq_append", "kvq_build_page
 class KvqCache(ctypes.Structure):
     _fields_ = [("B", c_int32), ("Hq", c_int32), ("Hkv", c_int32), ("D", c_int32),
                 ("page_size", c_int32), ("max_pages", c_int32), ("dtype", c_int32), ("reserved", c_int32),
-                ("block_table", c_void_p), ("seq_len", c_void_p), ("pool", c_void_p * 5),
-                ("pool_slots", c_int64 * 5), ("summary", c_void_p), ("open_ksum", c_void_p),
+                ("block_table", c_void_p), ("seq_len", c_void_p), ("pool", c_void_p * 6),
+                ("pool_slots", c_int64 * 6), ("summary", c_void_p), ("open_ksum", c_void_p),
                 ("err_word", c_void_p)]
 
 
@@ -246,7 +246,7 @@ class PagedCache:
         self.device = dev
         self.block_table = torch.full((B, max_pages), -1, dtype=torch.int32, device=dev)
         self.seq_len = torch.zeros(B, dtype=torch.int32, device=dev)
-        self.pool_slots = [int(x) for x in pool_slots]
+        self.pool_slots = [int(x) for x in pool_slots] + [0] * (6 - len(pool_slots))
         self.pools = []
         for tier, n in enumerate(self.pool_slots):
             if n > 0:
@@ -263,7 +263,7 @@ class PagedCache:
         s.B, s.Hq, s.Hkv, s.D, s.page_size, s.max_pages = B, Hq, Hkv, D, 16, max_pages
         s.dtype = DT_BF16 if dtype == "bf16" else DT_F16
         s.block_table, s.seq_len = _ptr(self.block_table), _ptr(self.seq_len)
-        for i in range(5):
+        for i in range(6):
             s.pool[i] = _ptr(self.pools[i]) if self.pools[i] is not None else None
             s.pool_slots[i] = self.pool_slots[i]
         s.summary, s.open_ksum, s.err_word = _ptr(self.summary), _ptr(self.open_ksum), _ptr(self.err)

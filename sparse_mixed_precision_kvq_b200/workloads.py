@@ -37,8 +37,8 @@ from typing import Dict, List, Optional
 import numpy as np
 
 PAGE = 16
-TIER_F16, TIER_I8, TIER_I4, TIER_I2, TIER_I1 = 0, 1, 2, 3, 4
-N_TIERS = 5
+TIER_F16, TIER_I8, TIER_I4, TIER_I2, TIER_I1, TIER_F8 = 0, 1, 2, 3, 4, 5
+N_TIERS = 6
 
 # stream tags (part of the seed key of each random stream)
 _S_KEY, _S_VAL, _S_Q, _S_KNEW, _S_VNEW, _S_OUTL, _S_PLANT, _S_TIER, _S_SLOT, _S_LEN, _S_QUAD = range(11)

@@ -63,7 +63,7 @@ int tier_mismatches() {
 
 int main() {
   const int bad = tier_mismatches<0>() + tier_mismatches<1>() + tier_mismatches<2>() + tier_mismatches<3>() +
-                  tier_mismatches<4>();
+                  tier_mismatches<4>() + tier_mismatches<5>();
   std::printf("layout inverse mismatches: %d\n", bad);
   return bad != 0;
 }

@@ -17,7 +17,7 @@ from tests.parity_helpers import (check_output, check_pages, check_selection, or
 
 pytestmark = pytest.mark.gpu
 
-ALL_TIERS = {W.TIER_F16: 0.2, W.TIER_I8: 0.2, W.TIER_I4: 0.2, W.TIER_I2: 0.2, W.TIER_I1: 0.2}
+ALL_TIERS = {W.TIER_F16: 0.16, W.TIER_I8: 0.17, W.TIER_I4: 0.17, W.TIER_I2: 0.17, W.TIER_I1: 0.17, W.TIER_F8: 0.16}
 CASES = {
     "bf16_d128": lambda: W.make("c1", B=2, Hq=16, Hkv=4, lens=np.array([700, 333]), tier_fracs=ALL_TIERS,
                                 k_frac_bp=2000),
@@ -32,9 +32,13 @@ def kvq():
     return k
 
 
+CASCADE = [W.TIER_F16, W.TIER_F8, W.TIER_I8, W.TIER_I4, W.TIER_I2, W.TIER_I1]  # hot to cold
+
+
 def demotion_plan(w, seed=7, frac=0.6):
-    """(b, page, new tier) for a seeded subset of the prefilled pages, each to a lower tier;
-    the last prefilled page of every sequence is always in the plan (when it can move)."""
+    """(b, page, new tier) for a seeded subset of the prefilled pages, each to a colder tier
+    of the cascade; the last prefilled page of every sequence is always in the plan (when
+    it can move)."""
     rng = np.random.default_rng(seed)
     plan = []
     for b in range(w.B):
@@ -42,15 +46,16 @@ def demotion_plan(w, seed=7, frac=0.6):
         P0 = w.pages_before(b)
         for p in range(P0):
             t = int(tiers[p])
+            pos = CASCADE.index(t)
             if t == W.TIER_I1 or (p != P0 - 1 and rng.random() > frac):
                 continue
-            plan.append((b, p, int(rng.integers(max(t, W.TIER_F16) + 1, W.TIER_I1 + 1))))
+            plan.append((b, p, CASCADE[int(rng.integers(pos + 1, len(CASCADE)))]))
     return plan
 
 
 def apply_plan(kvq, w, plan):
     """Cache with spare slots, demoted on the GPU; returns (cache, items, new entries)."""
-    spare = [0] * 5
+    spare = [0] * 6
     for _, _, t in plan:
         spare[t] += 1
     _, _, counts = w.slot_map()
@@ -116,7 +121,7 @@ def test_decode_step_on_a_demoted_cache(kvq, name):
 
 def test_invalid_items_are_skipped_with_an_error_bit(kvq):
     w = CASES["f16_d64"]()
-    cache = kvq.cache_from_workload(w, spare=[0, 1, 1, 1, 1])
+    cache = kvq.cache_from_workload(w, spare=[0, 1, 1, 1, 1, 1])
     bt0 = cache.block_table.clone()
     pools0 = [None if p is None else p.clone() for p in cache.pools]
     _, _, counts = w.slot_map()
@@ -134,6 +139,7 @@ def test_invalid_items_are_skipped_with_an_error_bit(kvq):
         (1, w.max_pages, ent(2, counts[2])),       # page out of range
         (1, 10, ent(2, counts[2])),                # a page holding no tokens (77 tokens: pages 0..4)
         (0, 3, ent(6, 0)),                         # no such tier
+        (0, 3, ent(7, 0)),                         # no such tier
     ]
     kvq.kvq_requantize_pages(cache, torch.tensor(bad, dtype=torch.int32, device="cuda"))
     torch.cuda.synchronize()
@@ -171,11 +177,12 @@ def _tie_values(D, L, seed=3):
 
 @pytest.mark.parametrize("D", [64, 128])
 def test_requantize_rounding_ties_and_signed_zeros(kvq, D):
-    """Page p (16-bit) moves to int8, int4, int2 in turn: every tie group takes the exact
-    fp64 route and rounds half to even; then int8 -> int2 and int4 -> 1-bit."""
+    """Pages 0-2 (16-bit) move to int8, int4, int2: every tie group takes the exact fp64
+    route and rounds half to even; then int8 -> int2, int4 -> 1-bit, int2 -> fp8, and
+    fp8 -> int4."""
     L, Hkv = 40, 2
     bits = [_tie_values(D, L, seed=g) for g in range(Hkv)]
-    cache = kvq.PagedCache(1, 2 * Hkv, Hkv, D, 3, "f16", [3, 3, 3, 3, 3], "cuda")
+    cache = kvq.PagedCache(1, 2 * Hkv, Hkv, D, 3, "f16", [3, 3, 3, 3, 3, 3], "cuda")
     cache.block_table.copy_(torch.from_numpy(kvq.encode_block_table(np.zeros((1, 3), np.int64),
                                                                     np.arange(3)[None])))
     cache.seq_len.fill_(L)
@@ -187,7 +194,7 @@ def test_requantize_rounding_ties_and_signed_zeros(kvq, D):
         return int(np.uint32((t << 29) | s).view(np.int32))
 
     heads = [ocache.build(b_[0], b_[1], "f16", np.zeros(3, np.int64)) for b_ in bits]
-    for plan in ([(0, 1, 0), (1, 2, 0), (2, 3, 0)], [(0, 3, 1), (1, 4, 1)]):
+    for plan in ([(0, 1, 0), (1, 2, 0), (2, 3, 0)], [(0, 3, 1), (1, 4, 1), (2, 5, 0)], [(2, 2, 1)]):
         items = torch.tensor([(0, p, ent(t, s)) for p, t, s in plan], dtype=torch.int32, device="cuda")
         kvq.kvq_requantize_pages(cache, items)
         torch.cuda.synchronize()

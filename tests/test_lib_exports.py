@@ -66,8 +66,8 @@ def test_every_binding_declares_its_argument_types():
 
 def test_host_helpers_without_gpu():
     from sparse_mixed_precision_kvq_b200 import kvq
-    assert [2 * kvq.kvq_chunk_bytes(t, 128) for t in range(5)] == [8192, 4608, 2560, 1536, 768]
-    assert kvq.kvq_chunk_bytes(5, 128) == 0 and kvq.kvq_chunk_bytes(0, 96) == 0
+    assert [2 * kvq.kvq_chunk_bytes(t, 128) for t in range(6)] == [8192, 4608, 2560, 1536, 768, 4352]
+    assert kvq.kvq_chunk_bytes(6, 128) == 0 and kvq.kvq_chunk_bytes(0, 96) == 0
     assert kvq.kvq_status_string(0) == "ok" and "workspace" in kvq.kvq_status_string(3)
 
 
