@@ -151,12 +151,15 @@ def kernel_traffic(kernel_file: str):
 
 
 # ----------------------------------------------------------------------------- ranks
-def rank_workload(config: str, rank: int, batch=None):
+def rank_workload(config: str, rank: int, batch=None, tier=None):
     """Rank r's batch: the workload's shapes with its own seeds (independent sequences per
-    rank: weak scaling, nothing exchanged on the data path)."""
+    rank: weak scaling, nothing exchanged on the data path).  ``tier`` stores every
+    prefilled page at that tier instead of the workload's mix."""
     from sparse_mixed_precision_kvq_b200 import workloads as W
     base = W.make(config)
     over = {} if batch is None else dict(B=batch)
+    if tier is not None:
+        over.update(tier_fracs={int(tier): 1.0}, hot_f16_planted=False)
     if batch is not None and config != "c4":
         over["lens"] = np.resize(base.lens, batch)
     return W.make(config, seed=base.seed + 1000 * rank, **over)
@@ -182,7 +185,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = rank_workload(args.config, rank, args.batch)
+    w = rank_workload(args.config, rank, args.batch, args.tier)
     quad_rank = args.quad_rank if args.score == "quad" else 0
     basis = None
     if quad_rank:
@@ -341,6 +344,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
                    "context": int(w.lens.max()), "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
                    "selected_pages": int(cnt.sum()),
                    "selection": "budget" if args.coverage is None else f"coverage {args.coverage}",
+                   "tiers": "the workload's" if args.tier is None else f"every prefilled page at tier {args.tier}",
                    "page_score": "mean-key" if not quad_rank else
                    f"quad (rank {quad_rank}, basis: eigenvectors of the key law's covariance)",
                    "l2": f"flushed ({args.flush_mib} MiB write) before every timed step",
@@ -520,6 +524,8 @@ def main():
     ap.add_argument("--score", default="mean", choices=["mean", "quad"],
                     help="page score: the mean-key score, or the quad (Gaussian-MGF) score (--path calls or three)")
     ap.add_argument("--quad-rank", type=int, default=16, help="r' of the quad score (8, 16, 24 or 32)")
+    ap.add_argument("--tier", type=int, default=None, choices=[0, 1, 2, 3, 4, 5],
+                    help="store every prefilled page at this tier (0 16-bit, 1 int8, 2 int4, 3 int2, 4 1-bit, 5 fp8)")
     ap.add_argument("--dense", action="store_true", help="also time attention over every page")
     ap.add_argument("--demote", type=int, default=None, choices=[1, 2, 3, 4, 5],
                     help="also time kvq_requantize_pages moving the workload's pages outside the sink and "
