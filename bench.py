@@ -190,7 +190,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     basis = None
     if quad_rank:
         basis = np.stack([w.quad_basis(g, quad_rank, "law") for g in range(w.Hkv)])
-    cache = kvq.cache_from_workload(w, device=dev, quad_basis=basis)
+    cache = kvq.cache_from_workload(w, device=dev, quad_basis=basis, host_tiers=args.host_tiers)
     step = kvq.DecodeStep(w, cache, device=dev, coverage=args.coverage, quad=bool(quad_rank))
     tier_tbl, _, _ = w.slot_map()
     flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
@@ -345,6 +345,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
                    "selected_pages": int(cnt.sum()),
                    "selection": "budget" if args.coverage is None else f"coverage {args.coverage}",
                    "tiers": "the workload's" if args.tier is None else f"every prefilled page at tier {args.tier}",
+                   "host_tiers": args.host_tiers,
                    "page_score": "mean-key" if not quad_rank else
                    f"quad (rank {quad_rank}, basis: eigenvectors of the key law's covariance)",
                    "l2": f"flushed ({args.flush_mib} MiB write) before every timed step",
@@ -370,6 +371,9 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     }
     if dense_ms is not None:
         line["dense_all_pages_ms"] = dense_ms
+    if args.host_tiers:
+        line["host_link"] = host_link(w, sel, cnt, tier_tbl, args.host_tiers, avg[names.index("sparse_decode_attn")]
+                                      if "sparse_decode_attn" in names else None, dev)
     if args.demote is not None:
         del step, cache
         line["demotion"] = time_demotion(w, args.demote, flush, stream, dev, peak, peak_kind)
@@ -402,6 +406,36 @@ def time_dense(w, cache, step, flush, stream, dev, reps=20):
         if r >= 3:
             ts.append(a.elapsed_time(b_))
     return float(np.mean(ts))
+
+
+def host_link(w, sel, cnt, tier_tbl, mask: int, attn_ms, dev, reps: int = 5):
+    """The attention's bytes read from pinned host memory, their rate over the kernel's
+    event-timed duration, against a pinned host -> device copy of 512 MiB timed here."""
+    import torch
+    from sparse_mixed_precision_kvq_b200.kvq import kvq_chunk_bytes
+    cb = np.array([2 * kvq_chunk_bytes(t, w.D) for t in range(6)], dtype=np.int64)
+    host = 0
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            tiers = tier_tbl[b, sel[b, g, :cnt[b, g]]]
+            host += int(sum(cb[t] for t in tiers if (mask >> int(t)) & 1))
+    src = torch.empty(512 << 20, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    ts = []
+    for r in range(reps + 1):
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dst.copy_(src, non_blocking=True)
+        b_.record()
+        torch.cuda.synchronize(dev)
+        if r:
+            ts.append(a.elapsed_time(b_))
+    peak = (512 << 20) / (np.mean(ts) * 1e-3) / 1e9
+    out = {"mask": mask, "attn_host_bytes": host, "h2d_copy_gbs": peak,
+           "peak_kind": "pinned host -> device copy of 512 MiB, timed in this run"}
+    if attn_ms:
+        out.update(achieved_gbs=host / (attn_ms * 1e-3) / 1e9, frac=host / (attn_ms * 1e-3) / 1e9 / peak)
+    return out
 
 
 CASCADE = [0, 5, 1, 2, 3, 4]  # tiers from hot to cold: 16-bit, fp8, int8, int4, int2, 1-bit
@@ -526,6 +560,8 @@ def main():
     ap.add_argument("--quad-rank", type=int, default=16, help="r' of the quad score (8, 16, 24 or 32)")
     ap.add_argument("--tier", type=int, default=None, choices=[0, 1, 2, 3, 4, 5],
                     help="store every prefilled page at this tier (0 16-bit, 1 int8, 2 int4, 3 int2, 4 1-bit, 5 fp8)")
+    ap.add_argument("--host-tiers", type=int, default=0,
+                    help="bit t: pool t lives in pinned host memory that the kernels read in place (DRAM value tier)")
     ap.add_argument("--dense", action="store_true", help="also time attention over every page")
     ap.add_argument("--demote", type=int, default=None, choices=[1, 2, 3, 4, 5],
                     help="also time kvq_requantize_pages moving the workload's pages outside the sink and "
@@ -539,6 +575,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.coverage is not None and args.path != "calls":
         ap.error("--coverage runs on the four-call path")
+    if args.host_tiers and args.path == "fused":
+        ap.error("--host-tiers: the fused step reads pages by bulk copies only")
     if args.score == "quad" and args.path not in ("calls", "three"):
         ap.error("--score quad runs on the four-call or the three-call path")
 

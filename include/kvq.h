@@ -106,7 +106,10 @@ typedef struct {
   int32_t page_size;       /* must be 16 */
   int32_t max_pages;       /* block-table row length (logical pages per sequence) */
   int32_t dtype;           /* kvq_dtype of keys, values, queries and outputs */
-  int32_t reserved;
+  int32_t host_tiers;      /* bit t set: pool[t] is pinned host memory mapped into the device address
+                              space (AMASS "What is in the box", Stage B: a host-DRAM pool read
+                              by the device); the attention kernel reads those pages with per-thread
+                              asynchronous loads instead of bulk copies; kvq_decode_step rejects it */
   int32_t* block_table;    /* device [B][max_pages] */
   int32_t* seq_len;        /* device [B] */
   void* pool[6];           /* device, per tier (NULL if unused) */

@@ -41,6 +41,8 @@ kvq_status to_dev(const kvq_cache* k, DevCache& c) {
   c.D = k->D;
   c.max_pages = k->max_pages;
   c.dtype = k->dtype;
+  if (static_cast<uint32_t>(k->host_tiers) >> kNumTiers) return KVQ_ERR_INVALID_ARG;
+  c.host_tiers = static_cast<uint32_t>(k->host_tiers);
   c.block_table = k->block_table;
   c.seq_len = k->seq_len;
   bool any = false;

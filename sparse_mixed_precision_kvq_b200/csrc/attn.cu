@@ -56,6 +56,7 @@ struct PageMeta {
   int end;       // monotonic end of the allocation (ring bytes issued so far)
   int tier;      // -1: page skipped
   int nv;        // valid tokens
+  int group;     // host-memory page: sequence number of its per-lane copy group, else -1
 };
 
 struct AttnArgs {
@@ -273,6 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
   const int f1 = min(total, f0 + W);
 
   int issued = 0, consumed = 0;  // pages of [f0, f1) issued / consumed
+  int groups = 0;                // per-lane copy groups committed (host-memory pages)
   int head = 0, tail = 0;        // monotonic ring byte counters
   int win_base = 0, win_n = 0;   // descriptor window: pages [f0 + win_base, f0 + win_base + win_n)
   PageDesc my{nullptr, -1, 0};
@@ -324,9 +326,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
       if (start + bytes - tail > kRing) break;  // no room yet
       const int slot = issued % kNBar;
       const uint32_t bar = smem_u32(&bars[slot]);
+      const bool host = bytes > 0 && ((c.host_tiers >> tier) & 1u);
+      if (host) {  // pinned host memory: every lane copies its 16-byte pieces, one group per page
+        const unsigned char* src = reinterpret_cast<const unsigned char*>(sp);
+        const uint32_t dst = smem_u32(ring + start % kRing);
+        for (int o = lane * 16; o < bytes; o += 32 * 16) cp_async16(dst + o, src + o);
+        cp_async_commit();
+      }
       if (lane == 0) {
-        pmeta[slot] = PageMeta{start % kRing, start + bytes, tier, nv};
-        if (bytes > 0) {
+        pmeta[slot] = PageMeta{start % kRing, start + bytes, tier, nv, host ? groups : -1};
+        if (bytes > 0 && !host) {
           mbar_expect_tx(bar, static_cast<uint32_t>(bytes));
           bulk_copy_g2s(smem_u32(ring + start % kRing), reinterpret_cast<const void*>(sp),
                         static_cast<uint32_t>(bytes), bar);
@@ -334,6 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
           mbar_arrive(bar);
         }
       }
+      groups += host ? 1 : 0;
       head = start + bytes;
       ++issued;
     }
@@ -372,7 +382,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
     }
     if (!failed) {
       const PageMeta pm = pmeta[slot];
+      if (pm.group >= 0) {  // wait for this page's group (later pages' groups may stay in flight)
+        cp_async_wait_pending(groups - 1 - pm.group);
+        __syncwarp();
+      }
       if (pm.tier >= 0) process_page<D, BF16, ONLY16>(ring_c + pm.ring_off, pm.tier, pm.nv, lane, a.scale_log2, st);
+      if (pm.group >= 0) fence_proxy_async();  // generic-proxy writes, before a bulk copy may reuse the bytes
       tail = pm.end;  // everything before this page's end is free again
     }
     __syncwarp();
@@ -392,6 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
   if (failed) {
     for (int k = consumed; k < issued; ++k) mbar_wait_bounded(smem_u32(&bars[k % kNBar]), (k / kNBar) & 1);
   }
+  if (groups > 0) cp_async_wait_pending(0);  // no per-lane copy may land after this point
 
   // CTA pre-merge: one partial per segment this CTA touched (written straight to the
   // output when the segment lies inside this CTA), then the last CTA of each segment

@@ -42,6 +42,7 @@ struct DevQuad {
 // Everything a kernel needs to locate pages (copied by value into kernel parameters).
 struct DevCache {
   int B, Hq, Hkv, G, D, max_pages, dtype;
+  uint32_t host_tiers;  // bit t: pool t is pinned host memory mapped into the device address space
   const int32_t* block_table;
   const int32_t* seq_len;
   unsigned char* pool[kNumTiers];

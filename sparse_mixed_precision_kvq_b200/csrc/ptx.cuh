@@ -75,6 +75,26 @@ __device__ inline void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t byt
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
+// Per-thread 16-byte asynchronous copy global -> shared (through L2): the copy path for
+// pools in pinned, device-mapped host memory, which are read by ordinary loads rather than
+// handed to the bulk-copy engine.  Both addresses 16-byte aligned.
+__device__ inline void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ inline void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+// Wait until at most n (0..7) of this thread's committed groups are still in flight.
+__device__ inline void cp_async_wait_pending(int n) {
+  switch (n) {
+    case 1: asm volatile("cp.async.wait_group 1;\n" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;\n" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;\n" ::: "memory"); break;
+    case 4: asm volatile("cp.async.wait_group 4;\n" ::: "memory"); break;
+    case 5: asm volatile("cp.async.wait_group 5;\n" ::: "memory"); break;
+    case 6: asm volatile("cp.async.wait_group 6;\n" ::: "memory"); break;
+    case 7: asm volatile("cp.async.wait_group 7;\n" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 0;\n" ::: "memory"); break;
+  }
+}
 // Bulk prefetch of a global range into L2 (16-byte aligned, size a multiple of 16).
 __device__ inline void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");

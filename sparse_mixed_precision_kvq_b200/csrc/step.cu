@@ -769,6 +769,7 @@ size_t attn_items_bound(const DevCache& c, int kmax) {
 }  // namespace
 
 bool step_supported(const DevCache& c) {
+  if (c.host_tiers != 0) return false;  // its pages are fetched by bulk copies only
   if ((long long)c.B * c.Hkv * 2 + kCtlWords > (long long)(kCounterBytes / sizeof(unsigned))) return false;
   return step_plan(c).ns >= kCW;
 }

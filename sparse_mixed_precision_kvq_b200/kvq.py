@@ -42,7 +42,7 @@ EXPORTS = ["kvq_chunk_bytes", "kvq_status_string", "kvq_append", "kvq_build_page
 
 class KvqCache(ctypes.Structure):
     _fields_ = [("B", c_int32), ("Hq", c_int32), ("Hkv", c_int32), ("D", c_int32),
-                ("page_size", c_int32), ("max_pages", c_int32), ("dtype", c_int32), ("reserved", c_int32),
+                ("page_size", c_int32), ("max_pages", c_int32), ("dtype", c_int32), ("host_tiers", c_int32),
                 ("block_table", c_void_p), ("seq_len", c_void_p), ("pool", c_void_p * 6),
                 ("pool_slots", c_int64 * 6), ("summary", c_void_p), ("open_ksum", c_void_p),
                 ("err_word", c_void_p)]
@@ -237,7 +237,7 @@ def encode_block_table(tier_tbl: np.ndarray, slot_tbl: np.ndarray) -> np.ndarray
 class PagedCache:
     """Device tensors of a paged cache plus the ``kvq_cache`` struct pointing at them."""
 
-    def __init__(self, B, Hq, Hkv, D, max_pages, dtype: str, pool_slots, device="cuda"):
+    def __init__(self, B, Hq, Hkv, D, max_pages, dtype: str, pool_slots, device="cuda", host_tiers: int = 0):
         import torch
         self.B, self.Hq, self.Hkv, self.D, self.max_pages = B, Hq, Hkv, D, max_pages
         self.dtype = dtype
@@ -248,10 +248,14 @@ class PagedCache:
         self.seq_len = torch.zeros(B, dtype=torch.int32, device=dev)
         self.pool_slots = [int(x) for x in pool_slots] + [0] * (6 - len(pool_slots))
         self.pools = []
+        self.host_tiers = int(host_tiers)
         for tier, n in enumerate(self.pool_slots):
             if n > 0:
                 nbytes = n * Hkv * 2 * kvq_chunk_bytes(tier, D)
-                self.pools.append(torch.zeros(nbytes, dtype=torch.uint8, device=dev))
+                if (self.host_tiers >> tier) & 1:  # pinned host memory, read by the device in place
+                    self.pools.append(torch.zeros(nbytes, dtype=torch.uint8, pin_memory=True))
+                else:
+                    self.pools.append(torch.zeros(nbytes, dtype=torch.uint8, device=dev))
             else:
                 self.pools.append(None)
         self.summary = torch.zeros((B, Hkv, max_pages, D), dtype=torch.float16, device=dev)
@@ -262,6 +266,7 @@ class PagedCache:
         s = self._s
         s.B, s.Hq, s.Hkv, s.D, s.page_size, s.max_pages = B, Hq, Hkv, D, 16, max_pages
         s.dtype = DT_BF16 if dtype == "bf16" else DT_F16
+        s.host_tiers = self.host_tiers
         s.block_table, s.seq_len = _ptr(self.block_table), _ptr(self.seq_len)
         for i in range(6):
             s.pool[i] = _ptr(self.pools[i]) if self.pools[i] is not None else None
@@ -307,20 +312,21 @@ class QuadState:
         return ctypes.byref(self._s)
 
 
-def cache_from_workload(w, device="cuda", threads: int = 8, spare=None, quad_basis=None):
+def cache_from_workload(w, device="cuda", threads: int = 8, spare=None, quad_basis=None, host_tiers: int = 0):
     """Allocate a cache for workload ``w`` and store its prefilled context with kvq_build_pages.
 
     After the call ``seq_len`` holds the prefilled lengths (before the step's append).
     ``spare`` (optional, per tier) adds free slots after the used ones of each pool.
     ``quad_basis`` (optional, fp32 ``[Hkv, rank, D]``) also builds the quad page-score state
-    (``cache.quad``) from the same keys with kvq_quad_build.
+    (``cache.quad``) from the same keys with kvq_quad_build.  ``host_tiers`` (bit t) puts
+    pool t in pinned host memory that the kernels read in place.
     """
     import torch
     from concurrent.futures import ThreadPoolExecutor
     tier_tbl, slot_tbl, counts = w.slot_map()
     if spare is not None:
         counts = [int(c) + int(x) for c, x in zip(counts, spare)]
-    cache = PagedCache(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.dtype, counts, device)
+    cache = PagedCache(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.dtype, counts, device, host_tiers=host_tiers)
     cache.block_table.copy_(torch.from_numpy(encode_block_table(tier_tbl, slot_tbl)))
     lens = np.asarray(w.lens, dtype=np.int64)
     cache.seq_len.copy_(torch.from_numpy(lens.astype(np.int32)))
