@@ -11,16 +11,19 @@
  *                          unpacking and dequantising cold pages in registers;
  *   kvq_append_scores      the first two in one launch (same results);
  *   kvq_score_select       the first three in one launch (same results);
- *   kvq_decode_step        the four above in one persistent launch (same results).
+ *   kvq_decode_step        the four above in one persistent launch (same results);
+ *   kvq_quad_*             the quad (Gaussian-MGF) page score and its per-page state;
+ *   kvq_requantize_pages   tier demotion: re-encode pages into a colder tier.
  *
  * Sources: AMASS "decode-time sparse KV-cache attention for vLLM" (amass-kv 0.1.1),
  * section "What is in the box" (per-page summary -> page score -> small selected working
  * set -> sparse paged kernel reading only those pages) and "Quickstart" (budget: fixed
  * selected fraction); ARGUS "Virtual Memory for Transformers" (argus_cache 0.1.7.1),
- * sections "The One-Minute Explanation" / "Visual Architecture" (fp16 hot pages, INT8,
- * INT4 2-way, INT2 4-way, 1-bit 8-way packed cold pages, reconstruction only when a query
- * touches a page), "Why It Works" (dequantise, then attend) and "Quickstart"
- * (sink_tokens).
+ * sections "The One-Minute Explanation" / "Visual Architecture" (fp16 hot pages; the
+ * cascade FP8, INT8, INT4 2-way, INT2 4-way, 1-bit 8-way packed for cold pages;
+ * reconstruction only when a query touches a page), "Why It Works" (dequantise, then
+ * attend) and "Quickstart" (sink_tokens); AMASS Stage B (a pinned, device-mapped
+ * host-DRAM pool: kvq_cache.host_tiers).
  *
  * Conventions (every call):
  *  - Pointers named "device" are device memory owned by the caller; the library never
@@ -39,8 +42,10 @@
  * Cache layout (all device memory, T = 16 tokens per page, D in {64, 128}):
  *  - block_table [B][max_pages] int32: entry = (tier << 29) | slot, tier in kvq_tier.
  *    A logical page's tier is shared by all kv heads.
- *  - pool[tier]: pool_slots[tier] physical slots; slot s holds, for kv head g and kind
- *    k (0 = K, 1 = V), one chunk of kvq_chunk_bytes(tier, D) bytes at byte offset
+ *  - pool[tier]: pool_slots[tier] physical slots (device memory, or pinned host memory
+ *    mapped into the device address space when bit tier of host_tiers is set); slot s
+ *    holds, for kv head g and kind k (0 = K, 1 = V), one chunk of
+ *    kvq_chunk_bytes(tier, D) bytes at byte offset
  *    ((s * Hkv + g) * 2 + k) * kvq_chunk_bytes(tier, D).  Base must be 16-byte aligned.
  *    Chunk = codes then meta.  Codes order: each element (t, d) belongs to lane
  *    lam, register pair R = 4*(d/16) + r and half h, with c = d % 16:
@@ -50,10 +55,12 @@
  *    b-bit tiers: lane word w = R/(16/b), slot j = R%(16/b); low code at bits b*j,
  *    high code at bits 16 + b*j; NW = D*b/64 words per lane, PW = min(4, NW); lane word
  *    w is uint32 ((w/PW)*32 + lam)*PW + w%PW of the codes area.  1-bit code 1 = +.
+ *    FP8 codes use the 8-bit layout (e4m3 bytes).
  *    Meta: b = 8/4/2: uint32 [T][D/32] = scale_fp16 | zero_fp16 << 16;
- *          1-bit:     uint16 [T][D/32] = magnitude fp16.  Empty slots are zero.
+ *          1-bit:     uint16 [T][D/32] = magnitude fp16;
+ *          fp8:       uint16 [T][D/32] = scale fp16.  Empty slots are zero.
  *    Value read back: 16-bit: as stored; b-bit: fp32(c * scale + zero) (one rounding);
- *    1-bit: +m or -m.
+ *    1-bit: +m or -m; fp8: e4m3(c) * scale (exact in fp32).
  *  - summary [B][Hkv][max_pages][D] fp16: fp16(mean of the page's keys as they arrived).
  *  - open_ksum [B][Hkv][D] double: running fp64 sum of the keys of the page that holds
  *    position seq_len-1 when that page is not full.
@@ -247,16 +254,6 @@ kvq_status kvq_sparse_decode_attn_noalloc(const kvq_cache* cache, const void* q,
 size_t kvq_noalloc_scratch_bytes(void);
 
 /*
- * kvq_score_select -- kvq_append (when pos is not NULL), kvq_page_scores and
- * kvq_select_topk in one launch, with the same results (AMASS "What is in the box":
- * score every page from its summary, keep the best).  The warp that scores the tile of a
- * sequence's appended token writes the token first; the CTA that finishes the last score
- * tile of a (b, kv head) selects its pages.  Arguments as those three calls; workspace:
- * any kvq workspace of at least 64 KiB prepared with kvq_workspace_init (per-(b, kv head)
- * tile counters at its head; the call leaves them zero).  B*Hkv <= 8192,
- * max_pages <= 51200.
- */
-/*
  * kvq_append_scores -- kvq_append followed by kvq_page_scores in one launch, with the same
  * results: the warp that scores the tile of a sequence's appended token writes the token
  * first.  Arguments as those two calls (pos, k_new, v_new required).
@@ -264,7 +261,16 @@ size_t kvq_noalloc_scratch_bytes(void);
 kvq_status kvq_append_scores(const kvq_cache* cache, const int32_t* pos, const void* k_new,
                              const void* v_new, const void* q, float* scores, kvq_stream_t stream);
 
-/* (coverage selection is not supported here: KVQ_ERR_UNSUPPORTED) */
+/*
+ * kvq_score_select -- kvq_append (when pos is not NULL), kvq_page_scores and
+ * kvq_select_topk in one launch, with the same results (AMASS "What is in the box":
+ * score every page from its summary, keep the best).  The warp that scores the tile of a
+ * sequence's appended token writes the token first; the CTA that finishes the last score
+ * tile of a (b, kv head) selects its pages.  Arguments as those three calls; workspace:
+ * any kvq workspace of at least 64 KiB prepared with kvq_workspace_init (per-(b, kv head)
+ * tile counters at its head; the call leaves them zero).  B*Hkv <= 8192,
+ * max_pages <= 51200.  Coverage selection is not supported here (KVQ_ERR_UNSUPPORTED).
+ */
 kvq_status kvq_score_select(const kvq_cache* cache, const int32_t* pos, const void* k_new,
                             const void* v_new, const void* q, const kvq_select_params* params,
                             float* scores, int32_t* sel, int32_t* cnt, int32_t kmax, void* workspace,
@@ -290,8 +296,8 @@ kvq_status kvq_step_workspace_size(const kvq_cache* cache, int32_t kmax, size_t*
  *            (entries past that are not written).
  *  workspace device scratch of at least kvq_step_workspace_size() bytes, prepared once
  *            with kvq_workspace_init.
- *  Returns KVQ_ERR_UNSUPPORTED for coverage selection, when B*Hkv > 8184, or when the
- *  per-CTA tables and selection keys
+ *  Returns KVQ_ERR_UNSUPPORTED for coverage selection, for pools in host memory
+ *  (host_tiers != 0), when B*Hkv > 8184, or when the per-CTA tables and selection keys
  *  (4 * (3B + max_pages) bytes) leave too little shared memory for the page ring.
  */
 kvq_status kvq_decode_step(const kvq_cache* cache, const int32_t* pos, const void* k_new,
@@ -359,7 +365,7 @@ kvq_status kvq_quad_append_scores(const kvq_cache* cache, const kvq_quad* quad, 
  *  slots past seq_len zero; then block_table[b][page] = new entry.  The page summary and
  *  open_ksum are unchanged (they follow the keys as they arrived), so later appends to an
  *  open page continue in the new tier.
- *  The new tier must be a quantised one (1..4) and the new (tier, slot) must differ from
+ *  The new tier must be a quantised one (1..5) and the new (tier, slot) must differ from
  *  the current one; an item that is out of range, names a page without tokens, has an
  *  invalid current or new entry, or aliases its own slot is skipped with
  *  KVQ_DERR_BAD_PAGE.  The caller owns slot allocation: new slots must not be referenced
@@ -372,7 +378,7 @@ kvq_status kvq_requantize_pages(const kvq_cache* cache, const int32_t* items, in
 /*
  * kvq_dequant_page -- values read back from storage for one logical page (testing aid).
  *  out device [Hkv][2][16][D] fp32: for each kv head, K then V, every token slot: the
- *  16-bit value, fp32(c * scale + zero), or +-m, per the page's tier.
+ *  16-bit value, fp32(c * scale + zero), +-m, or e4m3(c) * scale, per the page's tier.
  */
 kvq_status kvq_dequant_page(const kvq_cache* cache, int32_t b, int32_t page, float* out,
                             kvq_stream_t stream);
