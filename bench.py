@@ -2,7 +2,8 @@
 """Decode-step benchmark: sparse mixed-precision paged decode attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config c1] [--impl kvq|reference]
-                    [--path fused|calls]
+                    [--path calls|three|two|fused] [--score mean|quad] [--coverage C]
+                    [--tier T] [--host-tiers M] [--demote T]
 
 One step = one decode step of one attention layer for the whole batch, all of it in
 libkvq kernels: append the new token (quantise + pack + summary), score every page,
@@ -19,6 +20,12 @@ calls, replayed right after the timed loop.  The whole-step time is bracketed by
 (torchrun, one process per GPU, NCCL) every rank runs its own independent batch (weak
 scaling: sequences are independent problems, no collective on the data path) and the
 max time over ranks is used.  Rank 0 prints one JSON line.
+
+Options: ``--score quad`` scores pages with the quad (Gaussian-MGF) score; ``--coverage``
+selects by page-mass coverage; ``--tier T`` stores every prefilled page at tier T;
+``--host-tiers M`` keeps the pools of mask M in pinned host memory (the line gains a
+``host_link`` object); ``--demote T`` also times kvq_requantize_pages moving the
+workload's pages to tier T (a ``demotion`` object).
 
 ``--impl reference`` times the CPU oracle (the plain fp64 restatement of the method)
 on the host cores on a bounded sample of the same workload and prints the same line.

@@ -106,3 +106,27 @@ def test_quad_arguments_rejected_on_host():
     assert kvq._lib.kvq_quad_build(ref, qref, 4096, 4096, 16, None) == 1             # lambda not 16-byte aligned
     qd.lambda_, qd.basis = 4096, None
     assert kvq._lib.kvq_quad_append(ref, qref, 4096, 4096, None) == 1                # no basis
+
+
+def test_host_tiers_mask_checked_on_host():
+    """A host_tiers bit past the last tier is rejected before anything is enqueued."""
+    from sparse_mixed_precision_kvq_b200 import kvq
+    c = kvq.KvqCache()
+    c.B, c.Hq, c.Hkv, c.D, c.page_size, c.max_pages, c.dtype = 1, 8, 2, 64, 16, 4, 1
+    c.block_table = c.seq_len = c.summary = c.open_ksum = c.err_word = 4096
+    c.pool[0], c.pool_slots[0] = 4096, 4
+    c.host_tiers = 1 << 6
+    assert kvq._lib.kvq_page_scores(ctypes.byref(c), 4096, 4096, None) == 1
+    assert kvq._lib.kvq_append(ctypes.byref(c), 4096, 4096, 4096, None) == 1
+
+
+def test_single_tier_workload_override():
+    """bench --tier T: every prefilled page at tier T, the page opened by the append 16-bit."""
+    import numpy as np
+    import bench
+    for tier in range(6):
+        w = bench.rank_workload("c1", 0, batch=2, tier=tier)
+        for b in range(w.B):
+            t = w.tiers(b)
+            P0 = w.pages_before(b)
+            assert np.all(t[:P0] == tier) and np.all(t[P0:] == 0)
