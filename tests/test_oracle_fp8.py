@@ -94,3 +94,18 @@ def test_zero_group_and_token_meta():
     data = pack_chunk("k", TIER_F8, 128, 1, r["codes"][None], r["meta"][None])
     codes2, meta2 = unpack_chunk("k", TIER_F8, 128, data)
     assert np.array_equal(codes2[0], r["codes"]) and np.array_equal(meta2[0], r["meta"])
+
+
+def test_hand_derived_fixture():
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "fp8_examples.json")) as f:
+        fx = json.load(f)
+    for e in fx["rounding"]:
+        assert int(e4m3_rne(np.array(e["value"]))) == e["code"], e
+    g = fx["group"]
+    x = np.zeros(GROUP)
+    x[:len(g["x"])] = g["x"]
+    codes, scale, sbits, _ = quantise_fp8(x[None])
+    assert int(sbits[0]) == g["scale_bits"]
+    assert list(codes[0, :len(g["codes"])]) == g["codes"]
