@@ -130,3 +130,25 @@ def test_single_tier_workload_override():
             t = w.tiers(b)
             P0 = w.pages_before(b)
             assert np.all(t[:P0] == tier) and np.all(t[P0:] == 0)
+
+
+def test_algorithmic_bytes_by_hand():
+    """The roofline numerator: selected K+V chunks per tier + q + out + page lists for the
+    attention; every page summary + q + the fp32 scores for the page scores."""
+    import numpy as np
+    import bench
+    from sparse_mixed_precision_kvq_b200 import workloads as W
+    w = W.make("c0", lens=np.array([100]), tier_fracs={W.TIER_F16: 0.5, W.TIER_I4: 0.5})
+    tier_tbl, _, _ = w.slot_map()
+    sel = np.array([[[0, 3, 6], [1, 2, 0]]], dtype=np.int32)
+    cnt = np.array([[3, 2]], dtype=np.int32)
+    nb = bench.algorithmic_bytes(w, sel, cnt, tier_tbl)
+    chunk = {0: 2 * 16 * 64 * 2, 2: 2 * (16 * 64 // 2 + 16 * 2 * 4)}   # K+V at D = 64
+    pages = [int(tier_tbl[0, p]) for p in (0, 3, 6, 1, 2)]
+    qo = 2 * (1 * 8 * 64 * 2)
+    assert nb["attn"] == sum(chunk[t] for t in pages) + qo + 5 * 4
+    P = (100 + 15) // 16
+    assert nb["score"] == P * 2 * 64 * 2 + 8 * 64 * 2 + 2 * w.max_pages * 4
+    assert nb["append"] == 0 and nb["select"] == 2 * w.max_pages * 4 + 5 * 4
+    nq = bench.algorithmic_bytes(w, sel, cnt, tier_tbl, quad_rank=16)
+    assert nq["score"] - nb["score"] == P * 2 * 16 * 2
