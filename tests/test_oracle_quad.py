@@ -120,3 +120,16 @@ def test_projection_is_channel_ordered_dot():
             for d in range(8):
                 acc = acc + U[i, d] * keys[t, d]
             assert y[t, i] == acc
+
+
+def test_hand_derived_fixture():
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "quad_examples.json")) as f:
+        fx = json.load(f)
+    for e in fx["cases"]:
+        keys, basis = np.array(e["keys"]), np.array(e["basis"])
+        lam, _, _ = page_lambdas(keys, basis)
+        assert np.allclose(lam, e["lambda"], rtol=1e-6, atol=1e-7), e["why"]
+        got = quad_scores(np.array(e["q"]), keys.mean(0)[None], np.array(e["lambda"])[None], basis, e["s"], 1)[0]
+        assert np.isclose(got, e["score"], rtol=1e-12), e["why"]
