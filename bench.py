@@ -142,6 +142,23 @@ def algorithmic_bytes(w, sel: np.ndarray, cnt: np.ndarray, tier_tbl: np.ndarray,
     return dict(attn=attn, score=score, select=select, append=append)
 
 
+# algorithmic bytes of each launch of a path, by the names its timing parts carry
+PART_BYTES = {"append": ("append",), "page_scores": ("score",), "select_topk": ("select",),
+              "sparse_decode_attn": ("attn",), "append_scores": ("score", "append"),
+              "score_select": ("score", "select", "append"), "decode_step": ("attn", "score", "select", "append")}
+
+
+def kernel_rooflines(names, avg_ms, nbytes, peak: float):
+    """Per launch of the step: algorithmic bytes, GB/s over its event-timed duration, and
+    the fraction of the HBM peak."""
+    out = {}
+    for n, ms in zip(names, avg_ms):
+        b = sum(nbytes[k] for k in PART_BYTES[n])
+        gbs = b / (ms * 1e-3) / 1e9 if ms > 0 else 0.0
+        out[n] = {"bytes": int(b), "ms": float(ms), "gbs": gbs, "frac": gbs / peak}
+    return out
+
+
 def kernel_traffic(kernel_file: str):
     """ncu DRAM bytes per launch recorded for the current source of a kernel, else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -361,6 +378,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
                      "peak_gbs": peak, "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak,
                      "peak_kind": peak_kind},
         "kernels_ms": {n: float(a) for n, a in zip(names, avg)},
+        "kernels_roofline": kernel_rooflines(names, avg, nbytes, peak),
         "roofline": {"bound": "hbm", "kernel": names[dom], "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
                      "algorithmic_bytes_per_launch": dom_bytes,

@@ -152,3 +152,16 @@ def test_algorithmic_bytes_by_hand():
     assert nb["append"] == 0 and nb["select"] == 2 * w.max_pages * 4 + 5 * 4
     nq = bench.algorithmic_bytes(w, sel, cnt, tier_tbl, quad_rank=16)
     assert nq["score"] - nb["score"] == P * 2 * 16 * 2
+
+
+def test_kernel_rooflines_cover_every_path():
+    import bench
+    nbytes = dict(attn=1000, score=300, select=20, append=40)
+    paths = {"calls": ["append", "page_scores", "select_topk", "sparse_decode_attn"],
+             "three": ["append_scores", "select_topk", "sparse_decode_attn"],
+             "two": ["score_select", "sparse_decode_attn"], "fused": ["decode_step"]}
+    for names in paths.values():
+        r = bench.kernel_rooflines(names, [0.001] * len(names), nbytes, peak=1.0)
+        assert sum(v["bytes"] for v in r.values()) == 1360
+        for v in r.values():
+            assert abs(v["gbs"] - v["bytes"] / 1e-6 / 1e9) < 1e-9 and v["frac"] == v["gbs"]
