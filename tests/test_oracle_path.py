@@ -185,3 +185,21 @@ def test_step_pair_with_given_selection():
     r = step_pair(w, sh, 1, 3, q[1], kn[1, 3], vn[1, 3], sel=[0, 5, 62])
     assert list(r["used"]) == [0, 5, 62] and r["L"] == 1001
     assert r["out"].shape == (4, 128) and np.all(np.isfinite(r["out"]))
+
+
+def test_large_logits_and_empty_selection():
+    """Logits of magnitude ~1e3 stay finite and equal scipy's softmax / logsumexp; an empty
+    token set gives zeros and lse = -inf, and drops out of the combine."""
+    rng = np.random.default_rng(12)
+    q = rng.standard_normal(16) * 40
+    k = rng.standard_normal((50, 16)) * 40
+    v = rng.standard_normal((50, 16))
+    o, lse, _, _ = attend(q, k, v, 0.25)
+    logits = 0.25 * (k @ q)
+    assert np.abs(logits).max() > 500
+    assert np.allclose(o, softmax(logits) @ v, rtol=1e-12, atol=1e-13)
+    assert abs(lse - logsumexp(logits)) < 1e-9 * abs(lse)
+    oe, lse_e, me, le = attend(q, k[:0], v[:0], 0.25)
+    assert np.array_equal(oe, np.zeros(16)) and lse_e == -np.inf and le == 0.0
+    oc, lc = lse_combine([(oe, me, le), (o, *attend(q, k, v, 0.25)[2:])])
+    assert np.allclose(oc, o, rtol=1e-13) and abs(lc - lse) < 1e-9 * abs(lse)
