@@ -165,3 +165,22 @@ def test_kernel_rooflines_cover_every_path():
         assert sum(v["bytes"] for v in r.values()) == 1360
         for v in r.values():
             assert abs(v["gbs"] - v["bytes"] / 1e-6 / 1e9) < 1e-9 and v["frac"] == v["gbs"]
+
+
+def test_plain_c_caller(lib):
+    """The header compiles as C99 and a plain C program links libkvq and gets answers from
+    its host-only entry points (no GPU)."""
+    import shutil
+    import subprocess
+    import tempfile
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    libdir = os.path.join(ROOT, "sparse_mixed_precision_kvq_b200", "lib")
+    with tempfile.TemporaryDirectory() as tmp:
+        exe = os.path.join(tmp, "c_abi_check")
+        subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c_abi_check.c"), "-L", libdir, "-lkvq",
+                        "-Wl,-rpath," + libdir, "-o", exe], check=True, capture_output=True)
+        r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0 and "c abi ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
