@@ -1,0 +1,55 @@
+"""The attention kernel's exact code -> 16-bit operand conversions, replayed in numpy on
+every code (IEEE single roundings, subnormals kept, as the kernels are built):
+
+* integer tiers: the code placed in the mantissa of a 16-bit float with a magic exponent
+  (fp16 1024, bf16 128), minus (magic + 2^(b-1)), is the centred code c - 2^(b-1);
+* 8-bit codes for bf16 operands: 2^23 + c as fp32, minus 2^23 + 128, is c - 128 (exact in
+  bf16, whose 7-bit mantissa cannot hold 128 + c);
+* fp8: the e4m3 byte's exponent and mantissa placed in an fp32 pattern and multiplied by
+  2^120 give the e4m3 value, subnormals included."""
+import numpy as np
+
+from oracle.quant import e4m3_value
+
+
+def _f16(bits):
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def _bf16(bits):
+    return (np.asarray(bits, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def test_magic_exponent_centred_codes():
+    for b in (8, 4, 2):
+        c = np.arange(1 << b)
+        centre = 1 << (b - 1)
+        f16 = _f16(0x6400 | c) - _f16(0x6400 | centre)          # fp16 subtraction is exact here
+        assert np.array_equal(f16, c - centre)
+        if b < 8:
+            bf = _bf16(0x4300 | c) - _bf16(0x4300 | centre)
+            assert np.array_equal(bf, c - centre)
+    # why bf16 needs another route at 8 bits: 128 + c is not representable for odd c >= 128
+    assert _bf16(0x4300 | 0x81) != 128 + 0x81
+
+
+def test_fp32_route_for_8bit_codes_in_bf16():
+    c = np.arange(256, dtype=np.uint32)
+    v = (np.uint32(0x4B000000) | c).view(np.float32) - np.float32(8388736.0)
+    assert np.array_equal(v.astype(np.float64), c.astype(np.float64) - 128)
+    # every centred value is exact in bf16 (8 significant bits suffice for |c - 128| <= 128)
+    as_bf16 = (v.view(np.uint32) >> 16 << 16).view(np.float32)
+    assert np.array_equal(as_bf16, v)
+
+
+def test_e4m3_pattern_times_2_120():
+    b = np.arange(256, dtype=np.uint32)
+    pattern = (((b & 0x80) << 24) | ((b & 0x7F) << 20)).view(np.float32)
+    v = (pattern * np.float32(2.0 ** 120)).astype(np.float64)
+    ref = e4m3_value(b)
+    fin = np.isfinite(ref)
+    assert np.array_equal(v[fin], ref[fin])                       # subnormals: codes 1..7
+    assert np.all(np.isfinite(v))                                 # NaN codes come out finite (480)
+    # every e4m3 value is exact in bf16 and fp16 operands
+    assert np.array_equal(v[fin].astype(np.float16).astype(np.float64), v[fin])
+    assert np.array_equal(((v[fin].astype(np.float32).view(np.uint32) >> 16) << 16).view(np.float32), v[fin])
