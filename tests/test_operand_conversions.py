@@ -6,7 +6,9 @@ every code (IEEE single roundings, subnormals kept, as the kernels are built):
 * 8-bit codes for bf16 operands: 2^23 + c as fp32, minus 2^23 + 128, is c - 128 (exact in
   bf16, whose 7-bit mantissa cannot hold 128 + c);
 * fp8: the e4m3 byte's exponent and mantissa placed in an fp32 pattern and multiplied by
-  2^120 give the e4m3 value, subnormals included."""
+  2^120 give the e4m3 value, subnormals included;
+* the selection's score -> order key map is monotone, ranks -0 with +0 and NaN lowest,
+  and inverts."""
 import numpy as np
 
 from oracle.quant import e4m3_value
@@ -53,3 +55,31 @@ def test_e4m3_pattern_times_2_120():
     # every e4m3 value is exact in bf16 and fp16 operands
     assert np.array_equal(v[fin].astype(np.float16).astype(np.float64), v[fin])
     assert np.array_equal(((v[fin].astype(np.float32).view(np.uint32) >> 16) << 16).view(np.float32), v[fin])
+
+
+def _order_key(f: np.ndarray) -> np.ndarray:
+    """The selection's score -> key map (NaN -> 0, -0 -> +0, then the IEEE order trick)."""
+    f = np.where(f == 0, np.float32(0.0), f).astype(np.float32)
+    u = f.view(np.uint32)
+    k = np.where(u & 0x80000000, ~u, u | 0x80000000).astype(np.uint32)
+    return np.where(np.isnan(f), np.uint32(0), k)
+
+
+def test_selection_order_key_is_monotone_with_nan_lowest():
+    fi = np.finfo(np.float32)
+    vals = np.array([-np.inf, -fi.max, -1.0, -fi.tiny, -fi.smallest_subnormal, -0.0, 0.0,
+                     fi.smallest_subnormal, fi.tiny, 1.0, fi.max, np.inf], dtype=np.float32)
+    rng = np.random.default_rng(0)
+    more = np.sort(rng.standard_normal(5000).astype(np.float32) * 10.0 ** rng.uniform(-30, 30, 5000).astype(np.float32))
+    for seq in (vals, more):
+        k = _order_key(seq).astype(np.int64)
+        assert np.all(np.diff(k) >= 0)
+        strict = np.diff(seq.astype(np.float64)) > 0
+        assert np.all(np.diff(k)[strict] > 0)                    # strictly increasing where the scores are
+    assert _order_key(np.array([-0.0], np.float32))[0] == _order_key(np.array([0.0], np.float32))[0]
+    nan = _order_key(np.array([np.nan], np.float32))[0]
+    assert nan == 0 and np.all(_order_key(vals) > nan)            # NaN ranks below -inf
+    # the inverse map (key_score) returns the score for every non-NaN key
+    k = _order_key(vals)
+    back = np.where(k & 0x80000000, k & 0x7FFFFFFF, ~k).astype(np.uint32).view(np.float32)
+    assert np.array_equal(back, np.where(vals == 0, np.float32(0.0), vals))
