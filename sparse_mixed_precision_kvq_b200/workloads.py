@@ -27,6 +27,12 @@ Workload recipes (page size T = 16 everywhere):
 
 Planted pages hold keys ``2.4 * qhat + eps`` where ``qhat`` is the unit vector of the
 first query head of the kv head's group and ``eps`` follows the workload's key law.
+
+Overrides used by the tests and the benchmark: ``tier_fracs`` (any mix of the six tiers,
+fp8 included, assigned by seeded rank; ``{T: 1.0}`` puts every prefilled page at tier T),
+reduced batch / lengths (``small``), and ``quad_basis`` (the quad score's per-kv-head
+basis: unit vectors along the key law's largest-variance channels, or a seeded random
+orthonormal set).
 """
 from __future__ import annotations
 
