@@ -106,6 +106,11 @@ def test_quad_arguments_rejected_on_host():
     assert kvq._lib.kvq_quad_build(ref, qref, 4096, 4096, 16, None) == 1             # lambda not 16-byte aligned
     qd.lambda_, qd.basis = 4096, None
     assert kvq._lib.kvq_quad_append(ref, qref, 4096, 4096, None) == 1                # no basis
+    qd.basis, qd.rank = 4096, 12
+    assert kvq._lib.kvq_quad_append_scores(ref, qref, 4096, 4096, 4096, 4096, 0.1, 4096, None) == 2  # rank 12
+    qd.rank = 16
+    assert kvq._lib.kvq_quad_append_scores(ref, qref, None, 4096, 4096, 4096, 0.1, 4096, None) == 1  # no pos
+    assert kvq._lib.kvq_quad_append_scores(ref, qref, 4096, 4096, 4096, 4096, -1.0, 4096, None) == 1  # bad scale
 
 
 def test_host_tiers_mask_checked_on_host():
