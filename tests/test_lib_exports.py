@@ -189,3 +189,16 @@ def test_plain_c_caller(lib):
                         "-Wl,-rpath," + libdir, "-o", exe], check=True, capture_output=True)
         r = subprocess.run([exe], capture_output=True, text=True)
     assert r.returncode == 0 and "c abi ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
+
+
+def test_requantize_arguments_checked_on_host():
+    """n < 0 or missing items are rejected, n == 0 is a no-op, all before anything is enqueued."""
+    from sparse_mixed_precision_kvq_b200 import kvq
+    c = kvq.KvqCache()
+    c.B, c.Hq, c.Hkv, c.D, c.page_size, c.max_pages, c.dtype = 1, 8, 2, 64, 16, 4, 1
+    c.block_table = c.seq_len = c.summary = c.open_ksum = c.err_word = 4096
+    c.pool[0], c.pool_slots[0] = 4096, 4
+    ref = ctypes.byref(c)
+    assert kvq._lib.kvq_requantize_pages(ref, 4096, -1, None) == 1
+    assert kvq._lib.kvq_requantize_pages(ref, None, 3, None) == 1
+    assert kvq._lib.kvq_requantize_pages(ref, None, 0, None) == 0
