@@ -51,14 +51,26 @@ def select(scores: np.ndarray, P: int, k_abs: int, k_frac_bp: int, n_sink: int,
 
 def kth_margin(scores: np.ndarray, P: int, k_abs: int, k_frac_bp: int, n_sink: int,
                n_recent: int) -> float:
-    """Relative gap between the k-th and (k+1)-th best candidate scores (inf if none)."""
+    """Relative gap between the k-th and (k+1)-th best candidate scores, in the order the
+    selection ranks them (NaN below every number): ``(a - b) / max(|a|, |b|, 1e-30)``.
+
+    inf when no cut exists (k = 0 or every candidate chosen) or when the cut cannot move
+    under a rounding of the scores: ``b`` is NaN (a NaN never outranks a number and NaNs
+    are ordered by page index alone), or exactly one of ``a``, ``b`` is infinite.  Equal
+    scores (an exact tie, infinite ones included) give 0."""
     F = forced_pages(P, n_sink, n_recent)
-    c = np.array([scores[p] for p in range(P) if p not in F], dtype=np.float64)
-    k = min(budget(P, k_abs, k_frac_bp), c.size)
-    if k == 0 or k >= c.size:
+    c = [float(scores[p]) for p in range(P) if p not in F]
+    k = min(budget(P, k_abs, k_frac_bp), len(c))
+    if k == 0 or k >= len(c):
         return math.inf
-    s = np.sort(c)[::-1]
+    s = sorted(c, key=lambda v: (1, 0.0) if math.isnan(v) else (0, -v))
     a, b = s[k - 1], s[k]
+    if math.isnan(b):
+        return math.inf
+    if a == b:
+        return 0.0
+    if math.isinf(a) or math.isinf(b):
+        return math.inf
     return float((a - b) / max(abs(a), abs(b), 1e-30))
 
 
