@@ -242,9 +242,14 @@ kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const i
  *  scratch is a static device array of kvq_noalloc_scratch_bytes() (8 MiB) inside the
  *  library, held by every GPU that loads it until the process exits.  Allocates nothing
  *  (no cudaMalloc/cudaFree).  Returns KVQ_ERR_WORKSPACE when kvq_workspace_size() for
- *  this cache exceeds the static size.  The first call on a device looks up the array's
- *  device address (cudaGetSymbolAddress); make it before any stream capture.  All calls
- *  share the array: calls whose work overlaps on the GPU race.
+ *  this cache exceeds the static size, and KVQ_ERR_UNSUPPORTED for B*Hkv >= 6144 as
+ *  kvq_sparse_decode_attn does.  Each call made outside a stream capture looks up the
+ *  array's device address on the current device (cudaGetSymbolAddress; a re-created
+ *  context gets its new address); a call made while the stream captures reuses the last
+ *  lookup, so make the first call on each device before any stream capture.  Each call
+ *  clears the array's B*Hkv arrival counters with an asynchronous memset on `stream`
+ *  before the attention launch.  All calls share the array: calls whose work overlaps on
+ *  the GPU race.
  */
 kvq_status kvq_sparse_decode_attn_noalloc(const kvq_cache* cache, const void* q, const int32_t* sel,
                                           const int32_t* cnt, int32_t kmax, float sm_scale, void* out,

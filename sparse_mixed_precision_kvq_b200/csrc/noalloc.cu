@@ -10,13 +10,14 @@
 //
 // The array lives in every GPU that loads the library, for the life of the process.
 // Host code cannot pass the array's name to a kernel (on the host it is a stand-in, not
-// a device address), so the first call on each device looks its device address up with
-// cudaGetSymbolAddress while that device is current and caches it; make that first
-// call before any stream capture.  Every call shares the array, which keeps the last
-// call's contents: the split-K partials are fully rewritten before they are read, and the
-// per-segment arrival counters at its head must start at zero -- they are zero when the
-// library loads and every call leaves them zero.  Two calls whose work overlaps on the
-// GPU (different streams) race on the scratch.
+// a device address), so its device address is looked up with cudaGetSymbolAddress while
+// the device is current: on every call made outside a stream capture (so a context that
+// was reset and re-created gets the new address), and from the last such lookup during a
+// capture.  Make the first call on each device before any stream capture.  Every call
+// shares the array, which keeps the last call's contents: each call clears the
+// per-segment arrival counters at its head (an asynchronous memset on the caller's
+// stream; the split-K partials behind them are rewritten before they are read).  Two
+// calls whose work overlaps on the GPU (different streams) race on the scratch.
 #include <mutex>
 
 #include "kvq_internal.cuh"
@@ -32,11 +33,14 @@ constexpr int kMaxDevices = 64;
 void* g_scratch_addr[kMaxDevices] = {nullptr};
 std::mutex g_scratch_mu;
 
-// Device address of g_attn_scratch on the current device (looked up once per device).
-cudaError_t scratch_address(int device, void** out) {
+// Device address of g_attn_scratch on the current device: looked up again on every call
+// outside a stream capture, taken from the last lookup while `stream` is capturing.
+cudaError_t scratch_address(int device, cudaStream_t stream, void** out) {
   if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  const bool capturing = cudaStreamIsCapturing(stream, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[device] == nullptr) {
+  if (!capturing || g_scratch_addr[device] == nullptr) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_attn_scratch);
     if (e != cudaSuccess) return e;
@@ -61,11 +65,18 @@ kvq_status kvq_sparse_decode_attn_noalloc(const kvq_cache* cache, const void* q,
   size_t need = 0;
   kvq_status st = kvq_workspace_size(cache, kmax, &need);
   if (st != KVQ_OK) return st;
+  const long long segments = (long long)cache->B * cache->Hkv;
+  if (segments >= kMaxSegments) return KVQ_ERR_UNSUPPORTED;   // as kvq_sparse_decode_attn
   if (need > kNoAllocScratchBytes) return KVQ_ERR_WORKSPACE;  // batch too large for the static scratch
+  if (q == nullptr || sel == nullptr || cnt == nullptr || out == nullptr || !(sm_scale > 0.f))
+    return KVQ_ERR_INVALID_ARG;
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return KVQ_ERR_CUDA;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   void* scratch = nullptr;
-  if (scratch_address(device, &scratch) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (scratch_address(device, s, &scratch) != cudaSuccess) return KVQ_ERR_CUDA;
+  // the arrival counters start at zero whatever an earlier call left behind
+  if (cudaMemsetAsync(scratch, 0, (size_t)segments * sizeof(unsigned), s) != cudaSuccess) return KVQ_ERR_CUDA;
   return kvq_sparse_decode_attn(cache, q, sel, cnt, kmax, sm_scale, out, lse, scratch, kNoAllocScratchBytes,
                                 stream);
 }

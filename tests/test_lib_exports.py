@@ -71,7 +71,7 @@ def test_host_helpers_without_gpu():
     assert kvq.kvq_status_string(0) == "ok" and "workspace" in kvq.kvq_status_string(3)
 
 
-def test_invalid_arguments_rejected_on_host():
+def _check_invalid_arguments_rejected_on_host():
     """Argument checks run before any CUDA call, so they work without a device."""
     from sparse_mixed_precision_kvq_b200 import kvq
     c = kvq.KvqCache()
@@ -85,7 +85,7 @@ def test_invalid_arguments_rejected_on_host():
     assert kvq._lib.kvq_append(ctypes.byref(c), None, None, None, None) == 2
 
 
-def test_quad_arguments_rejected_on_host():
+def _check_quad_arguments_rejected_on_host():
     """Every case fails its host-side check before anything is enqueued (no device needed)."""
     from sparse_mixed_precision_kvq_b200 import kvq
     c = kvq.KvqCache()
@@ -113,7 +113,7 @@ def test_quad_arguments_rejected_on_host():
     assert kvq._lib.kvq_quad_append_scores(ref, qref, 4096, 4096, 4096, 4096, -1.0, 4096, None) == 1  # bad scale
 
 
-def test_host_tiers_mask_checked_on_host():
+def _check_host_tiers_mask_checked_on_host():
     """A host_tiers bit past the last tier is rejected before anything is enqueued."""
     from sparse_mixed_precision_kvq_b200 import kvq
     c = kvq.KvqCache()
@@ -191,7 +191,7 @@ def test_plain_c_caller(lib):
     assert r.returncode == 0 and "c abi ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
 
 
-def test_requantize_arguments_checked_on_host():
+def _check_requantize_arguments_checked_on_host():
     """n < 0 or missing items are rejected, n == 0 is a no-op, all before anything is enqueued."""
     from sparse_mixed_precision_kvq_b200 import kvq
     c = kvq.KvqCache()
@@ -202,3 +202,32 @@ def test_requantize_arguments_checked_on_host():
     assert kvq._lib.kvq_requantize_pages(ref, 4096, -1, None) == 1
     assert kvq._lib.kvq_requantize_pages(ref, None, 3, None) == 1
     assert kvq._lib.kvq_requantize_pages(ref, None, 0, None) == 0
+
+
+def _run_without_gpu(check: str):
+    """Run ``check`` (a function of this module) in a child process that sees no CUDA
+    device.  These checks hand made-up device addresses to the entry points and rely on
+    the host-side argument checks rejecting the call; if a check ever let one through,
+    the launch would fail with "no device" in the child instead of touching memory."""
+    import subprocess
+    import sys
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    code = f"import sys; sys.path.insert(0, {ROOT!r}); import tests.test_lib_exports as t; t.{check}()"
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
+def test_invalid_arguments_rejected_on_host():
+    _run_without_gpu('_check_invalid_arguments_rejected_on_host')
+
+
+def test_quad_arguments_rejected_on_host():
+    _run_without_gpu('_check_quad_arguments_rejected_on_host')
+
+
+def test_host_tiers_mask_checked_on_host():
+    _run_without_gpu('_check_host_tiers_mask_checked_on_host')
+
+
+def test_requantize_arguments_checked_on_host():
+    _run_without_gpu('_check_requantize_arguments_checked_on_host')

@@ -8,7 +8,9 @@ so that a run stopping at the first failure has run every other test first.
 The check: through the C ABI, on two calls in a row (two different workloads, so stale
 scratch from the first call cannot hide a bug in the second), the output and
 log-sum-exp equal those of kvq_sparse_decode_attn with a caller workspace, within the
-output tolerance the parity tests use.
+output tolerance the parity tests use.  Also: a batch beyond the static scratch is
+rejected, and a batch with too many (sequence, kv head) segments gets the same status
+from both entry points.
 """
 import numpy as np
 import pytest
@@ -59,3 +61,20 @@ def test_noalloc_rejects_a_batch_beyond_the_static_scratch():
     out = torch.empty_like(q)
     with pytest.raises(kvq.KvqError, match="workspace"):
         kvq.kvq_sparse_decode_attn_noalloc(cache, q, sel, cnt, 2, w.sm_scale, out, None)
+
+
+def test_noalloc_status_matches_the_workspace_entry_point():
+    """B*Hkv >= 6144 segments: both entry points answer "unsupported"."""
+    from sparse_mixed_precision_kvq_b200 import kvq
+    B, Hq, Hkv, D = 3100, 4, 2, 128
+    cache = kvq.PagedCache(B, Hq, Hkv, D, 1, "bf16", [B, 0, 0, 0, 0])
+    q = torch.zeros((B, Hq, D), dtype=torch.bfloat16, device="cuda")
+    sel = torch.zeros((B, Hkv, 1), dtype=torch.int32, device="cuda")
+    cnt = torch.zeros((B, Hkv), dtype=torch.int32, device="cuda")
+    out = torch.empty_like(q)
+    ws = torch.zeros(1 << 14, dtype=torch.float32, device="cuda")
+    with pytest.raises(kvq.KvqError, match="unsupported"):
+        kvq.kvq_sparse_decode_attn(cache, q, sel, cnt, 1, 0.1, out, None, ws)
+    with pytest.raises(kvq.KvqError, match="unsupported"):
+        kvq.kvq_sparse_decode_attn_noalloc(cache, q, sel, cnt, 1, 0.1, out, None)
+
