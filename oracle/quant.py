@@ -65,18 +65,26 @@ def e4m3_rne(v: np.ndarray) -> np.ndarray:
     return np.where(np.isnan(v), 0x7F, code).astype(np.int64)
 
 
+F8_NAN_SCALE_BITS = 0x7E00   # fp16 quiet NaN: the scale of a group holding a non-finite value
+
+
 def quantise_fp8(x: np.ndarray):
     """FP8 tier of groups ``x[..., 32]``: ``scale = fp16(amax / 448)`` (amax the largest
     magnitude, a zero amax is +0), ``code = e4m3(x / scale)`` (fp64 quotient, then one
     round-half-even to e4m3 with saturation; all codes 0 when scale == 0); read back as
-    ``e4m3(code) * scale`` (exact in fp32).  Returns ``(codes, scale, scale_bits, overflow)``."""
+    ``e4m3(code) * scale`` (exact in fp32).  A group holding a non-finite value (flagged as
+    such by the library) stores a NaN scale and zero codes, so every element reads back as
+    NaN.  Returns ``(codes, scale, scale_bits, overflow)``."""
     x = np.asarray(x, dtype=np.float64)
     assert x.shape[-1] == GROUP
-    amax = np.abs(x).max(axis=-1) + 0.0
+    bad = ~np.isfinite(x).all(axis=-1)
+    amax = np.where(bad, 0.0, np.abs(np.where(np.isfinite(x), x, 0.0)).max(axis=-1)) + 0.0
     scale, scale_bits, ov = fp16_rne_sat(amax / E4M3_MAX)
-    safe = np.where(scale == 0.0, 1.0, scale)
-    codes = e4m3_rne(x / safe[..., None])
-    codes = np.where((scale == 0.0)[..., None], 0, codes)
+    scale = np.where(bad, np.nan, scale)
+    scale_bits = np.where(bad, F8_NAN_SCALE_BITS, scale_bits).astype(scale_bits.dtype)
+    safe = np.where((scale == 0.0) | bad, 1.0, scale)
+    codes = e4m3_rne(np.where(bad[..., None], 0.0, x) / safe[..., None])
+    codes = np.where(((scale == 0.0) | bad)[..., None], 0, codes)
     return codes, scale, scale_bits, ov
 
 

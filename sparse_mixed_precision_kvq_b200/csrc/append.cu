@@ -233,10 +233,15 @@ __device__ inline void rq_quant(int gid, int n, const float (*vals)[kRqGroups + 
   uint32_t packed[kGroup / 4];
   if constexpr (NT == KVQ_TIER_F8) {  // scale fp16(amax / 448), code e4m3(x / scale) from the fp64 quotient
     float amax = 0.0f;
+    bool bad = false;
 #pragma unroll
-    for (int j = 0; j < kGroup; ++j) amax = fmaxf(amax, fabsf(v[j]));
-    const uint16_t sb = fp16_sat(static_cast<double>(amax) / 448.0, ov);
-    const double sc = static_cast<double>(__half2float(__ushort_as_half(sb)));
+    for (int j = 0; j < kGroup; ++j) {
+      amax = fmaxf(amax, fabsf(v[j]));
+      bad |= !isfinite(v[j]);
+    }
+    // a group holding a non-finite value: NaN scale and zero codes (it reads back as NaN)
+    const uint16_t sb = bad ? kF8NaNScale : fp16_sat(static_cast<double>(amax) / 448.0, ov);
+    const double sc = bad ? 0.0 : static_cast<double>(__half2float(__ushort_as_half(sb)));
 #pragma unroll
     for (int k = 0; k < kGroup / 4; ++k) {
       packed[k] = 0;

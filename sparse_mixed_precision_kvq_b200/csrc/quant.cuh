@@ -22,6 +22,9 @@ struct QOut {
   uint32_t meta;  // INT-b: scale | zero << 16 ; 1-bit: magnitude
 };
 
+// FP8 scale bits stored for a group that holds a non-finite value (an fp16 quiet NaN).
+constexpr uint16_t kF8NaNScale = 0x7E00u;
+
 // Warp-collective: lane j holds channel j of the group.
 __device__ inline QOut quant_group(double x, int tier, bool& ov) {
   const unsigned full = 0xffffffffu;
@@ -40,6 +43,8 @@ __device__ inline QOut quant_group(double x, int tier, bool& ov) {
     for (int o = 16; o; o >>= 1) a = fmax(a, __shfl_xor_sync(full, a, o));
     a += 0.0;
     const uint16_t sb = fp16_sat(a / 448.0, ov);
+    // a group holding a non-finite value: NaN scale and zero codes, so it reads back as NaN
+    if (__any_sync(full, !isfinite(x))) return {0u, kF8NaNScale};
     const double scale = static_cast<double>(__half2float(__ushort_as_half(sb)));
     const uint32_t code = scale != 0.0 ? __nv_cvt_double_to_fp8(x / scale, __NV_SATFINITE, __NV_E4M3) : 0u;
     return {code, sb};

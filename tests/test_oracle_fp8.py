@@ -109,3 +109,22 @@ def test_hand_derived_fixture():
     codes, scale, sbits, _ = quantise_fp8(x[None])
     assert int(sbits[0]) == g["scale_bits"]
     assert list(codes[0, :len(g["codes"])]) == g["codes"]
+
+
+def test_nonfinite_group_reads_back_nan():
+    """A group holding an infinite or NaN value (the library flags such input) stores the
+    fp16 quiet NaN 0x7E00 as its scale and zero codes: every element reads back as NaN,
+    whichever 16-bit type later consumes it.  Finite groups beside it are unchanged."""
+    rng = np.random.default_rng(9)
+    x = rng.normal(size=(4, GROUP)).astype(np.float16).astype(np.float64)
+    ref_codes, ref_scale, ref_bits, _ = quantise_fp8(x)
+    x[1, 5] = np.nan
+    x[2, 0] = np.inf
+    x[3, 31] = -np.inf
+    codes, scale, sbits, _ = quantise_fp8(x)
+    for i in (1, 2, 3):
+        assert int(sbits[i]) == 0x7E00 and np.isnan(scale[i]) and np.all(codes[i] == 0)
+        assert np.all(np.isnan(dequant_fp8(codes, scale)[i]))
+    assert int(sbits[0]) == int(ref_bits[0]) and np.array_equal(codes[0], ref_codes[0])
+    r = quantise_token(x.reshape(-1), TIER_F8)
+    assert list(r["meta"]) == [int(ref_bits[0]), 0x7E00, 0x7E00, 0x7E00]
