@@ -163,7 +163,7 @@ __device__ inline void quad_qterms(const DevQuad& qd, const QFrag<D, BF16>& qf, 
       x0[kk] = ok0 ? s0[kk] : make_float4(0.f, 0.f, 0.f, 0.f);
       x1[kk] = ok1 ? s1[kk] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    float cacc[4] = {0.f, 0.f, 0.f, 0.f};
+    float cacc[4] = {0.f, 0.f, 0.f, 0.f}, clo[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
       uint32_t ah[4], al[4];
@@ -173,8 +173,10 @@ __device__ inline void quad_qterms(const DevQuad& qd, const QFrag<D, BF16>& qf, 
       split_f32x2(x1[kk].z, x1[kk].w, ah[3], al[3]);
       mma16816<false>(cacc, ah, qf.bh[kk][0], qf.bh[kk][1]);
       mma16816<false>(cacc, al, qf.bh[kk][0], qf.bh[kk][1]);
-      if constexpr (BF16) mma16816<false>(cacc, ah, qf.bl[kk][0], qf.bl[kk][1]);
+      if constexpr (BF16) mma16816<false>(clo, ah, qf.bl[kk][0], qf.bl[kk][1]);  // query low part, x 2^24
     }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) cacc[j] += clo[j] * kQLoUnscale;
     // cacc: (row i0, head 2 q4), (i0, 2 q4 + 1), (i1, 2 q4), (i1, 2 q4 + 1)
     if (ok0) {
       zs[2 * q4][i0] = cacc[0] * cacc[0];
@@ -329,7 +331,7 @@ cudaError_t launch_quad_scores_r(const DevCache& c, const DevQuad& qd, const voi
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
   const int tiles_per_bg = (c.max_pages + 15) / 16;
   const long long total = (long long)c.B * c.Hkv * tiles_per_bg;
-  const long long warps = (long long)attn_num_ctas(dev) * kQuadWarps;  // one CTA per SM (registers)
+  const long long warps = (long long)sm_count(dev) * kQuadWarps;  // one CTA per SM (registers)
   const int per = (int)((total + warps - 1) / warps);
   const long long blocks = (total + (long long)per * kQuadWarps - 1) / ((long long)per * kQuadWarps);
   return launch_pdl(quad_score_kernel<D, BF16, RK>, dim3((unsigned)blocks), dim3(kQuadWarps * 32), 0, s, c, qd,

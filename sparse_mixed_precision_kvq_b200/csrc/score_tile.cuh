@@ -6,9 +6,14 @@
 //
 // One warp scores a tile of 16 page summaries on the tensor core (mma m16n8k16, fp16
 // inputs, fp32 accumulation): A = 16 summaries x 16 channels (fp16, as stored), B = the
-// kv head's query rows (heads as N <= 8).  The query is split into fp16 hi + lo parts (two
-// mmas), so every product is exact, as in an fp32 CUDA-core dot product; a 16-bit query
-// element beyond the fp16 range is flagged (KVQ_DERR_FP16_RANGE).  The channel order
+// kv head's query rows (heads as N <= 8).  A bf16 query is split into an fp16 high part
+// and an fp16 low part scaled by 2^24 (two mmas, the second accumulated apart and scaled
+// back by 2^-24, a power of two): fp16 holds a bf16 value exactly from 2^-17 up to its
+// range, and the scaled residual of a smaller one exactly down to 2^-41, so every product
+// is exact for |q| >= 2^-41 (below that an element loses at most 2^-49 of its product's
+// summary factor), as in an fp32 CUDA-core dot product.  An fp16 query is its own high
+// part.  A 16-bit query element beyond the fp16 range is flagged (KVQ_DERR_FP16_RANGE).
+// The channel order
 // inside each k-step is permuted -- the same way for A and B, which leaves the dot
 // product unchanged -- so that each lane reads its D/4 channels of a summary row as
 // contiguous 16-byte loads from a row-major [page][D] layout (global or shared memory).
@@ -24,14 +29,20 @@ namespace kvq {
 // NaN-propagating max (a NaN score ranks lowest later; here it must survive the max)
 __device__ inline float nanmax(float a, float b) { return (a != a || b != b) ? __int_as_float(0x7FC00000) : fmaxf(a, b); }
 
-// fp16 pair (hi) and residual pair (lo) of two 16-bit query values; *bad if out of range.
+// The low part of a split query is stored times kQLoScale; its products are summed
+// apart and multiplied by kQLoUnscale (both exact powers of two).
+constexpr float kQLoScale = 0x1p24f;
+constexpr float kQLoUnscale = 0x1p-24f;
+
+// fp16 pair (hi) and scaled residual pair (lo = fp16((x - hi) * 2^24)) of two 16-bit query
+// values; *bad if out of range.  x - hi is exact in fp32 (hi is x rounded, or 0).
 template <bool BF16>
 __device__ inline void split_q(uint32_t bits2, uint32_t& hi, uint32_t& lo, bool& bad) {
   const float x0 = bits_to_float<BF16>(static_cast<uint16_t>(bits2 & 0xFFFFu));
   const float x1 = bits_to_float<BF16>(static_cast<uint16_t>(bits2 >> 16));
   const __half2 h = __floats2half2_rn(x0, x1);
   const float2 hf = __half22float2(h);
-  const __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+  const __half2 l = __floats2half2_rn((x0 - hf.x) * kQLoScale, (x1 - hf.y) * kQLoScale);
   bad |= !(fabsf(x0) <= 65504.f) || !(fabsf(x1) <= 65504.f);
   hi = *reinterpret_cast<const uint32_t*>(&h);
   lo = *reinterpret_cast<const uint32_t*>(&l);
@@ -96,7 +107,7 @@ __device__ inline void tile_head_dots(const uint4 (&av)[2][D / 32], const QFrag<
     if constexpr (BF16) mma16816<false>(cl, a, qf.bl[kk][0], qf.bl[kk][1]);
   }
 #pragma unroll
-  for (int j = 0; j < 4; ++j) v[j] = ch[j] + cl[j];
+  for (int j = 0; j < 4; ++j) v[j] = ch[j] + cl[j] * kQLoUnscale;
 }
 
 // Max over the lane's valid heads of values laid out as tile_head_dots's, then over the

@@ -8,7 +8,9 @@ every code (IEEE single roundings, subnormals kept, as the kernels are built):
 * fp8: the e4m3 byte's exponent and mantissa placed in an fp32 pattern and multiplied by
   2^120 give the e4m3 value, subnormals included;
 * the selection's score -> order key map is monotone, ranks -0 with +0 and NaN lowest,
-  and inverts."""
+  and inverts;
+* the score kernels' split of a bf16 query into fp16 high and 2^24-scaled low parts is
+  exact for every element of magnitude >= 2^-41."""
 import numpy as np
 
 from oracle.quant import e4m3_value
@@ -83,3 +85,27 @@ def test_selection_order_key_is_monotone_with_nan_lowest():
     k = _order_key(vals)
     back = np.where(k & 0x80000000, k & 0x7FFFFFFF, ~k).astype(np.uint32).view(np.float32)
     assert np.array_equal(back, np.where(vals == 0, np.float32(0.0), vals))
+
+
+def test_bf16_query_split_is_exact_down_to_2_pow_minus_41():
+    """The score kernels split a bf16 query element x into hi = fp16(x) and
+    lo = fp16((x - hi) * 2^24), the low part's products scaled back by 2^-24.  Replayed on
+    every finite bf16 pattern in fp32 / fp16 (numpy rounds half to even, as cvt.rn):
+    hi + lo * 2^-24 == x for every |x| >= 2^-41 inside fp16's range, and misses a smaller x
+    by at most 2^-49."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    x = (bits << 16).view(np.float32)
+    fin = np.isfinite(x) & (np.abs(x) <= np.float32(65504.0))
+    x = x[fin]
+    with np.errstate(over="ignore"):
+        hi = x.astype(np.float16).astype(np.float32)
+        r = x - hi                                        # exact: hi is x rounded (or 0)
+        lo = (r * np.float32(2.0 ** 24)).astype(np.float16).astype(np.float64)
+    back = hi.astype(np.float64) + lo * 2.0 ** -24
+    xd = x.astype(np.float64)
+    big = np.abs(xd) >= 2.0 ** -41
+    assert np.array_equal(back[big], xd[big])
+    assert np.all(np.abs(back[~big] - xd[~big]) <= 2.0 ** -49)
+    # without the 2^24 scale the residual of a small element is lost
+    plain = hi.astype(np.float64) + (x - hi).astype(np.float16).astype(np.float64)
+    assert not np.array_equal(plain[big], xd[big])
