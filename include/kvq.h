@@ -210,8 +210,24 @@ kvq_status kvq_workspace_size(const kvq_cache* cache, int32_t kmax, size_t* byte
  * kvq_sparse_decode_attn and kvq_decode_step call leaves the counters zero again, so
  * this is needed once per workspace, not per call (and again after a call that flagged
  * KVQ_DERR_TIMEOUT).  One workspace may serve both calls.
+ * Word KVQ_WS_WAIT_LIMIT_WORD (uint32) of that head is never a counter: it is the limit,
+ * in microseconds, of every bounded wait of a kvq_sparse_decode_attn or kvq_decode_step
+ * call on this workspace (a wait on a copy in flight, or on another CTA's result).  0 (as
+ * kvq_workspace_init leaves it) means 2 s.  A wait that runs out sets KVQ_DERR_TIMEOUT,
+ * skips the rest of the work and returns; the workspace is then re-initialised.
  */
+#define KVQ_WS_WAIT_LIMIT_WORD 16383
 kvq_status kvq_workspace_init(void* workspace, size_t ws_bytes, kvq_stream_t stream);
+
+/*
+ * kvq_set_grid_override -- testing and tuning aid (the source pages have no counterpart):
+ * run the attention kernel and kvq_decode_step on `ctas` CTAs instead of one per SM, for
+ * every later call in the process (0 restores the default).  Fewer CTAs give each warp
+ * more pages, so small batches reach the deep-pipeline paths full-size batches take.
+ * kvq_workspace_size depends on it: size workspaces after setting it.  Not thread-safe
+ * with respect to calls running in other threads.  ctas in [0, 65535].
+ */
+kvq_status kvq_set_grid_override(int32_t ctas);
 
 /*
  * kvq_sparse_decode_attn -- attention of each query head over the tokens of its kv
@@ -273,7 +289,7 @@ kvq_status kvq_append_scores(const kvq_cache* cache, const int32_t* pos, const v
  * sequence's appended token writes the token first; the CTA that finishes the last score
  * tile of a (b, kv head) selects its pages.  Arguments as those three calls; workspace:
  * any kvq workspace of at least 64 KiB prepared with kvq_workspace_init (per-(b, kv head)
- * tile counters at its head; the call leaves them zero).  B*Hkv <= 8192,
+ * tile counters at its head; the call leaves them zero).  B*Hkv <= 8191,
  * max_pages <= 51200.  Coverage selection is not supported here (KVQ_ERR_UNSUPPORTED).
  */
 kvq_status kvq_score_select(const kvq_cache* cache, const int32_t* pos, const void* k_new,
@@ -302,7 +318,7 @@ kvq_status kvq_step_workspace_size(const kvq_cache* cache, int32_t kmax, size_t*
  *  workspace device scratch of at least kvq_step_workspace_size() bytes, prepared once
  *            with kvq_workspace_init.
  *  Returns KVQ_ERR_UNSUPPORTED for coverage selection, for pools in host memory
- *  (host_tiers != 0), when B*Hkv > 8184, or when the per-CTA tables and selection keys
+ *  (host_tiers != 0), when B*Hkv > 8183, or when the per-CTA tables and selection keys
  *  (4 * (3B + max_pages) bytes) leave too little shared memory for the page ring.
  */
 kvq_status kvq_decode_step(const kvq_cache* cache, const int32_t* pos, const void* k_new,

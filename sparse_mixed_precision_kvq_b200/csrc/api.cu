@@ -196,7 +196,7 @@ kvq_status kvq_score_select(const kvq_cache* cache, const int32_t* pos, const vo
   if (pos != nullptr && (k_new == nullptr || v_new == nullptr)) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
   if (params->coverage_ppm > 0) return KVQ_ERR_UNSUPPORTED;
-  if ((long long)c.B * c.Hkv > (long long)(kCounterBytes / 4 - kScoreSelectCounterWord)) return KVQ_ERR_UNSUPPORTED;
+  if ((long long)c.B * c.Hkv > (long long)(kWaitLimitWord - kScoreSelectCounterWord)) return KVQ_ERR_UNSUPPORTED;
   if ((size_t)c.max_pages * 4 > 200 * 1024) return KVQ_ERR_UNSUPPORTED;  // keys in shared memory
   if (ws_bytes < kCounterBytes) return KVQ_ERR_WORKSPACE;
   unsigned* done = static_cast<unsigned*>(workspace) + kScoreSelectCounterWord;
@@ -231,6 +231,12 @@ kvq_status kvq_decode_step(const kvq_cache* cache, const int32_t* pos, const voi
   if (ws_bytes < step_workspace_bytes(c, kmax)) return KVQ_ERR_WORKSPACE;
   return cuda_status(launch_step(c, pos, k_new, v_new, q, *params, scores, sel, cnt, kmax, sm_scale, out, lse,
                                  workspace, attn_num_ctas(current_device()), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_set_grid_override(int32_t ctas) {
+  if (ctas < 0 || ctas > 65535) return KVQ_ERR_INVALID_ARG;
+  set_grid_override(ctas);
+  return KVQ_OK;
 }
 
 kvq_status kvq_workspace_init(void* workspace, size_t ws_bytes, kvq_stream_t stream) {

@@ -39,6 +39,8 @@
 // overlaps the previous kernel's tail.
 #include <math.h>
 
+#include <atomic>
+
 #include "kvq_internal.cuh"
 #include "page_math.cuh"
 #include "ptx.cuh"
@@ -225,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
   __syncwarp();
 
   griddep_wait();  // the page lists and the cache come from earlier kernels
+  const unsigned long long wait_ns = wait_limit_ns(a.counters, kWaitLimitWord);
 
   // segment offsets: exclusive prefix sum of the (clamped) selected counts
   {
@@ -374,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
       begin_segment<D, BF16>(a.q, c.Hq, G, bg / c.Hkv, bg % c.Hkv, lane, st);
     }
     if (!failed) {
-      const bool ok = mbar_wait_bounded(smem_u32(&bars[slot]), parity);
+      const bool ok = mbar_wait_bounded(smem_u32(&bars[slot]), parity, wait_ns);
       if (__any_sync(0xffffffffu, !ok)) {
         failed = true;
         if (lane == 0) set_err(c.err, KVQ_DERR_TIMEOUT);
@@ -405,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
   if (lane == 0) s_pseg[warp] = failed ? -1 : cur;
   // after a timeout, give copies still in flight a bounded chance to land before exit
   if (failed) {
-    for (int k = consumed; k < issued; ++k) mbar_wait_bounded(smem_u32(&bars[k % kNBar]), (k / kNBar) & 1);
+    for (int k = consumed; k < issued; ++k) mbar_wait_bounded(smem_u32(&bars[k % kNBar]), (k / kNBar) & 1, wait_ns);
   }
   if (groups > 0) cp_async_wait_pending(0);  // no per-lane copy may land after this point
 
@@ -476,13 +479,24 @@ cudaError_t launch_attn_d(const AttnArgs& a, uint16_t* out, float* lse, cudaStre
 
 }  // namespace
 
-int attn_num_ctas(int device) {
+int sm_count(int device) {
   static int cache[64] = {0};
   if (device >= 0 && device < 64 && cache[device] > 0) return cache[device];
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0) sms = 148;
   if (device >= 0 && device < 64) cache[device] = sms;
   return sms;
+}
+
+namespace {
+std::atomic<int> g_grid_override{0};
+}
+
+void set_grid_override(int ctas) { g_grid_override.store(ctas > 0 ? ctas : 0); }
+
+int attn_num_ctas(int device) {
+  const int o = g_grid_override.load();
+  return o > 0 ? o : sm_count(device);
 }
 
 // Workspace: [kCounterBytes] per-segment arrival counters (zero between calls, at a fixed

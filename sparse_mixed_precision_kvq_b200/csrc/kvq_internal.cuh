@@ -20,6 +20,9 @@ constexpr int kMaxSegments = 6144;  // B * Hkv limit of the attention kernel (of
 // Head of every workspace: counters that must be zero when a call starts (every call
 // leaves them zero); kvq_workspace_init zeroes it once.
 constexpr size_t kCounterBytes = 65536;
+// Last word of that head: the limit of every bounded wait of a call on this workspace, in
+// microseconds (0: the default, kWaitNs).  No counter ever uses it.
+constexpr int kWaitLimitWord = static_cast<int>(kCounterBytes / 4) - 1;
 
 __host__ __device__ constexpr int tier_bits(int tier) {
   return tier == 0 ? 16 : tier == 1 ? 8 : tier == 2 ? 4 : tier == 3 ? 2 : tier == 4 ? 1 : 8;
@@ -259,7 +262,9 @@ cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_sele
                           int32_t* sel, int32_t* cnt, int kmax, cudaStream_t s);
 int coverage_sort_size(const DevCache& c, const kvq_select_params& prm);
 size_t attn_workspace_bytes(const DevCache& c, int num_ctas);
-int attn_num_ctas(int device);
+int sm_count(int device);      // streaming multiprocessors of the device (cached)
+int attn_num_ctas(int device);  // grid of the attention kernel and the fused step: sm_count, or the override
+void set_grid_override(int ctas);
 cudaError_t launch_attn(const DevCache& c, const void* q, const int32_t* sel, const int32_t* cnt, int kmax,
                         float sm_scale, void* out, float* lse, void* ws, int num_ctas, cudaStream_t s);
 bool step_supported(const DevCache& c);

@@ -8,7 +8,7 @@
 
 namespace kvq {
 
-constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded pipeline wait (2 s)
+constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded pipeline wait (2 s) unless a workspace sets one
 
 __device__ inline uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -58,14 +58,19 @@ __device__ inline bool bar_sync_or(int id, int nthreads, bool pred) {
       : "memory");
   return r != 0;
 }
-// Wait with a time limit; false if it ran out.
-__device__ inline bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+// Wait with a time limit (nanoseconds); false if it ran out.
+__device__ inline bool mbar_wait_bounded(uint32_t bar, uint32_t parity, unsigned long long limit_ns = kWaitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kWaitNs) return false;
+    if (globaltimer() - t0 > limit_ns) return false;
   }
   return true;
+}
+// The wait limit a workspace asks for: its head word `word` in microseconds, 0 = kWaitNs.
+__device__ inline unsigned long long wait_limit_ns(const unsigned* head, int word) {
+  const unsigned us = __ldcg(head + word);
+  return us ? 1000ull * us : kWaitNs;
 }
 // Bulk global -> shared copy (TMA engine), completion counted on mbarrier `bar`.
 // Addresses 16-byte aligned, bytes a multiple of 16.

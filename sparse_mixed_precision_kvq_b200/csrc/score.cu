@@ -197,7 +197,7 @@ cudaError_t launch_d(const DevCache& c, const void* q, float* scores, const Scor
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
   const int tiles_per_bg = (c.max_pages + 15) / 16;
   const long long total = (long long)c.B * c.Hkv * tiles_per_bg;
-  const long long blocks_max = 2LL * attn_num_ctas(dev);
+  const long long blocks_max = 2LL * sm_count(dev);
   const long long warps = blocks_max * kScoreWarps;
   const int per = (int)((total + warps - 1) / warps);
   const long long blocks = (total + (long long)per * kScoreWarps - 1) / ((long long)per * kScoreWarps);

@@ -86,7 +86,7 @@ cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_sele
                           int32_t* sel, int32_t* cnt, int kmax, cudaStream_t s) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-  const bool wide = (long long)c.B * c.Hkv * 4 <= attn_num_ctas(dev) && c.max_pages >= 4096;
+  const bool wide = (long long)c.B * c.Hkv * 4 <= sm_count(dev) && c.max_pages >= 4096;
   const int ncov = prm.coverage_ppm > 0 ? coverage_sort_size(c, prm) : 0;
   return wide ? launch_select_t<1024>(c, scores, prm, sel, cnt, kmax, ncov, s)
               : launch_select_t<512>(c, scores, prm, sel, cnt, kmax, ncov, s);

@@ -36,7 +36,7 @@
 //
 // No wait can deadlock: every score item is taken before any attention item, score items
 // never wait, so the units an attention item waits for are always being finished by CTAs
-// that are running.  Every wait is bounded (2 s); on a timeout the CTA flags
+// that are running.  Every wait is bounded (2 s, or the limit the workspace sets); on a timeout the CTA flags
 // KVQ_DERR_TIMEOUT, stops issuing copies, waits (bounded) for the copies in flight and
 // leaves.  Counters are returned to zero by the CTA that last uses them.
 #include <math.h>
@@ -144,12 +144,12 @@ __device__ inline int find_b(const int* tab, int B, int i) {
 // Bounded mbarrier wait (a spin on test_wait: no suspension, so no late wake-up) that
 // gives up at once when the CTA has given up (*abort), and makes the CTA give up when the
 // time runs out.
-__device__ inline bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ inline bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort, unsigned long long limit_ns) {
   if (mbar_test_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (!mbar_test_wait(bar, parity)) {
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
       return false;
     }
@@ -235,6 +235,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
     mbar_init_fence();
   }
   griddep_wait();  // the cache and the inputs come from earlier work on the stream
+  const unsigned long long wait_ns = wait_limit_ns(a.ctl, kWaitLimitWord);
 
   // item tables: exclusive prefix sums over b of the items of b's Hkv units
   constexpr int as = kASlots, bs = kBPages;
@@ -316,7 +317,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
       if (lane < n) {
         const int kk = k + lane;
         const int e = kk & (kNDesc - 1);
-        ok = wait_or_abort(smem_u32(&dempty[e]), ((kk / kNDesc) & 1) ^ 1, &s_abort);
+        ok = wait_or_abort(smem_u32(&dempty[e]), ((kk / kNDesc) & 1) ^ 1, &s_abort, wait_ns);
         if (ok) {
           desc[e] = d;
           mbar_arrive(smem_u32(&dfull[e]));
@@ -390,7 +391,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
                 ok = 1;
                 break;
               }
-              if (*reinterpret_cast<volatile int*>(&s_abort) || globaltimer() - t0 > kWaitNs) {
+              if (*reinterpret_cast<volatile int*>(&s_abort) || globaltimer() - t0 > wait_ns) {
                 ok = -1;
                 break;
               }
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
         const uint32_t par = (k / kNDesc) & 1;
         bool have;
         if (need && mi == m) {
-          have = wait_or_abort(smem_u32(&dfull[e]), par, &s_abort);
+          have = wait_or_abort(smem_u32(&dfull[e]), par, &s_abort, wait_ns);
           if (!have) return false;
         } else {
           have = mbar_test_wait(smem_u32(&dfull[e]), par);
@@ -507,7 +508,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
       if (!top_up(true)) return false;
       const int k = warp + m * kCW;
       slot = k % ns;
-      if (!wait_or_abort(smem_u32(&full[slot]), (k / ns) & 1, &s_abort)) return false;
+      if (!wait_or_abort(smem_u32(&full[slot]), (k / ns) & 1, &s_abort, wait_ns)) return false;
       d = desc[k & (kNDesc - 1)];
       return true;
     };
@@ -711,7 +712,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
       // let this warp's copies still in flight land before the CTA leaves (bounded)
       for (int j = m; j < mi; ++j) {
         const int k = warp + j * kCW;
-        mbar_wait_bounded(smem_u32(&full[k % ns]), (k / ns) & 1);
+        mbar_wait_bounded(smem_u32(&full[k % ns]), (k / ns) & 1, wait_ns);
       }
     }
   }
@@ -770,7 +771,7 @@ size_t attn_items_bound(const DevCache& c, int kmax) {
 
 bool step_supported(const DevCache& c) {
   if (c.host_tiers != 0) return false;  // its pages are fetched by bulk copies only
-  if ((long long)c.B * c.Hkv * 2 + kCtlWords > (long long)(kCounterBytes / sizeof(unsigned))) return false;
+  if ((long long)c.B * c.Hkv * 2 + kCtlWords > (long long)kWaitLimitWord) return false;
   return step_plan(c).ns >= kCW;
 }
 

@@ -31,13 +31,14 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "workspace too sm
 
 DERR_BAD_PAGE, DERR_FP16_RANGE, DERR_NAN_SCORE, DERR_KMAX = 0x1, 0x2, 0x4, 0x8
 DERR_NONFINITE, DERR_TIMEOUT, DERR_BAD_POS = 0x10, 0x20, 0x40
+WS_WAIT_LIMIT_WORD = 16383  # workspace head word: bounded-wait limit in microseconds (0: 2 s)
 
 EXPORTS = ["kvq_chunk_bytes", "kvq_status_string", "kvq_append", "kvq_build_pages", "kvq_page_scores",
            "kvq_select_topk", "kvq_workspace_size", "kvq_sparse_decode_attn", "kvq_dequant_page",
            "kvq_sparse_decode_attn_noalloc", "kvq_noalloc_scratch_bytes", "kvq_workspace_init",
            "kvq_step_workspace_size", "kvq_decode_step", "kvq_score_select", "kvq_append_scores",
            "kvq_requantize_pages", "kvq_quad_build", "kvq_quad_append", "kvq_quad_page_scores",
-           "kvq_quad_append_scores"]
+           "kvq_quad_append_scores", "kvq_set_grid_override"]
 
 
 class KvqCache(ctypes.Structure):
@@ -82,13 +83,15 @@ _lib.kvq_score_select.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, PO
                                   c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p]
 _lib.kvq_append_scores.argtypes = [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
 _lib.kvq_requantize_pages.argtypes = [_P, c_void_p, c_int32, c_void_p]
+_lib.kvq_set_grid_override.argtypes = [c_int32]
 _lib.kvq_quad_build.argtypes = [_P, _PQ, c_void_p, c_void_p, c_int64, c_void_p]
 _lib.kvq_quad_append.argtypes = [_P, _PQ, c_void_p, c_void_p, c_void_p]
 _lib.kvq_quad_page_scores.argtypes = [_P, _PQ, c_void_p, c_float, c_void_p, c_void_p]
 _lib.kvq_quad_append_scores.argtypes = [_P, _PQ, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_void_p, c_void_p]
 for _f in EXPORTS[2:9] + ["kvq_sparse_decode_attn_noalloc", "kvq_workspace_init", "kvq_step_workspace_size",
                           "kvq_decode_step", "kvq_score_select", "kvq_append_scores", "kvq_requantize_pages",
-                          "kvq_quad_build", "kvq_quad_append", "kvq_quad_page_scores", "kvq_quad_append_scores"]:
+                          "kvq_quad_build", "kvq_quad_append", "kvq_quad_page_scores", "kvq_quad_append_scores",
+                          "kvq_set_grid_override"]:
     getattr(_lib, _f).restype = c_int32
 
 
@@ -142,6 +145,11 @@ def kvq_workspace_size(cache, kmax: int) -> int:
     n = c_size_t(0)
     _check(_lib.kvq_workspace_size(cache.ref(), kmax, ctypes.byref(n)), "kvq_workspace_size")
     return int(n.value)
+
+
+def kvq_set_grid_override(ctas: int):
+    """Attention / fused-step grid of ``ctas`` CTAs for every later call (0: one per SM)."""
+    _check(_lib.kvq_set_grid_override(int(ctas)), "kvq_set_grid_override")
 
 
 def kvq_workspace_init(workspace, stream=None):

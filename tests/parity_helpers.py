@@ -4,6 +4,7 @@ from __future__ import annotations
 import numpy as np
 
 from oracle import cache as ocache
+from oracle.attention import attend, token_index
 from oracle.fp import bits16_to_f64
 from oracle.layout import chunk_bytes
 from oracle.select import kth_margin
@@ -110,3 +111,48 @@ def oracle_step(w, sh, b: int, g: int, q, kn, vn, sel=None, quad=None):
     (an ``oracle.quad.QuadState``) scores pages with the quad score."""
     return step_pair(w, sh, b, g, q[b], None if kn is None else kn[b, g], None if vn is None else vn[b, g],
                      sel=sel, quad=quad)
+
+
+def oracle_outputs_on(w, sh, b: int, g: int, q, pages):
+    """The oracle's attention of kv head g's query heads over the given pages of a
+    prepared (and already appended) cache: outputs [G, D] and lse [G]."""
+    G = w.G
+    idx = token_index(np.asarray(pages, dtype=np.int64), sh.L)
+    out, lse = np.zeros((G, w.D)), np.zeros(G)
+    for i in range(G):
+        o, l, _, _ = attend(q[b, g * G + i], sh.khat[idx], sh.vhat[idx], w.sm_scale)
+        out[i], lse[i] = o, l
+    return out, lse
+
+
+def check_unit(w, snap, scores, sel, cnt, out, lse, q, kn, vn, b: int, g: int, what: str, pages="all",
+               tail: bool = True) -> bool:
+    """One (sequence, kv head) unit of a GPU step against the oracle's step: the cache
+    after the append (every page's bytes, or those listed in ``pages`` plus the appended
+    one; summaries; the open page's key sum), the scores, the selected set and the outputs
+    and lse of the G query heads.  Where the sets legitimately differ (k-th margin <= 1e-5)
+    the outputs are compared with the oracle's attention over the GPU's set.  Returns
+    whether the sets were equal."""
+    sh = prepare(w, b, g)
+    r = oracle_step(w, sh, b, g, q, kn, vn)
+    P = r["P"]
+    if pages == "all":
+        pages = range(P)
+    pages = sorted(set(int(p) for p in pages if p < P) | ({int(w.lens[b]) // 16} if w.append and P else set()))
+    check_pages(snap, sh, w, b, g, pages)
+    check_summary(snap, sh, b, g, P)
+    if w.append or int(w.lens[b]) % 16:
+        assert np.array_equal(snap["ksum"][b, g], sh.ksum), f"{what}: open-page key sum differs"
+    G = w.G
+    check_scores(scores[b, g], r["scores"], q[b, g * G:(g + 1) * G], sh.summary, P, tail=tail)
+    got_sel = sel[b, g, :cnt[b, g]]
+    same = check_selection(got_sel, r["sel"], r["scores"], w, P)
+    ref_out, ref_lse = (r["out"], r["lse"]) if same else oracle_outputs_on(w, sh, b, g, q, got_sel)
+    for i in range(G):
+        h = g * G + i
+        check_output(out[b, h], ref_out[i], f"{what} b={b} h={h}", w.dtype)
+        if np.isfinite(ref_lse[i]):
+            assert abs(lse[b, h] - ref_lse[i]) <= 1e-3 * max(1.0, abs(ref_lse[i])), (what, b, h)
+        else:
+            assert not np.isfinite(lse[b, h])
+    return same

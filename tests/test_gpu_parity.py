@@ -16,7 +16,7 @@ from oracle import cache as ocache
 from oracle.step import prepare
 from sparse_mixed_precision_kvq_b200 import workloads as W
 from tests.parity_helpers import (check_output, check_pages, check_scores, check_selection, check_summary,
-                                  oracle_step, out_to_f64, query_and_new, snapshot)
+                                  check_unit, oracle_step, out_to_f64, query_and_new, snapshot)
 
 pytestmark = pytest.mark.gpu
 
@@ -75,7 +75,6 @@ def test_step_matches_oracle(kvq, name, path):
     cnt = step.cnt.cpu().numpy()
     out = out_to_f64(step.out, w.dtype)
     lse = step.lse.cpu().numpy()
-    n_same = 0
     for b in range(w.B):
         for g in range(w.Hkv):
             sh = prepare(w, b, g)
@@ -84,23 +83,8 @@ def test_step_matches_oracle(kvq, name, path):
             check_summary(pre, sh, b, g, P0)
             if int(w.lens[b]) % 16:
                 assert np.array_equal(pre["ksum"][b, g], sh.ksum)
-            r = oracle_step(w, sh, b, g, q, kn, vn)
-            P = r["P"]
-            if w.append:
-                pa = int(w.lens[b]) // 16
-                check_pages(post, sh, w, b, g, [pa])
-                check_summary(post, sh, b, g, P)
-                assert np.array_equal(post["ksum"][b, g], sh.ksum)
-            G = w.G
-            check_scores(scores[b, g], r["scores"], q[b, g * G:(g + 1) * G], sh.summary, P, tail=path != "fused")
-            got_sel = sel[b, g, :cnt[b, g]]
-            if check_selection(got_sel, r["sel"], r["scores"], w, P):
-                n_same += 1
-                for i in range(G):
-                    h = g * G + i
-                    check_output(out[b, h], r["out"][i], f"{name} b={b} h={h}", w.dtype)
-                    assert abs(lse[b, h] - r["lse"][i]) <= 1e-3 * max(1.0, abs(r["lse"][i]))
-    assert n_same >= (w.B * w.Hkv + 1) // 2
+            # after the step: the appended page, summaries, scores, selection, every output
+            check_unit(w, post, scores, sel, cnt, out, lse, q, kn, vn, b, g, name, pages=[], tail=path != "fused")
 
 
 @pytest.mark.parametrize("name", ["c0_alltiers_fp16_d64", "g1_alltiers", "c4"])
