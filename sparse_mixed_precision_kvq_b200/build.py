@@ -2,7 +2,7 @@
 
     python -m sparse_mixed_precision_kvq_b200.build [--force] [--verbose]
 
-Each ``csrc/*.cu`` is compiled to an object with
+Each ``csrc/*.cu`` is compiled (one nvcc per unit, in parallel) to an object with
 ``-gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`` (no fast-math; the
 quantise-and-pack and quad-state units also get ``-fmad=false`` so their fp64 metadata
 math is a fixed sequence of IEEE operations), then linked into ``lib/libkvq.so`` with the static CUDA
@@ -16,6 +16,7 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -54,15 +55,25 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     os.makedirs(LIBDIR, exist_ok=True)
     os.makedirs(OBJDIR, exist_ok=True)
-    objs = []
+    jobs = []
     for src in sources():
         obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
         cmd = [nvcc(), *ARCH, *COMMON, *PER_FILE.get(os.path.basename(src), []), "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
+        jobs.append((cmd, obj))
+    # one nvcc per translation unit, in parallel; output printed in source order
+    workers = max(1, min(len(jobs), os.cpu_count() or 1))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        done = list(ex.map(lambda j: subprocess.run(j[0], capture_output=True, text=True), jobs))
+    for (cmd, _), r in zip(jobs, done):
+        if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+            sys.stdout.write(r.stdout + r.stderr)
+        if r.returncode != 0:
+            sys.stderr.write(r.stdout + r.stderr)
+            raise subprocess.CalledProcessError(r.returncode, cmd)
+    objs = [obj for _, obj in jobs]
     tmp = LIB + ".tmp"
     subprocess.run([nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs], check=True)
     os.replace(tmp, LIB)
