@@ -201,46 +201,61 @@ def max_over_ranks(x: float, device) -> float:
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def run_kvq(args, rank: int, world: int, local_rank: int):
+PATHS = {"fused": "kvq_decode_step (one persistent launch)",
+         "two": "kvq_score_select -> kvq_sparse_decode_attn",
+         "three": "kvq_append_scores -> kvq_select_topk -> kvq_sparse_decode_attn",
+         "calls": "kvq_append -> kvq_page_scores -> kvq_select_topk -> kvq_sparse_decode_attn"}
+
+
+def step_parts(step, path: str):
+    """The launches of one step of ``path``, in order, as (name, callable) pairs."""
+    return {"fused": [("decode_step", step.run_fused)],
+            "two": [("score_select", step.score_select), ("sparse_decode_attn", step.attend)],
+            "three": [("append_scores", step.append_scores), ("select_topk", step.select),
+                      ("sparse_decode_attn", step.attend)],
+            "calls": [("append", step.append), ("page_scores", step.scores_), ("select_topk", step.select),
+                      ("sparse_decode_attn", step.attend)]}[path]
+
+
+def dominant_bytes(path: str, nbytes: dict, dom: int) -> int:
+    if path == "fused":
+        return nbytes["attn"] + nbytes["score"] + nbytes["select"] + nbytes["append"]
+    if path == "two":
+        return [nbytes["score"] + nbytes["select"] + nbytes["append"], nbytes["attn"]][dom]
+    if path == "three":
+        return [nbytes["score"] + nbytes["append"], nbytes["select"], nbytes["attn"]][dom]
+    return [nbytes["append"], nbytes["score"], nbytes["select"], nbytes["attn"]][dom]
+
+
+def kernel_files(path: str, quad: bool):
+    sc = "quad.cu" if quad else "score.cu"
+    return {"fused": ["step.cu"], "two": ["score.cu", "attn.cu"], "three": [sc, "select.cu", "attn.cu"],
+            "calls": ["append.cu", sc, "select.cu", "attn.cu"]}[path]
+
+
+def measure(w, cache, step, path: str, K: int, warmup: int, flush, stream, dev, world: int, peak: float,
+            quad_rank: int = 0, soak_s: float = 0.0, e2e: bool = True, eager: bool = True):
+    """Time one workload's decode step on this rank.
+
+    step time: K replays of a CUDA graph of the step, each after an L2 flush (outside the
+    events), timed with CUDA events around each replay, summed and maxed over ranks;
+    kernels: a second graph with events between the launches; eager: the same launches
+    issued directly (no graph); e2e: the graph with the step's host inputs copied in and
+    its outputs copied back inside the events.  ``soak_s`` seconds of further replays
+    follow the timed ones, so that the clock sampler running meanwhile has a record longer
+    than the timed steps themselves."""
     import torch
     import torch.distributed as dist
-    from sparse_mixed_precision_kvq_b200 import kvq
-    from sparse_mixed_precision_kvq_b200 import workloads as W
-
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    w = rank_workload(args.config, rank, args.batch, args.tier)
-    quad_rank = args.quad_rank if args.score == "quad" else 0
-    basis = None
-    if quad_rank:
-        basis = np.stack([w.quad_basis(g, quad_rank, "law") for g in range(w.Hkv)])
-    cache = kvq.cache_from_workload(w, device=dev, quad_basis=basis, host_tiers=args.host_tiers)
-    step = kvq.DecodeStep(w, cache, device=dev, coverage=args.coverage, quad=bool(quad_rank))
-    tier_tbl, _, _ = w.slot_map()
-    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    for _ in range(args.warmup):
+    parts = step_parts(step, path)
+    run_step = {"fused": step.run_fused, "two": step.run_two, "three": step.run_three, "calls": step.run}[path]
+    for _ in range(warmup):
         flush.fill_(1)
-        {"fused": step.run_fused, "two": step.run_two, "three": step.run_three, "calls": step.run}[args.path]()
+        run_step()
     torch.cuda.synchronize(dev)
     assert cache.err_bits() == 0, f"device error bits {cache.err_bits():#x}"
+    tier_tbl, _, _ = w.slot_map()
     sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
     nbytes = algorithmic_bytes(w, sel, cnt, tier_tbl, quad_rank)
-
-    K = args.steps
-    fused = args.path == "fused"
-    run_step = {"fused": step.run_fused, "two": step.run_two, "three": step.run_three, "calls": step.run}[args.path]
-    # kernels of one step, in launch order (one callable each)
-    parts = {"fused": [("decode_step", step.run_fused)],
-             "two": [("score_select", step.score_select), ("sparse_decode_attn", step.attend)],
-             "three": [("append_scores", step.append_scores), ("select_topk", step.select),
-                       ("sparse_decode_attn", step.attend)],
-             "calls": [("append", step.append), ("page_scores", step.scores_), ("select_topk", step.select),
-                       ("sparse_decode_attn", step.attend)]}[args.path]
-    # The step is replayed from CUDA graphs so the CPU never starves the GPU:
-    #  g_step: the step's launches, nothing between them (programmatic launch overlap intact);
-    #  g_prof: the same launches with timing events between them (per-kernel durations).
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
     with torch.cuda.stream(side):
@@ -267,11 +282,6 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
 
     e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[0])
-                          if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local_rank)
-    if rank == 0:
-        clocks.start()
-        time.sleep(1.0)  # let nvidia-smi start sampling
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -285,7 +295,14 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     if world > 1:
         dist.barrier()
     t1 = time.time()
-    # per-kernel durations: the same step with events between the kernels (one step at a time)
+    soak = 0
+    while time.time() - t1 < soak_s:   # the same replays, back to back, for the clock record
+        for _ in range(200):
+            flush.fill_(soak & 0xFF)
+            g_step.replay()
+            soak += 1
+        torch.cuda.synchronize(dev)
+    t2 = time.time()
     KP = min(K, 300)
     per = np.zeros((KP, len(parts)))
     for k in range(KP):
@@ -293,72 +310,157 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
         g_prof.replay()
         torch.cuda.synchronize(dev)
         per[k] = [pev[i].elapsed_time(pev[i + 1]) for i in range(len(parts))]
-    clocks.stop()
     step_ms = np.array([e0[k].elapsed_time(e1[k]) for k in range(K)])
     total_ms = max_over_ranks(float(step_ms.sum()), dev)
     ms_per_step = total_ms / K
-    tokens = world * w.B * K
-    value = tokens / (total_ms / 1e3)
 
-    # end to end through the public API: host q / new token in, host out / lse back
-    pin = dict(q=step.q.cpu().pin_memory())
-    if w.append:
-        pin["k"], pin["v"] = step.k_new.cpu().pin_memory(), step.v_new.cpu().pin_memory()
-    out_h = torch.empty_like(step.out, device="cpu").pin_memory()
-    lse_h = torch.empty_like(step.lse, device="cpu").pin_memory()
-    KE = max(1, min(K, 500))
-    e_start = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
-    e_end = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
-    for k in range(KE):
-        flush.fill_(k & 0xFF)
-        e_start[k].record(stream)
-        step.q.copy_(pin["q"], non_blocking=True)
+    out = {"ms_per_step": ms_per_step, "tokens_per_s": world * w.B * K / (total_ms / 1e3),
+           "nbytes": nbytes, "sel": sel, "cnt": cnt, "tier_tbl": tier_tbl, "names": [n for n, _ in parts],
+           "kernel_ms": per.mean(0), "clock_window": (t0, t2), "soak_steps": soak}
+    if eager:
+        KE = max(1, min(K, 200))
+        a = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
+        b_ = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
+        for k in range(KE):
+            flush.fill_(k & 0xFF)
+            a[k].record(stream)
+            run_step()
+            b_[k].record(stream)
+        torch.cuda.synchronize(dev)
+        out["ms_per_step_eager"] = max_over_ranks(float(np.mean([a[k].elapsed_time(b_[k]) for k in range(KE)])), dev)
+    if e2e:
+        pin = dict(q=step.q.cpu().pin_memory())
         if w.append:
-            step.k_new.copy_(pin["k"], non_blocking=True)
-            step.v_new.copy_(pin["v"], non_blocking=True)
-        g_step.replay()
-        out_h.copy_(step.out, non_blocking=True)
-        lse_h.copy_(step.lse, non_blocking=True)
-        e_end[k].record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(float(np.mean([e_start[k].elapsed_time(e_end[k]) for k in range(KE)])), dev)
-    h2d = pin["q"].numel() * 2 + (pin["k"].numel() * 2 * 2 if w.append else 0)
-    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+            pin["k"], pin["v"] = step.k_new.cpu().pin_memory(), step.v_new.cpu().pin_memory()
+        out_h = torch.empty_like(step.out, device="cpu").pin_memory()
+        lse_h = torch.empty_like(step.lse, device="cpu").pin_memory()
+        KE = max(1, min(K, 500))
+        es = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
+        ee = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
+        for k in range(KE):
+            flush.fill_(k & 0xFF)
+            es[k].record(stream)
+            step.q.copy_(pin["q"], non_blocking=True)
+            if w.append:
+                step.k_new.copy_(pin["k"], non_blocking=True)
+                step.v_new.copy_(pin["v"], non_blocking=True)
+            g_step.replay()
+            out_h.copy_(step.out, non_blocking=True)
+            lse_h.copy_(step.lse, non_blocking=True)
+            ee[k].record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(float(np.mean([es[k].elapsed_time(ee[k]) for k in range(KE)])), dev)
+        h2d = pin["q"].numel() * 2 + (pin["k"].numel() * 2 * 2 if w.append else 0)
+        d2h = out_h.numel() * 2 + lse_h.numel() * 4
+        out["e2e"] = {"value": world * w.B / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+                      "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
+    assert cache.err_bits() == 0, f"device error bits {cache.err_bits():#x}"
     del g_prof, g_step
+    step_bytes = sum(nbytes[k] for k in ("attn", "score", "select", "append"))
+    out["step_hbm"] = {"bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3) / 1e9,
+                       "peak_gbs": peak, "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak}
+    out["kernels_roofline"] = kernel_rooflines(out["names"], out["kernel_ms"], nbytes, peak)
+    return out
 
-    # optional dense reference point: every page selected (c1's dense run)
-    dense_ms = None
-    if args.dense and rank == 0:
-        dense_ms = time_dense(w, cache, step, flush, stream, dev)
 
-    if rank != 0:
-        return None
+def config_summary(name: str, w, m: dict, peak: float, dense_ms=None) -> dict:
+    """The per-workload object of the JSON line (other workloads than the headline one)."""
+    kr = m["kernels_roofline"]
+    d = {"workload": f"{name}: {DESCR[name]}", "batch": w.B, "context_max": int(w.lens.max()),
+         "selected_pages": int(m["cnt"].sum()), "ms_per_step": m["ms_per_step"], "tokens_per_s": m["tokens_per_s"],
+         "ms_per_step_eager": m.get("ms_per_step_eager"), "step_hbm": m["step_hbm"],
+         "kernels_ms": {n: float(a) for n, a in zip(m["names"], m["kernel_ms"])},
+         "attention_roofline": kr.get("sparse_decode_attn") or kr.get("decode_step"),
+         "e2e": m.get("e2e")}
+    if dense_ms is not None:
+        dense_bytes = dense_attn_bytes(w)
+        d["dense_all_pages"] = {"ms": dense_ms, "bytes": dense_bytes,
+                                "achieved_gbs": dense_bytes / (dense_ms * 1e-3) / 1e9,
+                                "frac": dense_bytes / (dense_ms * 1e-3) / 1e9 / peak,
+                                "speedup_of_sparse_step": dense_ms / m["ms_per_step"]}
+    return d
+
+
+def dense_attn_bytes(w) -> int:
+    """Attention over every page: all K+V chunks of every (sequence, kv head) + q + out."""
+    from sparse_mixed_precision_kvq_b200.kvq import kvq_chunk_bytes
+    tier_tbl, _, _ = w.slot_map()
+    cb = np.array([2 * kvq_chunk_bytes(t, w.D) for t in range(6)], dtype=np.int64)
+    tot = 0
+    for b in range(w.B):
+        P = w.pages_after(b)
+        tot += int(cb[tier_tbl[b, :P]].sum()) * w.Hkv + P * w.Hkv * 4
+    return tot + 2 * w.B * w.Hq * w.D * 2
+
+
+def run_kvq(args, rank: int, world: int, local_rank: int):
+    import torch
+    from sparse_mixed_precision_kvq_b200 import kvq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
     peak, peak_kind = load_peaks()
-    names = [n for n, _ in parts]
-    avg = per.mean(0)
+    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[0])
+                          if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local_rank)
+    if rank == 0:
+        clocks.start()
+        time.sleep(1.0)  # let nvidia-smi start sampling
+
+    w = rank_workload(args.config, rank, args.batch, args.tier)
+    quad_rank = args.quad_rank if args.score == "quad" else 0
+    basis = None
+    if quad_rank:
+        basis = np.stack([w.quad_basis(g, quad_rank, "law") for g in range(w.Hkv)])
+    cache = kvq.cache_from_workload(w, device=dev, quad_basis=basis, host_tiers=args.host_tiers)
+    step = kvq.DecodeStep(w, cache, device=dev, coverage=args.coverage, quad=bool(quad_rank))
+    m = measure(w, cache, step, args.path, args.steps, args.warmup, flush, stream, dev, world, peak,
+                quad_rank=quad_rank, soak_s=args.soak_s if rank == 0 else 0.0)
+    cw = m["clock_window"]
+    dense_ms = None
+    if args.dense and not args.no_dense and rank == 0:
+        dense_ms = time_dense(w, cache, step, flush, stream, dev)
+    names, avg, nbytes = m["names"], m["kernel_ms"], m["nbytes"]
     dom = int(np.argmax(avg))
-    step_bytes = nbytes["attn"] + nbytes["score"] + nbytes["select"] + nbytes["append"]
-    if fused:
-        dom_bytes, files = step_bytes, ["step.cu"]
-    elif args.path == "two":
-        dom_bytes = [nbytes["score"] + nbytes["select"] + nbytes["append"], nbytes["attn"]][dom]
-        files = ["score.cu", "attn.cu"]
-    elif args.path == "three":
-        dom_bytes = [nbytes["score"] + nbytes["append"], nbytes["select"], nbytes["attn"]][dom]
-        files = ["quad.cu" if quad_rank else "score.cu", "select.cu", "attn.cu"]
-    else:
-        dom_bytes = [nbytes["append"], nbytes["score"], nbytes["select"], nbytes["attn"]][dom]
-        files = ["append.cu", "quad.cu" if quad_rank else "score.cu", "select.cu", "attn.cu"]
+    dom_bytes = dominant_bytes(args.path, nbytes, dom)
+    files = kernel_files(args.path, bool(quad_rank))
     achieved = dom_bytes / (avg[dom] * 1e-3) / 1e9
     tr = kernel_traffic(files[dom])
+    sel, cnt, tier_tbl = m["sel"], m["cnt"], m["tier_tbl"]
+    host = None
+    if args.host_tiers:
+        host = host_link(w, sel, cnt, tier_tbl, args.host_tiers, avg[names.index("sparse_decode_attn")]
+                         if "sparse_decode_attn" in names else None, dev)
+    demotion = None
+    if args.demote is not None:
+        del step, cache
+        demotion = time_demotion(w, args.demote, flush, stream, dev, peak, peak_kind)
+    else:
+        del step, cache
+    torch.cuda.empty_cache()
+
+    # the other workloads, same path, default options (each rank its own batch)
+    configs = {}
+    for name in [c for c in args.configs.split(",") if c and c != args.config] if args.configs != "none" else []:
+        wc = rank_workload(name, rank)
+        cc = kvq.cache_from_workload(wc, device=dev)
+        sc = kvq.DecodeStep(wc, cc, device=dev)
+        mc = measure(wc, cc, sc, args.path, args.steps, args.warmup, flush, stream, dev, world, peak)
+        configs[name] = config_summary(name, wc, mc, peak)
+        del sc, cc
+        torch.cuda.empty_cache()
+    clocks.stop()
+    if rank != 0:
+        return None
     line = {
         "metric": METRIC,
-        "value": value,
+        "value": m["tokens_per_s"],
         "unit": "tokens/s",
         "n_gpus": world,
-        "steps": K,
+        "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": ms_per_step,
+        "ms_per_step": m["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -374,40 +476,46 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
                    f"quad (rank {quad_rank}, basis: eigenvectors of the key law's covariance)",
                    "l2": f"flushed ({args.flush_mib} MiB write) before every timed step",
                    "parallelism": f"replicas x{world} (independent batches)"},
-        "step_hbm": {"bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3) / 1e9,
-                     "peak_gbs": peak, "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak,
-                     "peak_kind": peak_kind},
+        "step_hbm": dict(m["step_hbm"], peak_kind=peak_kind),
+        "ms_per_step_eager": m.get("ms_per_step_eager"),
         "kernels_ms": {n: float(a) for n, a in zip(names, avg)},
-        "kernels_roofline": kernel_rooflines(names, avg, nbytes, peak),
+        "kernels_roofline": m["kernels_roofline"],
         "roofline": {"bound": "hbm", "kernel": names[dom], "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
                      "algorithmic_bytes_per_launch": dom_bytes,
                      "traffic": None if tr is None else tr["dram_bytes_per_launch"]},
-        "e2e": {"value": world * w.B / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
-        "gpu_launches": (len(parts) + (1 if quad_rank and w.append and args.path == "calls" else 0)) * K,
-        "path": {"fused": "kvq_decode_step (one persistent launch)",
-                 "two": "kvq_score_select -> kvq_sparse_decode_attn",
-                 "three": "kvq_append_scores -> kvq_select_topk -> kvq_sparse_decode_attn",
-                 "calls": "kvq_append -> kvq_page_scores -> kvq_select_topk -> kvq_sparse_decode_attn"}[args.path],
+        "e2e": m["e2e"],
+        "gpu_launches": (len(names) + (1 if quad_rank and w.append and args.path == "calls" else 0)) * args.steps,
+        "path": PATHS[args.path],
         "timing": "step: CUDA-graph replay of the step timed with events around each replay; "
-                  "kernels_ms: a second graph with events between the launches (no launch overlap)",
-        "clocks": clocks.summary(t0, t1),
+                  "kernels_ms: a second graph with events between the launches (no launch overlap); "
+                  "ms_per_step_eager: the same launches issued without a graph",
+        "clocks": dict(clocks.summary(cw[0], cw[1]),
+                       window=f"the {args.steps} timed steps and {m['soak_steps']} more replays of the same step "
+                              f"right after them ({args.soak_s:.1f} s)"),
     }
     if dense_ms is not None:
-        line["dense_all_pages_ms"] = dense_ms
-    if args.host_tiers:
-        line["host_link"] = host_link(w, sel, cnt, tier_tbl, args.host_tiers, avg[names.index("sparse_decode_attn")]
-                                      if "sparse_decode_attn" in names else None, dev)
-    if args.demote is not None:
-        del step, cache
-        line["demotion"] = time_demotion(w, args.demote, flush, stream, dev, peak, peak_kind)
+        dense_bytes = dense_attn_bytes(w)
+        line["dense_all_pages"] = {"op": "kvq_sparse_decode_attn over every page of every (sequence, kv head)",
+                                   "ms": dense_ms, "bytes": dense_bytes,
+                                   "achieved_gbs": dense_bytes / (dense_ms * 1e-3) / 1e9,
+                                   "frac": dense_bytes / (dense_ms * 1e-3) / 1e9 / peak,
+                                   "sparse_step_speedup": dense_ms / m["ms_per_step"]}
+    if configs:
+        line["configs"] = configs
+    if host is not None:
+        line["host_link"] = host
+    if demotion is not None:
+        line["demotion"] = demotion
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds or 12.0, config=args.config, seed_rank=rank,
+                                            batch=args.batch, tier=args.tier)
     return line
 
 
 def time_dense(w, cache, step, flush, stream, dev, reps=20):
+    """Attention over every page of every (sequence, kv head), L2 flushed, events around
+    each launch (c1's dense reference point)."""
     import torch
     from sparse_mixed_precision_kvq_b200 import kvq
     P = np.array([w.pages_after(b) for b in range(w.B)])
@@ -430,6 +538,7 @@ def time_dense(w, cache, step, flush, stream, dev, reps=20):
         torch.cuda.synchronize(dev)
         if r >= 3:
             ts.append(a.elapsed_time(b_))
+    assert cache.err_bits() == 0, f"device error bits {cache.err_bits():#x}"
     return float(np.mean(ts))
 
 
@@ -511,58 +620,99 @@ def time_demotion(w, tier: int, flush, stream, dev, peak: float, peak_kind: str,
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def cpu_baseline(w, budget_s: float = 15.0):
-    """The oracle's decode step timed on the host cores on a bounded sample of (b, g) pairs.
-
-    Cache construction (the oracle's quantise/pack of the prefilled context) is excluded;
-    each timed unit is the oracle step of one (sequence, kv head): append, score,
-    select, attention of its G query heads.  tokens/s = B / (mean unit time * B * Hkv).
-    """
+def _oracle_units(config: str, seed_rank: int, units, budget_s: float, batch=None, tier=None):
+    """Worker: prepare the listed (b, g) units of the workload (untimed), then run the
+    oracle's decode step on them round-robin for ``budget_s`` seconds, numpy/BLAS on one
+    thread.  Returns (unit steps run, seconds spent in them)."""
     from threadpoolctl import threadpool_limits
     from oracle.fp import bits16_to_f64
     from oracle.step import prepare, step_pair
-
+    w = rank_workload(config, seed_rank, batch, tier)
     q = bits16_to_f64(w.query_bits(), w.dtype)
     kn, vn = w.new_kv_bits() if w.append else (None, None)
-    pairs = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
-    rng = np.random.default_rng(0)
-    order = [pairs[i] for i in rng.permutation(len(pairs))][:4]
-    prepared = [(b, g, prepare(w, b, g)) for b, g in order]
-    times = []
-    spent = 0.0
-    saved = [(sh.L, sh.ksum.copy()) for _, _, sh in prepared]
     with threadpool_limits(limits=1):
-        while spent < budget_s and len(times) < 20000:
+        prepared = [(b, g, prepare(w, b, g)) for b, g in units]
+        saved = [(sh.L, sh.ksum.copy()) for _, _, sh in prepared]
+        n, spent = 0, 0.0
+        while spent < budget_s and n < 100000:
             for (b, g, sh), (L0, ks0) in zip(prepared, saved):
                 t0 = time.perf_counter()
                 step_pair(w, sh, b, g, q[b], None if kn is None else kn[b, g], None if vn is None else vn[b, g])
-                dt = time.perf_counter() - t0
-                times.append(dt)
-                spent += dt
+                spent += time.perf_counter() - t0
+                n += 1
                 sh.L, sh.ksum = L0, ks0.copy()   # undo the append so the next step repeats it
-    unit = float(np.mean(times))
-    t_step = unit * w.B * w.Hkv
-    return {"value": w.B / t_step, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{len(times)} timed oracle steps of single (sequence, kv head) units drawn from "
-                      f"{len(prepared)} units of the same workload; step time = mean unit time x {w.B * w.Hkv} "
-                      f"units; cache construction excluded (the appended token is rewritten each time); numpy/BLAS limited to 1 thread"}
+    return n, spent
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(w, budget_s: float = 12.0, config: str = "c1", seed_rank: int = 0, all_cores: bool = True,
+                 batch=None, tier=None):
+    """The oracle's decode step timed on the host cores, on a bounded sample of (b, g) units.
+
+    Cache construction (the oracle's quantise/pack of the prefilled context) is excluded;
+    each timed unit is the oracle step of one (sequence, kv head): append, score, select,
+    attention of its G query heads.  tokens/s = B / (B * Hkv / unit steps per second).
+    One thread: 4 units in one process.  All cores: one spawned worker process per core
+    (up to one per unit), each on its own unit(s), its rate summed over the workers."""
+    pairs = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+    rng = np.random.default_rng(0)
+    order = [pairs[i] for i in rng.permutation(len(pairs))]
+    n1, t1 = _oracle_units(config, seed_rank, order[:4], budget_s, batch, tier)
+    rate1 = n1 / t1
+    res = {"value": w.B / (w.B * w.Hkv / rate1), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+           "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+           "sample": f"{n1} timed oracle steps of single (sequence, kv head) units drawn from 4 units of the "
+                     f"same workload; step time = mean unit time x {w.B * w.Hkv} units; cache construction "
+                     f"excluded (the appended token is rewritten each time); numpy/BLAS on 1 thread"}
+    if all_cores:
+        import multiprocessing as mp
+        cores = max(1, min(os.cpu_count() or 1, len(pairs), 64))
+        groups = [order[i::cores] for i in range(cores)]
+        groups = [g[:2] for g in groups if g]
+        ctx = mp.get_context("spawn")
+        with ctx.Pool(len(groups)) as pool:
+            got = pool.starmap(_oracle_units, [(config, seed_rank, g, budget_s, batch, tier) for g in groups])
+        rate = sum(n / t for n, t in got if t > 0)
+        res["all_cores"] = {"value": w.B / (w.B * w.Hkv / rate), "unit": "tokens/s", "cores": len(groups),
+                            "unit_steps": int(sum(n for n, _ in got)),
+                            "sample": f"{len(groups)} spawned worker processes, one per core, each running the "
+                                      f"oracle step of its own 1-2 (sequence, kv head) units for {budget_s:.0f} s "
+                                      f"(numpy/BLAS on 1 thread each); rate = sum of the workers' unit rates"}
+    return res
 
 
 def run_reference(args, rank: int, world: int):
+    """The reference arm: the oracle (the plain fp64 restatement of the method) as it
+    stands, on the host cores, rank 0 only."""
     from sparse_mixed_precision_kvq_b200 import workloads as W
     if rank != 0:
         return None
     w = W.make(args.config)
     K = args.steps
-    budget = max(5.0, min(60.0, 150.0 / max(1, K + args.warmup)))
-    base = cpu_baseline(w, budget_s=budget)
+    budget = args.cpu_seconds if args.cpu_seconds is not None else max(3.0, min(30.0, 90.0 / max(1, K + args.warmup)))
+    base = cpu_baseline(w, budget_s=budget, config=args.config)
+    best = base.get("all_cores", base)
     line = {
-        "metric": METRIC, "value": base["value"], "unit": "tokens/s", "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": 1e3 * w.B / base["value"], "higher_is_better": True,
+        "metric": METRIC, "value": best["value"], "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": 1e3 * w.B / best["value"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{args.config}: {DESCR[args.config]}", "batch_per_gpu": w.B},
-        "impl": "reference", "cpu_baseline": base,
-        "e2e": {"value": base["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "config": {"workload": f"{args.config}: {DESCR[args.config]}", "batch_per_gpu": w.B,
+                   "context": int(w.lens.max()), "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D},
+        "impl": "reference",
+        "cpu_baseline": {"value": best["value"], "unit": "tokens/s", "cores": best["cores"], "kind": "oracle",
+                         "sample": best["sample"], "one_thread": base["value"], "cpu_model": base["cpu_model"],
+                         "nproc": base["nproc"]},
+        "e2e": {"value": best["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     return line
 
@@ -587,12 +737,20 @@ def main():
                     help="store every prefilled page at this tier (0 16-bit, 1 int8, 2 int4, 3 int2, 4 1-bit, 5 fp8)")
     ap.add_argument("--host-tiers", type=int, default=0,
                     help="bit t: pool t lives in pinned host memory that the kernels read in place (DRAM value tier)")
-    ap.add_argument("--dense", action="store_true", help="also time attention over every page")
+    ap.add_argument("--dense", action="store_true", default=None,
+                    help="also time attention over every page (on by default for c1)")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--configs", default="c2,c3,c4",
+                    help="comma-separated other workloads measured after the headline one (same path, default "
+                         "options) into the line's `configs` object; 'none' skips them")
+    ap.add_argument("--soak-s", type=float, default=1.5,
+                    help="seconds of further step replays after the timed ones, while clocks are sampled")
     ap.add_argument("--demote", type=int, default=None, choices=[1, 2, 3, 4, 5],
                     help="also time kvq_requantize_pages moving the workload's pages outside the sink and "
                          "recent windows to this tier (1 int8, 2 int4, 3 int2, 4 1-bit, 5 fp8)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=None,
+                    help="seconds of oracle steps per CPU leg (default 12; the reference arm sizes it by K + W)")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling runs)")
     ap.add_argument("--flush-mib", type=int, default=512, help="L2 flush buffer (must exceed the 126 MB L2)")
     args = ap.parse_args()
@@ -604,6 +762,12 @@ def main():
         ap.error("--host-tiers: the fused step reads pages by bulk copies only")
     if args.score == "quad" and args.path not in ("calls", "three"):
         ap.error("--score quad runs on the four-call or the three-call path")
+    if args.dense is None:
+        args.dense = args.config == "c1"
+    special = (args.coverage is not None or args.tier is not None or args.host_tiers or args.score != "mean"
+               or args.batch is not None or args.demote is not None)
+    if special and args.configs == "c2,c3,c4":
+        args.configs = "none"   # the other workloads are measured on plain runs only
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

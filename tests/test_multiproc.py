@@ -69,7 +69,7 @@ def test_reference_arm_prints_the_contract_line():
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--config", "c0",
-                        "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=300, cwd=root)
+                        "--steps", "1", "--warmup", "3", "--cpu-seconds", "2"], capture_output=True, text=True, timeout=300, cwd=root)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
@@ -78,4 +78,6 @@ def test_reference_arm_prints_the_contract_line():
                 "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
         assert key in d, key
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
-    assert d["cpu_baseline"]["cores"] == 1 and d["e2e"]["h2d_bytes_per_step"] == 0
+    # c0 has two (sequence, kv head) units: one worker process each on a host with two or more cores
+    assert d["cpu_baseline"]["cores"] == min(2, os.cpu_count()) and d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["one_thread"] > 0 and d["cpu_baseline"]["nproc"] == os.cpu_count()
