@@ -121,7 +121,7 @@ typedef struct {
   int32_t* seq_len;        /* device [B] */
   void* pool[6];           /* device, per tier (NULL if unused) */
   int64_t pool_slots[6];   /* slots in each pool */
-  uint16_t* summary;       /* device [B][Hkv][max_pages][D] fp16 bits */
+  uint16_t* summary;       /* device [B][Hkv][max_pages][D] fp16 bits, 16-byte aligned */
   double* open_ksum;       /* device [B][Hkv][D] */
   uint32_t* err_word;      /* device, 1 word */
 } kvq_cache;
@@ -237,7 +237,8 @@ kvq_status kvq_set_grid_override(int32_t ctas);
  *  sel, cnt  as written by kvq_select_topk (pages must be < ceil(seq_len/16)).
  *  sm_scale  softmax scale (1/sqrt(D) for standard attention).
  *  out       device [B][Hq][D] cache dtype out: softmax(sm_scale * q.k) v over the tokens
- *            of the selected pages; zeros when a kv head has no selected page.
+ *            of the selected pages; zeros when a kv head has no selected page; NaN (and a
+ *            NaN lse) when a key or value read back is NaN (non-finite input, flagged).
  *  lse       device [B][Hq] fp32 out (may be NULL): natural-log log-sum-exp of the
  *            scaled logits (-inf when nothing is selected).
  *  workspace device scratch of at least kvq_workspace_size() bytes, prepared once with

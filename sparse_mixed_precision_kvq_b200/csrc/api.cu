@@ -55,6 +55,8 @@ kvq_status to_dev(const kvq_cache* k, DevCache& c) {
     any |= k->pool[t] != nullptr;
   }
   if (!any) return KVQ_ERR_INVALID_ARG;
+  // the summary rows are read with 16-byte loads and bulk copies
+  if (reinterpret_cast<uintptr_t>(k->summary) % 16 != 0) return KVQ_ERR_INVALID_ARG;
   c.summary = k->summary;
   c.open_ksum = k->open_ksum;
   c.err = k->err_word;

@@ -28,6 +28,9 @@ __global__ void __launch_bounds__(128) append_kernel(DevCache c, const int32_t* 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bg = blockIdx.x;
   const int b = bg / c.Hkv, g = bg % c.Hkv;
+  // The page-score sweep that follows only prefetches until it waits for this grid, so it
+  // may launch at once: its summary traffic then overlaps this kernel.
+  griddep_launch_dependents();
   griddep_wait();
   const int P = pos[b];
   if (P >= c.max_pages * kPage) {
@@ -39,7 +42,6 @@ __global__ void __launch_bounds__(128) append_kernel(DevCache c, const int32_t* 
     __syncthreads();
     if (ok) append_phase2<BF16>(c, b, g, P, kr, vr, warp, 4, lane);
   }
-  griddep_launch_dependents();
 }
 
 // ----------------------------------------------------------------------------- build

@@ -85,9 +85,6 @@ struct PageDesc {
   int nv;
 };
 
-// Merge partial slots [s0, s1] (stride 1) of segment bg into `dst` slot (when dst >= 0)
-// or into the output (dst < 0), with all threads of the CTA.  Loads are issued in
-// batches of 8 so the merge costs a couple of L2 round trips, not one per partial.
 // Write the merged (M, L, o) of element (h, d) of segment bg: as a partial into slot `dst`
 // of (dst_o, dst_ml), or, with dst < 0, as the segment's output o / L and lse.
 template <bool BF16>
@@ -104,101 +101,99 @@ __device__ inline void put_merged(const AttnArgs& a, uint16_t* out, float* lse, 
     return;
   }
   const int b = bg / c.Hkv, g = bg % c.Hkv;
-  const float r = Ls > 0.f ? o / Ls : 0.f;
+  const bool any = !(Ls <= 0.f);  // a NaN sum (a NaN key or value) gives a NaN output
+  const float r = any ? o / Ls : 0.f;
   const size_t oi = ((size_t)b * c.Hq + (size_t)g * G + h) * D + d;
   if constexpr (BF16) out[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
   else out[oi] = __half_as_ushort(__float2half_rn(r));
   if (d == 0 && lse != nullptr)
-    lse[(size_t)b * c.Hq + (size_t)g * G + h] = Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
+    lse[(size_t)b * c.Hq + (size_t)g * G + h] = any ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
 }
 
-// CTA merge of segment bg: warps w0..w1 of this CTA hold one partial each, in their own
-// ring (shared memory: the warp's last segment) or in their global warp slot (u + bg).
-// All of an element's partials are loaded before any is used: one memory round trip.
+// CTA merge of element (h, d) of segment bg: warps w0..w1 of this CTA hold one partial
+// each, in their own ring (shared memory: the warp's last segment) or in their global warp
+// slot (u + bg).  All of the element's partials are loaded before any is used: one memory
+// round trip.  The result goes to CTA partial slot `dst`, or to the output (dst < 0).
 template <int D, bool BF16>
-__device__ inline void cta_merge(const AttnArgs& a, uint16_t* out, float* lse, const unsigned char* rings,
-                                 const int* pseg, int bg, int w0, int w1, int dst) {
+__device__ inline void cta_merge_elem(const AttnArgs& a, uint16_t* out, float* lse, const unsigned char* rings,
+                                      const int* pseg, int bg, int h, int d, int w0, int w1, int dst) {
   const int G = a.c.G;
-  for (int e = threadIdx.x; e < G * D; e += kThreads) {
-    const int h = e / D, d = e % D;
-    float mv[kWarps], lv[kWarps], ov[kWarps];
+  float mv[kWarps], lv[kWarps], ov[kWarps];
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    mv[w] = -INFINITY;
+    lv[w] = 0.f;
+    ov[w] = 0.f;
+    if (w >= w0 && w <= w1) {
+      if (pseg[w] == bg) {
+        const float* sp = reinterpret_cast<const float*>(rings + (size_t)w * kRing);
+        ov[w] = sp[h * D + d];
+        mv[w] = sp[G * D + 2 * h];
+        lv[w] = sp[G * D + 2 * h + 1];
+      } else {
+        const size_t slot = (size_t)blockIdx.x * kWarps + w + bg;
+        ov[w] = __ldcg(&a.wp_o[(slot * G + h) * D + d]);
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(&a.wp_ml[(slot * G + h) * 2]));
+        mv[w] = ml.x;
+        lv[w] = ml.y;
+      }
+    }
+  }
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mv[w]);
+  float o = 0.f, Ls = 0.f;
+  if (M != -INFINITY) {
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
-      mv[w] = -INFINITY;
-      lv[w] = 0.f;
-      ov[w] = 0.f;
-      if (w >= w0 && w <= w1) {
-        if (pseg[w] == bg) {
-          const float* sp = reinterpret_cast<const float*>(rings + (size_t)w * kRing);
-          ov[w] = sp[h * D + d];
-          mv[w] = sp[G * D + 2 * h];
-          lv[w] = sp[G * D + 2 * h + 1];
-        } else {
-          const size_t slot = (size_t)blockIdx.x * kWarps + w + bg;
-          ov[w] = __ldcg(&a.wp_o[(slot * G + h) * D + d]);
-          const float2 ml = __ldcg(reinterpret_cast<const float2*>(&a.wp_ml[(slot * G + h) * 2]));
-          mv[w] = ml.x;
-          lv[w] = ml.y;
-        }
-      }
+      const float f = mv[w] == -INFINITY ? 0.f : exp2f(mv[w] - M);
+      o += ov[w] * f;
+      Ls += lv[w] * f;
     }
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mv[w]);
-    float o = 0.f, Ls = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float f = mv[w] == -INFINITY ? 0.f : exp2f(mv[w] - M);
-        o += ov[w] * f;
-        Ls += lv[w] * f;
-      }
-    }
-    put_merged<BF16>(a, out, lse, bg, h, d, D, M, Ls, o, a.ws_o, a.ws_ml, dst);
   }
+  put_merged<BF16>(a, out, lse, bg, h, d, D, M, Ls, o, a.ws_o, a.ws_ml, dst);
 }
 
-// Final merge of segment bg from its CTA partial slots n0 + bg .. n1 + bg into the output;
-// partials are read in batches of 8 with an online rescale (one round trip per batch).
+// Final merge of element (h, d) of segment bg from its CTA partial slots n0 + bg .. n1 + bg
+// into the output; partials are read in batches of 8 with an online rescale (one round
+// trip per batch).
 template <int D, bool BF16>
-__device__ inline void final_combine(const AttnArgs& a, uint16_t* out, float* lse, int bg, int n0, int n1) {
+__device__ inline void final_combine_elem(const AttnArgs& a, uint16_t* out, float* lse, int bg, int h, int d, int n0,
+                                          int n1) {
   constexpr int NB = 8;
   const int G = a.c.G;
-  for (int e = threadIdx.x; e < G * D; e += kThreads) {
-    const int h = e / D, d = e % D;
-    float M = -INFINITY, o = 0.f, Ls = 0.f;
-    for (int j0 = n0; j0 <= n1; j0 += NB) {
-      float mv[NB], lv[NB], ov[NB];
+  float M = -INFINITY, o = 0.f, Ls = 0.f;
+  for (int j0 = n0; j0 <= n1; j0 += NB) {
+    float mv[NB], lv[NB], ov[NB];
 #pragma unroll
-      for (int i = 0; i < NB; ++i) {
-        mv[i] = -INFINITY;
-        lv[i] = 0.f;
-        ov[i] = 0.f;
-        if (j0 + i <= n1) {
-          const size_t slot = (size_t)(j0 + i) + bg;
-          const float2 ml = __ldcg(reinterpret_cast<const float2*>(&a.ws_ml[(slot * G + h) * 2]));
-          mv[i] = ml.x;
-          lv[i] = ml.y;
-          ov[i] = __ldcg(&a.ws_o[(slot * G + h) * D + d]);
-        }
+    for (int i = 0; i < NB; ++i) {
+      mv[i] = -INFINITY;
+      lv[i] = 0.f;
+      ov[i] = 0.f;
+      if (j0 + i <= n1) {
+        const size_t slot = (size_t)(j0 + i) + bg;
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(&a.ws_ml[(slot * G + h) * 2]));
+        mv[i] = ml.x;
+        lv[i] = ml.y;
+        ov[i] = __ldcg(&a.ws_o[(slot * G + h) * D + d]);
       }
-      float Mn = M;
-#pragma unroll
-      for (int i = 0; i < NB; ++i) Mn = fmaxf(Mn, mv[i]);
-      if (Mn == -INFINITY) continue;
-      const float r = M == -INFINITY ? 0.f : exp2f(M - Mn);
-      o *= r;
-      Ls *= r;
-#pragma unroll
-      for (int i = 0; i < NB; ++i) {
-        const float f = mv[i] == -INFINITY ? 0.f : exp2f(mv[i] - Mn);
-        o += ov[i] * f;
-        Ls += lv[i] * f;
-      }
-      M = Mn;
     }
-    put_merged<BF16>(a, out, lse, bg, h, d, D, M, Ls, o, nullptr, nullptr, -1);
+    float Mn = M;
+#pragma unroll
+    for (int i = 0; i < NB; ++i) Mn = fmaxf(Mn, mv[i]);
+    if (Mn == -INFINITY) continue;
+    const float r = M == -INFINITY ? 0.f : exp2f(M - Mn);
+    o *= r;
+    Ls *= r;
+#pragma unroll
+    for (int i = 0; i < NB; ++i) {
+      const float f = mv[i] == -INFINITY ? 0.f : exp2f(mv[i] - Mn);
+      o += ov[i] * f;
+      Ls += lv[i] * f;
+    }
+    M = Mn;
   }
+  put_merged<BF16>(a, out, lse, bg, h, d, D, M, Ls, o, nullptr, nullptr, -1);
 }
 
 template <int D, bool BF16, bool ONLY16>
@@ -226,6 +221,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
   fence_proxy_async();
   __syncwarp();
 
+  // L2 prefetch of the block table and the queries, overlapping the previous kernel's
+  // tail: the page lookups after the wait then hit L2 (a prefetch is only a hint; neither
+  // array is written by the kernels this launch may overlap).
+  {
+    const size_t stride = (size_t)gridDim.x * kThreads * 128;
+    const size_t nbt = (size_t)c.B * c.max_pages * sizeof(int32_t), nq = (size_t)c.B * c.Hq * D * 2;
+    for (size_t o = ((size_t)blockIdx.x * kThreads + tid) * 128; o < nbt; o += stride)
+      prefetch_l2_line(reinterpret_cast<const unsigned char*>(c.block_table) + o);
+    for (size_t o = ((size_t)blockIdx.x * kThreads + tid) * 128; o < nq; o += stride)
+      prefetch_l2_line(reinterpret_cast<const unsigned char*>(a.q) + o);
+  }
   griddep_wait();  // the page lists and the cache come from earlier kernels
   const unsigned long long wait_ns = wait_limit_ns(a.counters, kWaitLimitWord);
 
@@ -412,43 +418,64 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
   }
   if (groups > 0) cp_async_wait_pending(0);  // no per-lane copy may land after this point
 
-  // CTA pre-merge: one partial per segment this CTA touched (written straight to the
-  // output when the segment lies inside this CTA), then the last CTA of each segment
-  // (counted arrivals; no waiting) merges those into the output.
+  // Merge, in three phases over all the segments this CTA touched at once (a CTA-wide
+  // barrier between phases, so the tail costs a few memory round trips however many
+  // segments the CTA holds):
+  //  1. per (segment, element): merge this CTA's warp partials; a segment that lies inside
+  //     the CTA goes straight to the output, others to the CTA's partial slot;
+  //  2. per segment spanning CTAs: count this CTA's arrival; the last CTA to arrive
+  //     (no waiting) resets the counter and lists the segment;
+  //  3. per (listed segment, element): merge the segment's CTA partials into the output.
   __syncthreads();
   const int cw = kWarps * W;  // pages per CTA
   const int cta0 = min(total, (int)blockIdx.x * cw), cta1 = min(total, cta0 + cw);
-  __shared__ int s_last;
+  __shared__ int s_nlast;
+  // list of the segments this CTA completes: warp 0's ring past its partial (free now)
+  int16_t* last_list = reinterpret_cast<int16_t*>(smem + 8192);
   if (cta0 < cta1) {
-    int sbg = 0;
-    {
+    auto seg_of = [&](int f) {  // last segment starting at or before flat page f
       int lo = 0, hi = BH - 1;
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (off[mid] <= cta0) lo = mid; else hi = mid - 1;
+        if (off[mid] <= f) lo = mid; else hi = mid - 1;
       }
-      sbg = lo;
-    }
-    for (; sbg < BH && off[sbg] < cta1; ++sbg) {
-      if (off[sbg + 1] <= max(cta0, off[sbg])) continue;  // empty or before the CTA
-      const int w0 = max((int)blockIdx.x * kWarps, off[sbg] / W) - (int)blockIdx.x * kWarps;
-      const int w1 = min((int)blockIdx.x * kWarps + kWarps - 1, (off[sbg + 1] - 1) / W) - (int)blockIdx.x * kWarps;
+      return lo;
+    };
+    const int s0 = seg_of(cta0), s1 = seg_of(cta1 - 1);
+    const int nseg = s1 - s0 + 1, GD = G * D;
+    const int wb = (int)blockIdx.x * kWarps;
+    for (int e = tid; e < nseg * GD; e += kThreads) {
+      const int sbg = s0 + e / GD, el = e % GD;
+      if (off[sbg + 1] == off[sbg]) continue;  // empty segment: written at the start
+      const int w0 = max(wb, off[sbg] / W) - wb;
+      const int w1 = min(wb + kWarps - 1, (off[sbg + 1] - 1) / W) - wb;
       const int n0 = off[sbg] / cw, n1 = (off[sbg + 1] - 1) / cw;
-      cta_merge<D, BF16>(a, out, lse, smem, s_pseg, sbg, w0, w1, n0 == n1 ? -1 : (int)blockIdx.x + sbg);
+      cta_merge_elem<D, BF16>(a, out, lse, smem, s_pseg, sbg, el / D, el % D, w0, w1,
+                              n0 == n1 ? -1 : (int)blockIdx.x + sbg);
+    }
+    __threadfence();  // this thread's CTA partials are visible before any arrival is counted
+    if (tid == 0) s_nlast = 0;
+    __syncthreads();
+    for (int i = tid; i < nseg; i += kThreads) {
+      const int sbg = s0 + i;
+      if (off[sbg + 1] == off[sbg]) continue;
+      const int n0 = off[sbg] / cw, n1 = (off[sbg + 1] - 1) / cw;
       if (n0 == n1) continue;  // the whole segment was in this CTA: output written
-      __syncthreads();
-      if (tid == 0) {  // the barrier orders every thread's partial writes before this fence
-        __threadfence();
-        const unsigned old = atomicAdd(&a.counters[sbg], 1u);
-        s_last = old == static_cast<unsigned>(n1 - n0);
-        if (s_last) a.counters[sbg] = 0u;  // every CTA of this segment has arrived: reset for the next call
+      const unsigned old = atomicAdd(&a.counters[sbg], 1u);
+      if (old == static_cast<unsigned>(n1 - n0)) {  // every CTA of the segment has arrived
+        a.counters[sbg] = 0u;                          // ready for the next call
+        last_list[atomicAdd(&s_nlast, 1)] = static_cast<int16_t>(sbg);
       }
-      __syncthreads();
-      if (s_last) {
-        __threadfence();
-        final_combine<D, BF16>(a, out, lse, sbg, n0, n1);
+    }
+    __syncthreads();
+    const int nl = s_nlast;
+    if (nl > 0) {
+      __threadfence();
+      for (int e = tid; e < nl * GD; e += kThreads) {
+        const int sbg = last_list[e / GD], el = e % GD;
+        const int n0 = off[sbg] / cw, n1 = (off[sbg + 1] - 1) / cw;
+        final_combine_elem<D, BF16>(a, out, lse, sbg, el / D, el % D, n0, n1);
       }
-      __syncthreads();
     }
   }
   griddep_launch_dependents();

@@ -68,6 +68,19 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
   const int total = c.B * c.Hkv * tiles_per_bg;
   const int i0 = (blockIdx.x * kScoreWarps + warp) * per;
   const int i1 = min(total, i0 + per);
+  // Before waiting for the previous kernel (the append, which writes only the open page's
+  // summary row): ask L2 for this warp's summary rows, one bulk prefetch per (b, g) piece,
+  // so their DRAM traffic overlaps that kernel (a prefetch is only a hint).
+  if (lane == 0 && i0 < i1) {
+    for (int bg = i0 / tiles_per_bg; bg <= (i1 - 1) / tiles_per_bg; ++bg) {
+      const int L = c.seq_len[bg / c.Hkv];
+      const int P = min((L + kPage - 1) / kPage, c.max_pages);
+      const int p0 = max(i0, bg * tiles_per_bg) % tiles_per_bg * 16;
+      const int p1 = min(P, (min(i1, (bg + 1) * tiles_per_bg) - bg * tiles_per_bg) * 16);
+      if (p1 > p0)
+        bulk_prefetch_l2(c.summary + ((size_t)bg * c.max_pages + p0) * D, (uint32_t)(p1 - p0) * D * 2);
+    }
+  }
   griddep_wait();
 
   if (MODE != SCORES && f.pos != nullptr && i0 < i1) {  // appends whose page lies in this warp's tiles

@@ -196,10 +196,11 @@ __device__ inline void merge_warps(const float* wp, int G, int h, int d, float& 
 
 template <bool BF16>
 __device__ inline void write_out(uint16_t* out, float* lse, size_t row, int d, int D, float M, float Ls, float o) {
-  const float r = Ls > 0.f ? o / Ls : 0.f;
+  const bool any = !(Ls <= 0.f);  // a NaN sum (a NaN key or value) gives a NaN output
+  const float r = any ? o / Ls : 0.f;
   if constexpr (BF16) out[row * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
   else out[row * D + d] = __half_as_ushort(__float2half_rn(r));
-  if (d == 0 && lse != nullptr) lse[row] = Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
+  if (d == 0 && lse != nullptr) lse[row] = any ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
 }
 
 template <int D, bool BF16>
