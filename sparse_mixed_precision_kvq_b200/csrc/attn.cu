@@ -85,54 +85,56 @@ struct PageDesc {
   int nv;
 };
 
-// Write the merged (M, L, o) of element (h, d) of segment bg: as a partial into slot `dst`
-// of (dst_o, dst_ml), or, with dst < 0, as the segment's output o / L and lse.
+// Write the merged (M, L, o) of elements (h, d .. d+3) of segment bg: as a partial into
+// slot `dst` of (dst_o, dst_ml), or, with dst < 0, as the segment's output o / L and lse.
 template <bool BF16>
-__device__ inline void put_merged(const AttnArgs& a, uint16_t* out, float* lse, int bg, int h, int d, int D, float M,
-                                  float Ls, float o, float* dst_o, float* dst_ml, int dst) {
+__device__ inline void put_merged4(const AttnArgs& a, uint16_t* out, float* lse, int bg, int h, int d, int D, float M,
+                                   float Ls, float4 o, float* dst_o, float* dst_ml, int dst) {
   const DevCache& c = a.c;
   const int G = c.G;
   if (dst >= 0) {
-    dst_o[((size_t)dst * G + h) * D + d] = o;
-    if (d == 0) {
-      dst_ml[((size_t)dst * G + h) * 2] = M;
-      dst_ml[((size_t)dst * G + h) * 2 + 1] = Ls;
-    }
+    *reinterpret_cast<float4*>(&dst_o[((size_t)dst * G + h) * D + d]) = o;
+    if (d == 0) *reinterpret_cast<float2*>(&dst_ml[((size_t)dst * G + h) * 2]) = make_float2(M, Ls);
     return;
   }
   const int b = bg / c.Hkv, g = bg % c.Hkv;
   const bool any = !(Ls <= 0.f);  // a NaN sum (a NaN key or value) gives a NaN output
-  const float r = any ? o / Ls : 0.f;
+  const float ov[4] = {o.x, o.y, o.z, o.w};
   const size_t oi = ((size_t)b * c.Hq + (size_t)g * G + h) * D + d;
-  if constexpr (BF16) out[oi] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
-  else out[oi] = __half_as_ushort(__float2half_rn(r));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float r = any ? ov[i] / Ls : 0.f;
+    if constexpr (BF16) out[oi + i] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+    else out[oi + i] = __half_as_ushort(__float2half_rn(r));
+  }
   if (d == 0 && lse != nullptr)
     lse[(size_t)b * c.Hq + (size_t)g * G + h] = any ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
 }
 
-// CTA merge of element (h, d) of segment bg: warps w0..w1 of this CTA hold one partial
-// each, in their own ring (shared memory: the warp's last segment) or in their global warp
-// slot (u + bg).  All of the element's partials are loaded before any is used: one memory
-// round trip.  The result goes to CTA partial slot `dst`, or to the output (dst < 0).
+// CTA merge of elements (h, d .. d+3) of segment bg: warps w0..w1 of this CTA hold one
+// partial each, in their own ring (shared memory: the warp's last segment) or in their
+// global warp slot (u + bg).  Every partial is loaded before any is used (one memory round
+// trip).  The result goes to CTA partial slot `dst`, or to the output (dst < 0).
 template <int D, bool BF16>
-__device__ inline void cta_merge_elem(const AttnArgs& a, uint16_t* out, float* lse, const unsigned char* rings,
-                                      const int* pseg, int bg, int h, int d, int w0, int w1, int dst) {
+__device__ inline void cta_merge4(const AttnArgs& a, uint16_t* out, float* lse, const unsigned char* rings,
+                                  const int* pseg, int bg, int h, int d, int w0, int w1, int dst) {
   const int G = a.c.G;
-  float mv[kWarps], lv[kWarps], ov[kWarps];
+  float mv[kWarps], lv[kWarps];
+  float4 ov[kWarps];
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
     mv[w] = -INFINITY;
     lv[w] = 0.f;
-    ov[w] = 0.f;
+    ov[w] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (w >= w0 && w <= w1) {
       if (pseg[w] == bg) {
         const float* sp = reinterpret_cast<const float*>(rings + (size_t)w * kRing);
-        ov[w] = sp[h * D + d];
+        ov[w] = *reinterpret_cast<const float4*>(&sp[h * D + d]);
         mv[w] = sp[G * D + 2 * h];
         lv[w] = sp[G * D + 2 * h + 1];
       } else {
         const size_t slot = (size_t)blockIdx.x * kWarps + w + bg;
-        ov[w] = __ldcg(&a.wp_o[(slot * G + h) * D + d]);
+        ov[w] = __ldcg(reinterpret_cast<const float4*>(&a.wp_o[(slot * G + h) * D + d]));
         const float2 ml = __ldcg(reinterpret_cast<const float2*>(&a.wp_ml[(slot * G + h) * 2]));
         mv[w] = ml.x;
         lv[w] = ml.y;
@@ -142,40 +144,46 @@ __device__ inline void cta_merge_elem(const AttnArgs& a, uint16_t* out, float* l
   float M = -INFINITY;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mv[w]);
-  float o = 0.f, Ls = 0.f;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  float Ls = 0.f;
   if (M != -INFINITY) {
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
       const float f = mv[w] == -INFINITY ? 0.f : exp2f(mv[w] - M);
-      o += ov[w] * f;
+      o.x += ov[w].x * f;
+      o.y += ov[w].y * f;
+      o.z += ov[w].z * f;
+      o.w += ov[w].w * f;
       Ls += lv[w] * f;
     }
   }
-  put_merged<BF16>(a, out, lse, bg, h, d, D, M, Ls, o, a.ws_o, a.ws_ml, dst);
+  put_merged4<BF16>(a, out, lse, bg, h, d, D, M, Ls, o, a.ws_o, a.ws_ml, dst);
 }
 
-// Final merge of element (h, d) of segment bg from its CTA partial slots n0 + bg .. n1 + bg
-// into the output; partials are read in batches of 8 with an online rescale (one round
-// trip per batch).
+// Final merge of elements (h, d .. d+3) of segment bg from its CTA partial slots n0 + bg ..
+// n1 + bg into the output; partials are read in batches of 8 with an online rescale (one
+// round trip per batch).
 template <int D, bool BF16>
-__device__ inline void final_combine_elem(const AttnArgs& a, uint16_t* out, float* lse, int bg, int h, int d, int n0,
-                                          int n1) {
+__device__ inline void final_combine4(const AttnArgs& a, uint16_t* out, float* lse, int bg, int h, int d, int n0,
+                                      int n1) {
   constexpr int NB = 8;
   const int G = a.c.G;
-  float M = -INFINITY, o = 0.f, Ls = 0.f;
+  float M = -INFINITY, Ls = 0.f;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int j0 = n0; j0 <= n1; j0 += NB) {
-    float mv[NB], lv[NB], ov[NB];
+    float mv[NB], lv[NB];
+    float4 ov[NB];
 #pragma unroll
     for (int i = 0; i < NB; ++i) {
       mv[i] = -INFINITY;
       lv[i] = 0.f;
-      ov[i] = 0.f;
+      ov[i] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (j0 + i <= n1) {
         const size_t slot = (size_t)(j0 + i) + bg;
         const float2 ml = __ldcg(reinterpret_cast<const float2*>(&a.ws_ml[(slot * G + h) * 2]));
         mv[i] = ml.x;
         lv[i] = ml.y;
-        ov[i] = __ldcg(&a.ws_o[(slot * G + h) * D + d]);
+        ov[i] = __ldcg(reinterpret_cast<const float4*>(&a.ws_o[(slot * G + h) * D + d]));
       }
     }
     float Mn = M;
@@ -183,17 +191,23 @@ __device__ inline void final_combine_elem(const AttnArgs& a, uint16_t* out, floa
     for (int i = 0; i < NB; ++i) Mn = fmaxf(Mn, mv[i]);
     if (Mn == -INFINITY) continue;
     const float r = M == -INFINITY ? 0.f : exp2f(M - Mn);
-    o *= r;
+    o.x *= r;
+    o.y *= r;
+    o.z *= r;
+    o.w *= r;
     Ls *= r;
 #pragma unroll
     for (int i = 0; i < NB; ++i) {
       const float f = mv[i] == -INFINITY ? 0.f : exp2f(mv[i] - Mn);
-      o += ov[i] * f;
+      o.x += ov[i].x * f;
+      o.y += ov[i].y * f;
+      o.z += ov[i].z * f;
+      o.w += ov[i].w * f;
       Ls += lv[i] * f;
     }
     M = Mn;
   }
-  put_merged<BF16>(a, out, lse, bg, h, d, D, M, Ls, o, nullptr, nullptr, -1);
+  put_merged4<BF16>(a, out, lse, bg, h, d, D, M, Ls, o, nullptr, nullptr, -1);
 }
 
 template <int D, bool BF16, bool ONLY16>
@@ -442,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
       return lo;
     };
     const int s0 = seg_of(cta0), s1 = seg_of(cta1 - 1);
-    const int nseg = s1 - s0 + 1, GD = G * D;
+    const int nseg = s1 - s0 + 1, GD = G * D / 4;  // units of 4 consecutive channels
     const int wb = (int)blockIdx.x * kWarps;
     for (int e = tid; e < nseg * GD; e += kThreads) {
       const int sbg = s0 + e / GD, el = e % GD;
@@ -450,8 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
       const int w0 = max(wb, off[sbg] / W) - wb;
       const int w1 = min(wb + kWarps - 1, (off[sbg + 1] - 1) / W) - wb;
       const int n0 = off[sbg] / cw, n1 = (off[sbg + 1] - 1) / cw;
-      cta_merge_elem<D, BF16>(a, out, lse, smem, s_pseg, sbg, el / D, el % D, w0, w1,
-                              n0 == n1 ? -1 : (int)blockIdx.x + sbg);
+      cta_merge4<D, BF16>(a, out, lse, smem, s_pseg, sbg, el / (D / 4), 4 * (el % (D / 4)), w0, w1,
+                          n0 == n1 ? -1 : (int)blockIdx.x + sbg);
     }
     __threadfence();  // this thread's CTA partials are visible before any arrival is counted
     if (tid == 0) s_nlast = 0;
@@ -474,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
       for (int e = tid; e < nl * GD; e += kThreads) {
         const int sbg = last_list[e / GD], el = e % GD;
         const int n0 = off[sbg] / cw, n1 = (off[sbg + 1] - 1) / cw;
-        final_combine_elem<D, BF16>(a, out, lse, sbg, el / D, el % D, n0, n1);
+        final_combine4<D, BF16>(a, out, lse, sbg, el / (D / 4), 4 * (el % (D / 4)), n0, n1);
       }
     }
   }
@@ -527,9 +541,10 @@ int attn_num_ctas(int device) {
 }
 
 // Workspace: [kCounterBytes] per-segment arrival counters (zero between calls, at a fixed
-// place so that any later call, whatever its shapes, finds them zero), then the warp
-// partials ([wslots][G][D] o, [wslots][G][2] (m, l); wslots = warps + B*Hkv) and the CTA
-// partials ([slots][G][D], [slots][G][2]; slots = CTAs + B*Hkv).  A warp (CTA) u that
+// place so that any later call, whatever its shapes, finds them zero), then the o parts of
+// the warp partials ([wslots][G][D]; wslots = warps + B*Hkv) and of the CTA partials
+// ([slots][G][D]; slots = CTAs + B*Hkv), then their (m, l) parts ([wslots][G][2],
+// [slots][G][2]).  A warp (CTA) u that
 // covers segment bg writes slot u + bg: unique because ranges are contiguous and ordered.
 size_t attn_workspace_bytes(const DevCache& c, int num_ctas) {
   const size_t BH = (size_t)c.B * c.Hkv;
@@ -550,9 +565,9 @@ cudaError_t launch_attn(const DevCache& c, const void* q, const int32_t* sel, co
   const size_t wslots = (size_t)num_ctas * kWarps + BH, slots = (size_t)num_ctas + BH;
   a.counters = static_cast<unsigned*>(ws);
   a.wp_o = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + kCounterBytes);
-  a.wp_ml = a.wp_o + wslots * c.G * c.D;
-  a.ws_o = a.wp_ml + wslots * c.G * 2;
-  a.ws_ml = a.ws_o + slots * c.G * c.D;
+  a.ws_o = a.wp_o + wslots * c.G * c.D;  // o arrays first: every row 16-byte aligned
+  a.wp_ml = a.ws_o + slots * c.G * c.D;
+  a.ws_ml = a.wp_ml + wslots * c.G * 2;
   a.num_ctas = num_ctas;
   uint16_t* o = static_cast<uint16_t*>(out);
   const bool bf = c.dtype == KVQ_DT_BF16;
