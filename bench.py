@@ -23,8 +23,8 @@ max time over ranks is used.  Rank 0 prints one JSON line.
 
 Options: ``--score quad`` scores pages with the quad (Gaussian-MGF) score; ``--coverage``
 selects by page-mass coverage; ``--tier T`` stores every prefilled page at tier T;
-``--host-tiers M`` keeps the pools of mask M in pinned host memory (the line gains a
-``host_link`` object); ``--demote T`` also times kvq_requantize_pages moving the
+``--host-tiers M`` keeps the pools of mask M in pinned host memory and ``--host-v-tiers M``
+only their V chunks, K staying on the device (the line gains a ``host_link`` object); ``--demote T`` also times kvq_requantize_pages moving the
 workload's pages to tier T (a ``demotion`` object).
 
 ``--impl reference`` times the CPU oracle (the plain fp64 restatement of the method)
@@ -413,7 +413,8 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     basis = None
     if quad_rank:
         basis = np.stack([w.quad_basis(g, quad_rank, "law") for g in range(w.Hkv)])
-    cache = kvq.cache_from_workload(w, device=dev, quad_basis=basis, host_tiers=args.host_tiers)
+    cache = kvq.cache_from_workload(w, device=dev, quad_basis=basis, host_tiers=args.host_tiers,
+                                    host_v_tiers=args.host_v_tiers)
     step = kvq.DecodeStep(w, cache, device=dev, coverage=args.coverage, quad=bool(quad_rank))
     m = measure(w, cache, step, args.path, args.steps, args.warmup, flush, stream, dev, world, peak,
                 quad_rank=quad_rank, soak_s=args.soak_s if rank == 0 else 0.0)
@@ -429,9 +430,9 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     tr = kernel_traffic(files[dom])
     sel, cnt, tier_tbl = m["sel"], m["cnt"], m["tier_tbl"]
     host = None
-    if args.host_tiers:
+    if args.host_tiers or args.host_v_tiers:
         host = host_link(w, sel, cnt, tier_tbl, args.host_tiers, avg[names.index("sparse_decode_attn")]
-                         if "sparse_decode_attn" in names else None, dev)
+                         if "sparse_decode_attn" in names else None, dev, vmask=args.host_v_tiers)
     demotion = None
     if args.demote is not None:
         del step, cache
@@ -471,7 +472,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
                    "selected_pages": int(cnt.sum()),
                    "selection": "budget" if args.coverage is None else f"coverage {args.coverage}",
                    "tiers": "the workload's" if args.tier is None else f"every prefilled page at tier {args.tier}",
-                   "host_tiers": args.host_tiers,
+                   "host_tiers": args.host_tiers, "host_v_tiers": args.host_v_tiers,
                    "page_score": "mean-key" if not quad_rank else
                    f"quad (rank {quad_rank}, basis: eigenvectors of the key law's covariance)",
                    "l2": f"flushed ({args.flush_mib} MiB write) before every timed step",
@@ -542,17 +543,19 @@ def time_dense(w, cache, step, flush, stream, dev, reps=20):
     return float(np.mean(ts))
 
 
-def host_link(w, sel, cnt, tier_tbl, mask: int, attn_ms, dev, reps: int = 5):
-    """The attention's bytes read from pinned host memory, their rate over the kernel's
+def host_link(w, sel, cnt, tier_tbl, mask: int, attn_ms, dev, reps: int = 5, vmask: int = 0):
+    """The attention's bytes read from pinned host memory (K and V chunks of the pools in
+    ``mask``, V chunks of the V pools in ``vmask``), their rate over the kernel's
     event-timed duration, against a pinned host -> device copy of 512 MiB timed here."""
     import torch
     from sparse_mixed_precision_kvq_b200.kvq import kvq_chunk_bytes
-    cb = np.array([2 * kvq_chunk_bytes(t, w.D) for t in range(6)], dtype=np.int64)
+    cb = np.array([kvq_chunk_bytes(t, w.D) for t in range(6)], dtype=np.int64)
     host = 0
     for b in range(w.B):
         for g in range(w.Hkv):
-            tiers = tier_tbl[b, sel[b, g, :cnt[b, g]]]
-            host += int(sum(cb[t] for t in tiers if (mask >> int(t)) & 1))
+            for t in tier_tbl[b, sel[b, g, :cnt[b, g]]]:
+                t = int(t)
+                host += int(2 * cb[t] if (mask >> t) & 1 else (cb[t] if (vmask >> t) & 1 else 0))
     src = torch.empty(512 << 20, dtype=torch.uint8, pin_memory=True)
     dst = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     ts = []
@@ -565,7 +568,7 @@ def host_link(w, sel, cnt, tier_tbl, mask: int, attn_ms, dev, reps: int = 5):
         if r:
             ts.append(a.elapsed_time(b_))
     peak = (512 << 20) / (np.mean(ts) * 1e-3) / 1e9
-    out = {"mask": mask, "attn_host_bytes": host, "h2d_copy_gbs": peak,
+    out = {"mask": mask, "v_mask": vmask, "attn_host_bytes": host, "h2d_copy_gbs": peak,
            "peak_kind": "pinned host -> device copy of 512 MiB, timed in this run"}
     if attn_ms:
         out.update(achieved_gbs=host / (attn_ms * 1e-3) / 1e9, frac=host / (attn_ms * 1e-3) / 1e9 / peak)
@@ -737,6 +740,9 @@ def main():
                     help="store every prefilled page at this tier (0 16-bit, 1 int8, 2 int4, 3 int2, 4 1-bit, 5 fp8)")
     ap.add_argument("--host-tiers", type=int, default=0,
                     help="bit t: pool t lives in pinned host memory that the kernels read in place (DRAM value tier)")
+    ap.add_argument("--host-v-tiers", type=int, default=0,
+                    help="bit t: the V chunks of tier t live in their own pool in pinned host memory, the K chunks "
+                         "on the device (the mem-v variant of the DRAM value tier)")
     ap.add_argument("--dense", action="store_true", default=None,
                     help="also time attention over every page (on by default for c1)")
     ap.add_argument("--no-dense", action="store_true")
@@ -758,13 +764,14 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.coverage is not None and args.path != "calls":
         ap.error("--coverage runs on the four-call path")
-    if args.host_tiers and args.path == "fused":
-        ap.error("--host-tiers: the fused step reads pages by bulk copies only")
+    if (args.host_tiers or args.host_v_tiers) and args.path == "fused":
+        ap.error("--host-tiers / --host-v-tiers: the fused step reads adjacent device chunks only")
     if args.score == "quad" and args.path not in ("calls", "three"):
         ap.error("--score quad runs on the four-call or the three-call path")
     if args.dense is None:
         args.dense = args.config == "c1"
-    special = (args.coverage is not None or args.tier is not None or args.host_tiers or args.score != "mean"
+    special = (args.coverage is not None or args.tier is not None or args.host_tiers or args.host_v_tiers
+               or args.score != "mean"
                or args.batch is not None or args.demote is not None)
     if special and args.configs == "c2,c3,c4":
         args.configs = "none"   # the other workloads are measured on plain runs only

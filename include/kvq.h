@@ -124,6 +124,15 @@ typedef struct {
   uint16_t* summary;       /* device [B][Hkv][max_pages][D] fp16 bits, 16-byte aligned */
   double* open_ksum;       /* device [B][Hkv][D] */
   uint32_t* err_word;      /* device, 1 word */
+  void* vpool[6];          /* optional, per tier: a separate pool of V chunks (NULL: V chunks sit
+                              next to the K chunks in pool[t]).  When set, pool[t] holds the K
+                              chunk of (slot, kv head g) at byte (slot*Hkv + g) * chunk and
+                              vpool[t] its V chunk at the same offset; both have pool_slots[t]
+                              slots.  16-byte aligned. */
+  int32_t host_vtiers;     /* bit t set: vpool[t] is pinned host memory mapped into the device
+                              address space (AMASS "What is in the box", Stage B, the "mem-v"
+                              variant: values in host DRAM, keys resident on the device) */
+  int32_t reserved0;       /* must be 0 */
 } kvq_cache;
 
 typedef struct {

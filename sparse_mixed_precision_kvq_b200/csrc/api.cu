@@ -12,9 +12,9 @@ __global__ void dequant_kernel(DevCache c, int b, int page, float* __restrict__ 
   const int g = blockIdx.x >> 1, kind = blockIdx.x & 1;
   const int D = c.D;
   int tier;
-  const unsigned char* ck;
-  if (!page_chunk(c, b, page, g, tier, ck)) return;
-  const unsigned char* chunk = ck + (size_t)kind * c.chunk[tier];
+  const unsigned char *ck, *cv;
+  if (!page_chunks(c, b, page, g, tier, ck, cv)) return;
+  const unsigned char* chunk = kind ? cv : ck;
   for (int e = threadIdx.x; e < kPage * D; e += blockDim.x) {
     const int t = e / D, d = e % D;
     out[(((size_t)g * 2 + kind) * kPage + t) * D + d] = load_value(chunk, kind, tier, D, c.dtype == KVQ_DT_BF16, t, d);
@@ -46,7 +46,13 @@ kvq_status to_dev(const kvq_cache* k, DevCache& c) {
   c.block_table = k->block_table;
   c.seq_len = k->seq_len;
   bool any = false;
+  if (static_cast<uint32_t>(k->host_vtiers) >> kNumTiers || k->reserved0 != 0) return KVQ_ERR_INVALID_ARG;
+  c.host_vtiers = static_cast<uint32_t>(k->host_vtiers);
   for (int t = 0; t < kNumTiers; ++t) {
+    c.vpool[t] = static_cast<unsigned char*>(k->vpool[t]);
+    if (k->vpool[t] && (k->pool[t] == nullptr || reinterpret_cast<uintptr_t>(k->vpool[t]) % 16 != 0))
+      return KVQ_ERR_INVALID_ARG;
+    if (((c.host_vtiers >> t) & 1u) && k->vpool[t] == nullptr) return KVQ_ERR_INVALID_ARG;
     c.pool[t] = static_cast<unsigned char*>(k->pool[t]);
     c.pool_slots[t] = k->pool[t] ? k->pool_slots[t] : 0;
     c.chunk[t] = chunk_bytes(t, k->D);

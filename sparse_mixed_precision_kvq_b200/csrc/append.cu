@@ -64,9 +64,8 @@ __global__ void __launch_bounds__(128) build_kernel(DevCache c, const uint16_t* 
     return;
   }
   int tier;
-  const unsigned char* ck;
-  if (!page_chunk(c, b, p, g, tier, ck)) return;
-  unsigned char* out = const_cast<unsigned char*>(ck);
+  const unsigned char *ck, *cv;
+  if (!page_chunks(c, b, p, g, tier, ck, cv)) return;
   const int CB = c.chunk[tier];
 
   __shared__ __align__(16) uint32_t words[2][1024];  // chunk images (<= 4 KB each at D <= 128)
@@ -121,7 +120,7 @@ __global__ void __launch_bounds__(128) build_kernel(DevCache c, const uint16_t* 
   __syncthreads();
   for (int kind = 0; kind < 2; ++kind) {
     const uint4* src = reinterpret_cast<const uint4*>(words[kind]);
-    uint4* dst = reinterpret_cast<uint4*>(out + (size_t)kind * CB);
+    uint4* dst = reinterpret_cast<uint4*>(const_cast<unsigned char*>(kind ? cv : ck));
     for (int i = tid; i < CB / 16; i += blockDim.x) dst[i] = src[i];
   }
   if (ov) set_err(c.err, KVQ_DERR_FP16_RANGE);
@@ -218,11 +217,11 @@ __device__ inline void rq_decode(const uint32_t* oldw, int n, float (*vals)[kRqG
 
 template <int NT, int D>
 __device__ inline void rq_quant(int gid, int n, const float (*vals)[kRqGroups + 1], unsigned char* codes8,
-                                unsigned char* dst, bool& ov, bool& nonfinite) {
-  constexpr int ng = D / kGroup, NB = chunk_bytes(NT, D);
+                                unsigned char* dstK, unsigned char* dstV, bool& ov, bool& nonfinite) {
+  constexpr int ng = D / kGroup;
   const int kind = gid / (kPage * ng), t = (gid / ng) % kPage, grp = gid % ng;
   uint4* crow = reinterpret_cast<uint4*>(codes8 + (kind * kPage + t) * D + grp * kGroup);
-  unsigned char* meta = dst + kind * NB + codes_bytes(NT, D);
+  unsigned char* meta = (kind ? dstV : dstK) + codes_bytes(NT, D);
   if (t >= n) {  // token slot past the sequence: zero codes and metadata
     crow[0] = crow[1] = make_uint4(0, 0, 0, 0);
     if constexpr (NT == KVQ_TIER_I1 || NT == KVQ_TIER_F8) reinterpret_cast<uint16_t*>(meta)[t * ng + grp] = 0;
@@ -327,12 +326,11 @@ __device__ inline void rq_pack_kind(const unsigned char* codes8, uint32_t* d32, 
 }
 
 template <int NT, int D>
-__device__ inline void rq_pack(const unsigned char* codes8, unsigned char* dst) {
-  constexpr int wpk = codes_bytes(NT, D) / 4, cw = chunk_bytes(NT, D) / 4;
+__device__ inline void rq_pack(const unsigned char* codes8, unsigned char* dstK, unsigned char* dstV) {
+  constexpr int wpk = codes_bytes(NT, D) / 4;
   using Seq = std::make_integer_sequence<int, (wpk + 127) / 128>;
-  uint32_t* d32 = reinterpret_cast<uint32_t*>(dst);
-  rq_pack_kind<NT, 0, D>(codes8, d32, Seq{});
-  rq_pack_kind<NT, 1, D>(codes8 + kPage * D, d32 + cw, Seq{});
+  rq_pack_kind<NT, 0, D>(codes8, reinterpret_cast<uint32_t*>(dstK), Seq{});
+  rq_pack_kind<NT, 1, D>(codes8 + kPage * D, reinterpret_cast<uint32_t*>(dstV), Seq{});
 }
 
 template <bool BF16, int D>
@@ -346,14 +344,18 @@ __global__ void __launch_bounds__(128) requant_kernel(DevCache c, const int32_t*
   }
   const int ot = static_cast<int>(oe >> 29), nt = static_cast<int>(ne >> 29);
   const int OB = chunk_bytes(ot, D), NB = chunk_bytes(nt, D);
-  const unsigned char* src = c.pool[ot] + ((size_t)(oe & 0x1FFFFFFFu) * c.Hkv + g) * 2 * (size_t)OB;
-  unsigned char* dst = c.pool[nt] + ((size_t)(ne & 0x1FFFFFFFu) * c.Hkv + g) * 2 * (size_t)NB;
+  const unsigned char *srcK, *srcV, *dK, *dV;
+  slot_chunks(c, ot, oe & 0x1FFFFFFFu, g, srcK, srcV);
+  slot_chunks(c, nt, ne & 0x1FFFFFFFu, g, dK, dV);
+  unsigned char* dstK = const_cast<unsigned char*>(dK);
+  unsigned char* dstV = const_cast<unsigned char*>(dV);
 
   __shared__ __align__(16) uint32_t old_words[2 * chunk_bytes(KVQ_TIER_16, 128) / 4];
   __shared__ float vals[kGroup][kRqGroups + 1];
   __shared__ __align__(16) unsigned char codes8[2 * kPage * 128];
   for (int k = tid; k < 2 * OB / 16; k += blockDim.x)
-    reinterpret_cast<uint4*>(old_words)[k] = __ldcg(reinterpret_cast<const uint4*>(src) + k);
+    reinterpret_cast<uint4*>(old_words)[k] =
+        __ldcg(k < OB / 16 ? reinterpret_cast<const uint4*>(srcK) + k : reinterpret_cast<const uint4*>(srcV) + (k - OB / 16));
   __syncthreads();
   switch (ot) {
     case 0: rq_decode<0, D, BF16>(old_words, n, vals); break;
@@ -367,20 +369,20 @@ __global__ void __launch_bounds__(128) requant_kernel(DevCache c, const int32_t*
   bool ov = false, nonfinite = false;
   if (tid < 2 * kPage * (D / kGroup)) {
     switch (nt) {
-      case 1: rq_quant<1, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
-      case 2: rq_quant<2, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
-      case 3: rq_quant<3, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
-      case 4: rq_quant<4, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
-      default: rq_quant<5, D>(tid, n, vals, codes8, dst, ov, nonfinite); break;
+      case 1: rq_quant<1, D>(tid, n, vals, codes8, dstK, dstV, ov, nonfinite); break;
+      case 2: rq_quant<2, D>(tid, n, vals, codes8, dstK, dstV, ov, nonfinite); break;
+      case 3: rq_quant<3, D>(tid, n, vals, codes8, dstK, dstV, ov, nonfinite); break;
+      case 4: rq_quant<4, D>(tid, n, vals, codes8, dstK, dstV, ov, nonfinite); break;
+      default: rq_quant<5, D>(tid, n, vals, codes8, dstK, dstV, ov, nonfinite); break;
     }
   }
   __syncthreads();
   switch (nt) {
-    case 1: rq_pack<1, D>(codes8, dst); break;
-    case 2: rq_pack<2, D>(codes8, dst); break;
-    case 3: rq_pack<3, D>(codes8, dst); break;
-    case 4: rq_pack<4, D>(codes8, dst); break;
-    default: rq_pack<5, D>(codes8, dst); break;
+    case 1: rq_pack<1, D>(codes8, dstK, dstV); break;
+    case 2: rq_pack<2, D>(codes8, dstK, dstV); break;
+    case 3: rq_pack<3, D>(codes8, dstK, dstV); break;
+    case 4: rq_pack<4, D>(codes8, dstK, dstV); break;
+    default: rq_pack<5, D>(codes8, dstK, dstV); break;
   }
   if (ov) set_err(c.err, KVQ_DERR_FP16_RANGE);
   if (nonfinite) set_err(c.err, KVQ_DERR_NONFINITE);

@@ -80,7 +80,8 @@ struct AttnArgs {
 // i-th next page, so the dependent loads (page list -> block table) are paid once per
 // 32 pages instead of once per page.
 struct PageDesc {
-  const unsigned char* src;
+  const unsigned char* src;   // K chunk
+  const unsigned char* vsrc;  // V chunk (right after K unless the tier has a separate V pool)
   int tier;  // -1: skip
   int nv;
 };
@@ -300,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
   int groups = 0;                // per-lane copy groups committed (host-memory pages)
   int head = 0, tail = 0;        // monotonic ring byte counters
   int win_base = 0, win_n = 0;   // descriptor window: pages [f0 + win_base, f0 + win_base + win_n)
-  PageDesc my{nullptr, -1, 0};
+  PageDesc my{nullptr, nullptr, -1, 0};
   bool failed = false;
   const unsigned char* ring_c = ring;
 
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
   auto prefetch = [&]() {
     win_base = issued;
     win_n = min(32, (f1 - f0) - issued);
-    my = PageDesc{nullptr, -1, 0};
+    my = PageDesc{nullptr, nullptr, -1, 0};
     if (lane < win_n) {
       const int f = f0 + issued + lane;
       int lo = 0, hi = BH - 1;  // last bg with off[bg] <= f
@@ -323,9 +324,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
       const int P = min((L + kPage - 1) / kPage, c.max_pages);
       if (p >= 0 && p < P) {
         int tier;
-        const unsigned char* src;
-        if (page_chunk(c, b, p, g, tier, src)) {
+        const unsigned char *src, *vsrc;
+        if (page_chunks(c, b, p, g, tier, src, vsrc)) {
           my.src = src;
+          my.vsrc = vsrc;
           my.tier = tier;
           my.nv = min(kPage, L - p * kPage);
         }
@@ -340,28 +342,43 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
       if (issued == win_base + win_n) prefetch();
       const int k = issued - win_base;
       const unsigned long long sp = __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my.src), k);
+      const unsigned long long vp = __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my.vsrc), k);
       const int tier = __shfl_sync(0xffffffffu, my.tier, k);
       const int nv = __shfl_sync(0xffffffffu, my.nv, k);
-      const int bytes = tier >= 0 ? 2 * c.chunk[tier] : 0;
+      const int cb = tier >= 0 ? c.chunk[tier] : 0;
+      const int bytes = 2 * cb;
       int start = head;
       const int pos = head % kRing;
       if (pos + bytes > kRing) start += kRing - pos;
       if (start + bytes - tail > kRing) break;  // no room yet
       const int slot = issued % kNBar;
       const uint32_t bar = smem_u32(&bars[slot]);
-      const bool host = bytes > 0 && ((c.host_tiers >> tier) & 1u);
-      if (host) {  // pinned host memory: every lane copies its 16-byte pieces, one group per page
-        const unsigned char* src = reinterpret_cast<const unsigned char*>(sp);
-        const uint32_t dst = smem_u32(ring + start % kRing);
-        for (int o = lane * 16; o < bytes; o += 32 * 16) cp_async16(dst + o, src + o);
+      // K and V chunks of a pool in pinned host memory are fetched by every lane with
+      // 16-byte asynchronous loads (one commit group per page); device chunks by bulk copy
+      const bool khost = bytes > 0 && ((c.host_tiers >> tier) & 1u);
+      const bool vhost = bytes > 0 && (c.vpool[tier] != nullptr ? ((c.host_vtiers >> tier) & 1u) != 0u : khost);
+      const bool host = khost || vhost;
+      const uint32_t dst = smem_u32(ring + start % kRing);
+      if (host) {
+        const unsigned char* ks = reinterpret_cast<const unsigned char*>(sp);
+        const unsigned char* vs = reinterpret_cast<const unsigned char*>(vp);
+        if (khost)
+          for (int o = lane * 16; o < cb; o += 32 * 16) cp_async16(dst + o, ks + o);
+        if (vhost)
+          for (int o = lane * 16; o < cb; o += 32 * 16) cp_async16(dst + cb + o, vs + o);
         cp_async_commit();
       }
       if (lane == 0) {
         pmeta[slot] = PageMeta{start % kRing, start + bytes, tier, nv, host ? groups : -1};
-        if (bytes > 0 && !host) {
-          mbar_expect_tx(bar, static_cast<uint32_t>(bytes));
-          bulk_copy_g2s(smem_u32(ring + start % kRing), reinterpret_cast<const void*>(sp),
-                        static_cast<uint32_t>(bytes), bar);
+        const uint32_t tx = (khost ? 0u : (uint32_t)cb) + (vhost ? 0u : (uint32_t)cb);
+        if (bytes > 0 && tx > 0) {
+          mbar_expect_tx(bar, tx);
+          if (!host && vp == sp + (unsigned long long)cb) {  // adjacent K and V: one copy
+            bulk_copy_g2s(dst, reinterpret_cast<const void*>(sp), (uint32_t)bytes, bar);
+          } else {
+            if (!khost) bulk_copy_g2s(dst, reinterpret_cast<const void*>(sp), (uint32_t)cb, bar);
+            if (!vhost) bulk_copy_g2s(dst + cb, reinterpret_cast<const void*>(vp), (uint32_t)cb, bar);
+          }
         } else {
           mbar_arrive(bar);
         }

@@ -49,6 +49,8 @@ struct DevCache {
   const int32_t* block_table;
   const int32_t* seq_len;
   unsigned char* pool[kNumTiers];
+  unsigned char* vpool[kNumTiers];  // separate V chunks of a tier (nullptr: V next to K in pool)
+  uint32_t host_vtiers;             // bit t: vpool t is pinned host memory
   long long pool_slots[kNumTiers];
   int chunk[kNumTiers];  // chunk bytes per tier
   uint16_t* summary;
@@ -159,9 +161,24 @@ __device__ inline void set_err(uint32_t* err, uint32_t bits) {
   if (err) atomicOr(err, bits);
 }
 
-// Decode a block-table entry; false (and an error bit) if tier or slot is invalid.
-__device__ inline bool page_chunk(const DevCache& c, int b, int p, int g, int& tier,
-                                  const unsigned char*& chunkK) {
+// K and V chunks of (slot, kv head g) in tier `tier`: adjacent in pool[tier], or, with a
+// separate V pool, at the same offset in pool[tier] and vpool[tier].
+__device__ inline void slot_chunks(const DevCache& c, int tier, long long slot, int g, const unsigned char*& chunkK,
+                                   const unsigned char*& chunkV) {
+  const size_t i = (size_t)slot * c.Hkv + g, cb = (size_t)c.chunk[tier];
+  if (c.vpool[tier] != nullptr) {
+    chunkK = c.pool[tier] + i * cb;
+    chunkV = c.vpool[tier] + i * cb;
+  } else {
+    chunkK = c.pool[tier] + 2 * i * cb;
+    chunkV = chunkK + cb;
+  }
+}
+
+// Decode a block-table entry into the page's K and V chunks; false (and an error bit) if
+// tier or slot is invalid.
+__device__ inline bool page_chunks(const DevCache& c, int b, int p, int g, int& tier, const unsigned char*& chunkK,
+                                   const unsigned char*& chunkV) {
   const uint32_t e = static_cast<uint32_t>(c.block_table[(size_t)b * c.max_pages + p]);
   tier = static_cast<int>(e >> 29);
   const long long slot = static_cast<long long>(e & 0x1FFFFFFFu);
@@ -169,7 +186,7 @@ __device__ inline bool page_chunk(const DevCache& c, int b, int p, int g, int& t
     set_err(c.err, KVQ_DERR_BAD_PAGE);
     return false;
   }
-  chunkK = c.pool[tier] + ((size_t)(slot * c.Hkv + g) * 2) * (size_t)c.chunk[tier];
+  slot_chunks(c, tier, slot, g, chunkK, chunkV);
   return true;
 }
 

@@ -92,8 +92,8 @@ __device__ inline bool append_phase1(const DevCache& c, int b, int g, int pos, c
   const size_t bg = (size_t)b * c.Hkv + g;
   const int page = pos / kPage, t = pos % kPage;
   int tier;
-  const unsigned char* ck;
-  if (!page_chunk(c, b, page, g, tier, ck)) return false;
+  const unsigned char *ck, *cv;
+  if (!page_chunks(c, b, page, g, tier, ck, cv)) return false;
   bool ov = false;
   for (int d = t0; d < D; d += nt) {  // running key sum of the open page and its summary
     const double x = to_double<BF16>(krow[d]);
@@ -106,9 +106,10 @@ __device__ inline bool append_phase1(const DevCache& c, int b, int g, int pos, c
   }
   if (ov) set_err(c.err, KVQ_DERR_FP16_RANGE);
   if (t == 0) {  // a newly opened page starts from zero bytes
-    uint4* p4 = reinterpret_cast<uint4*>(const_cast<unsigned char*>(ck));
-    const int n16 = 2 * c.chunk[tier] / 16;
-    for (int i = t0; i < n16; i += nt) p4[i] = make_uint4(0, 0, 0, 0);
+    uint4* k4 = reinterpret_cast<uint4*>(const_cast<unsigned char*>(ck));
+    uint4* v4 = reinterpret_cast<uint4*>(const_cast<unsigned char*>(cv));
+    const int n16 = c.chunk[tier] / 16;
+    for (int i = t0; i < 2 * n16; i += nt) (i < n16 ? k4[i] : v4[i - n16]) = make_uint4(0, 0, 0, 0);
   }
   return true;
 }
@@ -119,14 +120,14 @@ __device__ inline bool append_phase2(const DevCache& c, int b, int g, int pos, c
   const int D = c.D;
   const int page = pos / kPage, t = pos % kPage;
   int tier;
-  const unsigned char* ck;
-  if (!page_chunk(c, b, page, g, tier, ck)) return false;
+  const unsigned char *ck, *cv;
+  if (!page_chunks(c, b, page, g, tier, ck, cv)) return false;
   bool ov = false, nonfinite = false;
   const int ng = D / kGroup;
   for (int gi = w; gi < 2 * ng; gi += nw) {
     const int kind = gi / ng, grp = gi % ng;
     const int d = grp * kGroup + lane;
-    unsigned char* chunk = const_cast<unsigned char*>(ck) + (kind ? c.chunk[tier] : 0);
+    unsigned char* chunk = const_cast<unsigned char*>(kind ? cv : ck);
     const uint16_t v = (kind ? vrow : krow)[d];
     const double x = to_double<BF16>(v);
     nonfinite |= !isfinite(x);

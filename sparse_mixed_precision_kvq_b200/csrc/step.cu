@@ -415,9 +415,9 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(StepArgs a) {
         const int p = __ldcg(&a.sel[(size_t)it.u * a.kmax + it.p0 + lane]);
         it.pg = p;
         if (p >= 0 && p < P) {
-          const unsigned char* s_;
+          const unsigned char *s_, *v_;
           int tier;
-          if (page_chunk(c, it.b, p, it.g, tier, s_)) {
+          if (page_chunks(c, it.b, p, it.g, tier, s_, v_)) {
             it.psrc = s_;
             it.tier = tier;
             it.nv = min(kPage, L - p * kPage);
@@ -772,6 +772,8 @@ size_t attn_items_bound(const DevCache& c, int kmax) {
 
 bool step_supported(const DevCache& c) {
   if (c.host_tiers != 0) return false;  // its pages are fetched by bulk copies only
+  for (int t = 0; t < kNumTiers; ++t)
+    if (c.vpool[t] != nullptr) return false;  // ... of adjacent K and V chunks
   if ((long long)c.B * c.Hkv * 2 + kCtlWords > (long long)kWaitLimitWord) return false;
   return step_plan(c).ns >= kCW;
 }

@@ -46,7 +46,7 @@ class KvqCache(ctypes.Structure):
                 ("page_size", c_int32), ("max_pages", c_int32), ("dtype", c_int32), ("host_tiers", c_int32),
                 ("block_table", c_void_p), ("seq_len", c_void_p), ("pool", c_void_p * 6),
                 ("pool_slots", c_int64 * 6), ("summary", c_void_p), ("open_ksum", c_void_p),
-                ("err_word", c_void_p)]
+                ("err_word", c_void_p), ("vpool", c_void_p * 6), ("host_vtiers", c_int32), ("reserved0", c_int32)]
 
 
 class SelectParams(ctypes.Structure):
@@ -243,9 +243,15 @@ def encode_block_table(tier_tbl: np.ndarray, slot_tbl: np.ndarray) -> np.ndarray
 
 
 class PagedCache:
-    """Device tensors of a paged cache plus the ``kvq_cache`` struct pointing at them."""
+    """Device tensors of a paged cache plus the ``kvq_cache`` struct pointing at them.
 
-    def __init__(self, B, Hq, Hkv, D, max_pages, dtype: str, pool_slots, device="cuda", host_tiers: int = 0):
+    ``host_tiers`` (bit t): pool t -- K and V chunks -- in pinned host memory.
+    ``v_tiers`` (bit t): tier t keeps its V chunks in a pool of their own; ``host_v_tiers``
+    (bit t, implies the v_tiers bit): that V pool in pinned host memory while the K pool
+    stays on the device (the "mem-v" variant of a host-DRAM value tier)."""
+
+    def __init__(self, B, Hq, Hkv, D, max_pages, dtype: str, pool_slots, device="cuda", host_tiers: int = 0,
+                 v_tiers: int = 0, host_v_tiers: int = 0):
         import torch
         self.B, self.Hq, self.Hkv, self.D, self.max_pages = B, Hq, Hkv, D, max_pages
         self.dtype = dtype
@@ -255,17 +261,28 @@ class PagedCache:
         self.block_table = torch.full((B, max_pages), -1, dtype=torch.int32, device=dev)
         self.seq_len = torch.zeros(B, dtype=torch.int32, device=dev)
         self.pool_slots = [int(x) for x in pool_slots] + [0] * (6 - len(pool_slots))
-        self.pools = []
+        self.pools, self.vpools = [], []
         self.host_tiers = int(host_tiers)
+        self.host_v_tiers = int(host_v_tiers)
+        self.v_tiers = int(v_tiers) | self.host_v_tiers
+
+        def alloc(nbytes, host):  # pinned host memory is read by the device in place
+            if host:
+                return torch.zeros(nbytes, dtype=torch.uint8, pin_memory=True)
+            return torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+
         for tier, n in enumerate(self.pool_slots):
-            if n > 0:
-                nbytes = n * Hkv * 2 * kvq_chunk_bytes(tier, D)
-                if (self.host_tiers >> tier) & 1:  # pinned host memory, read by the device in place
-                    self.pools.append(torch.zeros(nbytes, dtype=torch.uint8, pin_memory=True))
-                else:
-                    self.pools.append(torch.zeros(nbytes, dtype=torch.uint8, device=dev))
-            else:
+            if n <= 0:
                 self.pools.append(None)
+                self.vpools.append(None)
+                continue
+            cb = n * Hkv * kvq_chunk_bytes(tier, D)
+            if (self.v_tiers >> tier) & 1:
+                self.pools.append(alloc(cb, (self.host_tiers >> tier) & 1))
+                self.vpools.append(alloc(cb, (self.host_v_tiers >> tier) & 1))
+            else:
+                self.pools.append(alloc(2 * cb, (self.host_tiers >> tier) & 1))
+                self.vpools.append(None)
         self.summary = torch.zeros((B, Hkv, max_pages, D), dtype=torch.float16, device=dev)
         self.open_ksum = torch.zeros((B, Hkv, D), dtype=torch.float64, device=dev)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -278,7 +295,9 @@ class PagedCache:
         s.block_table, s.seq_len = _ptr(self.block_table), _ptr(self.seq_len)
         for i in range(6):
             s.pool[i] = _ptr(self.pools[i]) if self.pools[i] is not None else None
+            s.vpool[i] = _ptr(self.vpools[i]) if self.vpools[i] is not None else None
             s.pool_slots[i] = self.pool_slots[i]
+        s.host_vtiers = self.host_v_tiers
         s.summary, s.open_ksum, s.err_word = _ptr(self.summary), _ptr(self.open_ksum), _ptr(self.err)
 
     def ref(self):
@@ -288,13 +307,16 @@ class PagedCache:
         return int(self.err.item()) & 0xFFFFFFFF
 
     def pool_bytes(self) -> int:
-        return sum(p.numel() for p in self.pools if p is not None)
+        return sum(p.numel() for p in self.pools + self.vpools if p is not None)
 
     def chunk_view(self, b: int, page: int, g: int, kind: int):
         """Bytes (uint8 tensor view) of one chunk of logical page ``page`` (host-side lookup)."""
         e = int(self.block_table[b, page].item()) & 0xFFFFFFFF
         tier, slot = e >> 29, e & 0x1FFFFFFF
         cb = kvq_chunk_bytes(tier, self.D)
+        if self.vpools[tier] is not None:
+            o = (slot * self.Hkv + g) * cb
+            return tier, (self.vpools[tier] if kind else self.pools[tier])[o:o + cb]
         o = ((slot * self.Hkv + g) * 2 + kind) * cb
         return tier, self.pools[tier][o:o + cb]
 
@@ -320,21 +342,25 @@ class QuadState:
         return ctypes.byref(self._s)
 
 
-def cache_from_workload(w, device="cuda", threads: int = 8, spare=None, quad_basis=None, host_tiers: int = 0):
+def cache_from_workload(w, device="cuda", threads: int = 8, spare=None, quad_basis=None, host_tiers: int = 0,
+                        v_tiers: int = 0, host_v_tiers: int = 0):
     """Allocate a cache for workload ``w`` and store its prefilled context with kvq_build_pages.
 
     After the call ``seq_len`` holds the prefilled lengths (before the step's append).
     ``spare`` (optional, per tier) adds free slots after the used ones of each pool.
     ``quad_basis`` (optional, fp32 ``[Hkv, rank, D]``) also builds the quad page-score state
     (``cache.quad``) from the same keys with kvq_quad_build.  ``host_tiers`` (bit t) puts
-    pool t in pinned host memory that the kernels read in place.
+    pool t in pinned host memory that the kernels read in place; ``v_tiers`` /
+    ``host_v_tiers`` (bit t) give tier t a separate V pool, on the device or in pinned
+    host memory.
     """
     import torch
     from concurrent.futures import ThreadPoolExecutor
     tier_tbl, slot_tbl, counts = w.slot_map()
     if spare is not None:
         counts = [int(c) + int(x) for c, x in zip(counts, spare)]
-    cache = PagedCache(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.dtype, counts, device, host_tiers=host_tiers)
+    cache = PagedCache(w.B, w.Hq, w.Hkv, w.D, w.max_pages, w.dtype, counts, device, host_tiers=host_tiers,
+                       v_tiers=v_tiers, host_v_tiers=host_v_tiers)
     cache.block_table.copy_(torch.from_numpy(encode_block_table(tier_tbl, slot_tbl)))
     lens = np.asarray(w.lens, dtype=np.int64)
     cache.seq_len.copy_(torch.from_numpy(lens.astype(np.int32)))

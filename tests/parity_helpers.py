@@ -19,13 +19,19 @@ MARGIN = 1e-5
 
 
 def pools_to_cpu(cache):
-    return [None if p is None else p.cpu().numpy() for p in cache.pools]
+    """Every pool's bytes; a tier with a separate V pool gives a (K pool, V pool) pair."""
+    vpools = getattr(cache, "vpools", [None] * len(cache.pools))
+    return [None if p is None else (p.cpu().numpy() if v is None else (p.cpu().numpy(), v.cpu().numpy()))
+            for p, v in zip(cache.pools, vpools)]
 
 
 def gpu_chunk(pools, bt: np.ndarray, Hkv: int, D: int, b: int, p: int, g: int, kind: int):
     e = int(bt[b, p]) & 0xFFFFFFFF
     tier, slot = e >> 29, e & 0x1FFFFFFF
     cb = chunk_bytes(tier, D)
+    if isinstance(pools[tier], tuple):  # separate K and V pools
+        o = (slot * Hkv + g) * cb
+        return tier, pools[tier][kind][o:o + cb]
     o = ((slot * Hkv + g) * 2 + kind) * cb
     return tier, pools[tier][o:o + cb]
 
