@@ -297,7 +297,7 @@ class PagedCache:
             s.pool[i] = _ptr(self.pools[i]) if self.pools[i] is not None else None
             s.vpool[i] = _ptr(self.vpools[i]) if self.vpools[i] is not None else None
             s.pool_slots[i] = self.pool_slots[i]
-        s.host_vtiers = self.host_v_tiers
+        s.host_vtiers = sum(1 << i for i in range(6) if (self.host_v_tiers >> i) & 1 and self.vpools[i] is not None)
         s.summary, s.open_ksum, s.err_word = _ptr(self.summary), _ptr(self.open_ksum), _ptr(self.err)
 
     def ref(self):
