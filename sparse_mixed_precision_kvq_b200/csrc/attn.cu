@@ -306,9 +306,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
   const unsigned char* ring_c = ring;
 
   // lane i: descriptor of page f0 + issued + i (binary search of its segment in off[])
+  int my_rank = lane;  // issue position of this lane's page within the window
   auto prefetch = [&]() {
     win_base = issued;
     win_n = min(32, (f1 - f0) - issued);
+    int bgw = 0;  // segment of this lane's page
     my = PageDesc{nullptr, nullptr, -1, 0};
     if (lane < win_n) {
       const int f = f0 + issued + lane;
@@ -318,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
         if (off[mid] <= f) lo = mid; else hi = mid - 1;
       }
       const int bg = lo;
+      bgw = bg;
       const int b = bg / c.Hkv, g = bg % c.Hkv;
       const int p = __ldg(&a.sel[(size_t)bg * a.kmax + (f - off[bg])]);
       const int L = __ldg(&c.seq_len[b]);
@@ -335,18 +338,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
         set_err(c.err, KVQ_DERR_BAD_PAGE);
       }
     }
+    if constexpr (!ONLY16) {
+      // Issue the window's pages grouped by tier inside each segment (segments stay in
+      // order, so the k-th page issued is still in the segment of the k-th flat page):
+      // a warp then runs one tier's page math at a time, which keeps the instruction cache
+      // from cycling through every tier's code.  rank = position in (segment, tier, lane)
+      // order; the page issued k-th is the lane whose rank is k.
+      const int seg = bgw - __shfl_sync(0xffffffffu, bgw, 0);
+      const int key = lane < win_n ? seg * 8 + (my.tier < 0 ? 7 : my.tier) : 0x7FFFFFFF;
+      int rank = 0;
+#pragma unroll 8
+      for (int j = 0; j < 32; ++j) {
+        const int kj = __shfl_sync(0xffffffffu, key, j);
+        rank += (kj < key) || (kj == key && j < lane);
+      }
+      my_rank = rank;
+    }
   };
 
   auto issue_more = [&]() {
     while (issued - consumed < kNBar && issued < f1 - f0) {
       if (issued == win_base + win_n) prefetch();
-      const int k = issued - win_base;
+      const int k = ONLY16 ? issued - win_base
+                           : __ffs(__ballot_sync(0xffffffffu, my_rank == issued - win_base)) - 1;
       const unsigned long long sp = __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my.src), k);
       const unsigned long long vp = __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my.vsrc), k);
       const int tier = __shfl_sync(0xffffffffu, my.tier, k);
       const int nv = __shfl_sync(0xffffffffu, my.nv, k);
       const int cb = tier >= 0 ? c.chunk[tier] : 0;
       const int bytes = 2 * cb;
+      // An empty ring (every issued page consumed) restarts at offset 0, so a page of up to
+      // kRing bytes always fits; otherwise the page goes after the last one issued, or to
+      // the ring's start when it does not fit before the end, once that space is consumed.
+      if (issued == consumed) head = tail = 0;
       int start = head;
       const int pos = head % kRing;
       if (pos + bytes > kRing) start += kRing - pos;
