@@ -352,6 +352,10 @@ __global__ void __launch_bounds__(kThreads, kRing == kRingWide ? 1 : 2)
       const int nv = __shfl_sync(0xffffffffu, my.nv, k);
       const int cb = tier >= 0 ? c.chunk[tier] : 0;
       const int bytes = 2 * cb;
+      // An empty ring (every issued page consumed) restarts at offset 0, so a page of up to
+      // kRing bytes always fits; otherwise the page goes after the last one issued, or to
+      // the ring's start when it does not fit before the end, once that space is consumed.
+      if (issued == consumed) head = tail = 0;
       int start = head;
       const int pos = head % kRing;
       if (pos + bytes > kRing) start += kRing - pos;
