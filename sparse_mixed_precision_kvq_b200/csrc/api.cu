@@ -162,7 +162,7 @@ kvq_status kvq_workspace_size(const kvq_cache* cache, int32_t kmax, size_t* byte
   kvq_status st = to_dev(cache, c);
   if (st != KVQ_OK) return st;
   if (bytes == nullptr || kmax < 1) return KVQ_ERR_INVALID_ARG;
-  *bytes = attn_workspace_bytes(c, attn_num_ctas(current_device()));
+  *bytes = attn_workspace_bytes(c, attn_grid(c, current_device()));
   return KVQ_OK;
 }
 
@@ -176,7 +176,7 @@ kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const i
     return KVQ_ERR_INVALID_ARG;
   if (!aligned16(workspace) || !(sm_scale > 0.f)) return KVQ_ERR_INVALID_ARG;
   if ((long long)c.B * c.Hkv >= kMaxSegments) return KVQ_ERR_UNSUPPORTED;  // offsets live in shared memory
-  const int n = attn_num_ctas(current_device());
+  const int n = attn_grid(c, current_device());
   if (ws_bytes < attn_workspace_bytes(c, n)) return KVQ_ERR_WORKSPACE;
   return cuda_status(launch_attn(c, q, sel, cnt, kmax, sm_scale, out, lse, workspace, n,
                                  reinterpret_cast<cudaStream_t>(stream)));

@@ -50,7 +50,11 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kRing = 24576;  // bytes of page staging per warp (three 16-bit pages at D = 128)
+// Bytes of page staging per warp: three 16-bit pages at D = 128 with one CTA per SM (the
+// 16-bit-only kernel, whose pages are bandwidth-bound); half that with two CTAs per SM (the
+// kernel for caches with quantised pools, whose page math is latency-bound: twice the warps).
+constexpr int kRingWide = 24576;
+constexpr int kRingNarrow = 12288;
 constexpr int kNBar = 8;      // pages in flight per warp (max)
 
 struct PageMeta {
@@ -118,7 +122,7 @@ __device__ inline void put_merged4(const AttnArgs& a, uint16_t* out, float* lse,
 // trip).  The result goes to CTA partial slot `dst`, or to the output (dst < 0).
 template <int D, bool BF16>
 __device__ inline void cta_merge4(const AttnArgs& a, uint16_t* out, float* lse, const unsigned char* rings,
-                                  const int* pseg, int bg, int h, int d, int w0, int w1, int dst) {
+                                  int ring_bytes, const int* pseg, int bg, int h, int d, int w0, int w1, int dst) {
   const int G = a.c.G;
   float mv[kWarps], lv[kWarps];
   float4 ov[kWarps];
@@ -129,7 +133,7 @@ __device__ inline void cta_merge4(const AttnArgs& a, uint16_t* out, float* lse, 
     ov[w] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (w >= w0 && w <= w1) {
       if (pseg[w] == bg) {
-        const float* sp = reinterpret_cast<const float*>(rings + (size_t)w * kRing);
+        const float* sp = reinterpret_cast<const float*>(rings + (size_t)w * ring_bytes);
         ov[w] = *reinterpret_cast<const float4*>(&sp[h * D + d]);
         mv[w] = sp[G * D + 2 * h];
         lv[w] = sp[G * D + 2 * h + 1];
@@ -211,9 +215,9 @@ __device__ inline void final_combine4(const AttnArgs& a, uint16_t* out, float* l
   put_merged4<BF16>(a, out, lse, bg, h, d, D, M, Ls, o, nullptr, nullptr, -1);
 }
 
-template <int D, bool BF16, bool ONLY16>
-__global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t* __restrict__ out,
-                                                           float* __restrict__ lse) {
+template <int D, bool BF16, bool ONLY16, int kRing>
+__global__ void __launch_bounds__(kThreads, kRing == kRingWide ? 1 : 2)
+    attn_kernel(AttnArgs a, uint16_t* __restrict__ out, float* __restrict__ lse) {
   extern __shared__ __align__(128) unsigned char smem[];
   const DevCache& c = a.c;
   const int G = c.G;
@@ -227,6 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
   PageMeta* pmeta = reinterpret_cast<PageMeta*>(smem + (size_t)kWarps * kRing + kWarps * kNBar * 8) + warp * kNBar;
   int* off = reinterpret_cast<int*>(smem + (size_t)kWarps * kRing + kWarps * kNBar * 8 +
                                     kWarps * kNBar * sizeof(PageMeta));  // [BH + 1]
+  int16_t* last_list = reinterpret_cast<int16_t*>(off + BH + 1);       // [BH] segments this CTA completes
   __shared__ int scan_sh[kWarps + 1];
 
   if (lane == 0) {
@@ -485,8 +490,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
   const int cw = kWarps * W;  // pages per CTA
   const int cta0 = min(total, (int)blockIdx.x * cw), cta1 = min(total, cta0 + cw);
   __shared__ int s_nlast;
-  // list of the segments this CTA completes: warp 0's ring past its partial (free now)
-  int16_t* last_list = reinterpret_cast<int16_t*>(smem + 8192);
   if (cta0 < cta1) {
     auto seg_of = [&](int f) {  // last segment starting at or before flat page f
       int lo = 0, hi = BH - 1;
@@ -505,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
       const int w0 = max(wb, off[sbg] / W) - wb;
       const int w1 = min(wb + kWarps - 1, (off[sbg + 1] - 1) / W) - wb;
       const int n0 = off[sbg] / cw, n1 = (off[sbg + 1] - 1) / cw;
-      cta_merge4<D, BF16>(a, out, lse, smem, s_pseg, sbg, el / (D / 4), 4 * (el % (D / 4)), w0, w1,
+      cta_merge4<D, BF16>(a, out, lse, smem, kRing, s_pseg, sbg, el / (D / 4), 4 * (el % (D / 4)), w0, w1,
                           n0 == n1 ? -1 : (int)blockIdx.x + sbg);
     }
     __threadfence();  // this thread's CTA partials are visible before any arrival is counted
@@ -536,27 +539,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnArgs a, uint16_t*
   griddep_launch_dependents();
 }
 
-template <int D>
-constexpr size_t attn_smem_fixed() {
-  return (size_t)kWarps * kRing + kWarps * kNBar * 8 + kWarps * kNBar * sizeof(PageMeta);
+// Dynamic shared memory: the warps' rings, their mbarriers and page records, then the
+// segment offsets [BH + 1] and the list of segments a CTA completes [BH] (int16).
+size_t attn_smem_bytes(int ring, int BH) {
+  return (size_t)kWarps * ring + kWarps * kNBar * 8 + kWarps * kNBar * sizeof(PageMeta) + (size_t)(BH + 1) * 4 +
+         ((size_t)BH * 2 + 15) / 16 * 16;
 }
 
-template <int D, bool BF16, bool ONLY16>
+bool only16_cache(const DevCache& c) {
+  for (int t = 1; t < kNumTiers; ++t)
+    if (c.pool[t] != nullptr) return false;
+  return true;
+}
+
+// Two CTAs per SM when the cache has quantised pools and two narrow-ring CTAs fit (228 KB
+// of shared memory per SM, 1 KB of it reserved per CTA); one otherwise.
+int ctas_per_sm(const DevCache& c) {
+  if (only16_cache(c)) return 1;
+  return 2 * (attn_smem_bytes(kRingNarrow, c.B * c.Hkv) + 1024) <= 233472 ? 2 : 1;
+}
+
+template <int D, bool BF16, bool ONLY16, int RING>
 cudaError_t launch_attn_v(const AttnArgs& a, uint16_t* out, float* lse, cudaStream_t s) {
-  const int BH = a.c.B * a.c.Hkv;
-  const size_t smem = attn_smem_fixed<D>() + (size_t)(BH + 1) * 4;
-  cudaError_t e =
-      cudaFuncSetAttribute(attn_kernel<D, BF16, ONLY16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = attn_smem_bytes(RING, a.c.B * a.c.Hkv);
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, BF16, ONLY16, RING>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_kernel<D, BF16, ONLY16>, dim3(a.num_ctas), dim3(kThreads), smem, s, a, out, lse);
+  return launch_pdl(attn_kernel<D, BF16, ONLY16, RING>, dim3(a.num_ctas), dim3(kThreads), smem, s, a, out, lse);
 }
 
-// A cache whose only pool is the 16-bit one runs the 16-bit-only kernel.
+// A cache whose only pool is the 16-bit one runs the 16-bit-only kernel (one CTA per SM);
+// others the all-tier kernel, two CTAs per SM when they fit.
 template <int D, bool BF16>
 cudaError_t launch_attn_d(const AttnArgs& a, uint16_t* out, float* lse, cudaStream_t s) {
-  bool only16 = true;
-  for (int t = 1; t < kNumTiers; ++t) only16 = only16 && a.c.pool[t] == nullptr;
-  return only16 ? launch_attn_v<D, BF16, true>(a, out, lse, s) : launch_attn_v<D, BF16, false>(a, out, lse, s);
+  if (only16_cache(a.c)) return launch_attn_v<D, BF16, true, kRingWide>(a, out, lse, s);
+  return ctas_per_sm(a.c) == 2 ? launch_attn_v<D, BF16, false, kRingNarrow>(a, out, lse, s)
+                               : launch_attn_v<D, BF16, false, kRingWide>(a, out, lse, s);
 }
 
 }  // namespace
@@ -579,6 +597,11 @@ void set_grid_override(int ctas) { g_grid_override.store(ctas > 0 ? ctas : 0); }
 int attn_num_ctas(int device) {
   const int o = g_grid_override.load();
   return o > 0 ? o : sm_count(device);
+}
+
+int attn_grid(const DevCache& c, int device) {
+  const int o = g_grid_override.load();
+  return o > 0 ? o : sm_count(device) * ctas_per_sm(c);
 }
 
 // Workspace: [kCounterBytes] per-segment arrival counters (zero between calls, at a fixed

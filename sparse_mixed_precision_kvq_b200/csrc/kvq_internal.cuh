@@ -280,7 +280,8 @@ cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_sele
 int coverage_sort_size(const DevCache& c, const kvq_select_params& prm);
 size_t attn_workspace_bytes(const DevCache& c, int num_ctas);
 int sm_count(int device);      // streaming multiprocessors of the device (cached)
-int attn_num_ctas(int device);  // grid of the attention kernel and the fused step: sm_count, or the override
+int attn_num_ctas(int device);  // grid of the fused step: sm_count, or the override
+int attn_grid(const DevCache& c, int device);  // grid of the attention kernel for this cache (or the override)
 void set_grid_override(int ctas);
 cudaError_t launch_attn(const DevCache& c, const void* q, const int32_t* sel, const int32_t* cnt, int kmax,
                         float sm_scale, void* out, float* lse, void* ws, int num_ctas, cudaStream_t s);
