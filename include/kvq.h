@@ -265,7 +265,7 @@ kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const i
  *  allocate device memory at decode time, e.g. an engine that gave all device memory to
  *  its own KV page pool, or a plugin with no allocation hook.)
  *  Same arguments and results as kvq_sparse_decode_attn minus the workspace.  The split-K
- *  scratch is a static device array of kvq_noalloc_scratch_bytes() (8 MiB) inside the
+ *  scratch is a static device array of kvq_noalloc_scratch_bytes() (16 MiB) inside the
  *  library, held by every GPU that loads it until the process exits.  Allocates nothing
  *  (no cudaMalloc/cudaFree).  Returns KVQ_ERR_WORKSPACE when kvq_workspace_size() for
  *  this cache exceeds the static size, and KVQ_ERR_UNSUPPORTED for B*Hkv >= 6144 as

@@ -25,7 +25,7 @@
 namespace kvq {
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = 8u << 20;  // 8 MiB
+constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB
 
 static __device__ __align__(256) unsigned char g_attn_scratch[kNoAllocScratchBytes];
 

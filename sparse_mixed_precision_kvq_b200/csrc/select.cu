@@ -37,6 +37,9 @@ __global__ void __launch_bounds__(NT) select_kernel(DevCache c, const float* __r
   const int L = c.seq_len[b];
   const int P = min((L + kPage - 1) / kPage, c.max_pages);
   const float* sc = scores + (size_t)bg * c.max_pages;
+  const bool topk = prm.coverage_ppm <= 0;
+  // while loading the keys, the range of the candidates' scores (the selection's first
+  // pass) and the histogram's clearing, so that one barrier serves both
   bool nan_seen = false;
   for (int p0 = tid; p0 < P; p0 += 4 * NT) {  // four loads in flight per thread
     float v[4];
@@ -47,6 +50,32 @@ __global__ void __launch_bounds__(NT) select_kernel(DevCache c, const float* __r
       if (p0 + j * NT < P) keys[p0 + j * NT] = order_key(v[j], nan_seen);
   }
   if (nan_seen) set_err(c.err, KVQ_DERR_NAN_SCORE);
+  constexpr bool kPre = NT <= 512;  // (the 1024-thread instance keeps the separate pass: registers)
+  if (kPre && topk) {
+    // this thread's own keys (no barrier needed to read them back)
+    const SelectSplit sp = select_split(P, prm);
+    float lo = INFINITY, hi = -INFINITY;
+    for (int p = tid; p < sp.rs; p += NT) {
+      if (p < sp.ns) continue;
+      const uint32_t k = keys[p];
+      if (k != 0u) {
+        const float f = key_score(k);
+        lo = fminf(lo, f);
+        hi = fmaxf(hi, f);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if ((tid & 31) == 0) {
+      sh.wmin[tid >> 5] = lo;
+      sh.wmax[tid >> 5] = hi;
+    }
+    for (int i = tid; i < 257; i += NT) scratch[i] = 0u;
+    if (tid == 0) sh.ncand = 0;
+  }
   __syncthreads();
   SyncBar bar;
   if (prm.coverage_ppm > 0) {
@@ -55,7 +84,7 @@ __global__ void __launch_bounds__(NT) select_kernel(DevCache c, const float* __r
     select_coverage<NT>(keys, P, L, prm, mkey, mpage, scratch + kSelBitmapOff, sel + (size_t)bg * kmax, cnt + bg,
                         kmax, c.err, sh, tid, bar);
   } else {
-    select_pages<NT>(keys, P, prm, sel + (size_t)bg * kmax, cnt + bg, kmax, c.err, scratch, sh, tid, bar);
+    select_pages<NT, kPre>(keys, P, prm, sel + (size_t)bg * kmax, cnt + bg, kmax, c.err, scratch, sh, tid, bar);
   }
   griddep_launch_dependents();
 }

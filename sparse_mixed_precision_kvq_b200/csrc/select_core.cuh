@@ -138,7 +138,11 @@ __device__ inline void emit_chosen(const uint32_t* chosen, int nwords, int32_t* 
 // caller); writes the chosen pages in ascending order to out[0 .. min(n, kmax)) and
 // min(n, kmax) to *cnt_out (thread 0).  Flags KVQ_DERR_KMAX if n > kmax.  `scratch` is
 // kSelScratchWords words of shared memory; P <= kSelMaxPages.
-template <int NT, typename Bar>
+// PRE: the caller has already, before that barrier, put each warp's range of its
+// candidates' scores (NaN left out, -0 as +0; +inf/-inf when it has none) in
+// sh.wmin/sh.wmax, cleared scratch[0 .. 257) and set sh.ncand = 0 -- the first pass and
+// its barrier are then skipped.
+template <int NT, bool PRE = false, typename Bar>
 __device__ inline void select_pages(const uint32_t* keys, int P, const kvq_select_params& prm, int32_t* out,
                                     int32_t* cnt_out, int kmax, uint32_t* err, uint32_t* scratch, SelShared& sh,
                                     int tid, Bar& bar) {
@@ -178,26 +182,28 @@ __device__ inline void select_pages(const uint32_t* keys, int P, const kvq_selec
   if (mode == 2) {
     // 1) candidates' score range; clear the histogram
     float lo = INFINITY, hi = -INFINITY;
-    pages([&](int, int p, bool valid) {
-      const uint32_t k = valid ? keys[p] : 0u;
-      if (valid && is_cand(p) && k != 0u) {
-        const float f = key_score(k);
-        lo = fminf(lo, f);
-        hi = fmaxf(hi, f);
-      }
-    });
+    if constexpr (!PRE) {
+      pages([&](int, int p, bool valid) {
+        const uint32_t k = valid ? keys[p] : 0u;
+        if (valid && is_cand(p) && k != 0u) {
+          const float f = key_score(k);
+          lo = fminf(lo, f);
+          hi = fmaxf(hi, f);
+        }
+      });
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+      for (int o = 16; o; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+      }
+      if (lane == 0) {
+        sh.wmin[warp] = lo;
+        sh.wmax[warp] = hi;
+      }
+      for (int i = tid; i < 257; i += NT) hist[i] = 0;
+      if (tid == 0) sh.ncand = 0;
+      bar();
     }
-    if (lane == 0) {
-      sh.wmin[warp] = lo;
-      sh.wmax[warp] = hi;
-    }
-    for (int i = tid; i < 257; i += NT) hist[i] = 0;
-    if (tid == 0) sh.ncand = 0;
-    bar();
     lo = INFINITY;
     hi = -INFINITY;
 #pragma unroll
