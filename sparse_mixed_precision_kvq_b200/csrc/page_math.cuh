@@ -133,9 +133,26 @@ struct LaneWords {
   }
 };
 
+// N consecutive words with one vector load (src aligned to 4 * N bytes).
+template <int N>
+__device__ __forceinline__ void load_words(const uint32_t* src, uint32_t (&w)[N]) {
+  if constexpr (N == 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (N == 2) {
+    const uint2 v = *reinterpret_cast<const uint2*>(src);
+    w[0] = v.x; w[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) w[i] = src[i];
+  }
+}
+
 // Per-token metadata of one chunk for the lane's two token rows t0 = g8, t1 = g8 + 8:
 // the scale s and the zero offset of the centred codes, z + 2^(b-1) * s (1-bit: m, 0;
-// FP8: the scale, 0).
+// FP8: the scale, 0).  A token's NG metadata words (or half-words) are contiguous, and
+// aligned to their total size (the metadata area of every chunk is 16-byte aligned), so
+// they are read with one vector load.
 template <int TIER, int D>
 __device__ __forceinline__ void load_meta(const unsigned char* meta, int t0, float (&s)[2][D / 32],
                                           float (&z)[2][D / 32]) {
@@ -144,15 +161,17 @@ __device__ __forceinline__ void load_meta(const unsigned char* meta, int t0, flo
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int t = t0 + 8 * i;
-    if constexpr (TIER == KVQ_TIER_I1 || TIER == KVQ_TIER_F8) {
-      const uint16_t* m = reinterpret_cast<const uint16_t*>(meta) + t * NG;
+    if constexpr (TIER == KVQ_TIER_I1 || TIER == KVQ_TIER_F8) {  // NG fp16 values per token
+      uint32_t w[NG / 2];
+      load_words<NG / 2>(reinterpret_cast<const uint32_t*>(meta) + t * (NG / 2), w);
 #pragma unroll
       for (int gi = 0; gi < NG; ++gi) {
-        s[i][gi] = __half2float(__ushort_as_half(m[gi]));
+        s[i][gi] = __half2float(__ushort_as_half(static_cast<uint16_t>(w[gi / 2] >> (16 * (gi & 1)))));
         z[i][gi] = 0.f;
       }
     } else {
-      const uint32_t* m = reinterpret_cast<const uint32_t*>(meta) + t * NG;
+      uint32_t m[NG];
+      load_words<NG>(reinterpret_cast<const uint32_t*>(meta) + t * NG, m);
 #pragma unroll
       for (int gi = 0; gi < NG; ++gi) {
         const uint32_t v = m[gi];
@@ -305,19 +324,24 @@ __device__ __forceinline__ void process_page(const unsigned char* base, int tier
   p[3] = ex2(x[3] - mn1);
   st.l[0] = st.l[0] * a0 + p[0] + p[2];
   st.l[1] = st.l[1] * a1 + p[1] + p[3];
+  // rescale the accumulators only when some running maximum moved (else the factors are
+  // exactly 1): after the first pages of a segment that is the rare case
+  const bool moved = __any_sync(0xffffffffu, mn0 != st.m[0] || mn1 != st.m[1]);
   st.m[0] = mn0;
   st.m[1] = mn1;
+  if (moved) {
 #pragma unroll
-  for (int blk = 0; blk < KS; ++blk) {
-    st.o[blk][0] *= a0;
-    st.o[blk][1] *= a1;
-    st.o[blk][2] *= a0;
-    st.o[blk][3] *= a1;
-  }
+    for (int blk = 0; blk < KS; ++blk) {
+      st.o[blk][0] *= a0;
+      st.o[blk][1] *= a1;
+      st.o[blk][2] *= a0;
+      st.o[blk][3] *= a1;
+    }
 #pragma unroll
-  for (int gi = 0; gi < NG; ++gi) {
-    st.zacc[gi][0] *= a0;
-    st.zacc[gi][1] *= a1;
+    for (int gi = 0; gi < NG; ++gi) {
+      st.zacc[gi][0] *= a0;
+      st.zacc[gi][1] *= a1;
+    }
   }
   const unsigned char* vbase = base + chunk_bytes(tier, D);
   if constexpr (ONLY16) {
