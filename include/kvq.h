@@ -285,9 +285,12 @@ kvq_status kvq_sparse_decode_attn_noalloc(const kvq_cache* cache, const void* q,
 size_t kvq_noalloc_scratch_bytes(void);
 
 /*
- * kvq_append_scores -- kvq_append followed by kvq_page_scores in one launch, with the same
- * results: the warp that scores the tile of a sequence's appended token writes the token
- * first.  Arguments as those two calls (pos, k_new, v_new required).
+ * kvq_append_scores -- kvq_append followed by kvq_page_scores, with the same results, as
+ * two kernels chained by programmatic dependent launch: the score sweep starts while the
+ * append runs and scores every 16-page tile except those holding a page pos[b] / 16; it
+ * scores those after the append has completed.  Arguments as those two calls (pos, k_new,
+ * v_new required).  pos, q and seq_len must not be written by the append's own kernel
+ * (they are inputs of the call), and the sweep may read them before the append completes.
  */
 kvq_status kvq_append_scores(const kvq_cache* cache, const int32_t* pos, const void* k_new,
                              const void* v_new, const void* q, float* scores, kvq_stream_t stream);

@@ -28,10 +28,11 @@ __global__ void __launch_bounds__(128) append_kernel(DevCache c, const int32_t* 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bg = blockIdx.x;
   const int b = bg / c.Hkv, g = bg % c.Hkv;
-  // The page-score sweep that follows only prefetches until it waits for this grid, so it
-  // may launch at once: its summary traffic then overlaps this kernel.
-  griddep_launch_dependents();
+  // The page-score sweep that follows reads, before it waits for this grid, every summary
+  // row except the ones this grid writes; it may launch as soon as everything before this
+  // grid is complete, so that its sweep overlaps this kernel.
   griddep_wait();
+  griddep_launch_dependents();
   const int P = pos[b];
   if (P >= c.max_pages * kPage) {
     if (tid == 0) set_err(c.err, KVQ_DERR_BAD_POS);

@@ -49,11 +49,14 @@ struct ScoreSelect {
 // Grid of 2 CTAs per SM; warp w takes the contiguous run of 16-page tiles
 // [w * per, (w + 1) * per) of the flat list (b, g, tile), loading the next tile while
 // the current one is multiplied.
-// MODE 1 (kvq_append_scores) and 2 (kvq_score_select): the warp that owns the tile of a
-// (b, g)'s appended token writes the token first (so that tile is read after the new
-// summary row is stored).  MODE 2: after its tiles, the CTA counts them on each (b, g) it
-// touched, and the CTA that completes a (b, g) selects its pages (select_core.cuh) from
-// the scores in L2.
+// MODE 1 (kvq_append_scores): the append kernel runs just before this one and writes
+// only the summary row of page pos[b] / 16 of each (b, g).  Every other tile is scored
+// before waiting for that kernel, so the sweep overlaps the append; the tiles holding an
+// appended page are scored after the wait.
+// MODE 2 (kvq_score_select): the warp that owns the tile of a (b, g)'s appended token
+// writes the token first (so that tile is read after the new summary row is stored);
+// after its tiles, the CTA counts them on each (b, g) it touched, and the CTA that
+// completes a (b, g) selects its pages (select_core.cuh) from the scores in L2.
 enum { SCORES = 0, APPEND_SCORES = 1, APPEND_SCORES_SELECT = 2 };
 
 template <int D, bool BF16, int MODE>
@@ -70,8 +73,9 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
   const int i1 = min(total, i0 + per);
   // Before waiting for the previous kernel (the append, which writes only the open page's
   // summary row): ask L2 for this warp's summary rows, one bulk prefetch per (b, g) piece,
-  // so their DRAM traffic overlaps that kernel (a prefetch is only a hint).
-  if (lane == 0 && i0 < i1) {
+  // so their DRAM traffic overlaps that kernel (a prefetch is only a hint).  MODE 1 reads
+  // them at once instead (measured faster than a prefetch ahead of the sweep).
+  if (MODE != APPEND_SCORES && lane == 0 && i0 < i1) {
     for (int bg = i0 / tiles_per_bg; bg <= (i1 - 1) / tiles_per_bg; ++bg) {
       const int L = c.seq_len[bg / c.Hkv];
       const int P = min((L + kPage - 1) / kPage, c.max_pages);
@@ -81,9 +85,9 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
         bulk_prefetch_l2(c.summary + ((size_t)bg * c.max_pages + p0) * D, (uint32_t)(p1 - p0) * D * 2);
     }
   }
-  griddep_wait();
+  if constexpr (MODE != APPEND_SCORES) griddep_wait();
 
-  if (MODE != SCORES && f.pos != nullptr && i0 < i1) {  // appends whose page lies in this warp's tiles
+  if (MODE == APPEND_SCORES_SELECT && f.pos != nullptr && i0 < i1) {  // appends whose page lies in this warp's tiles
     for (int bg = i0 / tiles_per_bg; bg <= (i1 - 1) / tiles_per_bg; ++bg) {
       const int b = bg / c.Hkv, g = bg % c.Hkv;
       const int ps = f.pos[b];
@@ -107,9 +111,11 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
     uint4 av0[2][D / 32], av1[2][D / 32];  // double buffer (compile-time indexed)
 
     // where tile item i lives
+    // Reads before the wait (MODE 1) go to L2 (__ldcg): everything they touch was written
+    // by grids that are complete, and no stale L1 line may stand in for it.
     auto tile_src = [&](int i, int& Pn) -> const uint16_t* {
       const int bg = i / tiles_per_bg;
-      const int L = c.seq_len[bg / c.Hkv];
+      const int L = __ldcg(&c.seq_len[bg / c.Hkv]);
       Pn = min((L + kPage - 1) / kPage, c.max_pages);
       return c.summary + (size_t)bg * c.max_pages * D;
     };
@@ -118,7 +124,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
       if (bg != cur_bg) {  // new (b, g): its query fragments (hi + lo)
         cur_bg = bg;
         const int b = bg / c.Hkv, g = bg % c.Hkv;
-        const int L = c.seq_len[b];
+        const int L = __ldcg(&c.seq_len[b]);
         P = min((L + kPage - 1) / kPage, c.max_pages);
         out = scores + (size_t)bg * c.max_pages;
         qf.load(q, c.Hq, c.G, b, g, lane, bad);
@@ -132,21 +138,61 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
       }
     };
 
+    // MODE 1: the tile holding the appended page of each (b, g) in this warp's run; lane j
+    // keeps that of (b, g) bg0 + j (-1: none).  pos is the caller's, not the append's.
+    const int bg0 = i0 / tiles_per_bg;
+    int my_aff = -1;
+    auto aff_of = [&](int bg) {
+      const int ps = __ldcg(&f.pos[bg / c.Hkv]);
+      return ps >= 0 && ps < c.max_pages * kPage ? bg * tiles_per_bg + (ps / kPage) / 16 : -1;
+    };
+    if (MODE == APPEND_SCORES && bg0 + lane <= (i1 - 1) / tiles_per_bg) my_aff = aff_of(bg0 + lane);
+    auto held_back = [&](int i) {  // uniform over the warp
+      if constexpr (MODE != APPEND_SCORES) {
+        return false;
+      } else {
+        const int j = i / tiles_per_bg - bg0;
+        return (j < 32 ? __shfl_sync(0xffffffffu, my_aff, j) : aff_of(i / tiles_per_bg)) == i;
+      }
+    };
+    auto next_tile = [&](int i) {  // the next tile after i scored before the wait
+      for (++i; i < i1; ++i)
+        if (!held_back(i)) break;
+      return i;
+    };
     int Pn;
-    const uint16_t* src = tile_src(i0, Pn);
-    load_tile<D>(src, i0 % tiles_per_bg, Pn, lane, av0);
-    for (int i = i0; i < i1; i += 2) {
-      if (i + 1 < i1) {  // next tile into the odd buffer, then the even tile's math
-        src = tile_src(i + 1, Pn);
-        load_tile<D>(src, (i + 1) % tiles_per_bg, Pn, lane, av1);
+    if constexpr (MODE != APPEND_SCORES) {  // every tile of the run
+      load_tile<D>(tile_src(i0, Pn), i0 % tiles_per_bg, Pn, lane, av0);
+      for (int i = i0; i < i1; i += 2) {
+        if (i + 1 < i1) load_tile<D>(tile_src(i + 1, Pn), (i + 1) % tiles_per_bg, Pn, lane, av1);
+        compute(i, av0);
+        if (i + 1 >= i1) break;
+        if (i + 2 < i1) load_tile<D>(tile_src(i + 2, Pn), (i + 2) % tiles_per_bg, Pn, lane, av0);
+        compute(i + 1, av1);
       }
-      compute(i, av0);
-      if (i + 1 >= i1) break;
-      if (i + 2 < i1) {
-        src = tile_src(i + 2, Pn);
-        load_tile<D>(src, (i + 2) % tiles_per_bg, Pn, lane, av0);
+    }
+    int i = MODE == APPEND_SCORES ? next_tile(i0 - 1) : i1;
+    if (i < i1) {
+      load_tile<D>(tile_src(i, Pn), i % tiles_per_bg, Pn, lane, av0);
+      while (true) {  // next tile into the odd buffer, then the even tile's math
+        const int j = next_tile(i);
+        if (j < i1) load_tile<D>(tile_src(j, Pn), j % tiles_per_bg, Pn, lane, av1);
+        compute(i, av0);
+        if (j >= i1) break;
+        const int k = next_tile(j);
+        if (k < i1) load_tile<D>(tile_src(k, Pn), k % tiles_per_bg, Pn, lane, av0);
+        compute(j, av1);
+        if (k >= i1) break;
+        i = k;
       }
-      compute(i + 1, av1);
+    }
+    if constexpr (MODE == APPEND_SCORES) {
+      griddep_wait();  // the appended tokens' summary rows are written (and this grid ends after the append)
+      for (int t = i0; t < i1; ++t) {
+        if (!held_back(t)) continue;
+        load_tile<D>(tile_src(t, Pn), t % tiles_per_bg, Pn, lane, av0);
+        compute(t, av0);
+      }
     }
     if (bad) set_err(c.err, KVQ_DERR_FP16_RANGE);
   }
@@ -255,6 +301,8 @@ cudaError_t launch_score_select(const DevCache& c, const int32_t* pos, const voi
 cudaError_t launch_append_scores(const DevCache& c, const int32_t* pos, const void* k_new, const void* v_new,
                                  const void* q, float* scores, cudaStream_t s) {
   if (c.G > kMaxG) return cudaErrorInvalidValue;
+  const cudaError_t e = launch_append(c, pos, k_new, v_new, s);
+  if (e != cudaSuccess) return e;
   const bool bf = c.dtype == KVQ_DT_BF16;
   ScoreSelect f{};
   f.pos = pos;

@@ -61,7 +61,7 @@ struct QFrag {
       const uint4* src = reinterpret_cast<const uint4*>(q + ((size_t)b * Hq + (size_t)g * G + g8) * D + CW * q4);
 #pragma unroll
       for (int k = 0; k < CW / 8; ++k) {
-        const uint4 v = src[k];
+        const uint4 v = __ldcg(src + k);
         w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
       }
     } else {

@@ -379,6 +379,44 @@ def test_score_select_equals_calls(kvq, name):
                 assert torch.equal(sel0[b, g, :c[b, g]], sel1[b, g, :c[b, g]])
 
 
+@pytest.mark.parametrize("tiers", [None, ALL_TIERS])
+def test_append_scores_two_steps_equal_calls(kvq, tiers):
+    """Two decode steps back to back (the second append chained right after the first
+    step's attention, one sequence skipped, appended pages at a page start, mid-page and a
+    page end): kvq_append_scores, whose sweep scores the tiles without an appended page
+    before the append completes, leaves the bytes, scores, selection and outputs of the
+    four separate calls."""
+    over = dict(B=5, Hq=16, Hkv=2, lens=np.array([100, 47, 512, 1000, 40]))
+    if tiers is not None:
+        over["tier_fracs"] = tiers
+    w = W.make("c4", **over)
+    outs = []
+    for how in ("calls", "three"):
+        cache = kvq.cache_from_workload(w)
+        step = kvq.DecodeStep(w, cache)
+        run = step.run if how == "calls" else step.run_three
+        run()
+        step.pos += 1
+        step.pos[1] = -1
+        cache.seq_len += 1
+        cache.seq_len[1] -= 1
+        step.k_new.mul_(-0.5)
+        run()
+        torch.cuda.synchronize()
+        assert cache.err_bits() == 0, hex(cache.err_bits())
+        outs.append((snapshot(cache), step.scores.clone(), step.sel.clone(), step.cnt.clone(), step.out.clone()))
+    (s0, sc0, sel0, cnt0, o0), (s1, sc1, sel1, cnt1, o1) = outs
+    for t, (p0, p1) in enumerate(zip(s0["pools"], s1["pools"])):
+        assert (p0 is None) == (p1 is None) and (p0 is None or np.array_equal(p0, p1)), t
+    for k in ("bt", "summary", "ksum"):
+        assert np.array_equal(s0[k], s1[k]), k
+    assert torch.equal(sc0, sc1) and torch.equal(cnt0, cnt1) and torch.equal(o0, o1)
+    c = cnt0.cpu().numpy()
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            assert torch.equal(sel0[b, g, :c[b, g]], sel1[b, g, :c[b, g]])
+
+
 @pytest.mark.parametrize("P_cap", [700, 5000])
 def test_coverage_selection_matches_oracle(kvq, P_cap):
     """Coverage (nucleus) selection: the GPU set is the oracle's wherever the cut is not
