@@ -159,17 +159,40 @@ def kernel_rooflines(names, avg_ms, nbytes, peak: float):
     return out
 
 
+def kernel_source_hash(kernel_file: str) -> str:
+    """First 16 hex digits of the SHA-256 of a kernel's translation unit: the .cu file and
+    every header of the package it includes, directly or not, in a fixed order."""
+    import re
+    csrc = os.path.join(ROOT, "sparse_mixed_precision_kvq_b200", "csrc")
+    seen, order = set(), []
+
+    def visit(name):
+        if name in seen or not os.path.exists(os.path.join(csrc, name)):
+            return
+        seen.add(name)
+        order.append(name)
+        with open(os.path.join(csrc, name)) as f:
+            for inc in re.findall(r'^#include "([^"]+)"', f.read(), re.M):
+                visit(inc)
+
+    visit(kernel_file)
+    h = hashlib.sha256()
+    for name in order:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
 def kernel_traffic(kernel_file: str):
-    """ncu DRAM bytes per launch recorded for the current source of a kernel, else None."""
+    """ncu DRAM bytes per launch recorded for the current source of a kernel (its file and
+    the headers it includes), else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    src = os.path.join(ROOT, "sparse_mixed_precision_kvq_b200", "csrc", kernel_file)
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     e = d.get(kernel_file)
-    if not e or e.get("source_sha256_16") != h:
+    if not e or e.get("source_sha256_16") != kernel_source_hash(kernel_file):
         return None
     return e
 
