@@ -59,30 +59,109 @@ struct ScoreSelect {
 // completes a (b, g) selects its pages (select_core.cuh) from the scores in L2.
 enum { SCORES = 0, APPEND_SCORES = 1, APPEND_SCORES_SELECT = 2 };
 
-template <int D, bool BF16, int MODE>
+// REAL (modes 0 and 1): only the tiles that hold pages [0, P) of each (b, g) are divided
+// among the warps -- a ragged batch leaves most of a max_pages row empty, and an even split
+// of whole rows would give a few warps all the real tiles.  Each CTA first builds the tile
+// counts' exclusive prefix over (b, g) in shared memory; the scores past the real tiles are
+// -inf, written by a fill.
+template <int D, bool BF16, int MODE, bool REAL>
 __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, const uint16_t* __restrict__ q,
                                                                     float* __restrict__ scores, int tiles_per_bg,
                                                                     int per, ScoreSelect f) {
-  extern __shared__ __align__(16) uint32_t sel_smem[];  // MODE 2: keys [max_pages], then the scratch
+  // MODE 2: keys [max_pages], then the selection scratch; REAL: the tile prefix [B * Hkv + 1]
+  extern __shared__ __align__(16) uint32_t sel_smem[];
   __shared__ SelShared sel_sh;
   __shared__ int s_unit;
+  __shared__ int s_part[kScoreWarps];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, q4 = lane & 3;
-  const int total = c.B * c.Hkv * tiles_per_bg;
-  const int i0 = (blockIdx.x * kScoreWarps + warp) * per;
-  const int i1 = min(total, i0 + per);
+  const int BH = c.B * c.Hkv;
+  const int nw = gridDim.x * kScoreWarps, gw = blockIdx.x * kScoreWarps + warp;
+  int* pre = reinterpret_cast<int*>(sel_smem);
+  // Reads before the wait go to L2 (__ldcg): what they touch was written by grids that are
+  // complete, and no stale L1 line may stand in for it.
+  auto pages_of = [&](int bg) {
+    const int L = __ldcg(&c.seq_len[bg / c.Hkv]);
+    return min(max((L + kPage - 1) / kPage, 0), c.max_pages);
+  };
+  int total, i0, i1;
+  if constexpr (REAL) {
+    const int per_t = (BH + kScoreWarps * 32 - 1) / (kScoreWarps * 32);
+    const int lo = min(BH, tid * per_t), hi = min(BH, lo + per_t);
+    int s = 0;
+    for (int bg = lo; bg < hi; ++bg) {
+      const int t = (pages_of(bg) + 15) / 16;
+      pre[bg] = t;
+      s += t;
+    }
+    int x = s;  // inclusive prefix over the warp's lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_part[warp] = x;
+    __syncthreads();
+    int run = x - s, all = 0;
+#pragma unroll
+    for (int w = 0; w < kScoreWarps; ++w) {
+      const int v = s_part[w];
+      if (w < warp) run += v;
+      all += v;
+    }
+    for (int bg = lo; bg < hi; ++bg) {
+      const int t = pre[bg];
+      pre[bg] = run;
+      run += t;
+    }
+    if (tid == 0) pre[BH] = all;
+    __syncthreads();
+    total = all;
+    const int pw = (total + nw - 1) / nw;
+    i0 = min(total, gw * pw);
+    i1 = min(total, i0 + pw);
+  } else {
+    total = BH * tiles_per_bg;
+    i0 = gw * per;
+    i1 = min(total, i0 + per);
+  }
+  // (b, g) of item i: REAL, the last (b, g) whose prefix is <= i
+  auto bg_at = [&](int i) {
+    if constexpr (REAL) {
+      int lo = 0, hi = BH - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pre[mid] <= i) lo = mid; else hi = mid - 1;
+      }
+      return lo;
+    } else {
+      return i / tiles_per_bg;
+    }
+  };
+  // the same with a forward cursor (items visited in increasing order), and the tile
+  auto locate = [&](int i, int& cur, int& tile) {
+    if constexpr (REAL) {
+      while (pre[cur + 1] <= i) ++cur;
+      tile = i - pre[cur];
+      return cur;
+    } else {
+      tile = i % tiles_per_bg;
+      return i / tiles_per_bg;
+    }
+  };
   // Before waiting for the previous kernel (the append, which writes only the open page's
   // summary row): ask L2 for this warp's summary rows, one bulk prefetch per (b, g) piece,
   // so their DRAM traffic overlaps that kernel (a prefetch is only a hint).  MODE 1 reads
   // them at once instead (measured faster than a prefetch ahead of the sweep).
   if (MODE != APPEND_SCORES && lane == 0 && i0 < i1) {
-    for (int bg = i0 / tiles_per_bg; bg <= (i1 - 1) / tiles_per_bg; ++bg) {
-      const int L = c.seq_len[bg / c.Hkv];
-      const int P = min((L + kPage - 1) / kPage, c.max_pages);
-      const int p0 = max(i0, bg * tiles_per_bg) % tiles_per_bg * 16;
-      const int p1 = min(P, (min(i1, (bg + 1) * tiles_per_bg) - bg * tiles_per_bg) * 16);
-      if (p1 > p0)
-        bulk_prefetch_l2(c.summary + ((size_t)bg * c.max_pages + p0) * D, (uint32_t)(p1 - p0) * D * 2);
+    int cur = bg_at(i0);
+    for (int i = i0; i < i1;) {
+      int tile;
+      const int bg = locate(i, cur, tile);
+      const int n = min(i1, REAL ? pre[bg + 1] : (bg + 1) * tiles_per_bg) - i;  // tiles of this piece
+      const int p0 = tile * 16, p1 = min(pages_of(bg), (tile + n) * 16);
+      if (p1 > p0) bulk_prefetch_l2(c.summary + ((size_t)bg * c.max_pages + p0) * D, (uint32_t)(p1 - p0) * D * 2);
+      i += n;
     }
   }
   if constexpr (MODE != APPEND_SCORES) griddep_wait();
@@ -102,6 +181,12 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
       __syncwarp();
     }
   }
+  if constexpr (REAL) {  // -inf past each (b, g)'s real tiles
+    for (int bg = gw; bg < BH; bg += nw) {
+      float* row = scores + (size_t)bg * c.max_pages;
+      for (int p = (pre[bg + 1] - pre[bg]) * 16 + lane; p < c.max_pages; p += 32) row[p] = -INFINITY;
+    }
+  }
 
   if (i0 < i1) {
     QFrag<D, BF16> qf;
@@ -109,23 +194,20 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
     float* out = nullptr;
     bool bad = false;
     uint4 av0[2][D / 32], av1[2][D / 32];  // double buffer (compile-time indexed)
+    int lcur = bg_at(i0), ccur = lcur;      // cursors of the loads and of the math
 
-    // where tile item i lives
-    // Reads before the wait (MODE 1) go to L2 (__ldcg): everything they touch was written
-    // by grids that are complete, and no stale L1 line may stand in for it.
-    auto tile_src = [&](int i, int& Pn) -> const uint16_t* {
-      const int bg = i / tiles_per_bg;
-      const int L = __ldcg(&c.seq_len[bg / c.Hkv]);
-      Pn = min((L + kPage - 1) / kPage, c.max_pages);
+    auto tile_src = [&](int i, int& Pn, int& tile) -> const uint16_t* {
+      const int bg = locate(i, lcur, tile);
+      Pn = pages_of(bg);
       return c.summary + (size_t)bg * c.max_pages * D;
     };
     auto compute = [&](int i, const uint4 (&av)[2][D / 32]) {
-      const int bg = i / tiles_per_bg, tile = i % tiles_per_bg;
+      int tile;
+      const int bg = locate(i, ccur, tile);
       if (bg != cur_bg) {  // new (b, g): its query fragments (hi + lo)
         cur_bg = bg;
         const int b = bg / c.Hkv, g = bg % c.Hkv;
-        const int L = __ldcg(&c.seq_len[b]);
-        P = min((L + kPage - 1) / kPage, c.max_pages);
+        P = pages_of(bg);
         out = scores + (size_t)bg * c.max_pages;
         qf.load(q, c.Hq, c.G, b, g, lane, bad);
       }
@@ -137,22 +219,30 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
         if (p1 < c.max_pages) out[p1] = p1 < P ? m1 : -INFINITY;
       }
     };
+    auto load = [&](int i, uint4 (&av)[2][D / 32]) {
+      int Pn, tile;
+      const uint16_t* src = tile_src(i, Pn, tile);
+      load_tile<D>(src, tile, Pn, lane, av);
+    };
 
-    // MODE 1: the tile holding the appended page of each (b, g) in this warp's run; lane j
+    // MODE 1: the item holding the appended page of each (b, g) in this warp's run; lane j
     // keeps that of (b, g) bg0 + j (-1: none).  pos is the caller's, not the append's.
-    const int bg0 = i0 / tiles_per_bg;
-    int my_aff = -1;
+    const int bg0 = bg_at(i0), bg1 = bg_at(i1 - 1);
     auto aff_of = [&](int bg) {
       const int ps = __ldcg(&f.pos[bg / c.Hkv]);
-      return ps >= 0 && ps < c.max_pages * kPage ? bg * tiles_per_bg + (ps / kPage) / 16 : -1;
+      if (ps < 0 || ps >= c.max_pages * kPage) return -1;
+      const int t = (ps / kPage) / 16;
+      if constexpr (REAL) return t < pre[bg + 1] - pre[bg] ? pre[bg] + t : -1;
+      else return bg * tiles_per_bg + t;
     };
-    if (MODE == APPEND_SCORES && bg0 + lane <= (i1 - 1) / tiles_per_bg) my_aff = aff_of(bg0 + lane);
+    int my_aff = -1;
+    if (MODE == APPEND_SCORES && bg0 + lane <= bg1) my_aff = aff_of(bg0 + lane);
     auto held_back = [&](int i) {  // uniform over the warp
       if constexpr (MODE != APPEND_SCORES) {
         return false;
       } else {
-        const int j = i / tiles_per_bg - bg0;
-        return (j < 32 ? __shfl_sync(0xffffffffu, my_aff, j) : aff_of(i / tiles_per_bg)) == i;
+        if (bg1 - bg0 < 32) return __any_sync(0xffffffffu, my_aff == i) != 0;
+        return aff_of(bg_at(i)) == i;
       }
     };
     auto next_tile = [&](int i) {  // the next tile after i scored before the wait
@@ -160,27 +250,26 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
         if (!held_back(i)) break;
       return i;
     };
-    int Pn;
     if constexpr (MODE != APPEND_SCORES) {  // every tile of the run
-      load_tile<D>(tile_src(i0, Pn), i0 % tiles_per_bg, Pn, lane, av0);
+      load(i0, av0);
       for (int i = i0; i < i1; i += 2) {
-        if (i + 1 < i1) load_tile<D>(tile_src(i + 1, Pn), (i + 1) % tiles_per_bg, Pn, lane, av1);
+        if (i + 1 < i1) load(i + 1, av1);
         compute(i, av0);
         if (i + 1 >= i1) break;
-        if (i + 2 < i1) load_tile<D>(tile_src(i + 2, Pn), (i + 2) % tiles_per_bg, Pn, lane, av0);
+        if (i + 2 < i1) load(i + 2, av0);
         compute(i + 1, av1);
       }
     }
     int i = MODE == APPEND_SCORES ? next_tile(i0 - 1) : i1;
     if (i < i1) {
-      load_tile<D>(tile_src(i, Pn), i % tiles_per_bg, Pn, lane, av0);
+      load(i, av0);
       while (true) {  // next tile into the odd buffer, then the even tile's math
         const int j = next_tile(i);
-        if (j < i1) load_tile<D>(tile_src(j, Pn), j % tiles_per_bg, Pn, lane, av1);
+        if (j < i1) load(j, av1);
         compute(i, av0);
         if (j >= i1) break;
         const int k = next_tile(j);
-        if (k < i1) load_tile<D>(tile_src(k, Pn), k % tiles_per_bg, Pn, lane, av0);
+        if (k < i1) load(k, av0);
         compute(j, av1);
         if (k >= i1) break;
         i = k;
@@ -188,9 +277,10 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
     }
     if constexpr (MODE == APPEND_SCORES) {
       griddep_wait();  // the appended tokens' summary rows are written (and this grid ends after the append)
+      lcur = ccur = bg0;
       for (int t = i0; t < i1; ++t) {
         if (!held_back(t)) continue;
-        load_tile<D>(tile_src(t, Pn), t % tiles_per_bg, Pn, lane, av0);
+        load(t, av0);
         compute(t, av0);
       }
     }
@@ -255,20 +345,27 @@ cudaError_t launch_d(const DevCache& c, const void* q, float* scores, const Scor
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
   const int tiles_per_bg = (c.max_pages + 15) / 16;
-  const long long total = (long long)c.B * c.Hkv * tiles_per_bg;
+  const long long total = (long long)c.B * c.Hkv * tiles_per_bg;  // every row full: the most tiles
   const long long blocks_max = 2LL * sm_count(dev);
   const long long warps = blocks_max * kScoreWarps;
   const int per = (int)((total + warps - 1) / warps);
   const long long blocks = (total + (long long)per * kScoreWarps - 1) / ((long long)per * kScoreWarps);
-  size_t smem = 0;
-  if (MODE == APPEND_SCORES_SELECT) {
-    smem = ((size_t)(c.max_pages + 3) / 4 * 4 + kSelScratchWords) * sizeof(uint32_t);
-    const cudaError_t e =
-        cudaFuncSetAttribute(score_kernel<D, BF16, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if constexpr (MODE == APPEND_SCORES_SELECT) {
+    const size_t smem = ((size_t)(c.max_pages + 3) / 4 * 4 + kSelScratchWords) * sizeof(uint32_t);
+    const cudaError_t e = cudaFuncSetAttribute(score_kernel<D, BF16, MODE, false>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    return launch_pdl(score_kernel<D, BF16, MODE, false>, dim3((unsigned)blocks), dim3(kScoreWarps * 32), smem, s,
+                      c, static_cast<const uint16_t*>(q), scores, tiles_per_bg, per, f);
+  } else {
+    // the tile prefix in shared memory while it fits the default 48 KB; whole rows beyond
+    const size_t smem = ((size_t)c.B * c.Hkv + 1) * sizeof(int);
+    if (smem <= 48 * 1024)
+      return launch_pdl(score_kernel<D, BF16, MODE, true>, dim3((unsigned)blocks), dim3(kScoreWarps * 32), smem, s,
+                        c, static_cast<const uint16_t*>(q), scores, tiles_per_bg, per, f);
+    return launch_pdl(score_kernel<D, BF16, MODE, false>, dim3((unsigned)blocks), dim3(kScoreWarps * 32), 0, s, c,
+                      static_cast<const uint16_t*>(q), scores, tiles_per_bg, per, f);
   }
-  return launch_pdl(score_kernel<D, BF16, MODE>, dim3((unsigned)blocks), dim3(kScoreWarps * 32), smem, s, c,
-                    static_cast<const uint16_t*>(q), scores, tiles_per_bg, per, f);
 }
 
 }  // namespace

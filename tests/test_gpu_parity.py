@@ -417,6 +417,32 @@ def test_append_scores_two_steps_equal_calls(kvq, tiers):
             assert torch.equal(sel0[b, g, :c[b, g]], sel1[b, g, :c[b, g]])
 
 
+@pytest.mark.parametrize("B,Hkv", [(1600, 8), (300, 8)])
+def test_ragged_scores_both_splits(kvq, B, Hkv):
+    """kvq_page_scores on a ragged batch with empty sequences: with 12,800 (sequence, kv
+    head) rows the sweep divides whole max_pages rows among the warps, with 2,400 it
+    divides only the tiles that hold pages (and fills -inf past each length).  Scores of a
+    sample of units, the empty ones included, against the oracle's."""
+    rng = np.random.default_rng(B)
+    lens = rng.integers(0, 400, B)
+    lens[:4] = [0, 1, 16, 399]
+    lens[-1] = 0
+    w = W.make("c4", B=B, Hq=Hkv, Hkv=Hkv, lens=lens, append=False)
+    cache = kvq.cache_from_workload(w)
+    step = kvq.DecodeStep(w, cache)
+    step.scores_()
+    torch.cuda.synchronize()
+    assert cache.err_bits() == 0, hex(cache.err_bits())
+    scores = step.scores.cpu().numpy()
+    q, kn, vn = query_and_new(w)
+    units = {(0, 0), (1, Hkv - 1), (2, 3), (3, 5), (B - 1, Hkv - 1), (B - 1, 0)}
+    units |= {(int(b), int(g)) for b, g in zip(rng.integers(0, B, 6), rng.integers(0, Hkv, 6))}
+    for b, g in sorted(units):
+        sh = prepare(w, b, g)
+        r = oracle_step(w, sh, b, g, q, kn, vn)
+        check_scores(scores[b, g], r["scores"], q[b, g:g + 1], sh.summary, r["P"])
+
+
 @pytest.mark.parametrize("P_cap", [700, 5000])
 def test_coverage_selection_matches_oracle(kvq, P_cap):
     """Coverage (nucleus) selection: the GPU set is the oracle's wherever the cut is not
