@@ -23,6 +23,7 @@
 #include "ptx.cuh"
 #include "quant.cuh"
 #include "score_tile.cuh"
+#include "tile_split.cuh"
 
 namespace kvq {
 namespace {
@@ -209,10 +210,11 @@ __device__ inline void quad_load_tile(const uint16_t* sbase, const uint16_t* lba
   }
 }
 
-// Warp w takes tiles [w * per, (w + 1) * per) of the flat list (b, g, 16-page tile), as
-// kvq_page_scores does, loading the next tile (summary rows and lambda rows) while the
-// current one is multiplied; the two buffers take more registers than two CTAs per SM
-// leave, so one CTA of 8 warps runs per SM.
+// Warp w takes a contiguous run of the flat list of 16-page tiles, as kvq_page_scores
+// does -- REAL: only the tiles that hold pages, divided evenly (tile_split.cuh); else
+// [w * per, (w + 1) * per) of every row's max_pages / 16 tiles -- loading the next tile
+// (summary rows and lambda rows) while the current one is multiplied; the two buffers
+// take more registers than two CTAs per SM leave, so one CTA of 8 warps runs per SM.
 // With `ap.pos` set (kvq_quad_append_scores) the warp that owns the tile of a (b, g)'s
 // appended token first writes the token into the cache (quantise, pack, summary) and the
 // quad state, so that tile is read after both are stored.
@@ -222,19 +224,32 @@ struct QuadAppend {
   const uint16_t* v_new;
 };
 
-template <int D, bool BF16, int RK>
+template <int D, bool BF16, int RK, bool REAL>
 __global__ void __launch_bounds__(kQuadWarps * 32, 1)
     quad_score_kernel(DevCache c, DevQuad qd, const uint16_t* __restrict__ q, float sm_scale,
                       float* __restrict__ scores, int tiles_per_bg, int per, QuadAppend ap) {
+  extern __shared__ __align__(16) int pre[];             // REAL: the tile prefix [B * Hkv + 1]
   __shared__ float zs[kQuadWarps][kMaxG][kMaxQuadRank];  // (u_i . q_h)^2 of the warp's current (b, g)
+  __shared__ int s_part[kQuadWarps];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, q4 = lane & 3;
   const int r = qd.rank;
-  const int total = c.B * c.Hkv * tiles_per_bg;
-  const int i0 = (blockIdx.x * kQuadWarps + warp) * per;
-  const int i1 = min(total, i0 + per);
+  const int BH = c.B * c.Hkv;
+  const int nw = gridDim.x * kQuadWarps, gw = blockIdx.x * kQuadWarps + warp;
+  int total, i0, i1;
+  if constexpr (REAL) {  // (no append: the owner of an appended tile is defined on whole rows)
+    total = row_tile_prefix<kQuadWarps * 32>(c, pre, s_part, tid);
+    const int pw = (total + nw - 1) / nw;
+    i0 = min(total, gw * pw);
+    i1 = min(total, i0 + pw);
+  } else {
+    total = BH * tiles_per_bg;
+    i0 = gw * per;
+    i1 = min(total, i0 + per);
+  }
   griddep_wait();
-  if (ap.pos != nullptr && i0 < i1) {  // appends whose page lies in this warp's tiles
+  if constexpr (REAL) fill_past_tiles(c, pre, scores, gw, nw, lane);
+  if (!REAL && ap.pos != nullptr && i0 < i1) {  // appends whose page lies in this warp's tiles
     for (int bg = i0 / tiles_per_bg; bg <= (i1 - 1) / tiles_per_bg; ++bg) {
       const int b = bg / c.Hkv, g = bg % c.Hkv;
       const int ps = ap.pos[b];
@@ -259,20 +274,31 @@ __global__ void __launch_bounds__(kQuadWarps * 32, 1)
     uint4 av0[2][D / 32], av1[2][D / 32];
     uint4 lv0[2][RK], lv1[2][RK];
 
+    int lcur = REAL ? row_of_item(pre, BH, i0) : 0, ccur = lcur;  // forward cursors (REAL)
+    auto locate = [&](int i, int& cur, int& tile) {
+      if constexpr (REAL) {
+        advance_row(pre, cur, i);
+        tile = i - pre[cur];
+        return cur;
+      } else {
+        tile = i % tiles_per_bg;
+        return i / tiles_per_bg;
+      }
+    };
     auto load = [&](int i, uint4 (&av)[2][D / 32], uint4 (&lv)[2][RK]) {
-      const int bg = i / tiles_per_bg;
-      const int L = c.seq_len[bg / c.Hkv];
-      const int Pn = min((L + kPage - 1) / kPage, c.max_pages);
+      int tile;
+      const int bg = locate(i, lcur, tile);
+      const int Pn = row_pages(c, bg);
       quad_load_tile<D, RK>(c.summary + (size_t)bg * c.max_pages * D, qd.lambda + (size_t)bg * c.max_pages * r,
-                            i % tiles_per_bg, Pn, lane, av, lv);
+                            tile, Pn, lane, av, lv);
     };
     auto compute = [&](int i, const uint4 (&av)[2][D / 32], const uint4 (&lv)[2][RK]) {
-      const int bg = i / tiles_per_bg, tile = i % tiles_per_bg;
+      int tile;
+      const int bg = locate(i, ccur, tile);
       if (bg != cur_bg) {  // new (b, g): query fragments and (u_i . q_h)^2
         cur_bg = bg;
         const int b = bg / c.Hkv, g = bg % c.Hkv;
-        const int L = c.seq_len[b];
-        P = min((L + kPage - 1) / kPage, c.max_pages);
+        P = row_pages(c, bg);
         out = scores + (size_t)bg * c.max_pages;
         qf.load(q, c.Hq, c.G, b, g, lane, bad);
         quad_qterms<D, BF16>(qd, qf, g, lane, zs[warp]);
@@ -334,8 +360,12 @@ cudaError_t launch_quad_scores_r(const DevCache& c, const DevQuad& qd, const voi
   const long long warps = (long long)sm_count(dev) * kQuadWarps;  // one CTA per SM (registers)
   const int per = (int)((total + warps - 1) / warps);
   const long long blocks = (total + (long long)per * kQuadWarps - 1) / ((long long)per * kQuadWarps);
-  return launch_pdl(quad_score_kernel<D, BF16, RK>, dim3((unsigned)blocks), dim3(kQuadWarps * 32), 0, s, c, qd,
-                    static_cast<const uint16_t*>(q), sm_scale, scores, tiles_per_bg, per, ap);
+  const size_t smem = ((size_t)c.B * c.Hkv + 1) * sizeof(int);
+  if (ap.pos == nullptr && smem <= 32 * 1024)  // the tile prefix beside the 8 KB of (u_i . q_h)^2
+    return launch_pdl(quad_score_kernel<D, BF16, RK, true>, dim3((unsigned)blocks), dim3(kQuadWarps * 32), smem, s,
+                      c, qd, static_cast<const uint16_t*>(q), sm_scale, scores, tiles_per_bg, per, ap);
+  return launch_pdl(quad_score_kernel<D, BF16, RK, false>, dim3((unsigned)blocks), dim3(kQuadWarps * 32), 0, s, c,
+                    qd, static_cast<const uint16_t*>(q), sm_scale, scores, tiles_per_bg, per, ap);
 }
 
 template <int D, bool BF16>

@@ -14,6 +14,7 @@
 #include "quant.cuh"
 #include "score_tile.cuh"
 #include "select_core.cuh"
+#include "tile_split.cuh"
 
 namespace kvq {
 namespace {
@@ -59,11 +60,8 @@ struct ScoreSelect {
 // completes a (b, g) selects its pages (select_core.cuh) from the scores in L2.
 enum { SCORES = 0, APPEND_SCORES = 1, APPEND_SCORES_SELECT = 2 };
 
-// REAL (modes 0 and 1): only the tiles that hold pages [0, P) of each (b, g) are divided
-// among the warps -- a ragged batch leaves most of a max_pages row empty, and an even split
-// of whole rows would give a few warps all the real tiles.  Each CTA first builds the tile
-// counts' exclusive prefix over (b, g) in shared memory; the scores past the real tiles are
-// -inf, written by a fill.
+// REAL (modes 0 and 1): only the tiles that hold pages are divided among the warps
+// (tile_split.cuh); otherwise every row's max_pages / 16 tiles.
 template <int D, bool BF16, int MODE, bool REAL>
 __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, const uint16_t* __restrict__ q,
                                                                     float* __restrict__ scores, int tiles_per_bg,
@@ -80,43 +78,10 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
   int* pre = reinterpret_cast<int*>(sel_smem);
   // Reads before the wait go to L2 (__ldcg): what they touch was written by grids that are
   // complete, and no stale L1 line may stand in for it.
-  auto pages_of = [&](int bg) {
-    const int L = __ldcg(&c.seq_len[bg / c.Hkv]);
-    return min(max((L + kPage - 1) / kPage, 0), c.max_pages);
-  };
+  auto pages_of = [&](int bg) { return row_pages(c, bg); };
   int total, i0, i1;
   if constexpr (REAL) {
-    const int per_t = (BH + kScoreWarps * 32 - 1) / (kScoreWarps * 32);
-    const int lo = min(BH, tid * per_t), hi = min(BH, lo + per_t);
-    int s = 0;
-    for (int bg = lo; bg < hi; ++bg) {
-      const int t = (pages_of(bg) + 15) / 16;
-      pre[bg] = t;
-      s += t;
-    }
-    int x = s;  // inclusive prefix over the warp's lanes
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) s_part[warp] = x;
-    __syncthreads();
-    int run = x - s, all = 0;
-#pragma unroll
-    for (int w = 0; w < kScoreWarps; ++w) {
-      const int v = s_part[w];
-      if (w < warp) run += v;
-      all += v;
-    }
-    for (int bg = lo; bg < hi; ++bg) {
-      const int t = pre[bg];
-      pre[bg] = run;
-      run += t;
-    }
-    if (tid == 0) pre[BH] = all;
-    __syncthreads();
-    total = all;
+    total = row_tile_prefix<kScoreWarps * 32>(c, pre, s_part, tid);
     const int pw = (total + nw - 1) / nw;
     i0 = min(total, gw * pw);
     i1 = min(total, i0 + pw);
@@ -125,23 +90,15 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
     i0 = gw * per;
     i1 = min(total, i0 + per);
   }
-  // (b, g) of item i: REAL, the last (b, g) whose prefix is <= i
+  // (b, g) of item i
   auto bg_at = [&](int i) {
-    if constexpr (REAL) {
-      int lo = 0, hi = BH - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (pre[mid] <= i) lo = mid; else hi = mid - 1;
-      }
-      return lo;
-    } else {
-      return i / tiles_per_bg;
-    }
+    if constexpr (REAL) return row_of_item(pre, BH, i);
+    else return i / tiles_per_bg;
   };
   // the same with a forward cursor (items visited in increasing order), and the tile
   auto locate = [&](int i, int& cur, int& tile) {
     if constexpr (REAL) {
-      while (pre[cur + 1] <= i) ++cur;
+      advance_row(pre, cur, i);
       tile = i - pre[cur];
       return cur;
     } else {
@@ -181,12 +138,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2) score_kernel(DevCache c, 
       __syncwarp();
     }
   }
-  if constexpr (REAL) {  // -inf past each (b, g)'s real tiles
-    for (int bg = gw; bg < BH; bg += nw) {
-      float* row = scores + (size_t)bg * c.max_pages;
-      for (int p = (pre[bg + 1] - pre[bg]) * 16 + lane; p < c.max_pages; p += 32) row[p] = -INFINITY;
-    }
-  }
+  if constexpr (REAL) fill_past_tiles(c, pre, scores, gw, nw, lane);
 
   if (i0 < i1) {
     QFrag<D, BF16> qf;
