@@ -134,6 +134,82 @@ __device__ inline void emit_chosen(const uint32_t* chosen, int nwords, int32_t* 
   }
 }
 
+// Value bin of a candidate key between the candidates' minimum lo and 256 / range sc
+// (sc == 0: a single bin); NaN (key 0) in bin 256, below all others.
+__device__ inline int sel_bin(uint32_t k, float lo, float sc) {
+  if (k == 0u) return 256;  // NaN
+  const float v = (key_score(k) - lo) * sc;
+  return v >= 255.f ? 255 : (v > 0.f ? static_cast<int>(v) : 0);
+}
+
+// 256 / range of the candidates' scores [lo, hi], or 0 (one bin) when the range is empty,
+// zero or not finite.
+__device__ inline float sel_scale(float lo, float hi) {
+  const float range = hi - lo;
+  float scale = (range > 0.f && range <= 3.0e38f) ? 256.f / range : 0.f;
+  if (!(scale <= 3.0e38f)) scale = 0.f;
+  return scale;
+}
+
+// Warp 0 (lane = its lane): the bin T that holds the kk-th largest candidate (bins in rank
+// order 255 .. 0, then the NaN bin 256) and how many of T's pages are chosen, into
+// sh.prefix and sh.rem.
+__device__ inline void sel_find_bin(const int* hist, int kk, SelShared& sh, int lane) {
+  int h[8], tot = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    h[i] = hist[255 - (lane * 8 + i)];
+    tot += h[i];
+  }
+  int x = tot;  // inclusive prefix over lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  int cum = x - tot;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (cum < kk && kk <= cum + h[i]) {
+      sh.prefix = static_cast<uint32_t>(255 - (lane * 8 + i));
+      sh.rem = kk - cum;
+    }
+    cum += h[i];
+  }
+  if (lane == 31 && cum < kk) {  // the NaN bin
+    sh.prefix = 256u;
+    sh.rem = kk - cum;
+  }
+}
+
+// Warp 0: the radix digit (bits shift .. shift + 7) of the r-th largest key among those
+// matching `prefix` above it, from the digit histogram; new prefix and rank into
+// sh.prefix, sh.rem.
+__device__ inline void sel_find_digit(const int* hist, uint32_t prefix, int shift, int r, SelShared& sh, int lane) {
+  int h8[8], tot = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    h8[i] = hist[lane * 8 + i];
+    tot += h8[i];
+  }
+  int suf = tot;  // sum over lanes >= lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  int cum = suf - tot;  // keys in bins above this lane's bins
+#pragma unroll
+  for (int i = 7; i >= 0; --i) {
+    const int nxt = cum + h8[i];
+    if (cum < r && r <= nxt) {
+      sh.prefix = prefix | (static_cast<uint32_t>(lane * 8 + i) << shift);
+      sh.rem = r - cum;
+    }
+    cum = nxt;
+  }
+}
+
 // Select among the P keys in shared memory (written, and a barrier passed, by the
 // caller); writes the chosen pages in ascending order to out[0 .. min(n, kmax)) and
 // min(n, kmax) to *cnt_out (thread 0).  Flags KVQ_DERR_KMAX if n > kmax.  `scratch` is
@@ -174,11 +250,7 @@ __device__ inline void select_pages(const uint32_t* keys, int P, const kvq_selec
   float smin = 0.f, scale = 0.f;
   uint32_t thr = 0;
   int need = 0;
-  auto bin_of = [](uint32_t k, float lo, float sc) -> int {
-    if (k == 0u) return 256;  // NaN
-    const float v = (key_score(k) - lo) * sc;
-    return v >= 255.f ? 255 : (v > 0.f ? static_cast<int>(v) : 0);
-  };
+  auto bin_of = [](uint32_t k, float lo, float sc) -> int { return sel_bin(k, lo, sc); };
   if (mode == 2) {
     // 1) candidates' score range; clear the histogram
     float lo = INFINITY, hi = -INFINITY;
@@ -212,42 +284,14 @@ __device__ inline void select_pages(const uint32_t* keys, int P, const kvq_selec
       hi = fmaxf(hi, sh.wmax[w]);
     }
     smin = lo;
-    const float range = hi - lo;
-    scale = (range > 0.f && range <= 3.0e38f) ? 256.f / range : 0.f;  // 0: one bin (then the radix select)
-    if (!(scale <= 3.0e38f)) scale = 0.f;
+    scale = sel_scale(lo, hi);  // 0: one bin (then the radix select)
     // 2) histogram (shared atomics; the bins of a warp's pages are mostly distinct)
     pages([&](int, int p, bool valid) {
       if (valid && is_cand(p)) atomicAdd(&hist[bin_of(keys[p], smin, scale)], 1);
     });
     bar();
     // 3) warp 0: bin T holding the kk-th largest (bins in rank order: 255 .. 0, then NaN)
-    if (warp == 0) {
-      int h[8], tot = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        h[i] = hist[255 - (lane * 8 + i)];
-        tot += h[i];
-      }
-      int x = tot;  // inclusive prefix over lanes
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      int cum = x - tot;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (cum < kk && kk <= cum + h[i]) {
-          sh.prefix = static_cast<uint32_t>(255 - (lane * 8 + i));
-          sh.rem = kk - cum;
-        }
-        cum += h[i];
-      }
-      if (lane == 31 && cum < kk) {  // the NaN bin
-        sh.prefix = 256u;
-        sh.rem = kk - cum;
-      }
-    }
+    if (warp == 0) sel_find_bin(hist, kk, sh, lane);
     bar();
     const int T = static_cast<int>(sh.prefix);
     const int rem = sh.rem;
@@ -306,30 +350,7 @@ __device__ inline void select_pages(const uint32_t* keys, int P, const kvq_selec
           }
         });
         bar();
-        if (warp == 0) {
-          int h8[8], tot = 0;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            h8[i] = sh.hist[lane * 8 + i];
-            tot += h8[i];
-          }
-          int suf = tot;  // sum over lanes >= lane
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_down_sync(0xffffffffu, suf, o);
-            if (lane + o < 32) suf += y;
-          }
-          int cum = suf - tot;  // keys in bins above this lane's bins
-#pragma unroll
-          for (int i = 7; i >= 0; --i) {
-            const int nxt = cum + h8[i];
-            if (cum < r && r <= nxt) {
-              sh.prefix = prefix | (static_cast<uint32_t>(lane * 8 + i) << shift);
-              sh.rem = r - cum;
-            }
-            cum = nxt;
-          }
-        }
+        if (warp == 0) sel_find_digit(sh.hist, prefix, shift, r, sh, lane);
         bar();
         prefix = sh.prefix;
         r = sh.rem;

@@ -135,6 +135,38 @@ def test_select_isolated_ties_and_nans(kvq):
         assert bool(cache.err_bits() & kvq.DERR_NAN_SCORE) == nan_any
 
 
+def test_select_few_long_rows(kvq):
+    """Few long rows (the 1024-thread selection): ragged lengths with an empty row, a
+    one-page row, a row shorter than a bitmap word and rows of 4100-8193 pages; integer
+    scores with heavy ties (the radix path), NaNs, -0 and every budget form.  The
+    selection is the oracle's exactly."""
+    from oracle.select import select
+    rng = np.random.default_rng(11)
+    lens = np.array([0, 16, 16 * 20 + 3, 16 * 4100, 16 * 8193 - 5])
+    w = W.make("c4", B=5, Hq=4, Hkv=2, lens=lens, append=False)
+    cache = kvq.cache_from_workload(w)
+    P_cap = w.max_pages
+    sc = rng.integers(-4, 5, (w.B, w.Hkv, P_cap)).astype(np.float32)
+    sc[3, 1] = rng.normal(0, 1, P_cap).astype(np.float32)  # spread-out values: the value bins
+    sc[rng.random(sc.shape) < 0.02] = np.nan
+    sc[rng.random(sc.shape) < 0.02] = -0.0
+    for params in [(-1, 500, 1, 4), (-1, 800, 1, 4), (5, 0, 0, 0), (-1, 10000, 2, 2), (0, 0, 3, 0),
+                   (1000, 0, 1, 1), (40, 0, 0, 0)]:
+        prm = kvq.SelectParams(*params)
+        kmax = P_cap
+        selt = torch.full((w.B, w.Hkv, kmax), -7, dtype=torch.int32, device="cuda")
+        cntt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+        cache.err.zero_()
+        kvq.kvq_select_topk(cache, torch.from_numpy(sc).cuda(), prm, selt, cntt, kmax)
+        got_s, got_c = selt.cpu().numpy(), cntt.cpu().numpy()
+        for b in range(w.B):
+            P = (int(w.lens[b]) + 15) // 16
+            for g in range(w.Hkv):
+                want = select(sc[b, g].astype(np.float64), P, *params)
+                assert list(got_s[b, g, :got_c[b, g]]) == list(want), (params, b, g)
+        assert not (cache.err_bits() & ~kvq.DERR_NAN_SCORE)
+
+
 def test_select_kmax_truncation_flag(kvq):
     w = W.small("c1", append=False)
     cache = kvq.cache_from_workload(w)
