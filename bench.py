@@ -352,29 +352,30 @@ def measure(w, cache, step, path: str, K: int, warmup: int, flush, stream, dev, 
         torch.cuda.synchronize(dev)
         out["ms_per_step_eager"] = max_over_ranks(float(np.mean([a[k].elapsed_time(b_[k]) for k in range(KE)])), dev)
     if e2e:
-        pin = dict(q=step.q.cpu().pin_memory())
-        if w.append:
-            pin["k"], pin["v"] = step.k_new.cpu().pin_memory(), step.v_new.cpu().pin_memory()
-        out_h = torch.empty_like(step.out, device="cpu").pin_memory()
-        lse_h = torch.empty_like(step.lse, device="cpu").pin_memory()
+        # the step's inputs (q, k_new, v_new: one packed buffer) copied in from pinned host
+        # memory and its outputs (out, lse: one packed buffer) copied back, in one graph with
+        # the step's calls
+        pin_in = torch.empty_like(step.io_in, device="cpu").pin_memory()
+        pin_in.copy_(step.io_in)
+        pin_out = torch.empty_like(step.io_out, device="cpu").pin_memory()
+        g_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_e2e):
+            step.io_in.copy_(pin_in, non_blocking=True)
+            run_step()
+            pin_out.copy_(step.io_out, non_blocking=True)
         KE = max(1, min(K, 500))
         es = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
         ee = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
         for k in range(KE):
             flush.fill_(k & 0xFF)
             es[k].record(stream)
-            step.q.copy_(pin["q"], non_blocking=True)
-            if w.append:
-                step.k_new.copy_(pin["k"], non_blocking=True)
-                step.v_new.copy_(pin["v"], non_blocking=True)
-            g_step.replay()
-            out_h.copy_(step.out, non_blocking=True)
-            lse_h.copy_(step.lse, non_blocking=True)
+            g_e2e.replay()
             ee[k].record(stream)
         torch.cuda.synchronize(dev)
+        del g_e2e
         e2e_ms = max_over_ranks(float(np.mean([es[k].elapsed_time(ee[k]) for k in range(KE)])), dev)
-        h2d = pin["q"].numel() * 2 + (pin["k"].numel() * 2 * 2 if w.append else 0)
-        d2h = out_h.numel() * 2 + lse_h.numel() * 4
+        h2d = pin_in.numel()   # bytes of the packed input buffer
+        d2h = pin_out.numel()
         out["e2e"] = {"value": world * w.B / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                       "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
     assert cache.err_bits() == 0, f"device error bits {cache.err_bits():#x}"

@@ -398,8 +398,26 @@ def select_params(w, coverage=None) -> SelectParams:
     return SelectParams(-1, 0, w.n_sink, w.n_recent, int(round(coverage * 1e6)), w.sm_scale)
 
 
+def packed_buffer(specs, device):
+    """One device buffer holding tensors of the given (shape, dtype) at 256-byte aligned
+    offsets, so that one copy moves them all: returns the uint8 buffer and the typed views."""
+    import torch
+    sizes = [int(np.prod(shape)) * torch.empty((), dtype=dt).element_size() for shape, dt in specs]
+    offs, n = [], 0
+    for nb in sizes:
+        n = (n + 255) // 256 * 256
+        offs.append(n)
+        n += nb
+    buf = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+    return buf, [buf[o:o + nb].view(dt).view(shape) for (shape, dt), o, nb in zip(specs, offs, sizes)]
+
+
 class DecodeStep:
     """The buffers and calls of one decode step of workload ``w`` on ``cache``.
+
+    The step's inputs (q, and k_new, v_new when it appends) are views into one device
+    buffer ``io_in`` and its outputs (out, lse) into ``io_out``, so that a caller moves
+    each direction with a single copy.
 
     ``run()`` enqueues: kvq_append (if the workload appends) -> kvq_page_scores ->
     kvq_select_topk -> kvq_sparse_decode_attn, all on the current stream.  With
@@ -412,11 +430,17 @@ class DecodeStep:
         self.w, self.cache = w, cache
         dt = cache.tdtype
         bits = w.query_bits()
-        self.q = torch.from_numpy(bits.view(np.int16)).to(device).view(dt)
+        ins = [(bits.shape, dt)]
         if w.append:
             kn, vn = w.new_kv_bits()
-            self.k_new = torch.from_numpy(kn.view(np.int16)).to(device).view(dt)
-            self.v_new = torch.from_numpy(vn.view(np.int16)).to(device).view(dt)
+            ins += [(kn.shape, dt), (vn.shape, dt)]
+        self.io_in, views = packed_buffer(ins, device)
+        self.q = views[0]
+        self.q.copy_(torch.from_numpy(bits.view(np.int16)).view(dt))
+        if w.append:
+            self.k_new, self.v_new = views[1], views[2]
+            self.k_new.copy_(torch.from_numpy(kn.view(np.int16)).view(dt))
+            self.v_new.copy_(torch.from_numpy(vn.view(np.int16)).view(dt))
             self.pos = torch.from_numpy(np.asarray(w.lens, dtype=np.int32)).to(device)
         self.kmax = w.kmax() if coverage is None else w.max_pages
         self.quad = cache.quad if quad else None
@@ -428,8 +452,8 @@ class DecodeStep:
         self.scores = torch.empty((w.B, w.Hkv, w.max_pages), dtype=torch.float32, device=device)
         self.sel = torch.zeros((w.B, w.Hkv, self.kmax), dtype=torch.int32, device=device)
         self.cnt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device=device)
-        self.out = torch.empty((w.B, w.Hq, w.D), dtype=dt, device=device)
-        self.lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
+        self.io_out, (self.out, self.lse) = packed_buffer([((w.B, w.Hq, w.D), dt), ((w.B, w.Hq), torch.float32)],
+                                                          device)
         nws = max(kvq_workspace_size(cache, self.kmax), kvq_step_workspace_size(cache, self.kmax))
         self.ws = torch.empty((nws + 15) // 16 * 4, dtype=torch.float32, device=device)
         kvq_workspace_init(self.ws)
