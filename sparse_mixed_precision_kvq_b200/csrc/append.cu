@@ -25,6 +25,8 @@ template <bool BF16>
 __global__ void __launch_bounds__(128) append_kernel(DevCache c, const int32_t* __restrict__ pos,
                                                      const uint16_t* __restrict__ k_new,
                                                      const uint16_t* __restrict__ v_new) {
+  __shared__ uint16_t s_k[128], s_v[128];  // the token's K and V rows (D <= 128)
+  __shared__ double s_ks[128];              // the open page's fp64 key sums
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bg = blockIdx.x;
   const int b = bg / c.Hkv, g = bg % c.Hkv;
@@ -33,15 +35,21 @@ __global__ void __launch_bounds__(128) append_kernel(DevCache c, const int32_t* 
   // grid is complete, so that its sweep overlaps this kernel.
   griddep_wait();
   griddep_launch_dependents();
+  // The rows and the sums do not depend on the page: fetched in the same round trip as
+  // pos, ahead of the block-table lookup.
   const int P = pos[b];
+  if (tid < c.D) {
+    s_k[tid] = k_new[(size_t)bg * c.D + tid];
+    s_v[tid] = v_new[(size_t)bg * c.D + tid];
+    s_ks[tid] = c.open_ksum[(size_t)bg * c.D + tid];
+  }
+  __syncthreads();
   if (P >= c.max_pages * kPage) {
     if (tid == 0) set_err(c.err, KVQ_DERR_BAD_POS);
   } else if (P >= 0) {
-    const uint16_t* kr = k_new + (size_t)bg * c.D;
-    const uint16_t* vr = v_new + (size_t)bg * c.D;
-    const bool ok = append_phase1<BF16>(c, b, g, P, kr, tid, 128, nullptr);
+    const bool ok = append_phase1<BF16>(c, b, g, P, s_k, tid, 128, nullptr, s_ks);
     __syncthreads();
-    if (ok) append_phase2<BF16>(c, b, g, P, kr, vr, warp, 4, lane);
+    if (ok) append_phase2<BF16>(c, b, g, P, s_k, s_v, warp, 4, lane);
   }
 }
 

@@ -87,7 +87,7 @@ __device__ inline double to_double(uint16_t v) {
 // Both phases return false (nothing written) if the page's block-table entry is invalid.
 template <bool BF16>
 __device__ inline bool append_phase1(const DevCache& c, int b, int g, int pos, const uint16_t* krow, int t0, int nt,
-                                     uint16_t* patch) {
+                                     uint16_t* patch, const double* ksum_src = nullptr) {
   const int D = c.D;
   const size_t bg = (size_t)b * c.Hkv + g;
   const int page = pos / kPage, t = pos % kPage;
@@ -97,8 +97,8 @@ __device__ inline bool append_phase1(const DevCache& c, int b, int g, int pos, c
   bool ov = false;
   for (int d = t0; d < D; d += nt) {  // running key sum of the open page and its summary
     const double x = to_double<BF16>(krow[d]);
-    double* ks = c.open_ksum + bg * D + d;
-    const double S = (t == 0) ? x : (*ks + x);
+    double* ks = c.open_ksum + bg * D + d;  // ksum_src: the same sums, already fetched
+    const double S = (t == 0) ? x : ((ksum_src != nullptr ? ksum_src[d] : *ks) + x);
     *ks = S;
     const uint16_t m = fp16_sat(S / static_cast<double>(t + 1), ov);
     c.summary[(bg * c.max_pages + page) * D + d] = m;
