@@ -33,8 +33,10 @@ __global__ void __launch_bounds__(NT) select_kernel(DevCache c, const float* __r
   const int bg = blockIdx.x;
   const int b = bg / c.Hkv;
   const int tid = threadIdx.x;
+  // seq_len is an input of the call (no kernel of the step writes it): read through L2
+  // before the wait, so that the score loads go out as soon as the scores are complete
+  const int L = __ldcg(&c.seq_len[b]);
   griddep_wait();
-  const int L = c.seq_len[b];
   const int P = min((L + kPage - 1) / kPage, c.max_pages);
   const float* sc = scores + (size_t)bg * c.max_pages;
   const bool topk = prm.coverage_ppm <= 0;
