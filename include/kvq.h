@@ -9,7 +9,7 @@
  *   kvq_select_topk        pick the top pages plus forced sink/recent pages;
  *   kvq_sparse_decode_attn attend only the selected pages (split-K + log-sum-exp combine),
  *                          unpacking and dequantising cold pages in registers;
- *   kvq_append_scores      the first two in one launch (same results);
+ *   kvq_append_scores      the first two as one call (two chained kernels; same results);
  *   kvq_score_select       the first three in one launch (same results);
  *   kvq_decode_step        the four above in one persistent launch (same results);
  *   kvq_quad_*             the quad (Gaussian-MGF) page score and its per-page state;

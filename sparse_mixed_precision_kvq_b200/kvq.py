@@ -179,7 +179,7 @@ def kvq_decode_step(cache, pos, k_new, v_new, q, params: SelectParams, scores, s
 
 
 def kvq_append_scores(cache, pos, k_new, v_new, q, scores, stream=None):
-    """kvq_append + kvq_page_scores in one launch."""
+    """kvq_append + kvq_page_scores as one call: two chained kernels, the score sweep beside the append."""
     _check(_lib.kvq_append_scores(cache.ref(), _ptr(pos), _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(scores),
                                   _stream(stream)), "kvq_append_scores")
 
@@ -500,7 +500,7 @@ class DecodeStep:
             self.scores_()
 
     def run_three(self):
-        """The same step as ``run()`` in three launches: kvq_append_scores, select, attention."""
+        """The same step as ``run()`` in three calls: kvq_append_scores, select, attention."""
         self.append_scores()
         self.select()
         self.attend()
