@@ -43,12 +43,15 @@ __global__ void __launch_bounds__(NT) select_kernel(DevCache c, const float* __r
   // while loading the keys, the range of the candidates' scores (the selection's first
   // pass) and the histogram's clearing, so that one barrier serves both
   bool nan_seen = false;
-  for (int p0 = tid; p0 < P; p0 += 4 * NT) {  // four loads in flight per thread
-    float v[4];
+  // KB loads in flight per thread: rows of up to 8 * 512 (512 threads) or 9 * 1024 pages
+  // (a 2^k-token context and its appended token) take one round trip
+  constexpr int KB = NT >= 1024 ? 9 : 8;
+  for (int p0 = tid; p0 < P; p0 += KB * NT) {
+    float v[KB];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = p0 + j * NT < P ? sc[p0 + j * NT] : 0.f;
+    for (int j = 0; j < KB; ++j) v[j] = p0 + j * NT < P ? sc[p0 + j * NT] : 0.f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < KB; ++j)
       if (p0 + j * NT < P) keys[p0 + j * NT] = order_key(v[j], nan_seen);
   }
   if (nan_seen) set_err(c.err, KVQ_DERR_NAN_SCORE);
