@@ -3,7 +3,8 @@ kernel's deep-pipeline regime.
 
 * Full size: c1, c2, c3 and c4 with their own batch, heads and context (Llama-3-8B- and
   Qwen2.5-3B-shaped layers at 32k / 131k / ragged 2k-64k context), run through the four
-  C-ABI calls (and c1 through the one-launch fused step).  A seeded sample of (sequence,
+  C-ABI calls (c1 and c4 also through the one-launch fused step, c2 and c4 through
+  kvq_append_scores + select + attention).  A seeded sample of (sequence,
   kv head) units -- always the first and the last, and for c4 the longest and the
   shortest sequence -- is checked against the oracle's step: every page's bytes after the
   append, summaries, open-page key sums, scores, the selected set (bit-exact where the
@@ -94,14 +95,18 @@ def test_full_size_four_calls_match_oracle(kvq, name, n_units):
     _check_units(w, cache, res, sample_units(w, n_units, seed=1), f"{name} full")
 
 
-def test_full_size_fused_step_matches_oracle(kvq):
-    w = W.make("c1")
+@pytest.mark.parametrize("name, path", [("c1", "fused"), ("c4", "fused"), ("c2", "three"), ("c4", "three")])
+def test_full_size_other_paths_match_oracle(kvq, name, path):
+    """The one-launch fused step, and kvq_append_scores (its score sweep beside the append,
+    the appended pages' tiles held back) + select + attention, at full size."""
+    w = W.make(name)
     cache = kvq.cache_from_workload(w)
     step = kvq.DecodeStep(w, cache)
-    step.run_fused()
+    step.run_fused() if path == "fused" else step.run_three()
     res = _results(step, w)
     assert cache.err_bits() == 0, hex(cache.err_bits())
-    _check_units(w, cache, res, sample_units(w, 8, seed=2), "c1 full fused", tail=False)
+    _check_units(w, cache, res, sample_units(w, 12 if name == "c4" else 8, seed=2), f"{name} full {path}",
+                 tail=path != "fused")
 
 
 DEEP = {
