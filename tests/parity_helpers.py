@@ -162,3 +162,16 @@ def check_unit(w, snap, scores, sel, cnt, out, lse, q, kn, vn, b: int, g: int, w
         else:
             assert not np.isfinite(lse[b, h])
     return same
+
+
+def sample_units(w, n: int, seed: int = 0):
+    """n distinct (b, g) units: the first, the last, c4's longest and shortest sequences,
+    then seeded draws."""
+    units = {(0, 0), (w.B - 1, w.Hkv - 1)}
+    if w.name == "c4":
+        bl, bs = int(np.argmax(w.lens)), int(np.argmin(w.lens))
+        units |= {(bl, 0), (bl, w.Hkv - 1), (bs, 0), (bs, w.Hkv - 1)}
+    rng = np.random.default_rng(seed)
+    while len(units) < min(n, w.B * w.Hkv):
+        units.add((int(rng.integers(w.B)), int(rng.integers(w.Hkv))))
+    return sorted(units)

@@ -28,7 +28,8 @@ import torch
 
 from oracle.step import prepare
 from sparse_mixed_precision_kvq_b200 import workloads as W
-from tests.parity_helpers import check_pages, check_summary, check_unit, out_to_f64, query_and_new, snapshot
+from tests.parity_helpers import (check_pages, check_summary, check_unit, out_to_f64, query_and_new, sample_units,
+                                  snapshot)
 
 pytestmark = pytest.mark.gpu
 
@@ -40,19 +41,6 @@ def kvq():
     from sparse_mixed_precision_kvq_b200 import kvq as k
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     return k
-
-
-def sample_units(w, n: int, seed: int = 0):
-    """n distinct (b, g) units: the first, the last, c4's longest and shortest sequences,
-    then seeded draws."""
-    units = {(0, 0), (w.B - 1, w.Hkv - 1)}
-    if w.name == "c4":
-        bl, bs = int(np.argmax(w.lens)), int(np.argmin(w.lens))
-        units |= {(bl, 0), (bl, w.Hkv - 1), (bs, 0), (bs, w.Hkv - 1)}
-    rng = np.random.default_rng(seed)
-    while len(units) < min(n, w.B * w.Hkv):
-        units.add((int(rng.integers(w.B)), int(rng.integers(w.Hkv))))
-    return sorted(units)
 
 
 def _results(step, w):

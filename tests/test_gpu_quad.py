@@ -15,7 +15,7 @@ from oracle.quad import QuadState
 from oracle.select import kth_margin
 from oracle.step import prepare
 from sparse_mixed_precision_kvq_b200 import workloads as W
-from tests.parity_helpers import check_output, oracle_step, out_to_f64, query_and_new
+from tests.parity_helpers import check_output, oracle_step, out_to_f64, query_and_new, sample_units
 
 pytestmark = pytest.mark.gpu
 
@@ -124,6 +124,46 @@ def test_quad_step_matches_oracle(kvq, name):
             for i in range(w.G):
                 check_output(out[b, g * w.G + i], r["out"][i], f"b={b} g={g} h={i}", w.dtype)
     assert compared >= max(1, (w.B * w.Hkv) // 2)
+
+
+@pytest.mark.parametrize("name, n_units", [("c1", 8), ("c4", 12)])
+def test_quad_full_size_matches_oracle(kvq, name, n_units):
+    """The quad-scored step at the workloads' stated sizes (rank 16, the key law's basis;
+    c4: ragged rows, whose quad sweep divides only the tiles that hold pages), on a seeded
+    sample of units: scores within the bound, -inf past each length, the selected set, and
+    every head's output where the set is the oracle's."""
+    w = W.make(name)
+    basis = _basis(w, 16, "law")
+    cache = kvq.cache_from_workload(w, quad_basis=basis)
+    step = kvq.DecodeStep(w, cache, quad=True)
+    step.run()
+    torch.cuda.synchronize()
+    assert cache.err_bits() == 0, hex(cache.err_bits())
+    scores = step.scores.cpu().numpy()
+    sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
+    out = out_to_f64(step.out, w.dtype)
+    q, kn, vn = query_and_new(w)
+    compared = 0
+    units = sample_units(w, n_units, seed=3)
+    for b, g in units:
+        sh = prepare(w, b, g)
+        qs = _oracle_state(w, basis, b, g, sh)
+        r = oracle_step(w, sh, b, g, q, kn, vn, quad=qs)
+        P = r["P"]
+        qg = q[b, g * w.G:(g + 1) * w.G]
+        err = np.abs(scores[b, g, :P].astype(np.float64) - r["scores"][:P])
+        bound = _score_bound(qg, sh.summary, qs.lam, qs.basis, w.sm_scale, P)
+        assert np.all(err <= bound), f"b={b} g={g}: score error {err.max()} (bound {bound[np.argmax(err)]})"
+        assert np.all(np.isneginf(scores[b, g, P:]))
+        got = sel[b, g, :cnt[b, g]]
+        if not np.array_equal(got, r["sel"]):
+            m = kth_margin(r["scores"], P, w.k_abs, w.k_frac_bp, w.n_sink, w.n_recent)
+            assert m <= QUAD_MARGIN, f"b={b} g={g}: selection differs with margin {m}"
+            continue
+        compared += 1
+        for i in range(w.G):
+            check_output(out[b, g * w.G + i], r["out"][i], f"{name} b={b} g={g} h={i}", w.dtype)
+    assert compared >= max(1, len(units) // 2)
 
 
 def test_quad_scores_differ_from_the_plain_score(kvq):
