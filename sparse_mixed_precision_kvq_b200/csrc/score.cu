@@ -47,9 +47,9 @@ struct ScoreSelect {
   unsigned* done;  // [B * Hkv] tiles scored per (b, g) (zero between calls)
 };
 
-// Grid of 2 CTAs per SM; warp w takes the contiguous run of 16-page tiles
-// [w * per, (w + 1) * per) of the flat list (b, g, tile), loading the next tile while
-// the current one is multiplied.
+// Grid of 2 CTAs per SM; warp w takes a contiguous run of the flat list of 16-page tiles
+// in (b, g, tile) order (which tiles the list holds: REAL below), loading the next tile
+// while the current one is multiplied.
 // MODE 1 (kvq_append_scores): the append kernel runs just before this one and writes
 // only the summary row of page pos[b] / 16 of each (b, g).  Every other tile is scored
 // before waiting for that kernel, so the sweep overlaps the append; the tiles holding an
