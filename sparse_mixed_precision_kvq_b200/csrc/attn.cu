@@ -349,15 +349,21 @@ __global__ void __launch_bounds__(kThreads, kRing == kRingWide ? 1 : 2)
       // a warp then runs one tier's page math at a time, which keeps the instruction cache
       // from cycling through every tier's code.  rank = position in (segment, tier, lane)
       // order; the page issued k-th is the lane whose rank is k.
-      const int seg = bgw - __shfl_sync(0xffffffffu, bgw, 0);
-      const int key = lane < win_n ? seg * 8 + (my.tier < 0 ? 7 : my.tier) : 0x7FFFFFFF;
-      int rank = 0;
-#pragma unroll 8
-      for (int j = 0; j < 32; ++j) {
-        const int kj = __shfl_sync(0xffffffffu, key, j);
-        rank += (kj < key) || (kj == key && j < lane);
+      // Segments are contiguous in lane order (lanes past the window form a group of their
+      // own after them), so rank = lanes of earlier segments + lanes of this segment with a
+      // lower tier + lanes of this segment and tier before this one.
+      const int seg = lane < win_n ? bgw : 0x7FFFFFFF;
+      const int tier_k = lane < win_n && my.tier >= 0 ? my.tier : 7;
+      const unsigned same_seg = __match_any_sync(0xffffffffu, seg);
+      unsigned lower = 0u, same_tier = 0u;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const unsigned m = __ballot_sync(0xffffffffu, tier_k == t);
+        if (t < tier_k) lower |= m;
+        if (t == tier_k) same_tier = m;
       }
-      my_rank = rank;
+      const unsigned before = (1u << lane) - 1u;
+      my_rank = (__ffs(same_seg) - 1) + __popc(lower & same_seg) + __popc(same_tier & same_seg & before);
     }
   };
 
