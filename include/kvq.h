@@ -38,6 +38,12 @@
  *    a pipeline wait that ran out) set bits in *err_word (sticky; the caller clears it).
  *    The offending unit is skipped or clamped.  Kernels never trap.
  *  - Calls on different streams that write the same cache memory must not overlap.
+ *  - Kernels are launched with programmatic dependent launch: a call's kernel may start
+ *    while the previous kernel on the stream finishes, and reads some inputs of the call
+ *    (seq_len, the block table, pos, q) before it waits for that kernel.  A kernel of the
+ *    caller that lets its dependents launch early (griddepcontrol.launch_dependents) must
+ *    therefore have written those inputs before it does; kernels that do not (the
+ *    default) finish before the next call's kernels start.
  *
  * Cache layout (all device memory, T = 16 tokens per page, D in {64, 128}):
  *  - block_table [B][max_pages] int32: entry = (tier << 29) | slot, tier in kvq_tier.
