@@ -183,16 +183,17 @@ def kernel_source_hash(kernel_file: str) -> str:
     return h.hexdigest()[:16]
 
 
-def kernel_traffic(kernel_file: str):
+def kernel_traffic(kernel_file: str, workload):
     """ncu DRAM bytes per launch recorded for the current source of a kernel (its file and
-    the headers it includes), else None."""
+    the headers it includes) on `workload` (a plain run of that workload: its own budget
+    selection, mean-key scores, device pools), else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
+    if workload is None or not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel_file)
-    if not e or e.get("source_sha256_16") != kernel_source_hash(kernel_file):
+    if not e or e.get("source_sha256_16") != kernel_source_hash(kernel_file) or e.get("workload") != workload:
         return None
     return e
 
@@ -451,7 +452,9 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     dom_bytes = dominant_bytes(args.path, nbytes, dom)
     files = kernel_files(args.path, bool(quad_rank))
     achieved = dom_bytes / (avg[dom] * 1e-3) / 1e9
-    tr = kernel_traffic(files[dom])
+    plain = (args.coverage is None and args.tier is None and not args.host_tiers and not args.host_v_tiers
+             and args.score == "mean" and args.batch is None)
+    tr = kernel_traffic(files[dom], args.config if plain else None)
     sel, cnt, tier_tbl = m["sel"], m["cnt"], m["tier_tbl"]
     host = None
     if args.host_tiers or args.host_v_tiers:
