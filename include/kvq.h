@@ -209,7 +209,12 @@ kvq_status kvq_page_scores(const kvq_cache* cache, const void* q, float* scores,
  *  cnt     device [B][Hkv] int32 out: entries written to sel (<= kmax).
  *  kmax    row length of sel; a longer selection is truncated and flagged.
  *  With params->coverage_ppm > 0 the k best are replaced by the coverage choice; the
- *  candidates of a sequence (pages minus forced ones) must number at most 8192.
+ *  candidates of a sequence (pages minus forced ones) must number at most 8192 and
+ *  cache->max_pages at most 41984 (else KVQ_ERR_UNSUPPORTED).  The running mass that
+ *  decides the cut is summed in fixed point (2^-46 units, order-independent), so the
+ *  choice is deterministic and is the exact-arithmetic one except where the covered mass
+ *  lies within about 1e-10 of the total from the target; pages of zero mass (NaN or
+ *  underflowed scores) are never chosen as candidates.
  */
 kvq_status kvq_select_topk(const kvq_cache* cache, const float* scores,
                            const kvq_select_params* params, int32_t* sel, int32_t* cnt,

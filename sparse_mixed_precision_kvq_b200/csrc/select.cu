@@ -22,14 +22,16 @@ struct SyncBar {
 };
 
 // NT threads per (b, g): 512, or 1024 when a few long sequences leave most SMs idle.
-template <int NT>
+// COV: coverage selection (its own instance, so that the top-k instance keeps its
+// smaller register count).
+template <int NT, bool COV>
 __global__ void __launch_bounds__(NT) select_kernel(DevCache c, const float* __restrict__ scores,
                                                    kvq_select_params prm, int32_t* __restrict__ sel,
                                                    int32_t* __restrict__ cnt, int kmax, int ncov) {
-  // keys [max_pages, rounded to 2 words]; coverage: then mass keys [ncov] (u64), pages [ncov]
+  // keys [max_pages, rounded to 2 words]; coverage: then the candidates' mass keys [ncov] (u64)
   extern __shared__ __align__(16) uint32_t keys[];
   __shared__ SelShared sh;
-  __shared__ uint32_t scratch[kSelScratchWords];
+  __shared__ __align__(16) uint32_t scratch[kSelScratchWords];
   const int bg = blockIdx.x;
   const int b = bg / c.Hkv;
   const int tid = threadIdx.x;
@@ -39,7 +41,7 @@ __global__ void __launch_bounds__(NT) select_kernel(DevCache c, const float* __r
   griddep_wait();
   const int P = min((L + kPage - 1) / kPage, c.max_pages);
   const float* sc = scores + (size_t)bg * c.max_pages;
-  const bool topk = prm.coverage_ppm <= 0;
+  constexpr bool topk = !COV;
   // while loading the keys, the range of the candidates' scores (the selection's first
   // pass) and the histogram's clearing, so that one barrier serves both
   bool nan_seen = false;
@@ -83,37 +85,36 @@ __global__ void __launch_bounds__(NT) select_kernel(DevCache c, const float* __r
   }
   __syncthreads();
   SyncBar bar;
-  if (prm.coverage_ppm > 0) {
+  if constexpr (COV) {
     unsigned long long* mkey = reinterpret_cast<unsigned long long*>(keys + (c.max_pages + 1) / 2 * 2);
-    uint32_t* mpage = reinterpret_cast<uint32_t*>(mkey + ncov);
-    select_coverage<NT>(keys, P, L, prm, mkey, mpage, scratch + kSelBitmapOff, sel + (size_t)bg * kmax, cnt + bg,
-                        kmax, c.err, sh, tid, bar);
+    select_coverage<NT>(keys, P, L, prm, mkey, scratch, sel + (size_t)bg * kmax, cnt + bg, kmax, c.err, sh, tid,
+                        bar);
   } else {
     select_pages<NT, kPre>(keys, P, prm, sel + (size_t)bg * kmax, cnt + bg, kmax, c.err, scratch, sh, tid, bar);
   }
   griddep_launch_dependents();
 }
 
-template <int NT>
+template <int NT, bool COV>
 cudaError_t launch_select_t(const DevCache& c, const float* scores, const kvq_select_params& prm, int32_t* sel,
                             int32_t* cnt, int kmax, int ncov, cudaStream_t s) {
-  const size_t smem = (size_t)(c.max_pages + 1) / 2 * 2 * sizeof(uint32_t) + (size_t)ncov * 12;
+  const size_t smem = (size_t)(c.max_pages + 1) / 2 * 2 * sizeof(uint32_t) + (size_t)ncov * 8;
   // static (histogram scratch) + dynamic (keys) shared memory may pass the 48 KB default
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<NT, COV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(select_kernel<NT>, dim3(c.B * c.Hkv), dim3(NT), smem, s, c, scores, prm, sel, cnt, kmax, ncov);
+  return launch_pdl(select_kernel<NT, COV>, dim3(c.B * c.Hkv), dim3(NT), smem, s, c, scores, prm, sel, cnt, kmax,
+                    ncov);
 }
 
 }  // namespace
 
-// Sort slots coverage selection needs: a power of two >= the candidates of the longest
-// possible sequence (max_pages minus the forced pages); 0 if above kCovMaxCand.
+// Mass-key slots coverage selection needs: the candidates of the longest possible
+// sequence (max_pages minus the forced pages), at least 1; 0 if above kCovMaxCand or if
+// the sequence's pages exceed kCovMaxPages.
 int coverage_sort_size(const DevCache& c, const kvq_select_params& prm) {
   const int forced = max(prm.n_sink, 0) + max(prm.n_recent, 0);
   const int nc = max(1, c.max_pages - min(forced, c.max_pages));
-  int n = 1;
-  while (n < nc) n <<= 1;
-  return n <= kCovMaxCand ? n : 0;
+  return nc <= kCovMaxCand && c.max_pages <= kCovMaxPages ? nc : 0;
 }
 
 cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_select_params& prm,
@@ -122,8 +123,11 @@ cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_sele
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
   const bool wide = (long long)c.B * c.Hkv * 4 <= sm_count(dev) && c.max_pages >= 4096;
   const int ncov = prm.coverage_ppm > 0 ? coverage_sort_size(c, prm) : 0;
-  return wide ? launch_select_t<1024>(c, scores, prm, sel, cnt, kmax, ncov, s)
-              : launch_select_t<512>(c, scores, prm, sel, cnt, kmax, ncov, s);
+  if (ncov > 0)
+    return wide ? launch_select_t<1024, true>(c, scores, prm, sel, cnt, kmax, ncov, s)
+                : launch_select_t<512, true>(c, scores, prm, sel, cnt, kmax, ncov, s);
+  return wide ? launch_select_t<1024, false>(c, scores, prm, sel, cnt, kmax, 0, s)
+              : launch_select_t<512, false>(c, scores, prm, sel, cnt, kmax, 0, s);
 }
 
 }  // namespace kvq

@@ -71,6 +71,9 @@ struct SelShared {
   uint32_t prefix;
   int rem;
   int ncand;
+  // coverage selection
+  unsigned long long ckmin, ckmax, cabove;
+  int cbin, ccount;
 };
 
 // Exclusive prefix sum of one int per thread over NT threads; *total receives the sum.
@@ -407,11 +410,32 @@ __device__ inline void select_pages(const uint32_t* keys, int P, const kvq_selec
 // attention mass is estimated from its score as n_p * exp(sm_scale * (s_p - s_max)) (fp64;
 // n_p its valid tokens; NaN -> 0); the forced pages count as covered, and candidates are
 // added by mass (larger first, lower page first on ties) until the covered mass reaches
-// coverage * the total.  The candidates are sorted in shared memory (bitonic, N a power of
-// two >= their count), the sorted masses scanned (fp64), and the chosen pages emitted
-// through the same bitmap as the top-k selection.
+// coverage * the total.
+//
+// The chosen set is found without sorting, by an MSB-first radix search over the masses'
+// fp64 bit patterns (non-negative doubles order like their bits).  Each pass histograms
+// the candidates still undecided by the next (up to) 8 bits of their key, with a count and
+// a mass sum per bin, and one warp finds the bin in which the running mass, taken from the
+// heaviest bin down, reaches the target: heavier bins are chosen whole, lighter ones not,
+// and the search continues inside that bin until it holds one page or one exact mass (then
+// its lowest pages are taken, as many as reach the target).  The bin sums are fixed-point
+// integers (units of 2^-46, rounded down), kept as three 17-bit parts in 32-bit counters (a
+// mass is at most 16 = 2^50 units, so 8192 candidates sum below 2^30 in each part); they do
+// not depend on the order of the additions, and the selection is deterministic.  A warp
+// whose 32 candidates fall in at most 4 bins first merges the lanes of each bin (match +
+// warp reductions), so a bin that takes most candidates sees one shared atomic per warp,
+// not one per page; a warp spread over more bins adds lane by lane (warp reductions whose
+// lanes name many different groups ran several times slower).  Rounding 8192 masses down
+// loses under 2^-33 of a total of at least 1 (the page of the largest score has mass >= 1),
+// so the cut moves only where the covered mass is that close to the target.  Candidates
+// of zero mass are never taken: with coverage <= 1 the positive masses reach
+// the target in exact arithmetic, so when the rounded sums fall short of it (coverage 1)
+// every candidate of positive mass is taken, and no other.
 
-constexpr int kCovMaxCand = 8192;  // candidates one CTA sorts in shared memory
+constexpr int kCovMaxCand = 8192;  // candidates of one sequence (their mass keys sit in shared memory)
+constexpr int kCovFixBits = 46;    // fixed-point fraction bits of the bin sums
+constexpr int kCovEqOff = 1024;    // scratch: [0, 768) bin sums (3 parts), [768, 1024) counts, then the cut's pages
+constexpr int kCovMaxPages = (kSelBitmapOff - kCovEqOff) * 32;  // pages whose cut bitmap fits before the bitmap
 
 // Sum of one double per thread (fixed tree: the same order in every call).
 template <int NT, typename Bar>
@@ -429,43 +453,61 @@ __device__ inline double sel_block_sum(double v, SelShared& sh, int tid, Bar& ba
   return t;
 }
 
-// Inclusive prefix sums of the doubles a[0..n) in place, contiguous chunks per thread.
-template <int NT, typename Bar>
-__device__ inline void sel_prefix_sum(double* a, int n, SelShared& sh, int tid, Bar& bar) {
-  const int lane = tid & 31, warp = tid >> 5;
-  const int per = (n + NT - 1) / NT;
-  const int lo = min(n, tid * per), hi = min(n, lo + per);
-  double run = 0.0;
-  for (int i = lo; i < hi; ++i) run += a[i];
-  double x = run;  // inclusive scan over threads
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) sh.dsum[warp] = x;
-  bar();
-  double before = x - run;
-  for (int w = 0; w < warp; ++w) before += sh.dsum[w];
-  for (int i = lo; i < hi; ++i) {
-    before += a[i];
-    a[i] = before;
-  }
-  bar();
+// Fixed-point mass (units of 2^-kCovFixBits, rounded down) of a mass key.
+__device__ inline unsigned long long cov_fixed(unsigned long long key) {
+  return __double2ull_rz(__longlong_as_double(static_cast<long long>(key)) * 0x1p46);
 }
 
-// keys: the P order keys (scores) in shared memory; mkey/mpage: 2 * kCovMaxCand words
-// and kCovMaxCand words of shared memory; chosen: the bitmap area (ceil(P / 32) words).
+// Warp 0: the bin where the running mass from the top bin down first reaches need_q (the
+// mass above the bins is `above`), into sh.cbin (-1: the bins never reach it), sh.cabove
+// (the mass above that bin) and sh.ccount (its pages).  bs: the bins' three sum parts.
+__device__ inline void cov_find_bin(const uint32_t* bs, const int* bcnt, unsigned long long above,
+                                    unsigned long long need_q, SelShared& sh, int lane) {
+  unsigned long long s8[8], own = 0ull;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int b = 8 * lane + i;
+    s8[i] = static_cast<unsigned long long>(bs[b]) + (static_cast<unsigned long long>(bs[256 + b]) << 17) +
+            (static_cast<unsigned long long>(bs[512 + b]) << 34);
+    own += s8[i];
+  }
+  unsigned long long suf = own;  // mass of this lane's bins and every higher lane's
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  if (lane == 0 && above + suf < need_q) sh.cbin = -1;
+  unsigned long long cum = above + (suf - own);  // mass of the bins above this lane's
+#pragma unroll
+  for (int i = 7; i >= 0; --i) {
+    const unsigned long long nxt = cum + s8[i];
+    if (cum < need_q && need_q <= nxt) {
+      sh.cbin = 8 * lane + i;
+      sh.cabove = cum;
+      sh.ccount = bcnt[8 * lane + i];
+    }
+    cum = nxt;
+  }
+}
+
+// keys: the P order keys (scores) in shared memory; mkey: kCovMaxCand 64-bit slots of
+// shared memory (8-byte aligned); scratch: kSelScratchWords words of shared memory,
+// 8-byte aligned (bin sums and counts at its start, the bitmap at kSelBitmapOff).
 template <int NT, typename Bar>
 __device__ inline void select_coverage(const uint32_t* keys, int P, int L, const kvq_select_params& prm,
-                                       unsigned long long* mkey, uint32_t* mpage, uint32_t* chosen, int32_t* out,
-                                       int32_t* cnt_out, int kmax, uint32_t* err, SelShared& sh, int tid, Bar& bar) {
+                                       unsigned long long* mkey, uint32_t* scratch, int32_t* out, int32_t* cnt_out,
+                                       int kmax, uint32_t* err, SelShared& sh, int tid, Bar& bar) {
   constexpr int NW = NT / 32;
   const int lane = tid & 31, warp = tid >> 5;
   const SelectSplit sp = select_split(P, prm);
   const int ns = sp.ns, rs = sp.rs, nC = sp.nC;
   auto is_cand = [&](int p) { return p >= ns && p < rs; };
   const int nwords = (P + 31) / 32;
+  uint32_t* bs = scratch;                                                     // [3][256]
+  int* bcnt = reinterpret_cast<int*>(scratch + 768);                          // [256]
+  uint32_t* eqm = scratch + kCovEqOff;                                        // [nwords]
+  uint32_t* chosen = scratch + kSelBitmapOff;
   // 1) largest finite score
   float hi = -INFINITY;
   for (int p = tid; p < P; p += NT)
@@ -473,82 +515,165 @@ __device__ inline void select_coverage(const uint32_t* keys, int P, int L, const
 #pragma unroll
   for (int o = 16; o; o >>= 1) hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
   if (lane == 0) sh.wmax[warp] = hi;
+  if (tid == 0) {
+    sh.ckmin = ~0ull;
+    sh.ckmax = 0ull;
+  }
   bar();
   float smax = -INFINITY;
 #pragma unroll
   for (int w = 0; w < NW; ++w) smax = fmaxf(smax, sh.wmax[w]);
   const double scale = static_cast<double>(prm.sm_scale);
-  auto mass = [&](int p) -> double {
-    const uint32_t k = keys[p];
-    if (k == 0u || !(smax > -INFINITY)) return 0.0;
-    const double n = p == P - 1 ? static_cast<double>(L - kPage * (P - 1)) : static_cast<double>(kPage);
-    return n * exp(scale * (static_cast<double>(key_score(k)) - static_cast<double>(smax)));
-  };
-  // 2) the candidates' (mass, page) in sort slots 0..nC-1, padding after; the totals
-  int N = 1;
-  while (N < nC) N <<= 1;
+  // 2) every page's mass once: the candidates' keys into mkey[p - ns], the totals, the
+  //    candidates' key range
   double tot = 0.0, forced = 0.0;
+  unsigned long long kmin = ~0ull, kmx = 0ull;
   for (int p = tid; p < P; p += NT) {
-    const double m = mass(p);
+    const uint32_t k = keys[p];
+    double m = 0.0;
+    if (k != 0u && smax > -INFINITY) {
+      const double n = p == P - 1 ? static_cast<double>(L - kPage * (P - 1)) : static_cast<double>(kPage);
+      m = n * exp(scale * (static_cast<double>(key_score(k)) - static_cast<double>(smax)));
+    }
     tot += m;
-    if (!is_cand(p)) forced += m;
-  }
-  for (int i = tid; i < N; i += NT) {
-    if (i < nC) {  // the candidates are the pages ns .. rs - 1
-      mkey[i] = static_cast<unsigned long long>(__double_as_longlong(mass(ns + i)));
-      mpage[i] = static_cast<uint32_t>(ns + i);
+    if (is_cand(p)) {
+      const unsigned long long mk = static_cast<unsigned long long>(__double_as_longlong(m));
+      mkey[p - ns] = mk;
+      kmin = min(kmin, mk);
+      kmx = max(kmx, mk);
     } else {
-      mkey[i] = 0ull;
-      mpage[i] = 0x7FFFFFFFu;
+      forced += m;
     }
   }
-  for (int i = tid; i < nwords; i += NT) chosen[i] = 0u;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
+  }
+  if (lane == 0) {
+    atomicMin(&sh.ckmin, kmin);
+    atomicMax(&sh.ckmax, kmx);
+  }
   const double total = sel_block_sum<NT>(tot, sh, tid, bar);
   const double fsum = sel_block_sum<NT>(forced, sh, tid, bar);
   const double need = static_cast<double>(prm.coverage_ppm) * 1e-6 * total - fsum;
-  int kstar = 0;
+  // 3) the cut: every candidate whose key is above `prefix` in the bits >= shift, and the
+  //    r lowest pages of those equal to it there (mode 1); none (0); all of positive mass (2)
+  int mode = 0, shift = 0, r = 0;
+  unsigned long long prefix = 0ull;
   if (need > 0.0 && nC > 0) {
-    // 3) bitonic sort: mass descending, then page ascending (masses are >= 0: their bits
-    //    order like the values)
-    for (int size = 2; size <= N; size <<= 1) {
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int t = tid; t < N / 2; t += NT) {
-          const int i = 2 * t - (t & (stride - 1));
-          const int j = i + stride;
-          const bool down = (i & size) == 0;  // this run sorts "first before" (descending)
-          const unsigned long long ki = mkey[i], kj = mkey[j];
-          const uint32_t pi = mpage[i], pj = mpage[j];
-          const bool j_first = kj > ki || (kj == ki && pj < pi);
-          if (j_first == down) {
-            mkey[i] = kj;
-            mkey[j] = ki;
-            mpage[i] = pj;
-            mpage[j] = pi;
+    const unsigned long long need_q = __double2ull_ru(need * 0x1p46);  // >= 1 (2^kCovFixBits units)
+    const unsigned long long lo = sh.ckmin, hk = sh.ckmax;
+    shift = lo == hk ? 0 : 64 - __clzll(static_cast<long long>(lo ^ hk));  // bits below it are common
+    prefix = hk;
+    unsigned long long above = 0ull;
+    int count = nC;
+    mode = 1;
+    while (shift > 0 && count > 1) {
+      const int low = max(shift - 8, 0);
+      const unsigned long long hm = shift >= 64 ? 0ull : (~0ull << shift);
+      const unsigned long long want = prefix & hm;
+      for (int i = tid; i < 1024; i += NT) scratch[i] = 0u;  // sum parts and counts
+      bar();
+      for (int i0 = warp * 32; i0 < nC; i0 += NT) {  // warp-uniform rounds of 32 candidates
+        const int i = i0 + lane;
+        int bin = -1;
+        unsigned long long q = 0ull;
+        if (i < nC) {
+          const unsigned long long k = mkey[i];
+          if ((k & hm) == want) {
+            bin = static_cast<int>((k >> low) & ((1ull << (shift - low)) - 1ull));
+            q = cov_fixed(k);
           }
         }
-        bar();
+        const unsigned grp = __match_any_sync(0xffffffffu, bin);  // lanes of this lane's bin
+        const unsigned leads = __ballot_sync(0xffffffffu, bin >= 0 && lane == __ffs(grp) - 1);
+        if (__popc(leads) > 4) {  // spread over many bins: every lane adds its own (few conflicts)
+          if (bin >= 0) {
+            atomicAdd(&bs[bin], static_cast<unsigned>(q & 0x1FFFFull));
+            atomicAdd(&bs[256 + bin], static_cast<unsigned>((q >> 17) & 0x1FFFFull));
+            atomicAdd(&bs[512 + bin], static_cast<unsigned>(q >> 34));
+            atomicAdd(&bcnt[bin], 1);
+          }
+        } else if (bin >= 0) {  // a few bins: one addition per bin, the group's sums reduced first
+          const unsigned s0 = __reduce_add_sync(grp, static_cast<unsigned>(q & 0x1FFFFull));
+          const unsigned s1 = __reduce_add_sync(grp, static_cast<unsigned>((q >> 17) & 0x1FFFFull));
+          const unsigned s2 = __reduce_add_sync(grp, static_cast<unsigned>(q >> 34));
+          if (lane == __ffs(grp) - 1) {
+            atomicAdd(&bs[bin], s0);
+            atomicAdd(&bs[256 + bin], s1);
+            atomicAdd(&bs[512 + bin], s2);
+            atomicAdd(&bcnt[bin], __popc(grp));
+          }
+        }
+      }
+      bar();
+      if (warp == 0) cov_find_bin(bs, bcnt, above, need_q, sh, lane);
+      bar();
+      const int b = sh.cbin;
+      if (b < 0) {  // even every candidate left does not reach the target: all of positive mass
+        mode = 2;
+        break;
+      }
+      prefix = want | (static_cast<unsigned long long>(b) << low);
+      above = sh.cabove;
+      count = sh.ccount;
+      shift = low;  // (the next pass writes the bins and sh.c* only after two more barriers)
+    }
+    if (mode == 1) {
+      if (count <= 1) {
+        r = count;
+      } else {  // `count` candidates of one exact mass: the fewest of them that reach the target
+        const unsigned long long q = cov_fixed(prefix);
+        const unsigned long long rq = q > 0ull ? (need_q - above + q - 1ull) / q : static_cast<unsigned long long>(count);
+        r = rq < static_cast<unsigned long long>(count) ? static_cast<int>(rq) : count;
       }
     }
-    // 4) prefix sums of the sorted masses; the cut is the first prefix reaching `need`
-    double* pre = reinterpret_cast<double*>(mkey);
-    for (int i = tid; i < nC; i += NT) pre[i] = __longlong_as_double(static_cast<long long>(mkey[i]));
-    bar();
-    sel_prefix_sum<NT>(pre, nC, sh, tid, bar);
-    if (tid == 0) sh.rem = nC;
-    bar();
-    for (int i = tid; i < nC; i += NT)
-      if (pre[i] >= need && (i == 0 || pre[i - 1] < need)) sh.rem = i + 1;
-    bar();
-    kstar = sh.rem;
-    for (int i = tid; i < kstar; i += NT) {
-      const uint32_t p = mpage[i];
-      atomicOr(&chosen[p >> 5], 1u << (p & 31));
+  }
+  // 4) the bitmap: forced pages and the candidates above the cut (one ballot per word),
+  //    and the candidates at the cut in eqm
+  const unsigned long long hm = shift >= 64 ? 0ull : (~0ull << shift);
+  const unsigned long long want = prefix & hm;
+  for (int wd = warp; wd < nwords; wd += NW) {
+    const int p = 32 * wd + lane;
+    bool take = false, at = false;
+    if (p < P) {
+      if (!is_cand(p)) {
+        take = true;
+      } else if (mode == 2) {
+        take = mkey[p - ns] != 0ull;
+      } else if (mode == 1) {
+        const unsigned long long k = mkey[p - ns] & hm;
+        take = k > want;
+        at = k == want;
+      }
+    }
+    const unsigned tm = __ballot_sync(0xffffffffu, take), am = __ballot_sync(0xffffffffu, at);
+    if (lane == 0) {
+      chosen[wd] = tm;
+      eqm[wd] = am;
     }
   }
-  // 5) forced pages
-  for (int p = tid; p < P; p += NT)
-    if (!is_cand(p)) atomicOr(&chosen[p >> 5], 1u << (p & 31));
   bar();
+  if (mode == 1 && r > 0) {  // the r lowest pages at the cut (block scan over word ranges)
+    const int WPT = (nwords + NT - 1) / NT;
+    const int w_lo = min(nwords, tid * WPT), w_hi = min(nwords, w_lo + WPT);
+    int eq = 0;
+    for (int wd = w_lo; wd < w_hi; ++wd) eq += __popc(eqm[wd]);
+    int tot_eq;
+    int e = sel_exclusive_scan<NT>(eq, sh, &tot_eq, tid, bar);
+    for (int wd = w_lo; wd < w_hi && e < r; ++wd) {
+      unsigned m = eqm[wd], add = 0u;
+      while (m && e < r) {
+        const unsigned bit = m & (0u - m);
+        add |= bit;
+        m ^= bit;
+        ++e;
+      }
+      chosen[wd] |= add;
+    }
+    bar();
+  }
   emit_chosen<NT>(chosen, nwords, out, cnt_out, kmax, err, sh, tid, bar);
 }
 

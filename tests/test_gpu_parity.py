@@ -515,6 +515,64 @@ def test_coverage_selection_matches_oracle(kvq, P_cap):
     assert checked >= 40
 
 
+@pytest.mark.parametrize("kind", ["ties", "wide"])
+def test_coverage_exact_ties_and_wide_masses(kvq, kind):
+    """Coverage selection where the cut lands inside a group of exactly equal masses
+    (scores from four values: the group's lowest pages are taken, as many as reach the
+    target) or where the masses span hundreds of binades (the search descends through many
+    digit passes).  The set must be the oracle's wherever the covered mass is not within
+    1e-5 of the target; exact ties are part of the rule, not an ambiguity."""
+    from oracle.select import forced_pages, page_masses, select_coverage
+    import math
+    rng = np.random.default_rng(11 if kind == "ties" else 12)
+    B, Hkv = 8, 2
+    lens = rng.integers(200, 16 * 600 + 1, B)
+    w = W.make("c4", B=B, Hq=8, Hkv=Hkv, lens=lens, append=False)
+    cache = kvq.cache_from_workload(w)
+    if kind == "ties":
+        sc = (rng.integers(0, 4, (B, Hkv, w.max_pages)) * 2.0).astype(np.float32)
+        cases = [(0.3, 1.0, 1, 2), (0.5, 1.0, 0, 0), (0.7, 0.7, 2, 1), (0.9, 1.0, 0, 3), (0.97, 0.5, 1, 0)]
+    else:
+        sc = rng.normal(0, 40, (B, Hkv, w.max_pages)).astype(np.float32)
+        cases = [(0.999, 1.0, 1, 2), (0.9999, 0.5, 0, 0), (0.5, 2.0, 0, 1), (0.99, 0.25, 2, 0)]
+    checked = 0
+    for cov, scale, ns, nr in cases:
+        ppm = int(round(cov * 1e6))
+        prm = kvq.SelectParams(-1, 0, ns, nr, ppm, scale)
+        kmax = w.max_pages
+        selt = torch.full((B, Hkv, kmax), -7, dtype=torch.int32, device="cuda")
+        cntt = torch.zeros((B, Hkv), dtype=torch.int32, device="cuda")
+        cache.err.zero_()
+        kvq.kvq_select_topk(cache, torch.from_numpy(sc).cuda(), prm, selt, cntt, kmax)
+        got_s, got_c = selt.cpu().numpy(), cntt.cpu().numpy()
+        assert cache.err_bits() == 0
+        for b in range(B):
+            L = int(w.lens[b])
+            P = (L + 15) // 16
+            for g in range(Hkv):
+                s64 = sc[b, g].astype(np.float64)
+                want = select_coverage(s64, P, L, scale, ppm * 1e-6, ns, nr)
+                got = list(got_s[b, g, :got_c[b, g]])
+                # distance of the covered mass from the target, before and after the last page
+                m = page_masses(s64, P, L, scale)
+                F = forced_pages(P, ns, nr)
+                total, target = math.fsum(m), ppm * 1e-6 * math.fsum(m)
+                covered = math.fsum(m[p] for p in F)
+                order = sorted((p for p in range(P) if p not in F), key=lambda p: (-m[p], p))
+                k = 0
+                while k < len(order) and covered < target:
+                    covered += m[order[k]]
+                    k += 1
+                before = covered - (m[order[k - 1]] if k else 0.0)
+                dist = min(abs(target - before), abs(covered - target)) / total
+                gap_ok = not (0 < k < len(order)) or m[order[k - 1]] == m[order[k]] or \
+                    (m[order[k - 1]] - m[order[k]]) / m[order[k - 1]] > 1e-5
+                if dist > 1e-5 and gap_ok:
+                    assert got == list(want), (kind, cov, b, g, len(got), len(want))
+                    checked += 1
+    assert checked >= 40
+
+
 def test_coverage_step_through_attention(kvq):
     """A whole step with coverage selection: the pages chosen and the attention over them
     match the oracle's."""
