@@ -126,6 +126,43 @@ def test_quad_step_matches_oracle(kvq, name):
     assert compared >= max(1, (w.B * w.Hkv) // 2)
 
 
+@pytest.mark.parametrize("name", ["c1_r16_random", "c4_r24_random"])
+def test_quad_coverage_step_matches_oracle(kvq, name):
+    """Coverage selection on quad scores: the mass of page p is n_p * exp(quad_p) (the
+    score already carries the softmax scale, so the binding passes sm_scale = 1).  The
+    chosen set is the oracle's coverage set on its own quad scores wherever the cut is
+    clear of the scores' fp32 rounding (margin 1e-3), and the outputs are the oracle's
+    attention over the chosen pages."""
+    from oracle.select import coverage_margin, select_coverage
+    mk, rank, kind = CASES[name]
+    w = mk()
+    basis = _basis(w, rank, kind)
+    cache = kvq.cache_from_workload(w, quad_basis=basis)
+    step = kvq.DecodeStep(w, cache, coverage=0.9, quad=True)
+    assert step.params.sm_scale == 1.0
+    step.run()
+    torch.cuda.synchronize()
+    assert cache.err_bits() == 0, hex(cache.err_bits())
+    sel, cnt = step.sel.cpu().numpy(), step.cnt.cpu().numpy()
+    out = out_to_f64(step.out, w.dtype)
+    q, kn, vn = query_and_new(w)
+    compared = 0
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            sh = prepare(w, b, g)
+            r = oracle_step(w, sh, b, g, q, kn, vn, quad=_oracle_state(w, basis, b, g, sh))
+            L, P = int(w.final_lens()[b]), r["P"]
+            got = sel[b, g, :cnt[b, g]]
+            if coverage_margin(r["scores"], P, L, 1.0, 0.9, w.n_sink, w.n_recent) > 1e-3:
+                want = select_coverage(r["scores"], P, L, 1.0, 0.9, w.n_sink, w.n_recent)
+                assert list(got) == list(want), (b, g, len(got), len(want))
+                compared += 1
+            r2 = oracle_step(w, prepare(w, b, g), b, g, q, kn, vn, sel=got.astype(np.int64))
+            for i in range(w.G):
+                check_output(out[b, g * w.G + i], r2["out"][i], f"quad coverage b={b} g={g} h={i}", w.dtype)
+    assert compared >= max(1, (w.B * w.Hkv) // 2)
+
+
 @pytest.mark.parametrize("name, n_units", [("c1", 8), ("c4", 12)])
 def test_quad_full_size_matches_oracle(kvq, name, n_units):
     """The quad-scored step at the workloads' stated sizes (rank 16, the key law's basis;
