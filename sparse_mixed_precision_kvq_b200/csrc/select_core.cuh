@@ -454,6 +454,7 @@ __device__ inline double sel_block_sum(double v, SelShared& sh, int tid, Bar& ba
 }
 
 // Fixed-point mass (units of 2^-kCovFixBits, rounded down) of a mass key.
+static_assert(kCovFixBits == 46, "cov_fixed and the target scale by 2^46");
 __device__ inline unsigned long long cov_fixed(unsigned long long key) {
   return __double2ull_rz(__longlong_as_double(static_cast<long long>(key)) * 0x1p46);
 }
