@@ -13,8 +13,13 @@ kvq_select_topk -> kvq_sparse_decode_attn; ``--path fused`` as the single
 kvq_decode_step launch.
 
 Timing: W untimed steps, then K steps replayed from a CUDA graph of the step and timed
-on the device with CUDA events on the launching stream around each replay (L2 is
-flushed by writing a 512 MiB buffer before every timed step, outside the events).
+on the device with CUDA events on the launching stream around each replay.  Before every
+timed step, outside the events, L2 is flushed: a 512 MiB buffer is written (every L2 line
+replaced), then a 256 MiB buffer is read, so that the dirty lines of that write are
+written back before the step starts and L2 holds no line of the step's data and no
+dirty line (a decode loop enters a layer's step with L2 holding other layers' clean
+lines, not a backlog of write-backs).  The same steps after the write alone are reported
+as ``ms_per_step_write_only_flush``.
 Per-kernel durations come from a second graph of the same step with events between the
 calls, replayed right after the timed loop.  The whole-step time is bracketed by a barrier + synchronize; with N > 1
 (torchrun, one process per GPU, NCCL) every rank runs its own independent batch (weak
@@ -257,6 +262,24 @@ def kernel_files(path: str, quad: bool):
             "calls": ["append.cu", sc, "select.cu", "attn.cu"]}[path]
 
 
+class L2Flush:
+    """The L2 flush between timed steps: ``fill_(v)`` writes the whole write buffer (more
+    than L2), then reads the read buffer (more than L2), evicting the write's dirty lines;
+    ``write_only(v)`` does the write alone."""
+
+    def __init__(self, mib: int, dev):
+        import torch
+        self.w = torch.empty(mib << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(max(mib // 2, 160) << 18, dtype=torch.float32, device=dev)
+
+    def fill_(self, v: int):
+        self.w.fill_(v)
+        self.r.amax()
+
+    def write_only(self, v: int):
+        self.w.fill_(v)
+
+
 def measure(w, cache, step, path: str, K: int, warmup: int, flush, stream, dev, world: int, peak: float,
             quad_rank: int = 0, soak_s: float = 0.0, e2e: bool = True, eager: bool = True):
     """Time one workload's decode step on this rank.
@@ -337,10 +360,21 @@ def measure(w, cache, step, path: str, K: int, warmup: int, flush, stream, dev, 
     step_ms = np.array([e0[k].elapsed_time(e1[k]) for k in range(K)])
     total_ms = max_over_ranks(float(step_ms.sum()), dev)
     ms_per_step = total_ms / K
+    KD = min(K, 300)  # the same replays after the write alone (L2 left full of dirty lines)
+    d0 = [torch.cuda.Event(enable_timing=True) for _ in range(KD)]
+    d1 = [torch.cuda.Event(enable_timing=True) for _ in range(KD)]
+    for k in range(KD):
+        flush.write_only(k & 0xFF)
+        d0[k].record(stream)
+        g_step.replay()
+        d1[k].record(stream)
+    torch.cuda.synchronize(dev)
+    ms_dirty = max_over_ranks(float(np.mean([d0[k].elapsed_time(d1[k]) for k in range(KD)])), dev)
 
     out = {"ms_per_step": ms_per_step, "tokens_per_s": world * w.B * K / (total_ms / 1e3),
            "nbytes": nbytes, "sel": sel, "cnt": cnt, "tier_tbl": tier_tbl, "names": [n for n, _ in parts],
-           "kernel_ms": per.mean(0), "clock_window": (t0, t2), "soak_steps": soak}
+           "kernel_ms": per.mean(0), "clock_window": (t0, t2), "soak_steps": soak,
+           "ms_per_step_write_only_flush": ms_dirty}
     if eager:
         KE = max(1, min(K, 200))
         a = [torch.cuda.Event(enable_timing=True) for _ in range(KE)]
@@ -393,7 +427,8 @@ def config_summary(name: str, w, m: dict, peak: float, dense_ms=None) -> dict:
     kr = m["kernels_roofline"]
     d = {"workload": f"{name}: {DESCR[name]}", "batch": w.B, "context_max": int(w.lens.max()),
          "selected_pages": int(m["cnt"].sum()), "ms_per_step": m["ms_per_step"], "tokens_per_s": m["tokens_per_s"],
-         "ms_per_step_eager": m.get("ms_per_step_eager"), "step_hbm": m["step_hbm"],
+         "ms_per_step_eager": m.get("ms_per_step_eager"),
+         "ms_per_step_write_only_flush": m.get("ms_per_step_write_only_flush"), "step_hbm": m["step_hbm"],
          "kernels_ms": {n: float(a) for n, a in zip(m["names"], m["kernel_ms"])},
          "attention_roofline": kr.get("sparse_decode_attn") or kr.get("decode_step"),
          "e2e": m.get("e2e")}
@@ -425,7 +460,7 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     peak, peak_kind = load_peaks()
-    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(args.flush_mib, dev)
     stream = torch.cuda.current_stream(dev)
     clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[0])
                           if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local_rank)
@@ -502,10 +537,13 @@ def run_kvq(args, rank: int, world: int, local_rank: int):
                    "host_tiers": args.host_tiers, "host_v_tiers": args.host_v_tiers,
                    "page_score": "mean-key" if not quad_rank else
                    f"quad (rank {quad_rank}, basis: eigenvectors of the key law's covariance)",
-                   "l2": f"flushed ({args.flush_mib} MiB write) before every timed step",
+                   "l2": f"flushed before every timed step: {args.flush_mib} MiB written, then "
+                         f"{flush.r.numel() * 4 >> 20} MiB read (no line of the step's data and no dirty "
+                         f"line in L2); ms_per_step_write_only_flush: the same steps after the write alone",
                    "parallelism": f"replicas x{world} (independent batches)"},
         "step_hbm": dict(m["step_hbm"], peak_kind=peak_kind),
         "ms_per_step_eager": m.get("ms_per_step_eager"),
+        "ms_per_step_write_only_flush": m.get("ms_per_step_write_only_flush"),
         "kernels_ms": {n: float(a) for n, a in zip(names, avg)},
         "kernels_roofline": m["kernels_roofline"],
         "roofline": {"bound": "hbm", "kernel": names[dom], "achieved": achieved, "peak": peak, "unit": "GB/s",
