@@ -102,7 +102,12 @@ def page_masses(scores: np.ndarray, P: int, L: int, sm_scale: float) -> np.ndarr
 
 def select_coverage(scores: np.ndarray, P: int, L: int, sm_scale: float, coverage: float, n_sink: int,
                     n_recent: int) -> np.ndarray:
-    """Coverage selection of one (sequence, kv head), ascending, int64."""
+    """Coverage selection of one (sequence, kv head), ascending, int64.
+
+    Candidates of zero mass (NaN or underflowed scores) are never added: they come last in
+    the mass order, and with coverage <= 1 the positive masses reach the target in exact
+    arithmetic, so the running fp64 sum can stop short of it only by rounding (at coverage
+    1), where adding pages that carry no mass would not be the rule's choice."""
     F = forced_pages(P, n_sink, n_recent)
     m = page_masses(scores, P, L, sm_scale)
     total = math.fsum(m)
@@ -111,7 +116,7 @@ def select_coverage(scores: np.ndarray, P: int, L: int, sm_scale: float, coverag
     order = sorted((p for p in range(P) if p not in F), key=lambda p: (-m[p], p))
     chosen = []
     for p in order:
-        if covered >= target:
+        if covered >= target or m[p] == 0.0:
             break
         chosen.append(p)
         covered += m[p]
@@ -130,7 +135,7 @@ def coverage_margin(scores: np.ndarray, P: int, L: int, sm_scale: float, coverag
     order = sorted((p for p in range(P) if p not in F), key=lambda p: (-m[p], p))
     covered = math.fsum(m[p] for p in F)
     k = 0
-    while k < len(order) and covered < target:
+    while k < len(order) and covered < target and m[order[k]] > 0.0:
         covered += m[order[k]]
         k += 1
     out = math.inf

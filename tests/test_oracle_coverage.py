@@ -87,3 +87,29 @@ def test_margin_is_small_only_near_a_decision():
     m = page_masses(s, P, L, 1.0)
     cut = math.fsum(m[:2]) / math.fsum(m)   # covering exactly the top two pages
     assert coverage_margin(s, P, L, 1.0, cut, 0, 0) < 1e-12
+
+
+def test_zero_mass_pages_are_never_needed():
+    """With coverage 1 the target is the total mass, which the positive masses reach in
+    exact arithmetic; pages of zero mass (NaN scores) are never chosen, every page of
+    positive mass is.  The seed is one where the fp64 running sum of the sorted positive
+    masses ends 3.6e-15 short of fsum of all masses, so a loop that only compared the
+    running sum with the target would go on into the NaN pages."""
+    rng = np.random.default_rng(2)
+    P, L = 24, 16 * 24
+    s = rng.normal(0, 3, P).astype(np.float32)
+    s[rng.integers(0, P, 5)] = np.nan
+    m = page_masses(s, P, L, 1.0)
+    F = forced_pages(P, 1, 1)
+    order = sorted((p for p in range(P) if p not in F), key=lambda p: (-m[p], p))
+    covered = math.fsum(m[p] for p in F)
+    for p in order:
+        if m[p] > 0:
+            covered += m[p]
+    assert covered < math.fsum(m)  # the rounding this case is chosen for
+    got = set(select_coverage(s, P, L, 1.0, 1.0, 1, 1).tolist())
+    assert got == F | {p for p in range(P) if m[p] > 0}
+    assert not any(np.isnan(s[p]) for p in got - F)
+    # the same pages without the NaNs: every page
+    s2 = np.where(np.isnan(s), np.float32(-1.0), s)
+    assert select_coverage(s2, P, L, 1.0, 1.0, 1, 1).size == P
