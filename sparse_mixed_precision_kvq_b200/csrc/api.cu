@@ -151,7 +151,7 @@ kvq_status kvq_select_topk(const kvq_cache* cache, const float* scores, const kv
   if ((size_t)c.max_pages * 4 > 200 * 1024) return KVQ_ERR_UNSUPPORTED;  // keys in shared memory
   if (params->coverage_ppm > 0) {
     if (params->coverage_ppm > 1000000 || !(params->sm_scale > 0.f)) return KVQ_ERR_INVALID_ARG;
-    const int n = coverage_sort_size(c, *params);
+    const int n = coverage_key_slots(c, *params);
     if (n == 0 || ((size_t)c.max_pages + 1) / 2 * 8 + (size_t)n * 8 > 200 * 1024) return KVQ_ERR_UNSUPPORTED;
   }
   return cuda_status(launch_select(c, scores, *params, sel, cnt, kmax, reinterpret_cast<cudaStream_t>(stream)));

@@ -277,7 +277,7 @@ cudaError_t launch_append_scores(const DevCache& c, const int32_t* pos, const vo
 constexpr size_t kScoreSelectCounterWord = 8192;  // workspace word of the per-(b, g) tile counters
 cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_select_params& prm,
                           int32_t* sel, int32_t* cnt, int kmax, cudaStream_t s);
-int coverage_sort_size(const DevCache& c, const kvq_select_params& prm);
+int coverage_key_slots(const DevCache& c, const kvq_select_params& prm);
 size_t attn_workspace_bytes(const DevCache& c, int num_ctas);
 int sm_count(int device);      // streaming multiprocessors of the device (cached)
 int attn_num_ctas(int device);  // grid of the fused step: sm_count, or the override

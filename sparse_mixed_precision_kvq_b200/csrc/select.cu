@@ -111,7 +111,7 @@ cudaError_t launch_select_t(const DevCache& c, const float* scores, const kvq_se
 // Mass-key slots coverage selection needs: the candidates of the longest possible
 // sequence (max_pages minus the forced pages), at least 1; 0 if above kCovMaxCand or if
 // the sequence's pages exceed kCovMaxPages.
-int coverage_sort_size(const DevCache& c, const kvq_select_params& prm) {
+int coverage_key_slots(const DevCache& c, const kvq_select_params& prm) {
   const int forced = max(prm.n_sink, 0) + max(prm.n_recent, 0);
   const int nc = max(1, c.max_pages - min(forced, c.max_pages));
   return nc <= kCovMaxCand && c.max_pages <= kCovMaxPages ? nc : 0;
@@ -122,7 +122,7 @@ cudaError_t launch_select(const DevCache& c, const float* scores, const kvq_sele
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
   const bool wide = (long long)c.B * c.Hkv * 4 <= sm_count(dev) && c.max_pages >= 4096;
-  const int ncov = prm.coverage_ppm > 0 ? coverage_sort_size(c, prm) : 0;
+  const int ncov = prm.coverage_ppm > 0 ? coverage_key_slots(c, prm) : 0;
   if (ncov > 0)
     return wide ? launch_select_t<1024, true>(c, scores, prm, sel, cnt, kmax, ncov, s)
                 : launch_select_t<512, true>(c, scores, prm, sel, cnt, kmax, ncov, s);
