@@ -231,3 +231,20 @@ def test_host_tiers_mask_checked_on_host():
 
 def test_requantize_arguments_checked_on_host():
     _run_without_gpu('_check_requantize_arguments_checked_on_host')
+
+
+def test_recorded_traffic_applies_only_to_its_workload_and_source():
+    """bench reports the ncu DRAM bytes of profiles/traffic.json only for a plain run of the
+    workload they were captured on, and only while the kernel's source (its file and the
+    package headers it includes) is the one captured."""
+    import json
+    import bench
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["attn.cu"]
+    assert bench.kernel_traffic("attn.cu", None) is None
+    other = "c2" if rec["workload"] != "c2" else "c1"
+    assert bench.kernel_traffic("attn.cu", other) is None
+    got = bench.kernel_traffic("attn.cu", rec["workload"])
+    if rec["source_sha256_16"] == bench.kernel_source_hash("attn.cu"):
+        assert got is not None and got["dram_bytes_per_launch"] == rec["dram_bytes_per_launch"]
+    else:
+        assert got is None
