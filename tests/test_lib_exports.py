@@ -204,6 +204,27 @@ def _check_requantize_arguments_checked_on_host():
     assert kvq._lib.kvq_requantize_pages(ref, None, 0, None) == 0
 
 
+def _check_coverage_limits_on_host():
+    """Coverage selection's limits are checked before anything is enqueued: at most 8192
+    candidates, at most 41984 pages (the cut's scratch), coverage <= 1, sm_scale > 0."""
+    from sparse_mixed_precision_kvq_b200 import kvq
+    c = kvq.KvqCache()
+    c.B, c.Hq, c.Hkv, c.D, c.page_size, c.dtype = 1, 8, 2, 64, 16, 1
+    c.block_table = c.seq_len = c.summary = c.open_ksum = c.err_word = 4096
+    c.pool[0], c.pool_slots[0] = 4096, 4
+    ref = ctypes.byref(c)
+
+    def sel(max_pages, ns, nr, ppm, scale):
+        c.max_pages = max_pages
+        prm = kvq.SelectParams(-1, 0, ns, nr, ppm, scale)
+        return kvq._lib.kvq_select_topk(ref, 4096, ctypes.byref(prm), 4096, 4096, max_pages, None)
+
+    assert sel(9000, 0, 0, 950000, 0.1) == 2            # 9000 candidates > 8192
+    assert sel(42000, 1, 33999, 950000, 0.1) == 2       # 8000 candidates, but 42000 pages > 41984
+    assert sel(4000, 1, 4, 1000001, 0.1) == 1           # coverage above 1
+    assert sel(4000, 1, 4, 950000, 0.0) == 1            # sm_scale 0
+
+
 def _run_without_gpu(check: str):
     """Run ``check`` (a function of this module) in a child process that sees no CUDA
     device.  These checks hand made-up device addresses to the entry points and rely on
@@ -231,6 +252,10 @@ def test_host_tiers_mask_checked_on_host():
 
 def test_requantize_arguments_checked_on_host():
     _run_without_gpu('_check_requantize_arguments_checked_on_host')
+
+
+def test_coverage_limits_checked_on_host():
+    _run_without_gpu('_check_coverage_limits_on_host')
 
 
 def test_recorded_traffic_applies_only_to_its_workload_and_source():
