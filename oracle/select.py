@@ -81,7 +81,9 @@ def kth_margin(scores: np.ndarray, P: int, k_abs: int, k_frac_bp: int, n_sink: i
 # tokens, the score standing in for each token's logit), normalised over all pages of the
 # (sequence, kv head).  The forced pages are attended and count as covered; candidates are
 # then added by estimated mass (larger first, lower page index first on ties) until the
-# covered mass reaches ``coverage`` of the total.  A NaN score has mass 0.
+# covered mass reaches ``coverage`` of the total.  A NaN score has mass 0, and pages of
+# zero mass are never added (in exact arithmetic the positive masses reach any target up
+# to the total).
 
 def page_masses(scores: np.ndarray, P: int, L: int, sm_scale: float) -> np.ndarray:
     """Estimated mass of pages 0..P-1 (fp64), relative to the largest score's page."""
