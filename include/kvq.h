@@ -263,7 +263,7 @@ kvq_status kvq_set_grid_override(int32_t ctas);
  *            scaled logits (-inf when nothing is selected).
  *  workspace device scratch of at least kvq_workspace_size() bytes, prepared once with
  *            kvq_workspace_init (split-K partials; the last CTA of each (b, kv head) merges
- *            them, counted by arrival counters the call leaves at zero).  B*Hkv < 6144.
+ *            them, counted by arrival counters the call leaves at zero).  B*Hkv < 5632.
  */
 kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const int32_t* sel,
                                   const int32_t* cnt, int32_t kmax, float sm_scale, void* out,
@@ -279,7 +279,7 @@ kvq_status kvq_sparse_decode_attn(const kvq_cache* cache, const void* q, const i
  *  scratch is a static device array of kvq_noalloc_scratch_bytes() (16 MiB) inside the
  *  library, held by every GPU that loads it until the process exits.  Allocates nothing
  *  (no cudaMalloc/cudaFree).  Returns KVQ_ERR_WORKSPACE when kvq_workspace_size() for
- *  this cache exceeds the static size, and KVQ_ERR_UNSUPPORTED for B*Hkv >= 6144 as
+ *  this cache exceeds the static size, and KVQ_ERR_UNSUPPORTED for B*Hkv >= 5632 as
  *  kvq_sparse_decode_attn does.  Each call made outside a stream capture looks up the
  *  array's device address on the current device (cudaGetSymbolAddress; a re-created
  *  context gets its new address); a call made while the stream captures reuses the last

@@ -16,7 +16,10 @@ constexpr int kPage = 16;       // tokens per page
 constexpr int kGroup = 32;      // channels per quantisation group
 constexpr int kMaxG = 8;        // query heads per kv head handled by one mma N-tile
 constexpr int kNumTiers = 6;
-constexpr int kMaxSegments = 6144;  // B * Hkv limit of the attention kernel (offsets in shared memory)
+// B * Hkv limit of the attention kernel: its segment offsets and completion list live in
+// shared memory beside the one-CTA-per-SM 24 KB-per-warp page rings (196,608 + 1,792 +
+// 6 * B*Hkv bytes, within the 227 KB a CTA may hold up to 5,651 segments)
+constexpr int kMaxSegments = 5632;
 // Head of every workspace: counters that must be zero when a call starts (every call
 // leaves them zero); kvq_workspace_init zeroes it once.
 constexpr size_t kCounterBytes = 65536;

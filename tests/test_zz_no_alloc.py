@@ -64,7 +64,7 @@ def test_noalloc_rejects_a_batch_beyond_the_static_scratch():
 
 
 def test_noalloc_status_matches_the_workspace_entry_point():
-    """B*Hkv >= 6144 segments: both entry points answer "unsupported"."""
+    """B*Hkv >= 5632 segments: both entry points answer "unsupported"."""
     from sparse_mixed_precision_kvq_b200 import kvq
     B, Hq, Hkv, D = 3100, 4, 2, 128
     cache = kvq.PagedCache(B, Hq, Hkv, D, 1, "bf16", [B, 0, 0, 0, 0])
@@ -78,3 +78,35 @@ def test_noalloc_status_matches_the_workspace_entry_point():
     with pytest.raises(kvq.KvqError, match="unsupported"):
         kvq.kvq_sparse_decode_attn_noalloc(cache, q, sel, cnt, 1, 0.1, out, None)
 
+
+
+@pytest.mark.parametrize("B, ok", [(2815, True), (3000, False)])
+def test_segment_limit_boundary(B, ok):
+    """The attention's shared memory grows by 6 bytes per (sequence, kv head) segment beside
+    the 16-bit-only kernel's 24 KB-per-warp rings: 5630 segments launch (every one empty:
+    zero outputs, -inf lse), 6000 would exceed a CTA's 227 KB and are refused on the host
+    with "unsupported" by both entry points instead of failing the launch."""
+    from sparse_mixed_precision_kvq_b200 import kvq
+    Hq, Hkv, D = 4, 2, 128
+    cache = kvq.PagedCache(B, Hq, Hkv, D, 1, "bf16", [B, 0, 0, 0, 0])
+    q = torch.zeros((B, Hq, D), dtype=torch.bfloat16, device="cuda")
+    sel = torch.zeros((B, Hkv, 1), dtype=torch.int32, device="cuda")
+    cnt = torch.zeros((B, Hkv), dtype=torch.int32, device="cuda")
+    out = torch.full_like(q, 7.0)
+    lse = torch.zeros((B, Hq), dtype=torch.float32, device="cuda")
+    if ok:
+        ws = torch.zeros(kvq.kvq_workspace_size(cache, 1) // 4 + 4, dtype=torch.float32, device="cuda")
+        kvq.kvq_workspace_init(ws)
+        kvq.kvq_sparse_decode_attn(cache, q, sel, cnt, 1, 0.1, out, lse, ws)
+        torch.cuda.synchronize()
+        assert not out.float().abs().sum().item() and bool(torch.isneginf(lse).all())
+        out.fill_(7.0)
+        kvq.kvq_sparse_decode_attn_noalloc(cache, q, sel, cnt, 1, 0.1, out, lse)
+        torch.cuda.synchronize()
+        assert not out.float().abs().sum().item()
+    else:
+        ws = torch.zeros(1 << 14, dtype=torch.float32, device="cuda")
+        with pytest.raises(kvq.KvqError, match="unsupported"):
+            kvq.kvq_sparse_decode_attn(cache, q, sel, cnt, 1, 0.1, out, lse, ws)
+        with pytest.raises(kvq.KvqError, match="unsupported"):
+            kvq.kvq_sparse_decode_attn_noalloc(cache, q, sel, cnt, 1, 0.1, out, lse)
